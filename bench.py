@@ -1,0 +1,632 @@
+#!/usr/bin/env python
+"""Throughput of block top-k sparse decode attention on B200.
+
+One step = one decode step of one attention layer for a whole batch:
+  block-summary maintenance (last block) -> block scoring + top-k selection
+  -> gathered split-KV attention over the selected blocks,
+all three in libksa's CUDA kernels.  Metric: queries/s, one query = one
+sequence's decode step for one layer (all query heads).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ksa|reference]
+                  [--workload qwen3-0.6b|qwen3-8b|lessismore|sweep-L<ctx>-B<budget>|dense-L<ctx>]
+
+The default workload is the Qwen3-0.6B-shaped layer (batch 64, Hq 16, Hkv 8,
+D 128, context 16384, block 32, 32 blocks kept).  With N > 1 (torchrun, one
+rank per GPU) every rank runs the same per-GPU batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+Rank 0 prints one JSON line on stdout; diagnostics go to stderr.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "sparse decode-attn queries/s at 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
+UNIT = "queries/s"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=100)
+    p.add_argument("--impl", choices=["ksa", "reference"], default="ksa")
+    p.add_argument("--workload", default="qwen3-0.6b")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="wall-clock budget of the oracle CPU baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; no collective on the data path)
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            if torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        dev = f"cuda:{self.local}" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        dev = f"cuda:{self.local}" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# workloads
+
+
+def resolve_workload(name: str):
+    from block_top_sparse_ksa_b200 import synth
+    if name == "qwen3-0.6b":
+        return "block", synth.QWEN3_0_6B
+    if name == "qwen3-8b":
+        return "block", synth.QWEN3_8B
+    if name == "tiny":
+        return "block", synth.TINY
+    if name == "lessismore":
+        return "unified", synth.LESSISMORE
+    if name.startswith("sweep-L"):
+        ctx, budget = name[len("sweep-L"):].split("-B")
+        return "block", synth.sweep_shape(int(ctx), int(budget))
+    if name.startswith("dense-L"):
+        return "dense", synth.sweep_shape(int(name[len("dense-L"):]), 256)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def make_block_inputs(shape, device):
+    from block_top_sparse_ksa_b200 import synth
+    if shape.name == synth.QWEN3_0_6B.name:
+        return synth.qwen3_0_6b_inputs(device=device)
+    if shape.name == synth.QWEN3_8B.name:
+        return synth.qwen3_8b_inputs(device=device)
+    if shape.name == synth.TINY.name:
+        return synth.tiny_inputs(device=device)
+    return synth.sweep_inputs(shape, device=device)
+
+
+def query_sets(shape, count, device):
+    from block_top_sparse_ksa_b200 import synth
+    noise = 0.1 if shape.name.startswith("qwen3-0.6b") else None
+    return synth.make_queries(shape, 5000, count, device, group_noise=noise)
+
+
+def algorithmic_bytes(shape, seq_lens, kind: str):
+    """Per step: summaries read (when k < NB_b) + selected K/V + q + out (fp32).
+    Also returns the attention kernel's share (selected K/V + q + out)."""
+    bs, Hkv, Hq, D = shape.block_size, shape.num_kv_heads, shape.num_q_heads, shape.head_dim
+    k = shape.k_blocks
+    summ = kv = 0
+    for L in seq_lens:
+        nb = -(-int(L) // bs)
+        if kind == "dense":
+            kv += Hkv * int(L) * D * 2 * 2
+            continue
+        if k < nb:
+            summ += Hkv * nb * D * 4
+        kv += Hkv * min(k * bs, int(L)) * D * 2 * 2
+    qo = len(seq_lens) * Hq * D * (2 + 4)
+    return summ + kv + qo, kv + qo, summ
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and self.uuid not in parts[1] and parts[1] not in self.uuid:
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[6 + i]
+                          and "Not" not in r[6 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# timed runs
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source
+    is unchanged since the capture (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+        ent = rec[kernel][workload]
+        src = open(os.path.join(ROOT, ent["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha256_16"]:
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def run_block(args, dist, dev, kind):
+    import block_top_sparse_ksa_b200 as ksa
+    _, shape = resolve_workload(args.workload)
+    torch.manual_seed(0)
+    inp = make_block_inputs(shape, dev)
+    B, Hq, Hkv, D, T, bs = (shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
+                            shape.capacity, shape.block_size)
+    k = shape.k_blocks
+    nq = 16
+    qs = query_sets(shape, nq, dev)
+    S = ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs)  # prefill, untimed
+    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        q = qs[i % nq]
+        if kind == "dense":
+            ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, stream=stream)
+            return
+        ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, ksa.SUMMARY_LAST_BLOCK,
+                                      summaries=S, stream=stream)
+        ksa.ksa_select_blocks(q, S, inp.seq_lens, bs, T, k, block_idx=idx, num_sel=cnt,
+                              stream=stream)
+        ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt, tokens_per_idx=bs,
+                                   out=out, stream=stream)
+
+    launches_per_step = 1 if kind == "dense" else 3
+    for i in range(args.warmup):
+        step(i)
+    # per-kernel events on a sample of the timed steps
+    every = max(1, args.steps // 400)
+    marks = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index or 0)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        if i % every == 0:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            q = qs[i % nq]
+            ev[0].record(stream)
+            if kind == "dense":
+                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, stream=stream)
+                ev[1].record(stream)
+                ev[2].record(stream)
+            else:
+                ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, ksa.SUMMARY_LAST_BLOCK,
+                                              summaries=S, stream=stream)
+                ev[1].record(stream)
+                ksa.ksa_select_blocks(q, S, inp.seq_lens, bs, T, k, block_idx=idx, num_sel=cnt,
+                                      stream=stream)
+                ev[2].record(stream)
+                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt,
+                                           tokens_per_idx=bs, out=out, stream=stream)
+            ev[3].record(stream)
+            marks.append(ev)
+        else:
+            step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dist.barrier()
+    ms_local = start.elapsed_time(end)
+    ms = dist.max(ms_local)
+    t_sum = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    t_sel = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
+    t_att = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
+    lens = inp.seq_lens.cpu().tolist()
+    total_b, attn_b, summ_b = algorithmic_bytes(shape, lens, kind)
+    per_step_s = ms / 1e3 / args.steps
+    value = dist.sum(B) / per_step_s  # every rank processed B queries per step
+    peak, peak_kind = measured_peak()
+    attn_gbs = attn_b / (t_att * 1e-3) / 1e9
+    res = {
+        "ms_per_step": ms / args.steps,
+        "value": value,
+        "kernels_ms": {"summaries_last_block": t_sum, "select_blocks": t_sel,
+                       "sparse_decode_attn": t_att},
+        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": attn_gbs / peak,
+                     "traffic": stored_traffic("sparse_decode_attn", args.workload),
+                     "kernel": "sparse_decode_attn", "peak_source": peak_kind,
+                     "bytes_per_launch": attn_b},
+        "step_hbm": {"bytes_per_step": total_b, "gbs": total_b / per_step_s / 1e9,
+                     "frac": total_b / per_step_s / 1e9 / peak},
+        "select_hbm": {"bytes_per_launch": summ_b,
+                       "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "config": {"workload": shape.name, "batch_per_gpu": B, "num_q_heads": Hq,
+                   "num_kv_heads": Hkv, "head_dim": D, "capacity": T, "block_size": bs,
+                   "k_blocks": k if kind != "dense" else "all",
+                   "l2": "inputs larger than L2: K/V cache %.1f GB, %.0f MB read per step, %d "
+                         "rotating query sets" % (2 * inp.K.numel() * 2 / 1e9, total_b / 1e6, nq),
+                   "step": ("dense attention" if kind == "dense" else
+                            "summaries(last block) + select_blocks + sparse_decode_attn")},
+    }
+    if not args.no_e2e:
+        res["e2e"] = run_block_e2e(args, dist, dev, kind, inp, S, qs, shape)
+    res["_host"] = (inp, S, qs, shape, kind)
+    return res
+
+
+def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape):
+    """Same step through the public API with host buffers: per step the new
+    query and the new token's K/V rows go host->device (pinned), the output
+    comes back device->host.  Copies are inside the timed region."""
+    import block_top_sparse_ksa_b200 as ksa
+    B, Hq, Hkv, D, T, bs = (shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
+                            shape.capacity, shape.block_size)
+    k = shape.k_blocks
+    nq = qs.shape[0]
+    h_q = qs.cpu().pin_memory()
+    h_kv = torch.randn((nq, 2, B, Hkv, D), dtype=torch.float32).to(torch.bfloat16).pin_memory()
+    h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    d_q = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+    d_kv = torch.empty((2, B, Hkv, D), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    lens = inp.seq_lens
+    pos = (lens.long() - 1)  # the newest token's slot per row
+    ar_b = torch.arange(B, device=dev)
+
+    def step(i):
+        d_q.copy_(h_q[i % nq], non_blocking=True)
+        d_kv.copy_(h_kv[i % nq], non_blocking=True)
+        # append: write the new K/V rows into their cache slots
+        inp.K[ar_b, :, pos] = d_kv[0]
+        inp.V[ar_b, :, pos] = d_kv[1]
+        if kind == "dense":
+            ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, out=out, stream=stream)
+        else:
+            ksa.ksa_build_block_summaries(inp.K, lens, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S,
+                                          stream=stream)
+            ksa.ksa_select_blocks(d_q, S, lens, bs, T, k, block_idx=idx, num_sel=cnt,
+                                  stream=stream)
+            ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, idx, cnt, tokens_per_idx=bs,
+                                       out=out, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    steps = args.steps
+    for i in range(args.warmup):
+        step(i)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = dist.max(start.elapsed_time(end))
+    per = ms / 1e3 / steps
+    h2d = (B * Hq * D + 2 * B * Hkv * D) * 2
+    d2h = B * Hq * D * 4
+    return {"value": dist.sum(B) / per, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
+            "note": "cache append of the new token is a torch index copy"}
+
+
+def run_unified(args, dist, dev):
+    import block_top_sparse_ksa_b200 as ksa
+    from block_top_sparse_ksa_b200 import synth
+    sh = synth.LESSISMORE
+    inp = synth.lessismore_inputs(device=dev)
+    B, Hq, Hkv, D, T = sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, sh.capacity
+    ws = torch.empty((ksa.ksa_unified_select_workspace(B, Hq, Hkv, D, T, sh.per_head_topk,
+                                                       sh.token_budget),),
+                     dtype=torch.uint8, device=dev)
+    tok = torch.empty((B, sh.token_budget), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+    outs = [torch.empty((B, Hq, D), dtype=torch.float32, device=dev) for _ in inp.layers]
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        if ev:
+            ev[0].record(stream)
+        ksa.ksa_unified_select(inp.q_sel, inp.K_sel, inp.seq_lens, sh.per_head_topk,
+                               sh.token_budget, sh.recent_tokens, tok, cnt, ws, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        for li, (q, K, V) in enumerate(inp.layers):
+            ksa.ksa_sparse_decode_attn(q, K, V, inp.seq_lens, tok, cnt, tokens_per_idx=1,
+                                       idx_shared=True, out=outs[li], stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    every = max(1, args.steps // 200)
+    marks = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index or 0)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        if i % every == 0:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            step(i, ev)
+            marks.append(ev)
+        else:
+            step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = dist.max(start.elapsed_time(end))
+    t_sel = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    t_att = statistics.mean(m[1].elapsed_time(m[2]) for m in marks) / len(inp.layers)
+    per = ms / 1e3 / args.steps
+    sel_b = B * Hkv * sh.seq_len * D * 2 + B * Hq * D * 2
+    att_b = B * Hkv * sh.token_budget * D * 2 * 2 + B * Hq * D * 6
+    peak, peak_kind = measured_peak()
+    return {
+        "ms_per_step": ms / args.steps, "value": dist.sum(B) / per,
+        "kernels_ms": {"unified_select": t_sel, "sparse_decode_attn_per_layer": t_att},
+        "roofline": {"bound": "hbm", "achieved": att_b / (t_att * 1e-3) / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": att_b / (t_att * 1e-3) / 1e9 / peak,
+                     "traffic": stored_traffic("sparse_decode_attn", args.workload),
+                     "kernel": "sparse_decode_attn (token list)", "peak_source": peak_kind,
+                     "bytes_per_launch": att_b},
+        "select_hbm": {"bytes_per_launch": sel_b, "gbs": sel_b / (t_sel * 1e-3) / 1e9},
+        "step_hbm": {"bytes_per_step": sel_b + 3 * att_b,
+                     "gbs": (sel_b + 3 * att_b) / per / 1e9},
+        "gpu_launches": (3 + len(inp.layers)) * args.steps, "clocks": clk,
+        "config": {"workload": sh.name, "batch_per_gpu": B, "num_q_heads": Hq,
+                   "num_kv_heads": Hkv, "head_dim": D, "context": sh.seq_len,
+                   "per_head_topk": sh.per_head_topk, "token_budget": sh.token_budget,
+                   "recent_tokens": sh.recent_tokens, "sparse_layers": sh.sparse_layers,
+                   "l2": "inputs larger than L2 (4 x 1.3 GB K/V per layer)",
+                   "step": "unified_select + 3 x sparse_decode_attn (one query = one sequence's "
+                           "selection layer + 3 sparse layers)"},
+    }
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+
+
+def oracle_block_sample(shape, kind, n_rows, device):
+    """Host copies of n_rows rows of the workload, summaries by the oracle (untimed prefill)."""
+    from block_top_sparse_ksa_b200 import synth
+    from oracle import oracle as O
+    small = synth.dataclasses.replace(shape, batch=n_rows)
+    inp = make_block_inputs(small, device)
+    qs = query_sets(small, 4, device)
+    o = O.get()
+    lens = inp.seq_lens.cpu().numpy()
+    K, V = synth.bits(inp.K), synth.bits(inp.V)
+    qb = [synth.bits(qs[i]) for i in range(qs.shape[0])]
+    S = None if kind == "dense" else o.block_summaries(K, lens, shape.block_size)
+    return o, qb, K, V, S, lens
+
+
+def oracle_step_units(o, shape, kind, q, K, V, S, lens, rows):
+    """One oracle decode step over the given rows: scores, top-k, attention."""
+    bs, k = shape.block_size, shape.k_blocks
+    sel = np.asarray(rows)
+    qv, Kv, Vv, Lv = q[sel], K[sel], V[sel], lens[sel]
+    if kind == "dense":
+        o.attention(qv, Kv, Vv, Lv)
+        return
+    s = o.block_scores(qv, S[sel], Lv, bs)
+    n, hkv = s.shape[0], s.shape[1]
+    idx = np.full((n, hkv, k), -1, np.int32)
+    cnt = np.zeros((n, hkv), np.int32)
+    for b in range(n):
+        nb = -(-int(Lv[b]) // bs)
+        for g in range(hkv):
+            got = o.topk(s[b, g, :nb], k)
+            idx[b, g, :len(got)] = got
+            cnt[b, g] = len(got)
+    o.attention(qv, Kv, Vv, Lv, idx, cnt, bs)
+
+
+def cpu_baseline(args, dev, kind, budget_s):
+    _, shape = resolve_workload(args.workload)
+    n_rows = min(8, shape.batch)
+    o, qb, K, V, S, lens = oracle_block_sample(shape, kind, n_rows, dev)
+    o.set_threads(os.cpu_count() or 1)
+    rows_done = 0
+    t0 = time.perf_counter()
+    i = 0
+    while True:
+        oracle_step_units(o, shape, kind, qb[i % len(qb)], K, V, S, lens, list(range(n_rows)))
+        rows_done += n_rows
+        i += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": rows_done / el, "unit": UNIT, "cores": o.max_threads(), "kind": "oracle",
+            "sample": f"{n_rows} rows of {shape.name}, {i} steps of oracle block scores + top-k "
+                      f"+ attention (summaries precomputed, as the GPU prefill), {el:.1f} s"}
+
+
+def run_reference(args, dist):
+    """The oracle as the reference arm: same workload/metric, host cores."""
+    if dist.rank != 0:
+        return
+    kind, shape = resolve_workload(args.workload)
+    dev = torch.device("cuda", dist.local) if torch.cuda.is_available() else torch.device("cpu")
+    if kind == "unified":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the oracle arm covers the block top-k workloads only"}))
+        return
+    n_rows = min(8, shape.batch)
+    o, qb, K, V, S, lens = oracle_block_sample(shape, kind, n_rows, dev)
+    o.set_threads(os.cpu_count() or 1)
+    # size one step so that warmup + steps take about two minutes
+    t0 = time.perf_counter()
+    oracle_step_units(o, shape, kind, qb[0], K, V, S, lens, [0])
+    t_row = max(time.perf_counter() - t0, 1e-4)
+    per_step = min(n_rows, max(1, int(120.0 / (args.steps + args.warmup) / t_row)))
+    rows = list(range(per_step))
+    for i in range(args.warmup):
+        oracle_step_units(o, shape, kind, qb[i % 4], K, V, S, lens, rows)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step_units(o, shape, kind, qb[i % 4], K, V, S, lens, rows)
+    el = time.perf_counter() - t0
+    value = per_step * args.steps / el
+    sample = (f"{per_step} of {shape.batch} rows of {shape.name} per step (oracle block scores "
+              f"+ top-k + attention, fp64, summaries precomputed)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": shape.name, "batch_per_gpu": shape.batch,
+                   "sample_rows_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": o.max_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)  # rank 0 only; no process group is needed
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    dist.init("nccl")
+    import block_top_sparse_ksa_b200 as ksa
+    ksa.lib()  # fails loudly if libksa.so is missing
+    kind, _ = resolve_workload(args.workload)
+    try:
+        if kind == "unified":
+            res = run_unified(args, dist, dev)
+        else:
+            res = run_block(args, dist, dev, kind)
+        host = res.pop("_host", None)
+        del host
+        line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": dist.world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (seeded; no dataset or weights)",
+                "config": dict(res["config"], parallelism=f"dp{dist.world} (batch-sharded "
+                               "replicas, no data-path collective)"),
+                "roofline": res["roofline"], "kernels_ms": res["kernels_ms"],
+                "step_hbm": res["step_hbm"], "select_hbm": res.get("select_hbm"),
+                "gpu_launches": res["gpu_launches"], "clocks": res["clocks"]}
+        if "e2e" in res:
+            line["e2e"] = res["e2e"]
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and kind != "unified":
+            line["cpu_baseline"] = cpu_baseline(args, dev, kind, args.cpu_seconds)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

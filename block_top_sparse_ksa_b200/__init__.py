@@ -1,0 +1,244 @@
+"""block_top_sparse_ksa_b200 -- Python binding of libksa (include/ksa.h).
+
+Block top-k sparse decode attention over a GQA KV cache and LessIsMore unified
+token selection on NVIDIA B200.  This module only marshals arguments: it takes
+torch CUDA tensors (device memory) and the current torch CUDA stream, and calls
+the C ABI.  Every step of the computation runs in libksa's CUDA kernels; there
+is no CPU or PyTorch fallback.  If ``libksa.so`` is missing, loading fails with
+an error that says how to build it.
+
+Layouts (row-major, contiguous):
+  q [B, Hq, D] bf16;  K, V [B, Hkv, T, D] bf16;  seq_lens [B] int32;
+  summaries [B, Hkv, ceil(T/bs), D] fp32;  block_idx [B, Hkv, k] int32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "KsaError", "Shape", "lib", "library_path", "ksa_build_block_summaries",
+    "ksa_select_blocks", "ksa_sparse_decode_attn", "ksa_unified_select",
+    "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
+    "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "OUT_F32", "OUT_BF16", "FLAG_SEQ_LEN_CLAMPED",
+    "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libksa.so")
+
+SUMMARY_ALL, SUMMARY_LAST_BLOCK = 0, 1
+OUT_F32, OUT_BF16 = 0, 1
+FLAG_SEQ_LEN_CLAMPED, FLAG_INDEX_SKIPPED, FLAG_NONFINITE_SCORE, FLAG_WAIT_TIMEOUT = 1, 2, 4, 8
+_STATUS = {0: "KSA_OK", 1: "KSA_ERR_INVALID_ARG", 2: "KSA_ERR_UNSUPPORTED",
+           3: "KSA_ERR_WORKSPACE", 4: "KSA_ERR_CUDA"}
+
+
+class KsaError(RuntimeError):
+    """A libksa call returned a non-OK status."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("capacity", ctypes.c_int32), ("block_size", ctypes.c_int32)]
+
+
+_vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "ksa_build_block_summaries": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _i32, _vp, _vp, _vp]),
+    "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
+    "ksa_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz,
+                                 _vp, _vp]),
+    "ksa_sparse_decode_attn_workspace": (_sz, [ctypes.POINTER(Shape), _i32, _i32]),
+    "ksa_sparse_decode_attn": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                                      _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "ksa_unified_select_workspace": (_sz, [ctypes.POINTER(Shape), _i32, _i32]),
+    "ksa_unified_select": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _i32, _i32, _vp,
+                                  _vp, _vp, _sz, _vp, _vp]),
+    "ksa_status_string": (ctypes.c_char_p, [_i32]),
+    "ksa_last_error": (ctypes.c_char_p, []),
+    "ksa_version": (_i32, []),
+}
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libksa (raises if it was never built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(
+                f"{library_path} is missing: build it with "
+                "`python -m block_top_sparse_ksa_b200.build` (needs nvcc)")
+        handle = ctypes.CDLL(library_path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = handle
+    return _LIB
+
+
+def ksa_status_string(status: int) -> str:
+    return lib().ksa_status_string(int(status)).decode()
+
+
+def ksa_last_error() -> str:
+    return lib().ksa_last_error().decode()
+
+
+def ksa_version() -> int:
+    return int(lib().ksa_version())
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise KsaError(status, ksa_last_error())
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _shape(B, Hq, Hkv, D, T, bs=16) -> Shape:
+    return Shape(int(B), int(Hq), int(Hkv), int(D), int(T), int(bs))
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+
+
+def ksa_build_block_summaries(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                              mode: int = SUMMARY_ALL, summaries: Optional[torch.Tensor] = None,
+                              dev_status: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """Block mean keys S [B, Hkv, ceil(T/bs), D] fp32 (all blocks, or the last one)."""
+    _dev(K, "K", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hkv, T, D = K.shape
+    nb = -(-T // block_size)
+    if summaries is None:
+        summaries = torch.empty((B, Hkv, nb, D), dtype=torch.float32, device=K.device)
+    _dev(summaries, "summaries", torch.float32)
+    sh = _shape(B, Hkv, Hkv, D, T, block_size)
+    _check(lib().ksa_build_block_summaries(ctypes.byref(sh), _ptr(K), _ptr(seq_lens), int(mode),
+                                           _ptr(summaries), _ptr(dev_status), _stream(stream)))
+    return summaries
+
+
+def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.Tensor,
+                      block_size: int, capacity: int, k_blocks: int,
+                      block_idx: Optional[torch.Tensor] = None,
+                      num_sel: Optional[torch.Tensor] = None,
+                      dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Top-k blocks per (row, kv-head): (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv])."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(summaries, "summaries", torch.float32)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    Hkv = summaries.shape[1]
+    if block_idx is None:
+        block_idx = torch.empty((B, Hkv, k_blocks), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    sh = _shape(B, Hq, Hkv, D, capacity, block_size)
+    _check(lib().ksa_select_blocks(ctypes.byref(sh), _ptr(q), _ptr(summaries), _ptr(seq_lens),
+                                   int(k_blocks), _ptr(block_idx), _ptr(num_sel), None, 0,
+                                   _ptr(dev_status), _stream(stream)))
+    return block_idx, num_sel
+
+
+def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                           seq_lens: torch.Tensor, idx: Optional[torch.Tensor] = None,
+                           num_idx: Optional[torch.Tensor] = None, tokens_per_idx: int = 1,
+                           idx_shared: bool = False, scale: float = 0.0,
+                           out_dtype: int = OUT_F32, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None,
+                           dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Softmax attention over the selected tokens (dense when idx is None): (out, lse)."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(V, "V", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    cap = 0
+    if idx is not None:
+        _dev(idx, "idx", torch.int32)
+        _dev(num_idx, "num_idx", torch.int32)
+        cap = idx.shape[-1]
+    odt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=odt, device=q.device)
+    _dev(out, "out", odt)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32)
+    sh = _shape(B, Hq, Hkv, D, T, max(1, tokens_per_idx))
+    _check(lib().ksa_sparse_decode_attn(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx), _ptr(num_idx),
+        int(cap), int(tokens_per_idx), int(bool(idx_shared)), float(scale), int(out_dtype),
+        _ptr(out), _ptr(lse), None, 0, _ptr(dev_status), _stream(stream)))
+    return out, lse
+
+
+def ksa_unified_select_workspace(B: int, Hq: int, Hkv: int, D: int, T: int, per_head_topk: int,
+                                 token_budget: int) -> int:
+    sh = _shape(B, Hq, Hkv, D, T)
+    return int(lib().ksa_unified_select_workspace(ctypes.byref(sh), int(per_head_topk),
+                                                  int(token_budget)))
+
+
+def ksa_unified_select(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor,
+                       per_head_topk: int, token_budget: int, recent_tokens: int = -1,
+                       token_idx: Optional[torch.Tensor] = None,
+                       num_sel: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None,
+                       dev_status: Optional[torch.Tensor] = None, stream=None):
+    """LessIsMore selection: (token_idx [B, budget] ascending -1 padded, num_sel [B])."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    need = ksa_unified_select_workspace(B, Hq, Hkv, D, T, per_head_topk, token_budget)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    if token_idx is None:
+        token_idx = torch.empty((B, token_budget), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B,), dtype=torch.int32, device=q.device)
+    sh = _shape(B, Hq, Hkv, D, T)
+    _check(lib().ksa_unified_select(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(seq_lens), int(per_head_topk),
+        int(token_budget), int(recent_tokens), _ptr(token_idx), _ptr(num_sel), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+    return token_idx, num_sel

@@ -1,0 +1,328 @@
+// ksa_api.cu -- the C ABI of libksa (declared in include/ksa.h).
+//
+// Host-side argument validation, status codes and messages, TMA descriptor
+// encoding, and the launches.  Nothing here allocates device memory or
+// synchronises the host.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/ksa.h"
+#include "ksa_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ksa_status fail(ksa_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+ksa_status fail(ksa_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+ksa_status cuda_status(cudaError_t err, const char *what) {
+  if (err == cudaSuccess) {
+    g_last_error.clear();
+    return KSA_OK;
+  }
+  return fail(KSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+ksa_status check_shape(const ksa_shape *s, bool need_block) {
+  if (s == nullptr) return fail(KSA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->num_q_heads < 1 || s->num_kv_heads < 1 || s->capacity < 1)
+    return fail(KSA_ERR_INVALID_ARG, "batch, heads and capacity must be >= 1");
+  if (s->num_q_heads % s->num_kv_heads != 0)
+    return fail(KSA_ERR_INVALID_ARG, "num_q_heads (%d) is not a multiple of num_kv_heads (%d)",
+                s->num_q_heads, s->num_kv_heads);
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(KSA_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", s->head_dim);
+  if (need_block && s->block_size != 16 && s->block_size != 32 && s->block_size != 64)
+    return fail(KSA_ERR_UNSUPPORTED, "block_size %d not supported (16, 32 or 64)",
+                s->block_size);
+  const long long rows = static_cast<long long>(s->batch) * s->num_kv_heads * s->capacity;
+  if (rows >= (1LL << 31))
+    return fail(KSA_ERR_UNSUPPORTED, "batch * num_kv_heads * capacity must be < 2^31");
+  if (static_cast<long long>(s->batch) * s->num_kv_heads * 8 >= (1LL << 31))
+    return fail(KSA_ERR_UNSUPPORTED, "batch * num_kv_heads too large");
+  return KSA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+namespace ksa {
+
+bool encode_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int D,
+                          int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2u};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estride[2] = {1u, 1u};
+  const CUresult r =
+      fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace ksa
+
+extern "C" {
+
+ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
+                                     const int32_t *seq_lens, int32_t mode, float *summaries,
+                                     uint32_t *dev_status, void *stream) {
+  ksa_status st = check_shape(shape, true);
+  if (st != KSA_OK) return st;
+  if (K == nullptr || seq_lens == nullptr || summaries == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "K, seq_lens and summaries must be non-NULL");
+  if (mode != KSA_SUMMARY_ALL && mode != KSA_SUMMARY_LAST_BLOCK)
+    return fail(KSA_ERR_INVALID_ARG, "mode %d is neither ALL nor LAST_BLOCK", mode);
+  if (!aligned(K, 16) || !aligned(summaries, 16) || !aligned(seq_lens, 4))
+    return fail(KSA_ERR_INVALID_ARG, "K and summaries must be 16-byte aligned");
+  ksa::SummaryArgs a;
+  a.K = K;
+  a.seq_lens = seq_lens;
+  a.S = summaries;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hkv = shape->num_kv_heads;
+  a.T = shape->capacity;
+  a.D = shape->head_dim;
+  a.bs = shape->block_size;
+  a.mode = mode;
+  return cuda_status(ksa::launch_block_summaries(a, static_cast<cudaStream_t>(stream)),
+                     "ksa_build_block_summaries launch");
+}
+
+size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks) {
+  (void)shape;
+  (void)k_blocks;
+  return 0;
+}
+
+ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const float *summaries,
+                             const int32_t *seq_lens, int32_t k_blocks, int32_t *block_idx,
+                             int32_t *num_sel, void *ws, size_t ws_bytes, uint32_t *dev_status,
+                             void *stream) {
+  (void)ws;
+  (void)ws_bytes;
+  ksa_status st = check_shape(shape, true);
+  if (st != KSA_OK) return st;
+  if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
+      num_sel == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "q, summaries, seq_lens, block_idx, num_sel must be non-NULL");
+  if (k_blocks < 1) return fail(KSA_ERR_INVALID_ARG, "k_blocks must be >= 1 (got %d)", k_blocks);
+  const int nb_max = (shape->capacity + shape->block_size - 1) / shape->block_size;
+  if (nb_max > 16384)
+    return fail(KSA_ERR_UNSUPPORTED, "ceil(capacity/block_size) = %d exceeds 16384", nb_max);
+  if (!aligned(summaries, 16) || !aligned(q, 4))
+    return fail(KSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
+  ksa::SelectArgs a;
+  a.q = q;
+  a.S = summaries;
+  a.seq_lens = seq_lens;
+  a.block_idx = block_idx;
+  a.num_sel = num_sel;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hq = shape->num_q_heads;
+  a.Hkv = shape->num_kv_heads;
+  a.D = shape->head_dim;
+  a.T = shape->capacity;
+  a.bs = shape->block_size;
+  a.k = k_blocks;
+  return cuda_status(
+      ksa::launch_select_blocks(a, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      "ksa_select_blocks launch");
+}
+
+size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape, int32_t idx_capacity,
+                                        int32_t tokens_per_idx) {
+  (void)shape;
+  (void)idx_capacity;
+  (void)tokens_per_idx;
+  return 0;
+}
+
+ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                                  const uint16_t *V, const int32_t *seq_lens, const int32_t *idx,
+                                  const int32_t *num_idx, int32_t idx_capacity,
+                                  int32_t tokens_per_idx, int32_t idx_shared, float scale,
+                                  int32_t out_dtype, void *out, float *lse, void *ws,
+                                  size_t ws_bytes, uint32_t *dev_status, void *stream) {
+  (void)ws;
+  (void)ws_bytes;
+  ksa_status st = check_shape(shape, false);
+  if (st != KSA_OK) return st;
+  if (q == nullptr || K == nullptr || V == nullptr || seq_lens == nullptr || out == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "q, K, V, seq_lens and out must be non-NULL");
+  const int G = shape->num_q_heads / shape->num_kv_heads;
+  if (G > 8)
+    return fail(KSA_ERR_UNSUPPORTED, "query heads per kv-head = %d exceeds 8", G);
+  if (out_dtype != KSA_OUT_F32 && out_dtype != KSA_OUT_BF16)
+    return fail(KSA_ERR_INVALID_ARG, "out_dtype %d is neither F32 nor BF16", out_dtype);
+  if (!(scale >= 0.f) || isinf(scale))
+    return fail(KSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (idx != nullptr) {
+    if (num_idx == nullptr) return fail(KSA_ERR_INVALID_ARG, "num_idx is NULL with idx given");
+    if (idx_capacity < 1) return fail(KSA_ERR_INVALID_ARG, "idx_capacity must be >= 1");
+    if (tokens_per_idx < 1 || tokens_per_idx > 256 ||
+        (tokens_per_idx & (tokens_per_idx - 1)) != 0)
+      return fail(KSA_ERR_UNSUPPORTED, "tokens_per_idx %d is not a power of two in [1, 256]",
+                  tokens_per_idx);
+    if (idx_shared != 0 && idx_shared != 1)
+      return fail(KSA_ERR_INVALID_ARG, "idx_shared must be 0 or 1");
+    if (!aligned(idx, 4) || !aligned(num_idx, 4))
+      return fail(KSA_ERR_INVALID_ARG, "idx and num_idx must be 4-byte aligned");
+  }
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(q, 4) ||
+      !aligned(out, out_dtype == KSA_OUT_F32 ? 4 : 2) || (lse && !aligned(lse, 4)))
+    return fail(KSA_ERR_INVALID_ARG, "K and V must be 16-byte aligned, q and out element-aligned");
+  ksa::AttnArgs a;
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.seq_lens = seq_lens;
+  a.idx = idx;
+  a.num_idx = num_idx;
+  a.out_f32 = out_dtype == KSA_OUT_F32 ? static_cast<float *>(out) : nullptr;
+  a.out_bf16 = out_dtype == KSA_OUT_BF16 ? static_cast<uint16_t *>(out) : nullptr;
+  a.lse = lse;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hq = shape->num_q_heads;
+  a.Hkv = shape->num_kv_heads;
+  a.D = shape->head_dim;
+  a.T = shape->capacity;
+  a.cap = idx ? idx_capacity : 0;
+  a.tpi = idx ? tokens_per_idx : 1;
+  a.shared = idx ? idx_shared : 0;
+  a.scale = scale == 0.f ? static_cast<float>(1.0 / sqrt(static_cast<double>(shape->head_dim)))
+                         : scale;
+  return cuda_status(
+      ksa::launch_sparse_decode_attn(a, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      "ksa_sparse_decode_attn launch");
+}
+
+size_t ksa_unified_select_workspace(const ksa_shape *shape, int32_t per_head_topk,
+                                    int32_t token_budget) {
+  (void)per_head_topk;
+  (void)token_budget;
+  if (shape == nullptr || shape->batch < 1 || shape->num_q_heads < 1 || shape->capacity < 1)
+    return 0;
+  return ksa::unified_workspace_bytes(shape->batch, shape->num_q_heads, shape->capacity);
+}
+
+ksa_status ksa_unified_select(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                              const int32_t *seq_lens, int32_t per_head_topk,
+                              int32_t token_budget, int32_t recent_tokens, int32_t *token_idx,
+                              int32_t *num_sel, void *ws, size_t ws_bytes, uint32_t *dev_status,
+                              void *stream) {
+  ksa_status st = check_shape(shape, false);
+  if (st != KSA_OK) return st;
+  if (q == nullptr || K == nullptr || seq_lens == nullptr || token_idx == nullptr ||
+      num_sel == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "q, K, seq_lens, token_idx and num_sel must be non-NULL");
+  const int G = shape->num_q_heads / shape->num_kv_heads;
+  if (G > 8) return fail(KSA_ERR_UNSUPPORTED, "query heads per kv-head = %d exceeds 8", G);
+  if (shape->num_q_heads > 65535)
+    return fail(KSA_ERR_UNSUPPORTED, "num_q_heads above 65535 (vote counts are 16-bit)");
+  if (shape->capacity > 65536)
+    return fail(KSA_ERR_UNSUPPORTED, "capacity %d exceeds 65536", shape->capacity);
+  if (per_head_topk < 1) return fail(KSA_ERR_INVALID_ARG, "per_head_topk must be >= 1");
+  if (token_budget < 1 || token_budget > shape->capacity)
+    return fail(KSA_ERR_INVALID_ARG, "token_budget must be in [1, capacity]");
+  if (recent_tokens < 0) recent_tokens = token_budget / 4;
+  if (recent_tokens > token_budget)
+    return fail(KSA_ERR_INVALID_ARG, "recent_tokens (%d) exceeds token_budget (%d)",
+                recent_tokens, token_budget);
+  const size_t need =
+      ksa::unified_workspace_bytes(shape->batch, shape->num_q_heads, shape->capacity);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (!aligned(K, 16) || !aligned(q, 4))
+    return fail(KSA_ERR_INVALID_ARG, "K must be 16-byte aligned");
+  ksa::UnifiedArgs a;
+  a.q = q;
+  a.K = K;
+  a.seq_lens = seq_lens;
+  a.token_idx = token_idx;
+  a.num_sel = num_sel;
+  const size_t keys_bytes =
+      (static_cast<size_t>(shape->batch) * shape->num_q_heads * shape->capacity * 4 + 255) &
+      ~static_cast<size_t>(255);
+  a.keys = static_cast<uint32_t *>(ws);
+  a.votes = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + keys_bytes);
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hq = shape->num_q_heads;
+  a.Hkv = shape->num_kv_heads;
+  a.D = shape->head_dim;
+  a.T = shape->capacity;
+  a.P = per_head_topk;
+  a.budget = token_budget;
+  a.R = recent_tokens;
+  return cuda_status(
+      ksa::launch_unified_select(a, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      "ksa_unified_select launch");
+}
+
+const char *ksa_status_string(ksa_status status) {
+  switch (status) {
+    case KSA_OK: return "KSA_OK";
+    case KSA_ERR_INVALID_ARG: return "KSA_ERR_INVALID_ARG";
+    case KSA_ERR_UNSUPPORTED: return "KSA_ERR_UNSUPPORTED";
+    case KSA_ERR_WORKSPACE: return "KSA_ERR_WORKSPACE";
+    case KSA_ERR_CUDA: return "KSA_ERR_CUDA";
+  }
+  return "KSA_UNKNOWN_STATUS";
+}
+
+const char *ksa_last_error(void) { return g_last_error.c_str(); }
+
+int32_t ksa_version(void) { return 100; }
+
+}  // extern "C"

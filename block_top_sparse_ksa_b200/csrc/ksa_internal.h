@@ -1,0 +1,65 @@
+// ksa_internal.h -- launch entry points of the libksa kernels (host side).
+//
+// Every launcher assumes its arguments were validated by the C ABI layer
+// (ksa_api.cu) and returns the cudaError_t of its launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ksa {
+
+struct SummaryArgs {
+  const uint16_t *K;
+  const int32_t *seq_lens;
+  float *S;
+  uint32_t *status;
+  int B, Hkv, T, D, bs, mode;
+};
+cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream);
+
+struct SelectArgs {
+  const uint16_t *q;
+  const float *S;
+  const int32_t *seq_lens;
+  int32_t *block_idx;
+  int32_t *num_sel;
+  uint32_t *status;
+  int B, Hq, Hkv, D, T, bs, k;
+};
+cudaError_t launch_select_blocks(const SelectArgs &a, int num_sms, cudaStream_t stream);
+
+struct AttnArgs {
+  const uint16_t *q, *K, *V;
+  const int32_t *seq_lens;
+  const int32_t *idx;
+  const int32_t *num_idx;
+  float *out_f32;
+  uint16_t *out_bf16;
+  float *lse;
+  uint32_t *status;
+  int B, Hq, Hkv, D, T;
+  int cap, tpi, shared;
+  float scale;
+};
+cudaError_t launch_sparse_decode_attn(const AttnArgs &a, int num_sms, cudaStream_t stream);
+
+struct UnifiedArgs {
+  const uint16_t *q, *K;
+  const int32_t *seq_lens;
+  int32_t *token_idx;
+  int32_t *num_sel;
+  uint32_t *keys;   // workspace [B, Hq, T] score keys
+  int32_t *votes;   // workspace [B, T]
+  uint32_t *status;
+  int B, Hq, Hkv, D, T, P, budget, R;
+};
+size_t unified_workspace_bytes(int B, int Hq, int T);
+cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream);
+
+// TMA descriptor for a [rows, D] bf16 matrix, 128B swizzle, box = 64 x box_rows.
+bool encode_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int D,
+                          int box_rows);
+
+}  // namespace ksa

@@ -1,0 +1,262 @@
+// unified_select.cu -- LessIsMore unified token selection.
+//
+// LessIsMore (unified head selection, stable recency window; token selection
+// layer): every query head ranks all cached tokens, each head votes for its
+// top tokens, the votes are pooled into one token set shared by all heads,
+// and the budget is split between voted tokens and the most recent tokens.
+//
+// Three launches on the caller's stream:
+//  1. scores: one CTA per (row, kv-head, 1024-token chunk).  A producer warp
+//     streams the chunk's keys with TMA (128B swizzle); four consumer warps
+//     form S^T = K_tile q^T for the kv-group's G heads with mma.sync
+//     (fp32 accumulate) and store order-preserving uint32 score keys
+//     [B, Hq, T].  The g == 0 CTAs also clear the vote table.
+//  2. per-head picks: one CTA per (row, query head).  Exact radix select of the
+//     P-th largest key over the row's L keys (staged in shared memory), ties
+//     at the threshold to the lower token, then one atomic vote per pick.
+//  3. shared set: one CTA per row.  Radix select on the vote counts of
+//     [0, L - R) for the (budget - R) most voted tokens (ties to the lower
+//     token), written ascending, followed by the window [L - R, L).
+#include <string.h>
+
+#include "ksa_device.cuh"
+#include "ksa_internal.h"
+
+namespace ksa {
+
+namespace {
+
+constexpr int kTok = 32;            // tokens per pipeline stage
+constexpr int kChunk = 1024;        // tokens per scoring CTA
+constexpr int kScoreThreads = 160;  // 4 consumer warps + 1 producer warp
+constexpr int kPickThreads = 512;
+constexpr int kSetThreads = 1024;
+constexpr int kSmemKeys = 40960;    // keys of one head staged in shared memory
+
+template <int D>
+struct SCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kHalfBytes = kTok * 128;
+  static constexpr int kStageBytes = kHalves * kHalfBytes;
+  static constexpr int kStages = 8;
+  static constexpr size_t kSmemBytes =
+      1024 + static_cast<size_t>(kStages) * kStageBytes + 16 * kStages + 64;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads, 2)
+    unified_scores_kernel(const __grid_constant__ CUtensorMap kmap, const UnifiedArgs a,
+                          int n_chunks) {
+  using C = SCfg<D>;
+  constexpr int NS = C::kStages;
+  constexpr int KT = D / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + static_cast<size_t>(NS) * C::kStageBytes);
+  uint64_t *empty = full + NS;
+  uint32_t *timed_out = reinterpret_cast<uint32_t *>(empty + NS);
+
+  const int row = blockIdx.x / n_chunks, chunk = blockIdx.x % n_chunks;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int L = clamp_len(a.seq_lens[b], a.T,
+                          (g == 0 && chunk == 0 && tid == 0) ? a.status : nullptr);
+  if (L <= a.budget) return;  // every token is selected; no scores needed
+  const int t_begin = chunk * kChunk;
+  if (t_begin >= L) return;
+  const int t_end = min(L, t_begin + kChunk);
+  const int n_stage = (t_end - t_begin + kTok - 1) / kTok;
+
+  if (g == 0) {
+    for (int t = t_begin + tid; t < t_end; t += kScoreThreads)
+      a.votes[static_cast<size_t>(b) * a.T + t] = 0;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1u);
+      mbar_init(&empty[s], 1u);
+    }
+    *timed_out = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  uint32_t bad = 0u;
+  int issued = 0;
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&kmap);
+      for (int i = 0; i < n_stage; ++i) {
+        const int buf = i % NS;
+        if (i >= NS && !mbar_wait(&empty[buf], static_cast<uint32_t>((i / NS) - 1) & 1u)) {
+          bad |= KSA_FLAG_WAIT_TIMEOUT;
+          break;
+        }
+        issued = i + 1;
+        uint8_t *dst = smem + static_cast<size_t>(buf) * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[buf], C::kStageBytes);
+        const int y = static_cast<int>(static_cast<long long>(row) * a.T + t_begin + i * kTok);
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h)
+          tma_load_2d(dst + h * C::kHalfBytes, &kmap, h * 64, y, &full[buf]);
+      }
+    }
+  } else {
+    const int gid = lane >> 2, tig = lane & 3;
+    uint32_t qb[KT][2];
+    const uint16_t *qrow =
+        a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G + gid) * D;
+#pragma unroll
+    for (int ks = 0; ks < KT; ++ks) {
+      qb[ks][0] = gid < G ? *reinterpret_cast<const uint32_t *>(qrow + ks * 16 + tig * 2) : 0u;
+      qb[ks][1] = gid < G ? *reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 8 + tig * 2) : 0u;
+    }
+    const int mi = lane >> 3, lr = lane & 7;
+    for (int i = warp; i < n_stage; i += 4) {
+      const int buf = i % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[buf], static_cast<uint32_t>(i / NS) & 1u))) {
+        bad |= KSA_FLAG_WAIT_TIMEOUT;
+        break;
+      }
+      const uint32_t kbase = smem_addr(smem + static_cast<size_t>(buf) * C::kStageBytes);
+      float s[2][4];
+#pragma unroll
+      for (int tile = 0; tile < 2; ++tile) {
+        s[tile][0] = s[tile][1] = s[tile][2] = s[tile][3] = 0.f;
+        const int r = tile * 16 + lr + ((mi & 1) << 3);
+#pragma unroll
+        for (int ks = 0; ks < KT; ++ks) {
+          const int d = ks * 16 + ((mi >> 1) << 3);
+          uint32_t af[4];
+          ldsm_x4(af, kbase + (d >> 6) * C::kHalfBytes + swz128(r, (d & 63) >> 3));
+          mma_16816(s[tile], af, qb[ks][0], qb[ks][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[buf]);
+      const int t0 = t_begin + i * kTok;
+#pragma unroll
+      for (int tile = 0; tile < 2; ++tile) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int hh = tig * 2 + (c & 1);
+          const int t = t0 + tile * 16 + gid + ((c >> 1) << 3);
+          if (hh < G && t < t_end) {
+            bool nan;
+            const uint32_t key = score_key(s[tile][c], nan);
+            bad |= nan ? KSA_FLAG_NONFINITE_SCORE : 0u;
+            a.keys[(static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G + hh) * a.T + t] = key;
+          }
+        }
+      }
+    }
+  }
+  flag_status(a.status, bad);
+  if (bad & KSA_FLAG_WAIT_TIMEOUT) atomicExch(timed_out, 1u);
+  __syncthreads();
+  if (*timed_out != 0u && warp == 4 && lane == 0) {
+    // a wait gave up: let the issued copies land before the CTA exits (bounded)
+    for (int buf = 0; buf < NS && buf < issued; ++buf)
+      mbar_wait(&full[buf], static_cast<uint32_t>((issued - 1 - buf) / NS) & 1u);
+  }
+}
+
+// Per-head pick and vote: CTA per (row, query head).
+__global__ void __launch_bounds__(kPickThreads) unified_pick_kernel(const UnifiedArgs a,
+                                                                     int stage_in_smem) {
+  extern __shared__ uint32_t skeys[];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t info[4];
+  __shared__ uint32_t scratch[33];
+  const int b = blockIdx.x / a.Hq, h = blockIdx.x % a.Hq;
+  const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
+  if (L <= a.budget) return;
+  int32_t *votes = a.votes + static_cast<size_t>(b) * a.T;
+  if (a.P >= L) {
+    for (int t = threadIdx.x; t < L; t += kPickThreads) atomicAdd(&votes[t], 1);
+    return;
+  }
+  const uint32_t *gkeys = a.keys + (static_cast<size_t>(b) * a.Hq + h) * a.T;
+  const uint32_t *keys = gkeys;
+  if (stage_in_smem) {
+    for (int t = threadIdx.x; t < L; t += kPickThreads) skeys[t] = gkeys[t];
+    __syncthreads();
+    keys = skeys;
+  }
+  uint32_t tau, n_gt, n_eq;
+  radix_select_desc<kPickThreads>(keys, L, a.P, 32, hist, info, tau, n_gt, n_eq);
+  select_ascending<kPickThreads>(keys, L, tau, n_gt, n_eq, a.P, nullptr, scratch,
+                                 [&](int t) { atomicAdd(&votes[t], 1); });
+}
+
+// Shared set: CTA per row.
+__global__ void __launch_bounds__(kSetThreads) unified_set_kernel(const UnifiedArgs a) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t info[4];
+  __shared__ uint32_t scratch[33];
+  const int b = blockIdx.x;
+  const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
+  int32_t *out = a.token_idx + static_cast<size_t>(b) * a.budget;
+  if (L <= a.budget) {
+    for (int i = threadIdx.x; i < a.budget; i += kSetThreads) out[i] = i < L ? i : -1;
+    if (threadIdx.x == 0) a.num_sel[b] = L;
+    return;
+  }
+  const int n = L - a.R;       // candidates [0, L - R)
+  const int k = a.budget - a.R;
+  if (k > 0) {
+    const uint32_t *keys = reinterpret_cast<const uint32_t *>(a.votes + static_cast<size_t>(b) * a.T);
+    const int nbits = a.Hq < 256 ? 8 : 16;
+    uint32_t tau, n_gt, n_eq;
+    radix_select_desc<kSetThreads>(keys, n, k, nbits, hist, info, tau, n_gt, n_eq);
+    select_ascending<kSetThreads>(keys, n, tau, n_gt, n_eq, k, out, scratch, [](int) {});
+  }
+  for (int i = threadIdx.x; i < a.R; i += kSetThreads) out[k + i] = n + i;
+  if (threadIdx.x == 0) a.num_sel[b] = a.budget;
+}
+
+template <int D>
+cudaError_t launch_scores(const UnifiedArgs &a, cudaStream_t stream) {
+  CUtensorMap km;
+  memset(&km, 0, sizeof km);
+  if (!encode_kv_tensor_map(&km, a.K, static_cast<uint64_t>(a.B) * a.Hkv * a.T, D, kTok))
+    return cudaErrorInvalidValue;
+  const int n_chunks = (a.T + kChunk - 1) / kChunk;
+  const size_t smem = SCfg<D>::kSmemBytes;
+  cudaError_t err = cudaFuncSetAttribute(unified_scores_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const unsigned grid = static_cast<unsigned>(a.B) * a.Hkv * n_chunks;
+  unified_scores_kernel<D><<<grid, kScoreThreads, smem, stream>>>(km, a, n_chunks);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t unified_workspace_bytes(int B, int Hq, int T) {
+  const size_t keys = (static_cast<size_t>(B) * Hq * T * sizeof(uint32_t) + 255) & ~static_cast<size_t>(255);
+  const size_t votes = (static_cast<size_t>(B) * T * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  return keys + votes;
+}
+
+cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream) {
+  (void)num_sms;
+  cudaError_t err = a.D == 128 ? launch_scores<128>(a, stream) : launch_scores<64>(a, stream);
+  if (err != cudaSuccess) return err;
+  const int in_smem = a.T <= kSmemKeys ? 1 : 0;
+  const size_t pick_smem = in_smem ? static_cast<size_t>(a.T) * sizeof(uint32_t) : 0;
+  err = cudaFuncSetAttribute(unified_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(pick_smem));
+  if (err != cudaSuccess) return err;
+  unified_pick_kernel<<<static_cast<unsigned>(a.B) * a.Hq, kPickThreads, pick_smem, stream>>>(
+      a, in_smem);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  unified_set_kernel<<<static_cast<unsigned>(a.B), kSetThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ksa

@@ -1,0 +1,178 @@
+/*
+ * ksa.h -- C ABI of libksa: decode-phase block top-k sparse attention over a
+ * GQA KV cache, and LessIsMore unified token selection, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources of the method:
+ *   [KIN] Kinetics: Rethinking Test-Time Scaling Laws (press summary,
+ *         news.43u.com.cn), section 5 "from theory to practice: block top-k".
+ *   [LIM] LessIsMore (press summary, techwalker.com), section 2 "unified head
+ *         selection" / "stable recency window", section 5 "implementation".
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, dense row-major, owned by the
+ *     caller.  The library allocates nothing, keeps no state between calls,
+ *     and never synchronises the host: work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - bf16 tensors are passed as uint16_t* (the raw bf16 bit patterns).
+ *   - Shapes: B = batch, Hq / Hkv = query / kv heads (G = Hq/Hkv query heads
+ *     share one kv-head), D = head_dim, T = capacity (tokens per cache row),
+ *     bs = block_size, L_b = seq_lens[b] (tokens held by row b, the current
+ *     token included), NB_b = ceil(L_b / bs).
+ *   - Caches K, V: [B, Hkv, T, D] bf16.  Queries q: [B, Hq, D] bf16.
+ *   - Host-side validation failures return KSA_ERR_INVALID_ARG (bad argument)
+ *     or KSA_ERR_UNSUPPORTED (valid but not covered by the kernels) and
+ *     enqueue nothing.  A failed launch returns KSA_ERR_CUDA.
+ *     ksa_last_error() gives a message for the calling thread's last failure.
+ *   - dev_status (nullable): a device uint32 that kernels OR KSA_FLAG_* bits
+ *     into when device data is out of range.  It is never cleared by the
+ *     library; the caller zeroes it and reads it back when it wants to know.
+ *   - Bad device data never faults: a seq_len outside [1, T] is clamped to
+ *     [0, T] and flagged; an index entry outside the row is skipped and
+ *     flagged.
+ */
+#ifndef KSA_H
+#define KSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KSA_OK = 0,
+  KSA_ERR_INVALID_ARG = 1,
+  KSA_ERR_UNSUPPORTED = 2,
+  KSA_ERR_WORKSPACE = 3,
+  KSA_ERR_CUDA = 4
+} ksa_status;
+
+typedef struct {
+  int32_t batch;        /* B */
+  int32_t num_q_heads;  /* Hq */
+  int32_t num_kv_heads; /* Hkv; Hq % Hkv == 0 */
+  int32_t head_dim;     /* D: 64 or 128 */
+  int32_t capacity;     /* T: token slots per cache row */
+  int32_t block_size;   /* bs: 16, 32 or 64 for the block entry points */
+} ksa_shape;
+
+enum { KSA_SUMMARY_ALL = 0, KSA_SUMMARY_LAST_BLOCK = 1 };
+enum { KSA_OUT_F32 = 0, KSA_OUT_BF16 = 1 };
+
+enum {
+  KSA_FLAG_SEQ_LEN_CLAMPED = 1u << 0, /* some seq_len was outside [1, T] */
+  KSA_FLAG_INDEX_SKIPPED = 1u << 1,   /* some index entry named no valid token */
+  KSA_FLAG_NONFINITE_SCORE = 1u << 2, /* a NaN score was ranked lowest */
+  KSA_FLAG_WAIT_TIMEOUT = 1u << 3     /* a pipeline wait gave up: results invalid */
+};
+
+/*
+ * Block summaries (maintenance of the block mean representation) [KIN s.5].
+ *   S[b,g,j,:] = (1/n_j) * sum_{t=j*bs}^{j*bs+n_j-1} K[b,g,t,:],
+ *   n_j = min(bs, L_b - j*bs), computed in fp32 from bf16 keys.
+ * mode KSA_SUMMARY_ALL rebuilds every block j < NB_b (prefill);
+ * mode KSA_SUMMARY_LAST_BLOCK rebuilds only j = NB_b - 1 (one decode step
+ * after appending a token).  Entries j >= NB_b are not written.
+ *   K:         [B, Hkv, T, D] bf16 (read)
+ *   seq_lens:  [B] int32 (read)
+ *   summaries: [B, Hkv, ceil(T/bs), D] fp32 (written)
+ */
+ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
+                                     const int32_t *seq_lens, int32_t mode,
+                                     float *summaries, uint32_t *dev_status,
+                                     void *stream);
+
+/*
+ * Block scoring and top-k selection [KIN s.5]: for every (b, kv-head g)
+ *   s_j = sum_{h in group g} <q[b,h,:], S[b,g,j,:]>   (j < NB_b, fp32)
+ * and the k_blocks largest s_j are kept, ties to the lower j, listed in
+ * ascending j.  If NB_b <= k_blocks every block is kept and no summary is
+ * read.  A NaN score ranks lowest and sets KSA_FLAG_NONFINITE_SCORE.
+ *   q:         [B, Hq, D] bf16
+ *   summaries: [B, Hkv, ceil(T/bs), D] fp32 (from ksa_build_block_summaries)
+ *   block_idx: [B, Hkv, k_blocks] int32, ascending, -1 padded (written)
+ *   num_sel:   [B, Hkv] int32 = min(k_blocks, NB_b) (written)
+ *   ws:        unused (pass NULL, 0); kept for ABI stability.
+ * Limits: k_blocks >= 1; ceil(T/bs) <= 16384 (scores of one row live in
+ * on-chip memory), else KSA_ERR_UNSUPPORTED.
+ */
+size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks);
+ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q,
+                             const float *summaries, const int32_t *seq_lens,
+                             int32_t k_blocks, int32_t *block_idx,
+                             int32_t *num_sel, void *ws, size_t ws_bytes,
+                             uint32_t *dev_status, void *stream);
+
+/*
+ * Sparse decode attention over a selected token set [KIN s.5; LIM s.5
+ * "sparse attention layer", GQA kernel sharing one KV set per group].
+ * For query head h of row b (kv-head g = h / G) and selected tokens T_sel:
+ *   z_t = scale * <q[b,h,:], K[b,g,t,:]>,  w = softmax(z over T_sel),
+ *   out[b,h,:] = sum_t w_t V[b,g,t,:],   lse[b,h] = log sum_t exp(z_t).
+ * T_sel: idx == NULL -> dense, every t < L_b.  Otherwise entry e < num_idx
+ * of the list names tokens [idx*tpi, idx*tpi + tpi) with tpi =
+ * tokens_per_idx (block_size for block lists, 1 for token lists); tokens
+ * t >= L_b are dropped (partial tail block).  The list is [B, Hkv, cap]
+ * with num_idx [B, Hkv] (idx_shared == 0), or [B, cap] with num_idx [B]
+ * shared by every kv-head (idx_shared == 1, the LessIsMore layout).
+ * Entries are expected distinct; a negative entry or one naming no token
+ * below L_b is skipped and flagged.  An empty set gives out = 0,
+ * lse = -inf.  Accumulation is fp32; scale == 0 selects 1/sqrt(D).
+ *   out: [B, Hq, D] fp32 (out_dtype KSA_OUT_F32) or bf16 (KSA_OUT_BF16)
+ *   lse: [B, Hq] fp32, nullable
+ *   ws:  unused (pass NULL, 0); kept for ABI stability.
+ * Limits: D in {64, 128}; G <= 8; tokens_per_idx a power of two <= 256.
+ */
+size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape,
+                                        int32_t idx_capacity,
+                                        int32_t tokens_per_idx);
+ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q,
+                                  const uint16_t *K, const uint16_t *V,
+                                  const int32_t *seq_lens, const int32_t *idx,
+                                  const int32_t *num_idx, int32_t idx_capacity,
+                                  int32_t tokens_per_idx, int32_t idx_shared,
+                                  float scale, int32_t out_dtype, void *out,
+                                  float *lse, void *ws, size_t ws_bytes,
+                                  uint32_t *dev_status, void *stream);
+
+/*
+ * LessIsMore unified selection [LIM s.2, s.5 "token selection layer"].
+ * For each row b with L = L_b:
+ *   1. every query head h scores every token t < L: s_h[t] = <q[b,h], K[b,g(h),t]>
+ *      (fp32) and picks its per_head_topk best tokens, ties to the lower t;
+ *   2. votes[t] = number of heads that picked t;
+ *   3. the result is the (token_budget - recent_tokens) tokens of
+ *      [0, L - recent_tokens) with the most votes (ties to the lower t),
+ *      plus the window [L - recent_tokens, L), listed ascending.
+ *   If L <= token_budget every token [0, L) is selected.
+ *   token_idx: [B, token_budget] int32 ascending, -1 padded (written)
+ *   num_sel:   [B] int32 (written)
+ *   ws:        device scratch of at least ksa_unified_select_workspace() bytes,
+ *              256-byte aligned; contents need no initialisation.
+ * recent_tokens < 0 selects token_budget / 4 (the 25% window).
+ * Limits: 1 <= per_head_topk; 0 <= recent_tokens <= token_budget <= T;
+ * T <= 65536.
+ */
+size_t ksa_unified_select_workspace(const ksa_shape *shape,
+                                    int32_t per_head_topk, int32_t token_budget);
+ksa_status ksa_unified_select(const ksa_shape *shape, const uint16_t *q,
+                              const uint16_t *K, const int32_t *seq_lens,
+                              int32_t per_head_topk, int32_t token_budget,
+                              int32_t recent_tokens, int32_t *token_idx,
+                              int32_t *num_sel, void *ws, size_t ws_bytes,
+                              uint32_t *dev_status, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *ksa_status_string(ksa_status status);
+/* Message describing the calling thread's last failed call ("" if none). */
+const char *ksa_last_error(void);
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t ksa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KSA_H */

@@ -1,0 +1,107 @@
+"""The C ABI library builds, loads and exports every entry point of
+include/ksa.h; host-side validation rejects bad arguments before touching the
+device.  Runs without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "ksa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ksa_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def ksa():
+    from block_top_sparse_ksa_b200 import build
+    build.build()
+    import block_top_sparse_ksa_b200 as k
+    return k
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for n in ("ksa_build_block_summaries", "ksa_select_blocks", "ksa_sparse_decode_attn",
+              "ksa_unified_select"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ksa):
+    lib = ctypes.CDLL(ksa.library_path)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_wraps_every_entry_point(ksa):
+    for n in declared_functions():
+        if n.endswith("_workspace") and n != "ksa_unified_select_workspace":
+            continue  # workspace queries of calls that need none
+        assert hasattr(ksa, n), n
+
+
+def test_status_strings_and_version(ksa):
+    assert ksa.ksa_status_string(0) == "KSA_OK"
+    assert ksa.ksa_status_string(2) == "KSA_ERR_UNSUPPORTED"
+    assert ksa.ksa_version() >= 100
+
+
+def _shape(ksa, B=1, Hq=4, Hkv=2, D=128, T=64, bs=16):
+    return ksa.Shape(B, Hq, Hkv, D, T, bs)
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+
+
+def test_validation_rejects_bad_shapes(ksa):
+    lib = ksa.lib()
+    assert lib.ksa_select_blocks(None, FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, 0, None, None) == 1
+    for kw, want in [(dict(D=96), 2), (dict(Hq=3, Hkv=2), 1), (dict(bs=8), 2), (dict(B=0), 1)]:
+        sh = _shape(ksa, **kw)
+        st = lib.ksa_select_blocks(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, 0,
+                                   None, None)
+        assert st == want, (kw, st, ksa.ksa_last_error())
+        assert ksa.ksa_last_error() != ""
+
+
+def test_validation_rejects_bad_arguments(ksa):
+    lib = ksa.lib()
+    sh = _shape(ksa)
+    # k_blocks < 1
+    assert lib.ksa_select_blocks(ctypes.byref(sh), FAKE, FAKE, FAKE, 0, FAKE, FAKE, None, 0,
+                                 None, None) == 1
+    # NULL output
+    assert lib.ksa_select_blocks(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, None, FAKE, None, 0,
+                                 None, None) == 1
+    # summaries mode out of range
+    assert lib.ksa_build_block_summaries(ctypes.byref(sh), FAKE, FAKE, 7, FAKE, None, None) == 1
+    # attention: G = 16 unsupported, tokens_per_idx not a power of two, bad dtype
+    sh16 = _shape(ksa, Hq=32, Hkv=2)
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(sh16), FAKE, FAKE, FAKE, FAKE, None, None, 0,
+                                      1, 0, 0.0, 0, FAKE, None, None, 0, None, None) == 2
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 3,
+                                      0, 0.0, 0, FAKE, None, None, 0, None, None) == 2
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, None, None, 0, 1,
+                                      0, 0.0, 5, FAKE, None, None, 0, None, None) == 1
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, None, None, 0, 1,
+                                      0, -1.0, 0, FAKE, None, None, 0, None, None) == 1
+    # unified: recent > budget, budget > capacity, missing workspace
+    assert lib.ksa_unified_select(ctypes.byref(sh), FAKE, FAKE, FAKE, 8, 16, 17, FAKE, FAKE, FAKE,
+                                  1 << 20, None, None) == 1
+    assert lib.ksa_unified_select(ctypes.byref(sh), FAKE, FAKE, FAKE, 8, 65, 1, FAKE, FAKE, FAKE,
+                                  1 << 20, None, None) == 1
+    assert lib.ksa_unified_select(ctypes.byref(sh), FAKE, FAKE, FAKE, 8, 16, 4, FAKE, FAKE, None,
+                                  0, None, None) == 3
+
+
+def test_workspace_sizes(ksa):
+    lib = ksa.lib()
+    sh = _shape(ksa, B=16, Hq=32, Hkv=8, D=128, T=20000)
+    ws = lib.ksa_unified_select_workspace(ctypes.byref(sh), 4000, 4000)
+    assert ws >= 16 * 32 * 20000 * 4 + 16 * 20000 * 4
+    assert lib.ksa_select_blocks_workspace(ctypes.byref(sh), 128) == 0
+    assert lib.ksa_sparse_decode_attn_workspace(ctypes.byref(sh), 128, 16) == 0

@@ -1,0 +1,395 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Selected indices must match bit-exactly (inputs carry a planted score gap, or
+are dyadic so that every score is exact in fp32); attention outputs must meet
+max|d| <= 2e-3 and max|d| / max|ref| <= 1e-2, lse within 1e-4.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_top_sparse_ksa_b200 import synth
+from oracle.oracle import bf16_bits, bf16_value
+from tests.helpers import (DELTA, LSE_TOL, assert_out_close, gap_fix_row, min_boundary_gap,
+                           sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def ksa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import block_top_sparse_ksa_b200 as k
+    k.lib()
+    return k
+
+
+def to_dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(DEV)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return synth.bits(t)
+
+
+def rand_bits(rng, shape, scale=1.0):
+    return bf16_bits(rng.standard_normal(shape) * scale)
+
+
+def dyadic_bits(rng, shape, step=0.25, lim=4.0):
+    return bf16_bits(np.clip(np.round(rng.standard_normal(shape) / step) * step, -lim, lim))
+
+
+def status_tensor():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+# ---------------------------------------------------------------------------
+# A1 summaries
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32, 64])
+def test_summaries_all_and_last_block(ksa, oracle, D, bs):
+    rng = np.random.default_rng(100 + D + bs)
+    B, Hkv, T = 4, 3, 7 * bs + 5
+    K = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([T, 1, bs + 3, 5 * bs], np.int32)
+    Kd, Ld = to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    S = ksa.ksa_build_block_summaries(Kd, Ld, bs).cpu().numpy()
+    ref = oracle.block_summaries(K, lens, bs)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        np.testing.assert_allclose(S[b, :, :nb], ref[b, :, :nb], rtol=1e-6, atol=1e-6)
+    # LAST_BLOCK rewrites only block NB_b - 1
+    S2 = torch.full_like(torch.from_numpy(S), float("nan")).to(DEV)
+    ksa.ksa_build_block_summaries(Kd, Ld, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S2)
+    S2 = S2.cpu().numpy()
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        np.testing.assert_allclose(S2[b, :, nb - 1], ref[b, :, nb - 1], rtol=1e-6, atol=1e-6)
+        assert np.all(np.isnan(S2[b, :, :nb - 1])) and np.all(np.isnan(S2[b, :, nb:]))
+
+
+# ---------------------------------------------------------------------------
+# A2 + A3 selection
+
+
+def _select_case(ksa, oracle, rng, B, Hq, Hkv, D, T, bs, k, lens, dyadic=False, plant=True):
+    q = dyadic_bits(rng, (B, Hq, D)) if dyadic else rand_bits(rng, (B, Hq, D))
+    K = dyadic_bits(rng, (B, Hkv, T, D)) if dyadic else rand_bits(rng, (B, Hkv, T, D))
+    if plant:
+        for b in range(B):
+            K[b], _ = gap_fix_row(oracle, q[b], K[b], int(lens[b]), bs, k)
+            assert min_boundary_gap(oracle, q[b], K[b], int(lens[b]), bs, k) >= DELTA
+    qd, Kd, Ld = to_dev_bf16(q), to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    st = status_tensor()
+    S = ksa.ksa_build_block_summaries(Kd, Ld, bs, dev_status=st)
+    idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k, dev_status=st)
+    ref_idx, ref_cnt = oracle.select_blocks(q, K, lens, bs, k)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    assert st.item() == 0
+    return q, K, idx, cnt
+
+
+@pytest.mark.parametrize("D,bs,k", [(128, 16, 8), (64, 32, 5), (128, 64, 3), (128, 16, 64)])
+def test_select_blocks_planted_gap(ksa, oracle, D, bs, k):
+    rng = np.random.default_rng(200 + k)
+    B, Hq, Hkv, T = 3, 8, 2, 40 * bs + 7
+    lens = np.array([T, 13 * bs + 1, 3 * bs], np.int32)  # ragged, a 1-token tail, a short row
+    _select_case(ksa, oracle, rng, B, Hq, Hkv, D, T, bs, k, lens)
+
+
+def test_select_blocks_exact_ties(ksa, oracle):
+    """Dyadic inputs, full blocks: every score is exact in fp32, many tie
+    exactly, and both sides must break ties toward the lower block."""
+    rng = np.random.default_rng(210)
+    B, Hq, Hkv, D, bs = 2, 4, 2, 128, 16
+    T = 256 * bs
+    lens = np.array([T, 100 * bs], np.int32)
+    q = bf16_bits(np.round(rng.standard_normal((B, Hq, D))) * 0.25)
+    K = bf16_bits(np.clip(np.round(rng.standard_normal((B, Hkv, T, D)) * 0.5), -2, 2) * 0.25)
+    qd, Kd, Ld = to_dev_bf16(q), to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    S = ksa.ksa_build_block_summaries(Kd, Ld, bs)
+    for k in (1, 7, 50, 99, 100, 255):
+        idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k)
+        ref_idx, ref_cnt, scores = oracle.select_blocks(q, K, lens, bs, k, want_scores=True)
+        assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+        assert np.array_equal(idx.cpu().numpy(), ref_idx), k
+    nb = lens[0] // bs
+    assert len(np.unique(scores[0, 0, :nb])) < nb  # ties really occur
+
+
+def test_select_all_blocks_when_k_covers(ksa, oracle):
+    rng = np.random.default_rng(220)
+    B, Hq, Hkv, D, T, bs = 2, 4, 4, 64, 300, 32
+    lens = np.array([300, 31], np.int32)
+    _select_case(ksa, oracle, rng, B, Hq, Hkv, D, T, bs, 10, lens, plant=False)
+
+
+# ---------------------------------------------------------------------------
+# A4 + A5 attention
+
+
+def _attn_check(ksa, oracle, q, K, V, lens, idx=None, cnt=None, tpi=1, shared=False,
+                out_dtype=0):
+    qd, Kd, Vd = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V)
+    Ld = torch.from_numpy(lens).to(DEV)
+    idx_d = None if idx is None else torch.from_numpy(np.ascontiguousarray(idx)).to(DEV)
+    cnt_d = None if cnt is None else torch.from_numpy(np.ascontiguousarray(cnt)).to(DEV)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=DEV)
+    st = status_tensor()
+    out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, idx_d, cnt_d, tokens_per_idx=tpi,
+                                        idx_shared=shared, out_dtype=out_dtype, lse=lse,
+                                        dev_status=st)
+    ref, ref_lse, _ = oracle.attention(q, K, V, lens, idx, cnt, tpi, shared)
+    assert_out_close(out.float().cpu().numpy(), ref, bf16_output=(out_dtype == 1))
+    got_lse = lse.cpu().numpy()
+    fin = np.isfinite(ref_lse)
+    np.testing.assert_allclose(got_lse[fin], ref_lse[fin], rtol=0, atol=LSE_TOL)
+    assert np.all(np.isneginf(got_lse[~fin]))
+    return st.item()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_dense_attention(ksa, oracle, D, G):
+    rng = np.random.default_rng(300 + D + G)
+    B, Hkv, T = 3, 2, 700
+    q = rand_bits(rng, (B, G * Hkv, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([700, 33, 1], np.int32)
+    assert _attn_check(ksa, oracle, q, K, V, lens) == 0
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("out_dtype", [0, 1])
+def test_block_list_attention(ksa, oracle, bs, out_dtype):
+    rng = np.random.default_rng(400 + bs)
+    B, Hq, Hkv, D = 3, 8, 2, 128
+    T = 50 * bs + 9
+    q = rand_bits(rng, (B, Hq, D), 2.0)  # peaked softmax
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([T, 20 * bs + 3, 5], np.int32)
+    cap = 24
+    idx = np.full((B, Hkv, cap), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        for g in range(Hkv):
+            n = min(cap - g, nb)
+            sel = np.sort(rng.choice(nb, size=n, replace=False))
+            if b == 1:  # always include the partial tail block
+                sel = np.unique(np.append(sel[:-1], nb - 1))
+                n = len(sel)
+            idx[b, g, :n] = sel
+            cnt[b, g] = n
+    assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, bs, out_dtype=out_dtype) == 0
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("tpi", [1, 4, 16])
+def test_token_list_attention_shared(ksa, oracle, D, tpi):
+    rng = np.random.default_rng(500 + D + tpi)
+    B, Hq, Hkv = 2, 16, 4
+    T = 3000
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([3000, 1999], np.int32)
+    cap = 700 // tpi
+    idx = np.full((B, cap), -1, np.int32)
+    cnt = np.zeros((B,), np.int32)
+    for b in range(B):
+        n_units = -(-lens[b] // tpi)
+        n = cap - 3 * b
+        idx[b, :n] = np.sort(rng.choice(n_units, size=n, replace=False))
+        cnt[b] = n
+    assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, tpi, shared=True) == 0
+
+
+def test_attention_edge_cases(ksa, oracle):
+    rng = np.random.default_rng(600)
+    B, Hq, Hkv, D, T, bs = 3, 4, 2, 128, 256, 16
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([256, 100, 256], np.int32)
+    # row 0: empty lists; row 1: one single block; row 2: every block (== dense)
+    idx = np.full((B, Hkv, 16), -1, np.int32)
+    cnt = np.array([[0, 0], [1, 1], [16, 16]], np.int32)
+    idx[1, :, 0] = [6, 0]
+    idx[2] = np.arange(16)[None, :]
+    assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, bs) == 0
+    # all blocks selected == dense
+    dense_ref, _, _ = oracle.attention(q[2:], K[2:], V[2:], lens[2:])
+    blk_ref, _, _ = oracle.attention(q[2:], K[2:], V[2:], lens[2:], idx[2:], cnt[2:], bs)
+    np.testing.assert_allclose(blk_ref, dense_ref, rtol=0, atol=1e-12)
+
+
+def test_attention_flags_bad_entries(ksa, oracle):
+    rng = np.random.default_rng(610)
+    B, Hq, Hkv, D, T, bs = 1, 4, 1, 128, 128, 16
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([100], np.int32)
+    idx = np.array([[[1, -5, 3, 7, 2]]], np.int32)  # -5 invalid, block 7 starts past L=100
+    cnt = np.array([[5]], np.int32)
+    st = _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, bs)
+    assert st & 2  # KSA_FLAG_INDEX_SKIPPED
+
+
+def test_seq_len_out_of_range_is_clamped_and_flagged(ksa, oracle):
+    rng = np.random.default_rng(620)
+    B, Hq, Hkv, D, T = 2, 4, 2, 64, 96
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([500, 0], np.int32)
+    qd, Kd, Vd = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V)
+    st = status_tensor()
+    out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, torch.from_numpy(lens).to(DEV),
+                                        dev_status=st)
+    assert st.item() & 1  # KSA_FLAG_SEQ_LEN_CLAMPED
+    ref, _, _ = oracle.attention(q, K, V, np.array([T, 0], np.int32))
+    assert_out_close(out.cpu().numpy(), ref)
+
+
+# ---------------------------------------------------------------------------
+# A6 unified selection
+
+
+@pytest.mark.parametrize("L,P,budget,R", [(300, 50, 64, 16), (1500, 400, 300, 75),
+                                           (2500, 2600, 500, 125), (900, 120, 900, 225),
+                                           (4100, 1000, 1000, 1000), (5000, 800, 1200, 0)])
+def test_unified_select_exact(ksa, oracle, L, P, budget, R):
+    rng = np.random.default_rng(700 + L)
+    B, Hq, Hkv, D = 3, 16, 4, 128
+    T = L + 37
+    q = dyadic_bits(rng, (B, Hq, D))
+    K = dyadic_bits(rng, (B, Hkv, T, D))
+    lens = np.array([L, max(1, L // 3), max(1, budget - 5)], np.int32)
+    idx, cnt = ksa.ksa_unified_select(to_dev_bf16(q), to_dev_bf16(K),
+                                      torch.from_numpy(lens).to(DEV), P, budget, R)
+    ref_idx, ref_cnt = oracle.unified_select(q, K, lens, P, budget, R)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+
+
+def test_unified_default_window_is_quarter(ksa, oracle):
+    rng = np.random.default_rng(710)
+    B, Hq, Hkv, D, T = 1, 8, 2, 64, 1200
+    q = dyadic_bits(rng, (B, Hq, D))
+    K = dyadic_bits(rng, (B, Hkv, T, D))
+    lens = np.array([T], np.int32)
+    idx, cnt = ksa.ksa_unified_select(to_dev_bf16(q), to_dev_bf16(K),
+                                      torch.from_numpy(lens).to(DEV), 200, 400)
+    ref_idx, _ = oracle.unified_select(q, K, lens, 200, 400, 100)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+
+
+# ---------------------------------------------------------------------------
+# whole decode step on the named workloads
+
+
+def _decode_step(ksa, inp, k):
+    sh = inp.shape
+    S = ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, sh.block_size)
+    ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, sh.block_size, ksa.SUMMARY_LAST_BLOCK,
+                                  summaries=S)
+    idx, cnt = ksa.ksa_select_blocks(inp.q, S, inp.seq_lens, sh.block_size, sh.capacity, k)
+    lse = torch.empty((sh.batch, sh.num_q_heads), dtype=torch.float32, device=DEV)
+    out, _ = ksa.ksa_sparse_decode_attn(inp.q, inp.K, inp.V, inp.seq_lens, idx, cnt,
+                                        tokens_per_idx=sh.block_size, lse=lse)
+    return idx, cnt, out, lse
+
+
+def _check_rows(oracle, inp, rows, idx, cnt, out, lse, k):
+    sh = inp.shape
+    for b in rows:
+        L = int(inp.seq_lens[b].item())
+        qb, Kb, Vb = host_bits(inp.q[b:b + 1]), host_bits(inp.K[b:b + 1]), host_bits(inp.V[b:b + 1])
+        lens = np.array([L], np.int32)
+        ref_idx, ref_cnt = oracle.select_blocks(qb, Kb, lens, sh.block_size, k)
+        assert np.array_equal(cnt[b].cpu().numpy(), ref_cnt[0]), b
+        assert np.array_equal(idx[b].cpu().numpy(), ref_idx[0]), b
+        ref, ref_lse, _ = oracle.attention(qb, Kb, Vb, lens, ref_idx, ref_cnt, sh.block_size)
+        assert_out_close(out[b:b + 1].cpu().numpy(), ref, what=f"row {b}")
+        np.testing.assert_allclose(lse[b:b + 1].cpu().numpy(), ref_lse, rtol=0, atol=LSE_TOL)
+
+
+def _plant(oracle, inp, rows, k):
+    sh = inp.shape
+    for b in rows:
+        L = int(inp.seq_lens[b].item())
+        Kb, _ = gap_fix_row(oracle, host_bits(inp.q[b]), host_bits(inp.K[b]), L, sh.block_size, k)
+        inp.K[b] = to_dev_bf16(Kb)
+
+
+def test_decode_step_tiny(ksa, oracle):
+    inp = synth.tiny_inputs(device=DEV)
+    rows = [0]
+    _plant(oracle, inp, rows, synth.TINY.k_blocks)
+    res = _decode_step(ksa, inp, synth.TINY.k_blocks)
+    _check_rows(oracle, inp, rows, *res, synth.TINY.k_blocks)
+
+
+def test_decode_step_qwen3_0_6b_full_size(ksa, oracle):
+    inp = synth.qwen3_0_6b_inputs(device=DEV)
+    rows = sample_rows(inp.shape.batch, 5)
+    _plant(oracle, inp, rows, inp.shape.k_blocks)
+    res = _decode_step(ksa, inp, inp.shape.k_blocks)
+    _check_rows(oracle, inp, rows, *res, inp.shape.k_blocks)
+
+
+def test_decode_step_qwen3_8b_full_size(ksa, oracle):
+    inp = synth.qwen3_8b_inputs(device=DEV, poison_tail=64.0)
+    rows = sample_rows(inp.shape.batch, 6)
+    _plant(oracle, inp, rows, inp.shape.k_blocks)
+    res = _decode_step(ksa, inp, inp.shape.k_blocks)
+    _check_rows(oracle, inp, rows, *res, inp.shape.k_blocks)
+
+
+def test_lessismore_full_size(ksa, oracle):
+    sh = synth.LESSISMORE
+    inp = synth.lessismore_inputs(device=DEV)
+    tok, cnt = ksa.ksa_unified_select(inp.q_sel, inp.K_sel, inp.seq_lens, sh.per_head_topk,
+                                      sh.token_budget, sh.recent_tokens)
+    rows = sample_rows(sh.batch, 7, extra=1)
+    for b in rows:
+        ref_idx, ref_cnt = oracle.unified_select(host_bits(inp.q_sel[b:b + 1]),
+                                                 host_bits(inp.K_sel[b:b + 1]),
+                                                 np.array([sh.seq_len], np.int32),
+                                                 sh.per_head_topk, sh.token_budget,
+                                                 sh.recent_tokens)
+        assert cnt[b].item() == ref_cnt[0] == sh.token_budget
+        assert np.array_equal(tok[b].cpu().numpy(), ref_idx[0]), b
+    for (q, K, V) in inp.layers:
+        out, _ = ksa.ksa_sparse_decode_attn(q, K, V, inp.seq_lens, tok, cnt, tokens_per_idx=1,
+                                            idx_shared=True)
+        for b in rows[:2]:
+            ref, _, _ = oracle.attention(host_bits(q[b:b + 1]), host_bits(K[b:b + 1]),
+                                         host_bits(V[b:b + 1]), np.array([sh.seq_len], np.int32),
+                                         tok[b:b + 1].cpu().numpy(), cnt[b:b + 1].cpu().numpy(),
+                                         1, True)
+            assert_out_close(out[b:b + 1].cpu().numpy(), ref, what=f"row {b}")
+
+
+def test_dense_full_context_sampled(ksa, oracle):
+    """k = all: the dense path on a 32K-context sweep shape (few rows)."""
+    sh = synth.dataclasses.replace(synth.sweep_shape(32768, 1024), batch=4)
+    inp = synth.sweep_inputs(sh, device=DEV)
+    out, _ = ksa.ksa_sparse_decode_attn(inp.q, inp.K, inp.V, inp.seq_lens)
+    for b in (0, 3):
+        ref, _, _ = oracle.attention(host_bits(inp.q[b:b + 1]), host_bits(inp.K[b:b + 1]),
+                                     host_bits(inp.V[b:b + 1]), np.array([32768], np.int32))
+        assert_out_close(out[b:b + 1].cpu().numpy(), ref, what=f"row {b}")
