@@ -51,6 +51,8 @@ def parse_args():
                    help="wall-clock budget of the oracle CPU baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the per-GPU batch (small profiling cases only)")
     return p.parse_args()
 
 
@@ -105,7 +107,15 @@ class Dist:
 # workloads
 
 
-def resolve_workload(name: str):
+def resolve_workload(name: str, batch: int = 0):
+    kind, shape = _resolve(name)
+    if batch > 0:
+        from block_top_sparse_ksa_b200 import synth
+        shape = synth.dataclasses.replace(shape, batch=batch)
+    return kind, shape
+
+
+def _resolve(name: str):
     from block_top_sparse_ksa_b200 import synth
     if name == "qwen3-0.6b":
         return "block", synth.QWEN3_0_6B
@@ -126,9 +136,9 @@ def resolve_workload(name: str):
 def make_block_inputs(shape, device):
     from block_top_sparse_ksa_b200 import synth
     if shape.name == synth.QWEN3_0_6B.name:
-        return synth.qwen3_0_6b_inputs(device=device)
+        return synth.qwen3_0_6b_inputs(device=device, shape=shape)
     if shape.name == synth.QWEN3_8B.name:
-        return synth.qwen3_8b_inputs(device=device)
+        return synth.qwen3_8b_inputs(device=device, shape=shape)
     if shape.name == synth.TINY.name:
         return synth.tiny_inputs(device=device)
     return synth.sweep_inputs(shape, device=device)
@@ -243,7 +253,7 @@ def stored_traffic(kernel: str, workload: str):
 
 def run_block(args, dist, dev, kind):
     import block_top_sparse_ksa_b200 as ksa
-    _, shape = resolve_workload(args.workload)
+    _, shape = resolve_workload(args.workload, args.batch)
     torch.manual_seed(0)
     inp = make_block_inputs(shape, dev)
     B, Hq, Hkv, D, T, bs = (shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
@@ -252,6 +262,10 @@ def run_block(args, dist, dev, kind):
     nq = 16
     qs = query_sets(shape, nq, dev)
     S = ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs)  # prefill, untimed
+    ws_sel = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
+                         dtype=torch.uint8, device=dev)
+    ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
+                         dtype=torch.uint8, device=dev)
     idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
     cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
@@ -260,14 +274,15 @@ def run_block(args, dist, dev, kind):
     def step(i):
         q = qs[i % nq]
         if kind == "dense":
-            ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, stream=stream)
+            ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, workspace=ws_att,
+                                       stream=stream)
             return
         ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, ksa.SUMMARY_LAST_BLOCK,
                                       summaries=S, stream=stream)
         ksa.ksa_select_blocks(q, S, inp.seq_lens, bs, T, k, block_idx=idx, num_sel=cnt,
-                              stream=stream)
+                              workspace=ws_sel, stream=stream)
         ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt, tokens_per_idx=bs,
-                                   out=out, stream=stream)
+                                   out=out, workspace=ws_att, stream=stream)
 
     launches_per_step = 1 if kind == "dense" else 3
     for i in range(args.warmup):
@@ -289,7 +304,8 @@ def run_block(args, dist, dev, kind):
             q = qs[i % nq]
             ev[0].record(stream)
             if kind == "dense":
-                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, stream=stream)
+                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out,
+                                           workspace=ws_att, stream=stream)
                 ev[1].record(stream)
                 ev[2].record(stream)
             else:
@@ -297,10 +313,11 @@ def run_block(args, dist, dev, kind):
                                               summaries=S, stream=stream)
                 ev[1].record(stream)
                 ksa.ksa_select_blocks(q, S, inp.seq_lens, bs, T, k, block_idx=idx, num_sel=cnt,
-                                      stream=stream)
+                                      workspace=ws_sel, stream=stream)
                 ev[2].record(stream)
                 ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt,
-                                           tokens_per_idx=bs, out=out, stream=stream)
+                                           tokens_per_idx=bs, out=out, workspace=ws_att,
+                                           stream=stream)
             ev[3].record(stream)
             marks.append(ev)
         else:
@@ -345,12 +362,12 @@ def run_block(args, dist, dev, kind):
                             "summaries(last block) + select_blocks + sparse_decode_attn")},
     }
     if not args.no_e2e:
-        res["e2e"] = run_block_e2e(args, dist, dev, kind, inp, S, qs, shape)
+        res["e2e"] = run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att)
     res["_host"] = (inp, S, qs, shape, kind)
     return res
 
 
-def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape):
+def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att):
     """Same step through the public API with host buffers: per step the new
     query and the new token's K/V rows go host->device (pinned), the output
     comes back device->host.  Copies are inside the timed region."""
@@ -379,14 +396,15 @@ def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape):
         inp.K[ar_b, :, pos] = d_kv[0]
         inp.V[ar_b, :, pos] = d_kv[1]
         if kind == "dense":
-            ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, out=out, stream=stream)
+            ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, out=out, workspace=ws_att,
+                                       stream=stream)
         else:
             ksa.ksa_build_block_summaries(inp.K, lens, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S,
                                           stream=stream)
             ksa.ksa_select_blocks(d_q, S, lens, bs, T, k, block_idx=idx, num_sel=cnt,
-                                  stream=stream)
+                                  workspace=ws_sel, stream=stream)
             ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, idx, cnt, tokens_per_idx=bs,
-                                       out=out, stream=stream)
+                                       out=out, workspace=ws_att, stream=stream)
         h_out.copy_(out, non_blocking=True)
 
     steps = args.steps
@@ -422,6 +440,9 @@ def run_unified(args, dist, dev):
     tok = torch.empty((B, sh.token_budget), dtype=torch.int32, device=dev)
     cnt = torch.empty((B,), dtype=torch.int32, device=dev)
     outs = [torch.empty((B, Hq, D), dtype=torch.float32, device=dev) for _ in inp.layers]
+    ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T,
+                                                               sh.token_budget, 1),),
+                         dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(i, ev=None):
@@ -433,7 +454,8 @@ def run_unified(args, dist, dev):
             ev[1].record(stream)
         for li, (q, K, V) in enumerate(inp.layers):
             ksa.ksa_sparse_decode_attn(q, K, V, inp.seq_lens, tok, cnt, tokens_per_idx=1,
-                                       idx_shared=True, out=outs[li], stream=stream)
+                                       idx_shared=True, out=outs[li], workspace=ws_att,
+                                       stream=stream)
         if ev:
             ev[2].record(stream)
 
@@ -528,7 +550,7 @@ def oracle_step_units(o, shape, kind, q, K, V, S, lens, rows):
 
 
 def cpu_baseline(args, dev, kind, budget_s):
-    _, shape = resolve_workload(args.workload)
+    _, shape = resolve_workload(args.workload, args.batch)
     n_rows = min(8, shape.batch)
     o, qb, K, V, S, lens = oracle_block_sample(shape, kind, n_rows, dev)
     o.set_threads(os.cpu_count() or 1)
@@ -551,7 +573,7 @@ def run_reference(args, dist):
     """The oracle as the reference arm: same workload/metric, host cores."""
     if dist.rank != 0:
         return
-    kind, shape = resolve_workload(args.workload)
+    kind, shape = resolve_workload(args.workload, args.batch)
     dev = torch.device("cuda", dist.local) if torch.cuda.is_available() else torch.device("cpu")
     if kind == "unified":
         print(json.dumps({"impl": "reference", "unavailable":

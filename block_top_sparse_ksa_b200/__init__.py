@@ -22,6 +22,7 @@ import torch
 __all__ = [
     "KsaError", "Shape", "lib", "library_path", "ksa_build_block_summaries",
     "ksa_select_blocks", "ksa_sparse_decode_attn", "ksa_unified_select",
+    "ksa_select_blocks_workspace", "ksa_sparse_decode_attn_workspace",
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "OUT_F32", "OUT_BF16", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -155,10 +156,25 @@ def ksa_build_block_summaries(K: torch.Tensor, seq_lens: torch.Tensor, block_siz
     return summaries
 
 
+def _workspace(ws: Optional[torch.Tensor], need: int, device) -> torch.Tensor:
+    """The caller's workspace, or a fresh zero-filled one (see include/ksa.h)."""
+    if ws is None:
+        return torch.zeros((max(need, 1),), dtype=torch.uint8, device=device)
+    _dev(ws, "workspace", ws.dtype)
+    return ws
+
+
+def ksa_select_blocks_workspace(B: int, Hq: int, Hkv: int, D: int, T: int, block_size: int,
+                                k_blocks: int) -> int:
+    sh = _shape(B, Hq, Hkv, D, T, block_size)
+    return int(lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)))
+
+
 def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.Tensor,
                       block_size: int, capacity: int, k_blocks: int,
                       block_idx: Optional[torch.Tensor] = None,
                       num_sel: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None,
                       dev_status: Optional[torch.Tensor] = None, stream=None):
     """Top-k blocks per (row, kv-head): (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv])."""
     _dev(q, "q", torch.bfloat16)
@@ -171,9 +187,12 @@ def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.
     if num_sel is None:
         num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     sh = _shape(B, Hq, Hkv, D, capacity, block_size)
+    ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
+                    q.device)
     _check(lib().ksa_select_blocks(ctypes.byref(sh), _ptr(q), _ptr(summaries), _ptr(seq_lens),
-                                   int(k_blocks), _ptr(block_idx), _ptr(num_sel), None, 0,
-                                   _ptr(dev_status), _stream(stream)))
+                                   int(k_blocks), _ptr(block_idx), _ptr(num_sel), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _ptr(dev_status),
+                                   _stream(stream)))
     return block_idx, num_sel
 
 
@@ -183,6 +202,7 @@ def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                            idx_shared: bool = False, scale: float = 0.0,
                            out_dtype: int = OUT_F32, out: Optional[torch.Tensor] = None,
                            lse: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None,
                            dev_status: Optional[torch.Tensor] = None, stream=None):
     """Softmax attention over the selected tokens (dense when idx is None): (out, lse)."""
     _dev(q, "q", torch.bfloat16)
@@ -203,11 +223,21 @@ def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     if lse is not None:
         _dev(lse, "lse", torch.float32)
     sh = _shape(B, Hq, Hkv, D, T, max(1, tokens_per_idx))
+    ws = _workspace(workspace, lib().ksa_sparse_decode_attn_workspace(
+        ctypes.byref(sh), int(cap), int(tokens_per_idx)), q.device)
     _check(lib().ksa_sparse_decode_attn(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx), _ptr(num_idx),
         int(cap), int(tokens_per_idx), int(bool(idx_shared)), float(scale), int(out_dtype),
-        _ptr(out), _ptr(lse), None, 0, _ptr(dev_status), _stream(stream)))
+        _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
     return out, lse
+
+
+def ksa_sparse_decode_attn_workspace(B: int, Hq: int, Hkv: int, D: int, T: int,
+                                     idx_capacity: int = 0, tokens_per_idx: int = 1) -> int:
+    sh = _shape(B, Hq, Hkv, D, T, max(1, tokens_per_idx))
+    return int(lib().ksa_sparse_decode_attn_workspace(ctypes.byref(sh), int(idx_capacity),
+                                                      int(tokens_per_idx)))
 
 
 def ksa_unified_select_workspace(B: int, Hq: int, Hkv: int, D: int, T: int, per_head_topk: int,
@@ -230,7 +260,7 @@ def ksa_unified_select(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor,
     B, Hq, D = q.shape
     _, Hkv, T, _ = K.shape
     need = ksa_unified_select_workspace(B, Hq, Hkv, D, T, per_head_topk, token_budget)
-    if workspace is None:
+    if workspace is None:  # the unified workspace needs no initialisation
         workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     if token_idx is None:
         token_idx = torch.empty((B, token_budget), dtype=torch.int32, device=q.device)

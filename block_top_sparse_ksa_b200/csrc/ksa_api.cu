@@ -137,17 +137,16 @@ ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
 }
 
 size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks) {
-  (void)shape;
   (void)k_blocks;
-  return 0;
+  if (check_shape(shape, true) != KSA_OK) return 0;
+  return ksa::select_workspace_bytes(shape->batch, shape->num_kv_heads, shape->capacity,
+                                     shape->block_size);
 }
 
 ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const float *summaries,
                              const int32_t *seq_lens, int32_t k_blocks, int32_t *block_idx,
                              int32_t *num_sel, void *ws, size_t ws_bytes, uint32_t *dev_status,
                              void *stream) {
-  (void)ws;
-  (void)ws_bytes;
   ksa_status st = check_shape(shape, true);
   if (st != KSA_OK) return st;
   if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
@@ -159,6 +158,11 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const fl
     return fail(KSA_ERR_UNSUPPORTED, "ceil(capacity/block_size) = %d exceeds 16384", nb_max);
   if (!aligned(summaries, 16) || !aligned(q, 4))
     return fail(KSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
+  const size_t need = ksa::select_workspace_bytes(shape->batch, shape->num_kv_heads,
+                                                  shape->capacity, shape->block_size);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   ksa::SelectArgs a;
   a.q = q;
   a.S = summaries;
@@ -174,16 +178,17 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const fl
   a.bs = shape->block_size;
   a.k = k_blocks;
   return cuda_status(
-      ksa::launch_select_blocks(a, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      ksa::launch_select_blocks(a, ws, device_sm_count(), static_cast<cudaStream_t>(stream)),
       "ksa_select_blocks launch");
 }
 
 size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape, int32_t idx_capacity,
                                         int32_t tokens_per_idx) {
-  (void)shape;
   (void)idx_capacity;
   (void)tokens_per_idx;
-  return 0;
+  if (check_shape(shape, false) != KSA_OK) return 0;
+  return ksa::attn_workspace_bytes(shape->batch, shape->num_q_heads, shape->num_kv_heads,
+                                   shape->head_dim, device_sm_count());
 }
 
 ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
@@ -192,8 +197,6 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, con
                                   int32_t tokens_per_idx, int32_t idx_shared, float scale,
                                   int32_t out_dtype, void *out, float *lse, void *ws,
                                   size_t ws_bytes, uint32_t *dev_status, void *stream) {
-  (void)ws;
-  (void)ws_bytes;
   ksa_status st = check_shape(shape, false);
   if (st != KSA_OK) return st;
   if (q == nullptr || K == nullptr || V == nullptr || seq_lens == nullptr || out == nullptr)
@@ -220,6 +223,12 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, con
   if (!aligned(K, 16) || !aligned(V, 16) || !aligned(q, 4) ||
       !aligned(out, out_dtype == KSA_OUT_F32 ? 4 : 2) || (lse && !aligned(lse, 4)))
     return fail(KSA_ERR_INVALID_ARG, "K and V must be 16-byte aligned, q and out element-aligned");
+  const int sms = device_sm_count();
+  const size_t need = ksa::attn_workspace_bytes(shape->batch, shape->num_q_heads,
+                                                shape->num_kv_heads, shape->head_dim, sms);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   ksa::AttnArgs a;
   a.q = q;
   a.K = K;
@@ -242,7 +251,7 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, con
   a.scale = scale == 0.f ? static_cast<float>(1.0 / sqrt(static_cast<double>(shape->head_dim)))
                          : scale;
   return cuda_status(
-      ksa::launch_sparse_decode_attn(a, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      ksa::launch_sparse_decode_attn(a, ws, sms, static_cast<cudaStream_t>(stream)),
       "ksa_sparse_decode_attn launch");
 }
 

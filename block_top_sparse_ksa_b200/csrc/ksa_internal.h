@@ -28,7 +28,9 @@ struct SelectArgs {
   uint32_t *status;
   int B, Hq, Hkv, D, T, bs, k;
 };
-cudaError_t launch_select_blocks(const SelectArgs &a, int num_sms, cudaStream_t stream);
+// workspace: semaphores [B*Hkv] (zero between calls) + score keys [B*Hkv, ceil(T/bs)]
+size_t select_workspace_bytes(int B, int Hkv, int T, int bs);
+cudaError_t launch_select_blocks(const SelectArgs &a, void *ws, int num_sms, cudaStream_t stream);
 
 struct AttnArgs {
   const uint16_t *q, *K, *V;
@@ -43,7 +45,12 @@ struct AttnArgs {
   int cap, tpi, shared;
   float scale;
 };
-cudaError_t launch_sparse_decode_attn(const AttnArgs &a, int num_sms, cudaStream_t stream);
+// Resident CTAs per SM the attention workspace is sized for (the launch never exceeds it).
+constexpr int kAttnMaxCtasPerSm = 4;
+// workspace: semaphores [B*Hkv] (zero between calls) + split-row partials
+size_t attn_workspace_bytes(int B, int Hq, int Hkv, int D, int num_sms);
+cudaError_t launch_sparse_decode_attn(const AttnArgs &a, void *ws, int num_sms,
+                                      cudaStream_t stream);
 
 struct UnifiedArgs {
   const uint16_t *q, *K;

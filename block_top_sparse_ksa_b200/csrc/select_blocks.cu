@@ -5,14 +5,15 @@
 // (the source gives no formula): the dot product of the block mean with the
 // sum of the kv-group's query heads, one selection per kv-head.
 //
-// One thread-block cluster per (row b, kv-head g).  Each CTA of the cluster
-// streams a contiguous slice of the row's fp32 summaries (8 lanes per 512-byte
-// summary row, 128-bit loads, two row groups in flight per warp), reduces the
-// dot products with warp shuffles, and stores order-preserving uint32 score
-// keys straight into the shared memory of CTA rank 0 (distributed shared
-// memory).  After a cluster barrier, rank 0 runs an exact radix select (k-th
-// largest key; ties at the threshold resolved toward the lower block index)
-// and writes the winners in ascending block order.  Scores never touch HBM.
+// One CTA per (row b, kv-head g, chunk of up to 128 blocks).  The CTA pulls its
+// chunk of fp32 summaries (<= 64 KB, contiguous) into shared memory with one
+// TMA bulk copy, so the whole chunk is in flight at once, forms the group
+// query sum meanwhile, scores the blocks (8 lanes per summary row, warp
+// shuffles) and stores order-preserving uint32 score keys in the workspace.
+// The row's chunks count themselves on a semaphore; the CTA finishing last
+// stages the row's keys in shared memory and runs an exact radix select
+// (k-th largest key; ties at the threshold go to the lower block index),
+// writes the winners in ascending block order, and resets the semaphore.
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
 
@@ -22,140 +23,179 @@ namespace {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelRows = 128;  // summary rows per CTA
+
+struct SelDev {
+  SelectArgs a;
+  int chunks;      // CTAs per (row, kv-head)
+  uint32_t *keys;  // workspace [B*Hkv, nb_max]
+  int32_t *sem;    // workspace [B*Hkv], zero between calls
+};
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
 
 template <int D>
-__global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a, int csize) {
+__global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw);  // [nb_max], used on rank 0
+  float *sbuf = reinterpret_cast<float *>(smem_raw);  // chunk summaries, later the row's keys
+  __shared__ uint64_t bar;
+  __shared__ __align__(16) float qsum[D];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t info[4];
   __shared__ uint32_t scratch[33];
-  __shared__ __align__(16) float qsum[D];
+  __shared__ int is_last;
+  __shared__ int timed_out;
 
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
+  const SelectArgs &a = p.a;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = blockIdx.x / csize;
+  const int row = blockIdx.x / p.chunks, chunk = blockIdx.x % p.chunks;
   const int b = row / a.Hkv, g = row % a.Hkv;
   const int G = a.Hq / a.Hkv;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
-  const int L = clamp_len(a.seq_lens[b], a.T, (rank == 0 && tid == 0) ? a.status : nullptr);
+  const int L = clamp_len(a.seq_lens[b], a.T, (chunk == 0 && tid == 0) ? a.status : nullptr);
   const int nb = (L + a.bs - 1) / a.bs;
   const int k = a.k;
   int32_t *out = a.block_idx + static_cast<size_t>(row) * k;
 
-  if (nb <= k) {  // every block is kept; no summary is read (same branch for the whole cluster)
-    if (rank == 0) {
+  if (nb <= k) {  // every block is kept; no summary is read
+    if (chunk == 0) {
       for (int i = tid; i < k; i += kSelThreads) out[i] = i < nb ? i : -1;
       if (tid == 0) a.num_sel[row] = nb;
     }
     return;
   }
-
+  const int j0 = static_cast<int>(static_cast<long long>(chunk) * nb / p.chunks);
+  const int j1 = static_cast<int>(static_cast<long long>(chunk + 1) * nb / p.chunks);
+  const int n = j1 - j0;
+  if (tid == 0) {
+    mbar_init(&bar, 1u);
+    timed_out = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0 && n > 0) {
+    const uint32_t bytes = static_cast<uint32_t>(n) * D * 4u;
+    mbar_arrive_expect_tx(&bar, bytes);
+    bulk_g2s(sbuf, a.S + (static_cast<size_t>(row) * nb_max + j0) * D, bytes, &bar);
+  }
+  // group query sum while the chunk is in flight
   for (int d = tid; d < D; d += kSelThreads) {
     const uint16_t *qp = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * D + d;
     float s = 0.f;
     for (int h = 0; h < G; ++h) s += bf16_bits_to_f32(qp[static_cast<size_t>(h) * D]);
     qsum[d] = s;
   }
-  cluster.sync();  // all CTAs of the cluster are running before any remote store
+  __syncthreads();
 
-  constexpr int PER = D / 32;  // float4 chunks per lane: chunk (sub + 8*i) of the row
-  const int sub = lane & 7;
-  float4 qv[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) qv[i] = reinterpret_cast<const float4 *>(qsum)[sub + 8 * i];
-
-  const int j0 = static_cast<int>(static_cast<long long>(rank) * nb / csize);
-  const int j1 = static_cast<int>(static_cast<long long>(rank + 1) * nb / csize);
-  uint32_t *keys0 = cluster.map_shared_rank(keys, 0);
-  const float4 *srow =
-      reinterpret_cast<const float4 *>(a.S + static_cast<size_t>(row) * nb_max * D);
   uint32_t bad = 0u;
-  constexpr int kStride = kSelWarps * 4;  // summary rows covered by the CTA per step
-  for (int jb = j0 + warp * 4; jb < j1; jb += 2 * kStride) {
-    const int ja = jb + (lane >> 3);
-    const int jc = ja + kStride;
-    float4 va[PER], vc[PER];
+  if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar, 0u))) {
+    bad |= KSA_FLAG_WAIT_TIMEOUT;
+    timed_out = 1;
+  }
+  if (n > 0 && bad == 0u) {
+    constexpr int PER = D / 32;  // float4 chunks per lane: chunk (sub + 8*i) of the row
+    const int sub = lane & 7;
+    float4 qv[PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      va[i] = ja < j1 ? __ldg(srow + static_cast<size_t>(ja) * (D / 4) + sub + 8 * i)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      vc[i] = jc < j1 ? __ldg(srow + static_cast<size_t>(jc) * (D / 4) + sub + 8 * i)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float sa = 0.f, sc = 0.f;
+    for (int i = 0; i < PER; ++i) qv[i] = reinterpret_cast<const float4 *>(qsum)[sub + 8 * i];
+    uint32_t *krow = p.keys + static_cast<size_t>(row) * nb_max;
+    // warp-uniform trip count: every lane reaches the full-mask shuffles
+    for (int jw = warp * 4; jw < n; jw += kSelWarps * 4) {
+      const int jr = jw + (lane >> 3);
+      const bool live = jr < n;
+      const float4 *srow = reinterpret_cast<const float4 *>(sbuf + static_cast<size_t>(jr) * D);
+      float s = 0.f;
+      if (live) {
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      sa = fmaf(qv[i].x, va[i].x, sa);
-      sa = fmaf(qv[i].y, va[i].y, sa);
-      sa = fmaf(qv[i].z, va[i].z, sa);
-      sa = fmaf(qv[i].w, va[i].w, sa);
-      sc = fmaf(qv[i].x, vc[i].x, sc);
-      sc = fmaf(qv[i].y, vc[i].y, sc);
-      sc = fmaf(qv[i].z, vc[i].z, sc);
-      sc = fmaf(qv[i].w, vc[i].w, sc);
-    }
-#pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
-      sa += __shfl_xor_sync(0xffffffffu, sa, off);
-      sc += __shfl_xor_sync(0xffffffffu, sc, off);
-    }
-    if (sub == 0) {
-      bool nan;
-      if (ja < j1) {
-        keys0[ja] = score_key(sa, nan);
-        bad |= nan ? KSA_FLAG_NONFINITE_SCORE : 0u;
+        for (int i = 0; i < PER; ++i) {
+          const float4 v = srow[sub + 8 * i];
+          s = fmaf(qv[i].x, v.x, s);
+          s = fmaf(qv[i].y, v.y, s);
+          s = fmaf(qv[i].z, v.z, s);
+          s = fmaf(qv[i].w, v.w, s);
+        }
       }
-      if (jc < j1) {
-        keys0[jc] = score_key(sc, nan);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (live && sub == 0) {
+        bool nan;
+        krow[j0 + jr] = score_key(s, nan);
         bad |= nan ? KSA_FLAG_NONFINITE_SCORE : 0u;
       }
     }
   }
   flag_status(a.status, bad);
-  cluster.sync();  // every key of the row is in rank 0's shared memory
-  if (rank != 0) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = (atomicAdd(&p.sem[row], 1) == p.chunks - 1) ? 1 : 0;
+  __syncthreads();
+  if (timed_out) {  // block-uniform: read after the barrier above
+    if (tid == 0) mbar_wait(&bar, 0u);  // let the copy land before the smem is reused
+    __syncthreads();
+  }
+  if (!is_last) return;
 
+  // ---- last chunk of the row: exact top-k over the row's keys
+  __threadfence();
+  uint32_t *kb = reinterpret_cast<uint32_t *>(sbuf);
+  const uint32_t *krow = p.keys + static_cast<size_t>(row) * nb_max;
+  for (int j = tid; j < nb; j += kSelThreads) kb[j] = __ldcg(krow + j);
+  __syncthreads();
   uint32_t tau, n_gt, n_eq;
-  radix_select_desc<kSelThreads>(keys, nb, k, 32, hist, info, tau, n_gt, n_eq);
-  select_ascending<kSelThreads>(keys, nb, tau, n_gt, n_eq, k, out, scratch, [](int) {});
-  if (tid == 0) a.num_sel[row] = k;
+  radix_select_desc<kSelThreads>(kb, nb, k, 32, hist, info, tau, n_gt, n_eq);
+  select_ascending<kSelThreads>(kb, nb, tau, n_gt, n_eq, k, out, scratch, [](int) {});
+  if (tid == 0) {
+    a.num_sel[row] = k;
+    p.sem[row] = 0;  // ready for the next call
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_select_blocks(const SelectArgs &a, int num_sms, cudaStream_t stream) {
+size_t select_workspace_bytes(int B, int Hkv, int T, int bs) {
+  const size_t rows = static_cast<size_t>(B) * Hkv;
+  const size_t nb_max = static_cast<size_t>((T + bs - 1) / bs);
+  const size_t sems = (rows * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  const size_t keys = (rows * nb_max * sizeof(uint32_t) + 255) & ~static_cast<size_t>(255);
+  return sems + keys;
+}
+
+cudaError_t launch_select_blocks(const SelectArgs &a, void *ws, int num_sms,
+                                 cudaStream_t stream) {
   (void)num_sms;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
-  int csize = (nb_max + 255) / 256;
-  csize = csize < 1 ? 1 : (csize > 8 ? 8 : csize);
-  const size_t smem = static_cast<size_t>(nb_max) * sizeof(uint32_t);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.B) * a.Hkv * csize, 1, 1);
-  cfg.blockDim = dim3(kSelThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  SelDev p;
+  p.a = a;
+  p.chunks = (nb_max + kSelRows - 1) / kSelRows;
+  const size_t rows = static_cast<size_t>(a.B) * a.Hkv;
+  const size_t sems = (rows * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  p.sem = static_cast<int32_t *>(ws);
+  p.keys = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + sems);
+  size_t smem = static_cast<size_t>(kSelRows) * a.D * sizeof(float);
+  if (static_cast<size_t>(nb_max) * sizeof(uint32_t) > smem)
+    smem = static_cast<size_t>(nb_max) * sizeof(uint32_t);
+  const unsigned grid = static_cast<unsigned>(rows * p.chunks);
   cudaError_t err;
   if (a.D == 128) {
     err = cudaFuncSetAttribute(select_blocks_kernel<128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = cudaLaunchKernelEx(&cfg, select_blocks_kernel<128>, a, csize);
+    select_blocks_kernel<128><<<grid, kSelThreads, smem, stream>>>(p);
   } else {
     err = cudaFuncSetAttribute(select_blocks_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = cudaLaunchKernelEx(&cfg, select_blocks_kernel<64>, a, csize);
+    select_blocks_kernel<64><<<grid, kSelThreads, smem, stream>>>(p);
   }
-  return err;
+  return cudaGetLastError();
 }
 
 }  // namespace ksa

@@ -4,10 +4,11 @@
 // and every block is represented by its mean key,
 //   S[b,g,j,:] = (1/n_j) sum_{t in block j, t < L_b} K[b,g,t,:],  n_j = min(bs, L_b - j*bs).
 //
-// One warp per block: lane l owns D/32 consecutive dims, so every warp-wide
-// load reads one whole 2*D-byte key row (fully coalesced); the bs rows of a
-// block are independent loads kept in flight by unrolling.  Sums are fp32 in
-// token order, then one IEEE division by n_j.
+// One warp per block.  Lane l reads 16-byte chunk (l % (D/8)) of the block's
+// rows l / (D/8), l / (D/8) + 32/(D/8), ... so every warp-wide load covers
+// 2 (D = 128) or 4 (D = 64) whole key rows and all of a block's loads are
+// independent (in flight together).  Partial sums meet through warp shuffles;
+// then one IEEE division by n_j, in fp32.
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
 
@@ -16,24 +17,11 @@ namespace ksa {
 namespace {
 
 template <int D>
-__device__ __forceinline__ void load_dims(const uint16_t *p, float (&v)[D / 32]) {
-  if constexpr (D == 128) {
-    const uint2 x = __ldg(reinterpret_cast<const uint2 *>(p));
-    v[0] = bf16_lo(x.x);
-    v[1] = bf16_hi(x.x);
-    v[2] = bf16_lo(x.y);
-    v[3] = bf16_hi(x.y);
-  } else {
-    const uint32_t x = __ldg(reinterpret_cast<const uint32_t *>(p));
-    v[0] = bf16_lo(x);
-    v[1] = bf16_hi(x);
-  }
-}
-
-template <int D>
 __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
-  constexpr int DPL = D / 32;
+  constexpr int CH = D / 8;     // 16-byte chunks per key row
+  constexpr int RP = 32 / CH;   // rows covered by one warp-wide load
   const int lane = threadIdx.x & 31;
+  const int c = lane % CH, rp = lane / CH;
   const int wpc = blockDim.x >> 5;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   const bool all = (a.mode == KSA_SUMMARY_ALL);
@@ -54,25 +42,35 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
       j = nb - 1;
     }
     const int n = min(a.bs, L - j * a.bs);
-    const uint16_t *src = a.K + (static_cast<size_t>(bg) * a.T + static_cast<size_t>(j) * a.bs) * D +
-                          lane * DPL;
-    float acc[DPL];
+    const uint16_t *src =
+        a.K + (static_cast<size_t>(bg) * a.T + static_cast<size_t>(j) * a.bs) * D + c * 8;
+    float acc[8];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll 8
-    for (int t = 0; t < n; ++t) {
-      float v[DPL];
-      load_dims<D>(src + static_cast<size_t>(t) * D, v);
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] += v[i];
+    for (int t = rp; t < n; t += RP) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + static_cast<size_t>(t) * D));
+      acc[0] += bf16_lo(x.x);
+      acc[1] += bf16_hi(x.x);
+      acc[2] += bf16_lo(x.y);
+      acc[3] += bf16_hi(x.y);
+      acc[4] += bf16_lo(x.z);
+      acc[5] += bf16_hi(x.z);
+      acc[6] += bf16_lo(x.w);
+      acc[7] += bf16_hi(x.w);
     }
-    float *dst = a.S + (static_cast<size_t>(bg) * nb_max + j) * D + lane * DPL;
-    const float fn = static_cast<float>(n);
-    if constexpr (DPL == 4) {
-      *reinterpret_cast<float4 *>(dst) =
+#pragma unroll
+    for (int off = CH; off < 32; off <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+    }
+    if (rp == 0) {
+      const float fn = static_cast<float>(n);
+      float *dst = a.S + (static_cast<size_t>(bg) * nb_max + j) * D + c * 8;
+      reinterpret_cast<float4 *>(dst)[0] =
           make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
-    } else {
-      *reinterpret_cast<float2 *>(dst) = make_float2(acc[0] / fn, acc[1] / fn);
+      reinterpret_cast<float4 *>(dst)[1] =
+          make_float4(acc[4] / fn, acc[5] / fn, acc[6] / fn, acc[7] / fn);
     }
   }
 }

@@ -38,7 +38,8 @@ struct SCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kHalfBytes = kTok * 128;
   static constexpr int kStageBytes = kHalves * kHalfBytes;
-  static constexpr int kStages = 8;
+  static constexpr int kStages = 8;  // multiple of the 4 consumer warps: one owner per buffer
+  static_assert(kStages % 4 == 0, "stage buffers must map to one consumer warp each");
   static constexpr size_t kSmemBytes =
       1024 + static_cast<size_t>(kStages) * kStageBytes + 16 * kStages + 64;
 };

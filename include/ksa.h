@@ -30,6 +30,14 @@
  *   - Bad device data never faults: a seq_len outside [1, T] is clamped to
  *     [0, T] and flagged; an index entry outside the row is skipped and
  *     flagged.
+ *   - Workspaces (ws): caller-allocated device scratch of the size the
+ *     matching *_workspace() query returns for the same shape on the current
+ *     device, 256-byte aligned.  The select and attention workspaces begin with
+ *     per-row semaphores that must be zero when a call starts: zero-fill the
+ *     buffer once after allocating it; every call that completes leaves them
+ *     zero again, so one buffer serves any number of calls issued one after
+ *     another.  Calls that may run concurrently need separate workspaces.
+ *     After a KSA_FLAG_WAIT_TIMEOUT the workspace must be zero-filled again.
  */
 #ifndef KSA_H
 #define KSA_H
@@ -94,9 +102,10 @@ ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
  *   summaries: [B, Hkv, ceil(T/bs), D] fp32 (from ksa_build_block_summaries)
  *   block_idx: [B, Hkv, k_blocks] int32, ascending, -1 padded (written)
  *   num_sel:   [B, Hkv] int32 = min(k_blocks, NB_b) (written)
- *   ws:        unused (pass NULL, 0); kept for ABI stability.
- * Limits: k_blocks >= 1; ceil(T/bs) <= 16384 (scores of one row live in
- * on-chip memory), else KSA_ERR_UNSUPPORTED.
+ *   ws:        device scratch of ksa_select_blocks_workspace() bytes, 256-byte
+ *              aligned (see "Workspaces" above).
+ * Limits: k_blocks >= 1; ceil(T/bs) <= 16384 (the scores of one row are
+ * ranked in on-chip memory), else KSA_ERR_UNSUPPORTED.
  */
 size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks);
 ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q,
@@ -122,7 +131,9 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q,
  * lse = -inf.  Accumulation is fp32; scale == 0 selects 1/sqrt(D).
  *   out: [B, Hq, D] fp32 (out_dtype KSA_OUT_F32) or bf16 (KSA_OUT_BF16)
  *   lse: [B, Hq] fp32, nullable
- *   ws:  unused (pass NULL, 0); kept for ABI stability.
+ *   ws:  device scratch of ksa_sparse_decode_attn_workspace() bytes, 256-byte
+ *        aligned (see "Workspaces" above); rows whose tokens are split between
+ *        CTAs leave partial results there.
  * Limits: D in {64, 128}; G <= 8; tokens_per_idx a power of two <= 256.
  */
 size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape,

@@ -39,8 +39,6 @@ def test_library_exports_every_declared_symbol(ksa):
 
 def test_binding_wraps_every_entry_point(ksa):
     for n in declared_functions():
-        if n.endswith("_workspace") and n != "ksa_unified_select_workspace":
-            continue  # workspace queries of calls that need none
         assert hasattr(ksa, n), n
 
 
@@ -103,5 +101,17 @@ def test_workspace_sizes(ksa):
     sh = _shape(ksa, B=16, Hq=32, Hkv=8, D=128, T=20000)
     ws = lib.ksa_unified_select_workspace(ctypes.byref(sh), 4000, 4000)
     assert ws >= 16 * 32 * 20000 * 4 + 16 * 20000 * 4
-    assert lib.ksa_select_blocks_workspace(ctypes.byref(sh), 128) == 0
-    assert lib.ksa_sparse_decode_attn_workspace(ctypes.byref(sh), 128, 16) == 0
+    sh16 = _shape(ksa, B=32, Hq=32, Hkv=8, D=128, T=32768, bs=16)
+    assert lib.ksa_select_blocks_workspace(ctypes.byref(sh16), 128) >= 32 * 8 * 2048 * 4 + 32 * 8 * 4
+    assert lib.ksa_sparse_decode_attn_workspace(ctypes.byref(sh16), 128, 16) >= 32 * 8 * 4
+    bad = _shape(ksa, D=96)
+    assert lib.ksa_select_blocks_workspace(ctypes.byref(bad), 8) == 0
+
+
+def test_missing_workspace_is_rejected(ksa):
+    lib = ksa.lib()
+    sh = _shape(ksa)
+    assert lib.ksa_select_blocks(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, 0, None,
+                                 None) == 3
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, None, None, 0, 1,
+                                      0, 0.0, 0, FAKE, None, None, 0, None, None) == 3

@@ -393,3 +393,28 @@ def test_dense_full_context_sampled(ksa, oracle):
         ref, _, _ = oracle.attention(host_bits(inp.q[b:b + 1]), host_bits(inp.K[b:b + 1]),
                                      host_bits(inp.V[b:b + 1]), np.array([32768], np.int32))
         assert_out_close(out[b:b + 1].cpu().numpy(), ref, what=f"row {b}")
+
+
+@pytest.mark.parametrize("mode", ["dense", "blocks", "tokens"])
+def test_long_pipelines(ksa, oracle, mode):
+    """Few rows, long selections: every CTA cycles its stage buffers dozens of
+    times (the pipeline's barrier phases wrap many times)."""
+    rng = np.random.default_rng(800)
+    B, Hq, Hkv, D, T, bs = 1, 8, 2, 128, 32768, 16
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([T - 5], np.int32)
+    if mode == "dense":
+        assert _attn_check(ksa, oracle, q, K, V, lens) == 0
+    elif mode == "blocks":
+        nb = -(-lens[0] // bs)
+        idx = np.stack([np.sort(rng.choice(nb, size=1024, replace=False)) for _ in range(Hkv)])
+        idx[:, -1] = nb - 1  # keep the partial tail block
+        idx = np.sort(idx, axis=1)[None].astype(np.int32)
+        cnt = np.full((B, Hkv), 1024, np.int32)
+        assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, bs) == 0
+    else:
+        idx = np.sort(rng.choice(lens[0], size=8192, replace=False))[None].astype(np.int32)
+        cnt = np.array([8192], np.int32)
+        assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, 1, shared=True) == 0
