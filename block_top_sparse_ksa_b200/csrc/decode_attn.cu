@@ -5,7 +5,7 @@
 // GQA group, so the G query heads of a kv-head read each K/V row once.
 //
 // Design (B200, sm_100a):
-//  * persistent, stream-K split: the work is the flat sequence of 32-token
+//  * persistent, stream-K split: the work is the flat sequence of 16-token
 //    stages of all (row b, kv-head g) pairs, each row padded to V stages (the
 //    most any row can hold); a fixed grid of (SMs x resident CTAs) CTAs takes
 //    equal contiguous slices of it, so every CTA streams about the same number
@@ -14,7 +14,7 @@
 //    no multicast) of the selected K and V rows -- whole blocks / dense runs --
 //    or, for token lists, 16-byte cp.async into the same swizzled layout; each
 //    stage buffer has a full and an empty mbarrier (bounded waits) and belongs
-//    to one consumer warp, so its phases are awaited in order;
+//    to one consumer warp (two buffers per warp, so loads overlap compute);
 //  * warps 0-3 consume the stages round-robin.  The G (<= 8) query heads of
 //    the group form the N dimension of mma.sync m16n8k16 tiles: S^T = K_tile q^T
 //    (16 tokens x 8 heads, fp32 accumulate), online softmax in fp32 registers,
@@ -36,7 +36,9 @@ namespace ksa {
 
 namespace {
 
-constexpr int kStageTok = 32;
+constexpr int kStageTok = 16;  // tokens per pipeline stage (16 or 32: one or two mma tiles)
+constexpr int kTiles = kStageTok / 16;
+constexpr uint32_t kFullMask = kStageTok >= 32 ? 0xffffffffu : ((1u << kStageTok) - 1u);
 constexpr int kConsumers = 4;
 constexpr int kAttnThreads = (kConsumers + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -46,7 +48,7 @@ enum { kModeDense = 0, kModeTma = 1, kModeCp = 2 };
 template <int D>
 struct Cfg {
   static constexpr int kHalves = D / 64;              // 64-column (128-byte) halves of a row
-  static constexpr int kHalfBytes = kStageTok * 128;  // one half of a 32-row tile
+  static constexpr int kHalfBytes = kStageTok * 128;  // one 64-column half of a stage tile
   static constexpr int kTileBytes = kHalves * kHalfBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;  // K tile + V tile
   // A multiple of the consumer-warp count: stage i lives in buffer i % kStages
@@ -54,7 +56,8 @@ struct Cfg {
   // the same warp and that warp awaits the buffer's phases strictly in order.
   // (With buffers shared between warps a fast warp could wait on a phase two
   // ahead of the barrier, which a parity wait cannot tell from a finished one.)
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  // Two buffers per warp: a warp computes on one while its next stage lands.
+  static constexpr int kStages = (kStageTok == 16 ? 8 : 4) * (D == 128 ? 1 : 2);
   static_assert(kStages % kConsumers == 0, "stage buffers must map to one consumer warp each");
   static constexpr int kKT = D / 16;
   // stage buffers, 2 mbarriers + 1 mask per stage, flags; plus 1 KB alignment slack
@@ -119,45 +122,6 @@ __device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int r, uint32_t *
   return ri;
 }
 
-struct StageSpan {
-  long long t0;  // first token of the segment
-  int nvalid;    // rows of the segment below L
-  bool entry;    // the segment comes from a real list entry
-};
-
-// Segment u (one per lane) of stage `stage` of a row.  Dense and TMA modes.
-__device__ __forceinline__ StageSpan stage_segment(int mode, int stage, int u, int tpi,
-                                                   const RowInfo &ri) {
-  StageSpan sp{0, 0, false};
-  if (mode == kModeDense) {
-    if (u == 0) {
-      sp.t0 = static_cast<long long>(stage) * kStageTok;
-      sp.nvalid = static_cast<int>(min(static_cast<long long>(kStageTok), ri.L - sp.t0));
-      sp.entry = true;
-    }
-    return sp;
-  }
-  const int seg = tpi < kStageTok ? tpi : kStageTok;
-  const int nseg = kStageTok / seg;
-  if (u >= nseg) return sp;
-  int e, part;
-  if (tpi >= kStageTok) {
-    e = stage / (tpi / kStageTok);
-    part = stage % (tpi / kStageTok);
-  } else {
-    e = stage * nseg + u;
-    part = 0;
-  }
-  if (e >= ri.n_idx) return sp;
-  const int id = ri.list[e];
-  sp.entry = true;
-  if (id < 0) return sp;
-  sp.t0 = static_cast<long long>(id) * tpi + static_cast<long long>(part) * kStageTok;
-  const long long left = ri.L - sp.t0;
-  sp.nvalid = static_cast<int>(left <= 0 ? 0 : (left < seg ? left : seg));
-  return sp;
-}
-
 __device__ __forceinline__ void store_out(const AttnArgs &a, size_t oi, float v) {
   if (a.out_f32 != nullptr)
     a.out_f32[oi] = v;
@@ -200,76 +164,141 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
     *abort_flag = 0u;
     fence_mbar_init();
   }
+  if (MODE != kModeCp && tid == kConsumers * 32) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
 
-  int issued = 0;  // stages the producer filled
+  int issued = 0;  // stages the producer filled (TMA modes: uses of the lane's own buffer)
 
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
-    if (MODE != kModeCp && lane == 0) {
-      prefetch_tensormap(&kmap);
-      prefetch_tensormap(&vmap);
-    }
     uint32_t skipped = 0u;
-    bool stop = false;
-    int i = 0;
-    for (int r = r_first; r <= r_last && !stop; ++r) {
-      const long long rv0 = static_cast<long long>(r) * p.V;
-      // the CTA holding the row's first stage reports the row's bad device data
-      const bool reporter = lane == 0 && rv0 >= s0;
-      const RowInfo ri = row_info<MODE>(a, r, reporter ? a.status : nullptr);
-      const int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
-      const int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
-      for (int j = ja; j < jb; ++j, ++i) {
-        const int buf = i % NS;
-        if (i >= NS &&
-            !__all_sync(0xffffffffu,
-                        mbar_wait(&empty[buf], static_cast<uint32_t>((i / NS) - 1) & 1u))) {
-          if (lane == 0) {
-            *abort_flag = 1u;
-            flag_status(a.status, KSA_FLAG_WAIT_TIMEOUT);
+    if (MODE != kModeCp) {
+      // TMA modes, lane-parallel: lane l < NS owns stage buffer l and fills the
+      // CTA's stages l, l + NS, l + 2 NS, ...  Each lane runs its own chain
+      // (wait for the buffer, read the block index, arm the barrier, issue the
+      // boxes), so up to NS such chains are in flight at once.
+      if (lane < NS) {
+        const int seg = (MODE == kModeDense || tpi >= kStageTok) ? kStageTok : tpi;
+        const int nseg = kStageTok / seg;                        // 1 or 2 segments
+        const int spe = tpi >= kStageTok ? tpi / kStageTok : 1;  // stages per entry
+        int r = r_first;
+        long long rv0 = static_cast<long long>(r) * p.V;
+        RowInfo ri = row_info<MODE>(a, r, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
+        int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
+        int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
+        int cnt = jb > ja ? jb - ja : 0;
+        int row_base = 0;  // CTA ordinal of the row's first stage
+        for (int i = lane;; i += NS) {
+          while (i >= row_base + cnt && r <= r_last) {
+            row_base += cnt;
+            if (++r > r_last) break;
+            rv0 = static_cast<long long>(r) * p.V;
+            ri = row_info<MODE>(a, r, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
+            ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
+            jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
+            cnt = jb > ja ? jb - ja : 0;
           }
-          stop = true;
-          break;
-        }
-        issued = i + 1;
-        uint8_t *sK = stages + static_cast<size_t>(buf) * C::kStageBytes;
-        uint8_t *sV = sK + C::kTileBytes;
-        if (MODE != kModeCp) {
-          const StageSpan sp = stage_segment(MODE, j, lane, tpi, ri);
-          const int seg = (MODE == kModeDense || tpi >= kStageTok) ? kStageTok : tpi;
-          if (sp.entry && sp.nvalid == 0 && (MODE == kModeDense || sp.t0 % tpi == 0))
-            skipped = KSA_FLAG_INDEX_SKIPPED;
-          uint32_t bits = 0u;
-          if (sp.nvalid > 0)
-            bits = (sp.nvalid >= 32 ? 0xffffffffu : ((1u << sp.nvalid) - 1u)) << (lane * seg);
-          const uint32_t mask = __reduce_or_sync(0xffffffffu, bits);
-          const uint32_t issuing = __ballot_sync(0xffffffffu, sp.nvalid > 0);
-          const uint32_t bytes =
-              static_cast<uint32_t>(__popc(issuing)) * seg * 128u * C::kHalves * 2u;
-          if (lane == 0) {
-            stage_mask[buf] = mask;
-            mbar_arrive_expect_tx(&full[buf], bytes);
-          }
-          __syncwarp();
-          if (sp.nvalid > 0) {
-            const int yrow = static_cast<int>(static_cast<long long>(r) * a.T + sp.t0);
+          if (r > r_last) break;
+          const int j = ja + (i - row_base);
+          long long t0[kTiles];
+          int nv[kTiles];
+          uint32_t mask = 0u, bytes = 0u;
 #pragma unroll
-            for (int h = 0; h < C::kHalves; ++h) {
-              tma_load_2d(sK + h * C::kHalfBytes + lane * seg * 128, &kmap, h * 64, yrow,
-                          &full[buf]);
-              tma_load_2d(sV + h * C::kHalfBytes + lane * seg * 128, &vmap, h * 64, yrow,
-                          &full[buf]);
+          for (int u = 0; u < kTiles; ++u) {  // nseg <= kTiles segments
+            nv[u] = 0;
+            t0[u] = 0;
+            if (u >= nseg) continue;
+            bool ok = true;
+            if (MODE == kModeDense) {
+              t0[u] = static_cast<long long>(j) * kStageTok;
+            } else {
+              const int e = (tpi >= kStageTok) ? j / spe : j * nseg + u;
+              const int part = (tpi >= kStageTok) ? j % spe : 0;
+              const int id = e < ri.n_idx ? __ldg(ri.list + e) : -1;
+              ok = e < ri.n_idx && id >= 0;
+              t0[u] = static_cast<long long>(id) * tpi + static_cast<long long>(part) * kStageTok;
+              if (e < ri.n_idx && (id < 0 || (part == 0 && t0[u] >= ri.L)))
+                skipped = KSA_FLAG_INDEX_SKIPPED;
+            }
+            const long long left = ri.L - t0[u];
+            nv[u] = (!ok || left <= 0) ? 0 : (left < seg ? static_cast<int>(left) : seg);
+            if (nv[u] > 0) {
+              mask |= (nv[u] >= 32 ? 0xffffffffu : ((1u << nv[u]) - 1u)) << (u * seg);
+              bytes += static_cast<uint32_t>(seg) * 128u * C::kHalves * 2u;
             }
           }
-        } else {
-          // token lists: stage row u <- entry j*32/tpi + u/tpi, token offset u%tpi
-          const int per = kStageTok / tpi;
-          const int e = j * per + lane / tpi;
+          if (issued > 0 &&
+              !mbar_wait(&empty[lane], static_cast<uint32_t>(issued - 1) & 1u)) {
+            *abort_flag = 1u;
+            flag_status(a.status, KSA_FLAG_WAIT_TIMEOUT);
+            break;
+          }
+          ++issued;  // uses of this lane's buffer
+          uint8_t *sK = stages + static_cast<size_t>(lane) * C::kStageBytes;
+          uint8_t *sV = sK + C::kTileBytes;
+          stage_mask[lane] = mask;
+          mbar_arrive_expect_tx(&full[lane], bytes);
+#pragma unroll
+          for (int u = 0; u < kTiles; ++u) {
+            if (nv[u] <= 0) continue;
+            const int yrow = static_cast<int>(static_cast<long long>(r) * a.T + t0[u]);
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h) {
+              tma_load_2d(sK + h * C::kHalfBytes + u * seg * 128, &kmap, h * 64, yrow, &full[lane]);
+              tma_load_2d(sV + h * C::kHalfBytes + u * seg * 128, &vmap, h * 64, yrow, &full[lane]);
+            }
+          }
+        }
+      }
+    } else {
+      // token lists: the warp fills one stage at a time with 16-byte cp.async
+      // (row u of a stage <- list entry j*eps + u/tpi, token offset u%tpi); the
+      // list is read 32 entries at a time, one per lane, the next 32 in flight
+      bool stop = false;
+      int i = 0;
+      for (int r = r_first; r <= r_last && !stop; ++r) {
+        const long long rv0 = static_cast<long long>(r) * p.V;
+        const bool reporter = lane == 0 && rv0 >= s0;
+        const RowInfo ri = row_info<MODE>(a, r, reporter ? a.status : nullptr);
+        const int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
+        const int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
+        const int eps = kStageTok / tpi;  // entries per stage
+        int wbase = 0, cur = -1, nxt = -1;
+        if (ja < jb) {
+          wbase = (ja * eps) & ~31;
+          cur = (wbase + lane < ri.n_idx) ? ri.list[wbase + lane] : -1;
+          nxt = (wbase + 32 + lane < ri.n_idx) ? ri.list[wbase + 32 + lane] : -1;
+        }
+        for (int j = ja; j < jb; ++j, ++i) {
+          const int buf = i % NS;
+          if (i >= NS &&
+              !__all_sync(0xffffffffu,
+                          mbar_wait(&empty[buf], static_cast<uint32_t>((i / NS) - 1) & 1u))) {
+            if (lane == 0) {
+              *abort_flag = 1u;
+              flag_status(a.status, KSA_FLAG_WAIT_TIMEOUT);
+            }
+            stop = true;
+            break;
+          }
+          issued = i + 1;
+          uint8_t *sK = stages + static_cast<size_t>(buf) * C::kStageBytes;
+          uint8_t *sV = sK + C::kTileBytes;
+          if (j * eps >= wbase + 32) {  // stages advance by at most one window
+            wbase += 32;
+            cur = nxt;
+            nxt = (wbase + 32 + lane < ri.n_idx) ? ri.list[wbase + 32 + lane] : -1;
+          }
+          const int e = j * eps + lane / tpi;
+          const int id = __shfl_sync(0xffffffffu, cur, (e - wbase) & 31);
           bool valid = false;
           long long t = 0;
-          if (e < ri.n_idx) {
-            const int id = ri.list[e];
+          if (lane < kStageTok && e < ri.n_idx) {
             t = static_cast<long long>(id) * tpi + (lane % tpi);
             valid = id >= 0 && t < ri.L;
             if (!valid && (lane % tpi) == 0 &&
@@ -299,6 +328,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         }
       }
     }
+    __syncwarp();
     skipped = __reduce_or_sync(0xffffffffu, skipped);
     if (skipped && lane == 0) flag_status(a.status, skipped);
   } else {
@@ -354,7 +384,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         const uint32_t mask = stage_mask[buf];
         uint8_t *sK = stages + static_cast<size_t>(buf) * C::kStageBytes;
         uint8_t *sV = sK + C::kTileBytes;
-        if (mask != 0xffffffffu) {
+        if (mask != kFullMask) {
           // rows past L / skipped entries: zero V so that p = 0 meets finite values
           for (int u = 0; u < kStageTok; ++u) {
             if (!((mask >> u) & 1u) && lane < C::kHalves * 8) {
@@ -367,7 +397,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         }
         const uint32_t kbase = smem_addr(sK), vbase = smem_addr(sV);
 #pragma unroll
-        for (int tile = 0; tile < 2; ++tile) {
+        for (int tile = 0; tile < kTiles; ++tile) {
           float s[4] = {0.f, 0.f, 0.f, 0.f};
           {
             const int rr = tile * 16 + lr + ((mi & 1) << 3);
@@ -527,12 +557,16 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
   }
 
   __syncthreads();
-  if (*abort_flag != 0u && warp == kConsumers && lane == 0) {
+  if (*abort_flag != 0u && warp == kConsumers) {
     // a wait gave up: let every copy the producer issued land before the CTA
     // exits (each wait bounded again)
-    for (int buf = 0; buf < NS && buf < issued; ++buf) {
-      const int uses = (issued - 1 - buf) / NS + 1;
-      mbar_wait(&full[buf], static_cast<uint32_t>(uses - 1) & 1u);
+    if (MODE != kModeCp) {
+      if (lane < NS && issued > 0) mbar_wait(&full[lane], static_cast<uint32_t>(issued - 1) & 1u);
+    } else if (lane == 0) {
+      for (int buf = 0; buf < NS && buf < issued; ++buf) {
+        const int uses = (issued - 1 - buf) / NS + 1;
+        mbar_wait(&full[buf], static_cast<uint32_t>(uses - 1) & 1u);
+      }
     }
   }
 }
@@ -555,8 +589,8 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   if (n > p.W) n = p.W;
   if (n < 1) n = 1;
   p.N = static_cast<int>(n);
-  sparse_decode_attn_kernel<D, MODE><<<p.N, kAttnThreads, smem, stream>>>(km, vm, p);
-  return cudaGetLastError();
+  return launch_pdl(sparse_decode_attn_kernel<D, MODE>, dim3(p.N), dim3(kAttnThreads), smem,
+                    stream, km, vm, p);
 }
 
 }  // namespace

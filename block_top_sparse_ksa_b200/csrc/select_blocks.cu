@@ -5,8 +5,8 @@
 // (the source gives no formula): the dot product of the block mean with the
 // sum of the kv-group's query heads, one selection per kv-head.
 //
-// One CTA per (row b, kv-head g, chunk of up to 128 blocks).  The CTA pulls its
-// chunk of fp32 summaries (<= 64 KB, contiguous) into shared memory with one
+// One CTA per (row b, kv-head g, chunk of up to 64 blocks).  The CTA pulls its
+// chunk of fp32 summaries (<= 32 KB, contiguous) into shared memory with one
 // TMA bulk copy, so the whole chunk is in flight at once, forms the group
 // query sum meanwhile, scores the blocks (8 lanes per summary row, warp
 // shuffles) and stores order-preserving uint32 score keys in the workspace.
@@ -23,7 +23,7 @@ namespace {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSelRows = 128;  // summary rows per CTA
+constexpr int kSelRows = 64;  // summary rows per CTA (32 KB at D = 128: many CTAs resident)
 
 struct SelDev {
   SelectArgs a;
@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev
   const SelectArgs &a = p.a;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x / p.chunks, chunk = blockIdx.x % p.chunks;
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = row / a.Hkv, g = row % a.Hkv;
   const int G = a.Hq / a.Hkv;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
@@ -188,14 +190,13 @@ cudaError_t launch_select_blocks(const SelectArgs &a, void *ws, int num_sms,
     err = cudaFuncSetAttribute(select_blocks_kernel<128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    select_blocks_kernel<128><<<grid, kSelThreads, smem, stream>>>(p);
+    return launch_pdl(select_blocks_kernel<128>, dim3(grid), dim3(kSelThreads), smem, stream, p);
   } else {
     err = cudaFuncSetAttribute(select_blocks_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    select_blocks_kernel<64><<<grid, kSelThreads, smem, stream>>>(p);
+    return launch_pdl(select_blocks_kernel<64>, dim3(grid), dim3(kSelThreads), smem, stream, p);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace ksa

@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
   const int wpc = blockDim.x >> 5;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   const bool all = (a.mode == KSA_SUMMARY_ALL);
+  pdl_wait();
+  pdl_launch_dependents();
   const long long total =
       all ? static_cast<long long>(a.B) * a.Hkv * nb_max : static_cast<long long>(a.B) * a.Hkv;
   for (long long w = static_cast<long long>(blockIdx.x) * wpc + (threadIdx.x >> 5); w < total;
@@ -82,15 +84,16 @@ cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream) {
   const long long warps = (a.mode == KSA_SUMMARY_ALL)
                               ? static_cast<long long>(a.B) * a.Hkv * nb_max
                               : static_cast<long long>(a.B) * a.Hkv;
-  const int threads = 256;
-  long long blocks = (warps + 7) / 8;
-  if (blocks > 148LL * 32) blocks = 148LL * 32;
+  // last-block updates are few and latency-bound: one warp per CTA spreads them
+  // over every SM; full rebuilds stream with 8 warps per CTA
+  const int threads = (a.mode == KSA_SUMMARY_ALL) ? 256 : 32;
+  const int wpc = threads / 32;
+  long long blocks = (warps + wpc - 1) / wpc;
+  if (blocks > 148LL * 64) blocks = 148LL * 64;
   if (blocks < 1) blocks = 1;
-  if (a.D == 128)
-    block_summaries_kernel<128><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
-  else
-    block_summaries_kernel<64><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
-  return cudaGetLastError();
+  const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
+  if (a.D == 128) return launch_pdl(block_summaries_kernel<128>, grid, block, 0, stream, a);
+  return launch_pdl(block_summaries_kernel<64>, grid, block, 0, stream, a);
 }
 
 }  // namespace ksa

@@ -62,6 +62,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
   const int b = row / a.Hkv, g = row % a.Hkv;
   const int G = a.Hq / a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
   const int L = clamp_len(a.seq_lens[b], a.T,
                           (g == 0 && chunk == 0 && tid == 0) ? a.status : nullptr);
   if (L <= a.budget) return;  // every token is selected; no scores needed
@@ -88,7 +90,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
   int issued = 0;
   if (warp == 4) {
     if (lane == 0) {
-      prefetch_tensormap(&kmap);
       for (int i = 0; i < n_stage; ++i) {
         const int buf = i % NS;
         if (i >= NS && !mbar_wait(&empty[buf], static_cast<uint32_t>((i / NS) - 1) & 1u)) {
@@ -172,6 +173,8 @@ __global__ void __launch_bounds__(kPickThreads) unified_pick_kernel(const Unifie
   __shared__ uint32_t info[4];
   __shared__ uint32_t scratch[33];
   const int b = blockIdx.x / a.Hq, h = blockIdx.x % a.Hq;
+  pdl_wait();
+  pdl_launch_dependents();
   const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
   if (L <= a.budget) return;
   int32_t *votes = a.votes + static_cast<size_t>(b) * a.T;
@@ -198,6 +201,8 @@ __global__ void __launch_bounds__(kSetThreads) unified_set_kernel(const UnifiedA
   __shared__ uint32_t info[4];
   __shared__ uint32_t scratch[33];
   const int b = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
   int32_t *out = a.token_idx + static_cast<size_t>(b) * a.budget;
   if (L <= a.budget) {
@@ -231,8 +236,8 @@ cudaError_t launch_scores(const UnifiedArgs &a, cudaStream_t stream) {
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const unsigned grid = static_cast<unsigned>(a.B) * a.Hkv * n_chunks;
-  unified_scores_kernel<D><<<grid, kScoreThreads, smem, stream>>>(km, a, n_chunks);
-  return cudaGetLastError();
+  return launch_pdl(unified_scores_kernel<D>, dim3(grid), dim3(kScoreThreads), smem, stream, km,
+                    a, n_chunks);
 }
 
 }  // namespace
@@ -252,12 +257,11 @@ cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_
   err = cudaFuncSetAttribute(unified_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(pick_smem));
   if (err != cudaSuccess) return err;
-  unified_pick_kernel<<<static_cast<unsigned>(a.B) * a.Hq, kPickThreads, pick_smem, stream>>>(
-      a, in_smem);
-  err = cudaGetLastError();
+  err = launch_pdl(unified_pick_kernel, dim3(static_cast<unsigned>(a.B) * a.Hq),
+                   dim3(kPickThreads), pick_smem, stream, a, in_smem);
   if (err != cudaSuccess) return err;
-  unified_set_kernel<<<static_cast<unsigned>(a.B), kSetThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(unified_set_kernel, dim3(static_cast<unsigned>(a.B)), dim3(kSetThreads), 0,
+                    stream, a);
 }
 
 }  // namespace ksa
