@@ -103,6 +103,15 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def weak_scaling(dist: Dist, queries_per_rank: int, ms_local: float, steps: int):
+    """Whole-job throughput of K timed steps: every rank processed its own
+    batch each step; the job took the slowest rank's time.
+    Returns (queries/s over all ranks, ms per step)."""
+    ms = dist.max(ms_local)
+    total = dist.sum(float(queries_per_rank))
+    return total / (ms / 1e3 / steps), ms / steps
+
+
 # ---------------------------------------------------------------------------
 # workloads
 
@@ -326,15 +335,14 @@ def run_block(args, dist, dev, kind):
     torch.cuda.synchronize()
     clk = clocks.stop()
     dist.barrier()
-    ms_local = start.elapsed_time(end)
-    ms = dist.max(ms_local)
+    value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), args.steps)
+    ms = ms_step * args.steps
     t_sum = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     t_sel = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
     t_att = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
     lens = inp.seq_lens.cpu().tolist()
     total_b, attn_b, summ_b = algorithmic_bytes(shape, lens, kind)
     per_step_s = ms / 1e3 / args.steps
-    value = dist.sum(B) / per_step_s  # every rank processed B queries per step
     peak, peak_kind = measured_peak()
     attn_gbs = attn_b / (t_att * 1e-3) / 1e9
     res = {
@@ -419,12 +427,11 @@ def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att):
         step(i)
     end.record(stream)
     torch.cuda.synchronize()
-    ms = dist.max(start.elapsed_time(end))
-    per = ms / 1e3 / steps
+    value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), steps)
     h2d = (B * Hq * D + 2 * B * Hkv * D) * 2
     d2h = B * Hq * D * 4
-    return {"value": dist.sum(B) / per, "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
             "note": "cache append of the new token is a torch index copy"}
 
 
@@ -480,7 +487,8 @@ def run_unified(args, dist, dev):
     end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms = dist.max(start.elapsed_time(end))
+    value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), args.steps)
+    ms = ms_step * args.steps
     t_sel = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     t_att = statistics.mean(m[1].elapsed_time(m[2]) for m in marks) / len(inp.layers)
     per = ms / 1e3 / args.steps
@@ -488,7 +496,7 @@ def run_unified(args, dist, dev):
     att_b = B * Hkv * sh.token_budget * D * 2 * 2 + B * Hq * D * 6
     peak, peak_kind = measured_peak()
     return {
-        "ms_per_step": ms / args.steps, "value": dist.sum(B) / per,
+        "ms_per_step": ms_step, "value": value,
         "kernels_ms": {"unified_select": t_sel, "sparse_decode_attn_per_layer": t_att},
         "roofline": {"bound": "hbm", "achieved": att_b / (t_att * 1e-3) / 1e9, "peak": peak,
                      "unit": "GB/s", "frac": att_b / (t_att * 1e-3) / 1e9 / peak,
