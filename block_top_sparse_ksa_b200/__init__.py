@@ -23,6 +23,7 @@ __all__ = [
     "KsaError", "Shape", "lib", "library_path", "ksa_build_block_summaries",
     "ksa_select_blocks", "ksa_sparse_decode_attn", "ksa_unified_select",
     "ksa_select_blocks_workspace", "ksa_sparse_decode_attn_workspace",
+    "ksa_sparse_decode_attn_noalloc",
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "OUT_F32", "OUT_BF16", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -61,6 +62,9 @@ _SIGS = {
     "ksa_sparse_decode_attn_workspace": (_sz, [ctypes.POINTER(Shape), _i32, _i32]),
     "ksa_sparse_decode_attn": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                       _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "ksa_sparse_decode_attn_noalloc": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                              _vp, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp,
+                                              _vp]),
     "ksa_unified_select_workspace": (_sz, [ctypes.POINTER(Shape), _i32, _i32]),
     "ksa_unified_select": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _i32, _i32, _vp,
                                   _vp, _vp, _sz, _vp, _vp]),
@@ -230,6 +234,43 @@ def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         int(cap), int(tokens_per_idx), int(bool(idx_shared)), float(scale), int(out_dtype),
         _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status),
         _stream(stream)))
+    return out, lse
+
+
+def ksa_sparse_decode_attn_noalloc(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                                   seq_lens: torch.Tensor, idx: Optional[torch.Tensor] = None,
+                                   num_idx: Optional[torch.Tensor] = None,
+                                   tokens_per_idx: int = 1, idx_shared: bool = False,
+                                   scale: float = 0.0, out_dtype: int = OUT_F32,
+                                   out: Optional[torch.Tensor] = None,
+                                   lse: Optional[torch.Tensor] = None,
+                                   dev_status: Optional[torch.Tensor] = None, stream=None):
+    """ksa_sparse_decode_attn on the library's fixed scratch (no workspace argument).
+
+    For callers that must not allocate device memory; see include/ksa.h.  Calls
+    that may overlap on the GPU share the scratch and race."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(V, "V", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    cap = 0
+    if idx is not None:
+        _dev(idx, "idx", torch.int32)
+        _dev(num_idx, "num_idx", torch.int32)
+        cap = idx.shape[-1]
+    odt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=odt, device=q.device)
+    _dev(out, "out", odt)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32)
+    sh = _shape(B, Hq, Hkv, D, T, max(1, tokens_per_idx))
+    _check(lib().ksa_sparse_decode_attn_noalloc(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx), _ptr(num_idx),
+        int(cap), int(tokens_per_idx), int(bool(idx_shared)), float(scale), int(out_dtype),
+        _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
     return out, lse
 
 

@@ -91,6 +91,16 @@ EncodeTiledFn encode_fn() {
 
 namespace ksa {
 
+ksa_status set_last_error(ksa_status status, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
 bool encode_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int D,
                           int box_rows) {
   EncodeTiledFn fn = encode_fn();

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/ksa.h"
+
 namespace ksa {
 
 struct SummaryArgs {
@@ -64,6 +66,10 @@ struct UnifiedArgs {
 };
 size_t unified_workspace_bytes(int B, int Hq, int T);
 cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream);
+
+// Records a message for ksa_last_error() and returns `status`.
+ksa_status set_last_error(ksa_status status, const char *fmt, ...)
+    __attribute__((format(printf, 2, 3)));
 
 // TMA descriptor for a [rows, D] bf16 matrix, 128B swizzle, box = 64 x box_rows.
 bool encode_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int D,

@@ -149,6 +149,33 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q,
                                   uint32_t *dev_status, void *stream);
 
 /*
+ * ksa_sparse_decode_attn without a workspace argument: the same computation,
+ * arguments and results, for callers that must not allocate device memory
+ * (a serving loop that allows no new device memory after start-up, code
+ * recorded into a CUDA graph while capture is active, or a layer handed only
+ * its input and output buffers).  The sources describe no such entry point;
+ * it is an integration convenience with no counterpart in the method.
+ * The library keeps one fixed 8 MiB scratch area per GPU (held from the first
+ * call on that GPU, or from library load when CUDA loads modules eagerly,
+ * until the process exits) and uses it in place of the workspace.  Shapes whose
+ * ksa_sparse_decode_attn_workspace() exceeds 8 MiB return KSA_ERR_UNSUPPORTED
+ * with a message.  It allocates nothing: it clears the scratch's semaphores
+ * with cudaMemsetAsync on `stream` and launches the attention kernel.
+ * The first call on a device looks up the scratch's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call shares the one scratch area, so calls that may overlap on the
+ * GPU (different streams, or different host threads) race: issue them one
+ * after another on one stream.
+ */
+ksa_status ksa_sparse_decode_attn_noalloc(const ksa_shape *shape, const uint16_t *q,
+                                          const uint16_t *K, const uint16_t *V,
+                                          const int32_t *seq_lens, const int32_t *idx,
+                                          const int32_t *num_idx, int32_t idx_capacity,
+                                          int32_t tokens_per_idx, int32_t idx_shared,
+                                          float scale, int32_t out_dtype, void *out,
+                                          float *lse, uint32_t *dev_status, void *stream);
+
+/*
  * LessIsMore unified selection [LIM s.2, s.5 "token selection layer"].
  * For each row b with L = L_b:
  *   1. every query head h scores every token t < L: s_h[t] = <q[b,h], K[b,g(h),t]>
