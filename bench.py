@@ -2,9 +2,9 @@
 """Throughput of block top-k sparse decode attention on B200.
 
 One step = one decode step of one attention layer for a whole batch:
-  block-summary maintenance (last block) -> block scoring + top-k selection
-  -> gathered split-KV attention over the selected blocks,
-all three in libksa's CUDA kernels.  Metric: queries/s, one query = one
+  block-summary maintenance (last block) + block scoring + top-k selection
+  (one fused kernel) -> gathered split-KV attention over the selected blocks,
+all in libksa's CUDA kernels.  Metric: queries/s, one query = one
 sequence's decode step for one layer (all query heads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ksa|reference]
@@ -286,14 +286,12 @@ def run_block(args, dist, dev, kind):
             ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, workspace=ws_att,
                                        stream=stream)
             return
-        ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, ksa.SUMMARY_LAST_BLOCK,
-                                      summaries=S, stream=stream)
-        ksa.ksa_select_blocks(q, S, inp.seq_lens, bs, T, k, block_idx=idx, num_sel=cnt,
-                              workspace=ws_sel, stream=stream)
+        ksa.ksa_decode_select_blocks(q, inp.K, S, inp.seq_lens, bs, k, block_idx=idx,
+                                     num_sel=cnt, workspace=ws_sel, stream=stream)
         ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt, tokens_per_idx=bs,
                                    out=out, workspace=ws_att, stream=stream)
 
-    launches_per_step = 1 if kind == "dense" else 3
+    launches_per_step = 1 if kind == "dense" else 2
     for i in range(args.warmup):
         step(i)
     # per-kernel events on a sample of the timed steps
@@ -318,11 +316,9 @@ def run_block(args, dist, dev, kind):
                 ev[1].record(stream)
                 ev[2].record(stream)
             else:
-                ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, ksa.SUMMARY_LAST_BLOCK,
-                                              summaries=S, stream=stream)
                 ev[1].record(stream)
-                ksa.ksa_select_blocks(q, S, inp.seq_lens, bs, T, k, block_idx=idx, num_sel=cnt,
-                                      workspace=ws_sel, stream=stream)
+                ksa.ksa_decode_select_blocks(q, inp.K, S, inp.seq_lens, bs, k, block_idx=idx,
+                                             num_sel=cnt, workspace=ws_sel, stream=stream)
                 ev[2].record(stream)
                 ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt,
                                            tokens_per_idx=bs, out=out, workspace=ws_att,
@@ -337,7 +333,6 @@ def run_block(args, dist, dev, kind):
     dist.barrier()
     value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), args.steps)
     ms = ms_step * args.steps
-    t_sum = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     t_sel = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
     t_att = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
     lens = inp.seq_lens.cpu().tolist()
@@ -348,8 +343,7 @@ def run_block(args, dist, dev, kind):
     res = {
         "ms_per_step": ms / args.steps,
         "value": value,
-        "kernels_ms": {"summaries_last_block": t_sum, "select_blocks": t_sel,
-                       "sparse_decode_attn": t_att},
+        "kernels_ms": {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att},
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                      "frac": attn_gbs / peak,
                      "traffic": stored_traffic("sparse_decode_attn", args.workload),
@@ -367,7 +361,8 @@ def run_block(args, dist, dev, kind):
                    "l2": "inputs larger than L2: K/V cache %.1f GB, %.0f MB read per step, %d "
                          "rotating query sets" % (2 * inp.K.numel() * 2 / 1e9, total_b / 1e6, nq),
                    "step": ("dense attention" if kind == "dense" else
-                            "summaries(last block) + select_blocks + sparse_decode_attn")},
+                            "decode_select_blocks (last-block summary refresh + scoring + "
+                            "top-k) + sparse_decode_attn")},
     }
     if not args.no_e2e:
         res["e2e"] = run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att)
@@ -407,10 +402,8 @@ def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att):
             ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, out=out, workspace=ws_att,
                                        stream=stream)
         else:
-            ksa.ksa_build_block_summaries(inp.K, lens, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S,
-                                          stream=stream)
-            ksa.ksa_select_blocks(d_q, S, lens, bs, T, k, block_idx=idx, num_sel=cnt,
-                                  workspace=ws_sel, stream=stream)
+            ksa.ksa_decode_select_blocks(d_q, inp.K, S, lens, bs, k, block_idx=idx,
+                                         num_sel=cnt, workspace=ws_sel, stream=stream)
             ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, idx, cnt, tokens_per_idx=bs,
                                        out=out, workspace=ws_att, stream=stream)
         h_out.copy_(out, non_blocking=True)

@@ -23,7 +23,7 @@ __all__ = [
     "KsaError", "Shape", "lib", "library_path", "ksa_build_block_summaries",
     "ksa_select_blocks", "ksa_sparse_decode_attn", "ksa_unified_select",
     "ksa_select_blocks_workspace", "ksa_sparse_decode_attn_workspace",
-    "ksa_sparse_decode_attn_noalloc",
+    "ksa_sparse_decode_attn_noalloc", "ksa_decode_select_blocks",
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "OUT_F32", "OUT_BF16", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -59,6 +59,8 @@ _SIGS = {
     "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]),
+    "ksa_decode_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _i32, _vp,
+                                        _vp, _vp, _sz, _vp, _vp]),
     "ksa_sparse_decode_attn_workspace": (_sz, [ctypes.POINTER(Shape), _i32, _i32]),
     "ksa_sparse_decode_attn": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                       _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -197,6 +199,33 @@ def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.
                                    int(k_blocks), _ptr(block_idx), _ptr(num_sel), _ptr(ws),
                                    ws.numel() * ws.element_size(), _ptr(dev_status),
                                    _stream(stream)))
+    return block_idx, num_sel
+
+
+def ksa_decode_select_blocks(q: torch.Tensor, K: torch.Tensor, summaries: torch.Tensor,
+                             seq_lens: torch.Tensor, block_size: int, k_blocks: int,
+                             block_idx: Optional[torch.Tensor] = None,
+                             num_sel: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None,
+                             dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Refresh every row's last-block summary from K, then select (one launch)."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(summaries, "summaries", torch.float32)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    if block_idx is None:
+        block_idx = torch.empty((B, Hkv, k_blocks), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    sh = _shape(B, Hq, Hkv, D, T, block_size)
+    ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
+                    q.device)
+    _check(lib().ksa_decode_select_blocks(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(summaries), _ptr(seq_lens), int(k_blocks),
+        _ptr(block_idx), _ptr(num_sel), _ptr(ws), ws.numel() * ws.element_size(),
+        _ptr(dev_status), _stream(stream)))
     return block_idx, num_sel
 
 

@@ -175,7 +175,7 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const fl
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   ksa::SelectArgs a;
   a.q = q;
-  a.S = summaries;
+  a.S = const_cast<float *>(summaries);  // read only: no K is given, so nothing is refreshed
   a.seq_lens = seq_lens;
   a.block_idx = block_idx;
   a.num_sel = num_sel;
@@ -188,8 +188,51 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const fl
   a.bs = shape->block_size;
   a.k = k_blocks;
   return cuda_status(
-      ksa::launch_select_blocks(a, ws, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      ksa::launch_select_blocks(a, nullptr, ws, device_sm_count(),
+                                static_cast<cudaStream_t>(stream)),
       "ksa_select_blocks launch");
+}
+
+ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                                    float *summaries, const int32_t *seq_lens, int32_t k_blocks,
+                                    int32_t *block_idx, int32_t *num_sel, void *ws,
+                                    size_t ws_bytes, uint32_t *dev_status, void *stream) {
+  if (K == nullptr) return fail(KSA_ERR_INVALID_ARG, "K must be non-NULL");
+  if (!aligned(K, 16)) return fail(KSA_ERR_INVALID_ARG, "K must be 16-byte aligned");
+  // same validation as the selection alone
+  ksa_status st = check_shape(shape, true);
+  if (st != KSA_OK) return st;
+  if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
+      num_sel == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "q, summaries, seq_lens, block_idx, num_sel must be non-NULL");
+  if (k_blocks < 1) return fail(KSA_ERR_INVALID_ARG, "k_blocks must be >= 1 (got %d)", k_blocks);
+  const int nb_max = (shape->capacity + shape->block_size - 1) / shape->block_size;
+  if (nb_max > 16384)
+    return fail(KSA_ERR_UNSUPPORTED, "ceil(capacity/block_size) = %d exceeds 16384", nb_max);
+  if (!aligned(summaries, 16) || !aligned(q, 4))
+    return fail(KSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
+  const size_t need = ksa::select_workspace_bytes(shape->batch, shape->num_kv_heads,
+                                                  shape->capacity, shape->block_size);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  ksa::SelectArgs a;
+  a.q = q;
+  a.S = summaries;
+  a.seq_lens = seq_lens;
+  a.block_idx = block_idx;
+  a.num_sel = num_sel;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hq = shape->num_q_heads;
+  a.Hkv = shape->num_kv_heads;
+  a.D = shape->head_dim;
+  a.T = shape->capacity;
+  a.bs = shape->block_size;
+  a.k = k_blocks;
+  return cuda_status(ksa::launch_select_blocks(a, K, ws, device_sm_count(),
+                                               static_cast<cudaStream_t>(stream)),
+                     "ksa_decode_select_blocks launch");
 }
 
 size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape, int32_t idx_capacity,

@@ -233,6 +233,47 @@ __device__ __forceinline__ uint32_t swz128(int r, int c) {
 }
 
 // ---------------------------------------------------------------------------
+// block mean (the block summary of the method), one warp per block
+
+// Mean of the n consecutive bf16 key rows starting at `rows` (row stride D),
+// computed by one warp: lane l sums 16-byte chunk l % (D/8) of rows l / (D/8),
+// l / (D/8) + 32 / (D/8), ... in row order (every row of the block is one
+// in-flight load), partial sums meet by xor-shuffles, then one IEEE division.
+// Lanes l < D/8 receive dims [8 (l % (D/8)), +8) in mean[] and return true.
+// All 32 lanes must call it with the same arguments.
+template <int D>
+__device__ __forceinline__ bool warp_block_mean(const uint16_t *rows, int n, float (&mean)[8]) {
+  constexpr int CH = D / 8;    // 16-byte chunks per key row
+  constexpr int RP = 32 / CH;  // rows covered by one warp-wide load
+  const int lane = threadIdx.x & 31;
+  const int c = lane % CH, rp = lane / CH;
+  const uint16_t *src = rows + c * 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mean[i] = 0.f;
+#pragma unroll 8
+  for (int t = rp; t < n; t += RP) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + static_cast<size_t>(t) * D));
+    mean[0] += bf16_lo(x.x);
+    mean[1] += bf16_hi(x.x);
+    mean[2] += bf16_lo(x.y);
+    mean[3] += bf16_hi(x.y);
+    mean[4] += bf16_lo(x.z);
+    mean[5] += bf16_hi(x.z);
+    mean[6] += bf16_lo(x.w);
+    mean[7] += bf16_hi(x.w);
+  }
+#pragma unroll
+  for (int off = CH; off < 32; off <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mean[i] += __shfl_xor_sync(0xffffffffu, mean[i], off);
+  }
+  const float fn = static_cast<float>(n);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mean[i] = mean[i] / fn;
+  return rp == 0;
+}
+
+// ---------------------------------------------------------------------------
 // block-wide helpers
 
 // Exclusive prefix count of `flag` over the block (thread order) plus the total.

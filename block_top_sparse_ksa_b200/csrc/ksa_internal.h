@@ -23,7 +23,7 @@ cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream);
 
 struct SelectArgs {
   const uint16_t *q;
-  const float *S;
+  float *S;  // read; written only by the fused last-block refresh
   const int32_t *seq_lens;
   int32_t *block_idx;
   int32_t *num_sel;
@@ -32,7 +32,9 @@ struct SelectArgs {
 };
 // workspace: semaphores [B*Hkv] (zero between calls) + score keys [B*Hkv, ceil(T/bs)]
 size_t select_workspace_bytes(int B, int Hkv, int T, int bs);
-cudaError_t launch_select_blocks(const SelectArgs &a, void *ws, int num_sms, cudaStream_t stream);
+// K non-null: first refresh each row's last-block summary from K (fused maintenance).
+cudaError_t launch_select_blocks(const SelectArgs &a, const uint16_t *K, void *ws, int num_sms,
+                                 cudaStream_t stream);
 
 struct AttnArgs {
   const uint16_t *q, *K, *V;

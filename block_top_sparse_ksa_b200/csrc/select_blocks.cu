@@ -14,6 +14,11 @@
 // stages the row's keys in shared memory and runs an exact radix select
 // (k-th largest key; ties at the threshold go to the lower block index),
 // writes the winners in ascending block order, and resets the semaphore.
+//
+// With a key cache given (the fused decode-step entry point), the CTA whose
+// chunk holds a row's last block first recomputes that block's mean from the
+// keys -- the per-step maintenance of the block representation -- while its
+// chunk is in flight, stores it in the summaries and scores the fresh value.
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
 
@@ -27,6 +32,7 @@ constexpr int kSelRows = 64;  // summary rows per CTA (32 KB at D = 128: many CT
 
 struct SelDev {
   SelectArgs a;
+  const uint16_t *K;  // non-null: refresh each row's last-block summary from K first
   int chunks;      // CTAs per (row, kv-head)
   uint32_t *keys;  // workspace [B*Hkv, nb_max]
   int32_t *sem;    // workspace [B*Hkv], zero between calls
@@ -47,6 +53,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev
   float *sbuf = reinterpret_cast<float *>(smem_raw);  // chunk summaries, later the row's keys
   __shared__ uint64_t bar;
   __shared__ __align__(16) float qsum[D];
+  __shared__ __align__(16) float fresh[D];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t info[4];
   __shared__ uint32_t scratch[33];
@@ -70,6 +77,18 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev
     if (chunk == 0) {
       for (int i = tid; i < k; i += kSelThreads) out[i] = i < nb ? i : -1;
       if (tid == 0) a.num_sel[row] = nb;
+      if (p.K != nullptr && nb > 0 && warp == 0) {
+        // fused maintenance still keeps the last block's mean current
+        float mean[8];
+        const int jl = nb - 1;
+        const uint16_t *rows =
+            p.K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
+        if (warp_block_mean<D>(rows, L - jl * a.bs, mean)) {
+          float *dst = a.S + (static_cast<size_t>(row) * nb_max + jl) * D + (lane % (D / 8)) * 8;
+          reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+          reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+        }
+      }
     }
     return;
   }
@@ -94,6 +113,22 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev
     for (int h = 0; h < G; ++h) s += bf16_bits_to_f32(qp[static_cast<size_t>(h) * D]);
     qsum[d] = s;
   }
+  // fused maintenance: the chunk holding the row's last block refreshes its mean
+  const bool refresh = p.K != nullptr && n > 0 && j1 == nb;
+  if (refresh && warp == 0) {
+    float mean[8];
+    const int jl = nb - 1;
+    const uint16_t *rows =
+        p.K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
+    if (warp_block_mean<D>(rows, L - jl * a.bs, mean)) {
+      const int c8 = (lane % (D / 8)) * 8;
+      float *dst = a.S + (static_cast<size_t>(row) * nb_max + jl) * D + c8;
+      reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+      reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) fresh[c8 + i] = mean[i];
+    }
+  }
   __syncthreads();
 
   uint32_t bad = 0u;
@@ -101,6 +136,10 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev
     bad |= KSA_FLAG_WAIT_TIMEOUT;
     timed_out = 1;
   }
+  if (refresh && bad == 0u) {  // after the copy landed: overwrite the stale summary
+    for (int d = tid; d < D; d += kSelThreads) sbuf[static_cast<size_t>(n - 1) * D + d] = fresh[d];
+  }
+  __syncthreads();
   if (n > 0 && bad == 0u) {
     constexpr int PER = D / 32;  // float4 chunks per lane: chunk (sub + 8*i) of the row
     const int sub = lane & 7;
@@ -170,12 +209,13 @@ size_t select_workspace_bytes(int B, int Hkv, int T, int bs) {
   return sems + keys;
 }
 
-cudaError_t launch_select_blocks(const SelectArgs &a, void *ws, int num_sms,
+cudaError_t launch_select_blocks(const SelectArgs &a, const uint16_t *K, void *ws, int num_sms,
                                  cudaStream_t stream) {
   (void)num_sms;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   SelDev p;
   p.a = a;
+  p.K = K;
   p.chunks = (nb_max + kSelRows - 1) / kSelRows;
   const size_t rows = static_cast<size_t>(a.B) * a.Hkv;
   const size_t sems = (rows * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);

@@ -18,10 +18,7 @@ namespace {
 
 template <int D>
 __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
-  constexpr int CH = D / 8;     // 16-byte chunks per key row
-  constexpr int RP = 32 / CH;   // rows covered by one warp-wide load
   const int lane = threadIdx.x & 31;
-  const int c = lane % CH, rp = lane / CH;
   const int wpc = blockDim.x >> 5;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   const bool all = (a.mode == KSA_SUMMARY_ALL);
@@ -44,35 +41,13 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
       j = nb - 1;
     }
     const int n = min(a.bs, L - j * a.bs);
-    const uint16_t *src =
-        a.K + (static_cast<size_t>(bg) * a.T + static_cast<size_t>(j) * a.bs) * D + c * 8;
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 8
-    for (int t = rp; t < n; t += RP) {
-      const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + static_cast<size_t>(t) * D));
-      acc[0] += bf16_lo(x.x);
-      acc[1] += bf16_hi(x.x);
-      acc[2] += bf16_lo(x.y);
-      acc[3] += bf16_hi(x.y);
-      acc[4] += bf16_lo(x.z);
-      acc[5] += bf16_hi(x.z);
-      acc[6] += bf16_lo(x.w);
-      acc[7] += bf16_hi(x.w);
-    }
-#pragma unroll
-    for (int off = CH; off < 32; off <<= 1) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-    }
-    if (rp == 0) {
-      const float fn = static_cast<float>(n);
-      float *dst = a.S + (static_cast<size_t>(bg) * nb_max + j) * D + c * 8;
-      reinterpret_cast<float4 *>(dst)[0] =
-          make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
-      reinterpret_cast<float4 *>(dst)[1] =
-          make_float4(acc[4] / fn, acc[5] / fn, acc[6] / fn, acc[7] / fn);
+    float mean[8];
+    const uint16_t *rows =
+        a.K + (static_cast<size_t>(bg) * a.T + static_cast<size_t>(j) * a.bs) * D;
+    if (warp_block_mean<D>(rows, n, mean)) {
+      float *dst = a.S + (static_cast<size_t>(bg) * nb_max + j) * D + (lane % (D / 8)) * 8;
+      reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+      reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
     }
   }
 }

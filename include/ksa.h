@@ -115,6 +115,21 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q,
                              uint32_t *dev_status, void *stream);
 
 /*
+ * One decode step's selection in a single launch [KIN s.5]: for every row b
+ * and kv-head g, first recompute the mean of the last block j = NB_b - 1 from
+ * K and store it in `summaries` (what ksa_build_block_summaries does with
+ * KSA_SUMMARY_LAST_BLOCK, bit for bit), then score and select exactly as
+ * ksa_select_blocks.  Use after appending the step's token to K.
+ * Arguments as ksa_select_blocks, plus K [B, Hkv, T, D] bf16 (read);
+ * `summaries` is read and its last-block entries are written.
+ */
+ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q,
+                                    const uint16_t *K, float *summaries,
+                                    const int32_t *seq_lens, int32_t k_blocks,
+                                    int32_t *block_idx, int32_t *num_sel, void *ws,
+                                    size_t ws_bytes, uint32_t *dev_status, void *stream);
+
+/*
  * Sparse decode attention over a selected token set [KIN s.5; LIM s.5
  * "sparse attention layer", GQA kernel sharing one KV set per group].
  * For query head h of row b (kv-head g = h / G) and selected tokens T_sel:

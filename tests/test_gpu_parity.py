@@ -418,3 +418,58 @@ def test_long_pipelines(ksa, oracle, mode):
         idx = np.sort(rng.choice(lens[0], size=8192, replace=False))[None].astype(np.int32)
         cnt = np.array([8192], np.int32)
         assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, 1, shared=True) == 0
+
+
+@pytest.mark.parametrize("D,bs,k", [(128, 16, 8), (64, 32, 6)])
+def test_decode_select_fuses_last_block_refresh(ksa, oracle, D, bs, k):
+    """ksa_decode_select_blocks == LAST_BLOCK refresh followed by selection:
+    the same summaries bit for bit, the same blocks, and the oracle's blocks."""
+    rng = np.random.default_rng(900 + D)
+    B, Hq, Hkv = 4, 8, 2
+    T = 40 * bs + 9
+    lens = np.array([T, 3 * bs + 1, 5, 20 * bs], np.int32)  # rows 1 and 2 keep every block
+    q = rand_bits(rng, (B, Hq, D))
+    K_new = rand_bits(rng, (B, Hkv, T, D))
+    for b in range(B):
+        K_new[b], _ = gap_fix_row(oracle, q[b], K_new[b], int(lens[b]), bs, k)
+    K_old = K_new.copy()  # the cache before this step's token: the last block differs
+    for b in range(B):
+        jl = (lens[b] - 1) // bs
+        K_old[b, :, jl * bs:lens[b]] = rand_bits(rng, (Hkv, lens[b] - jl * bs, D))
+    qd, Ld = to_dev_bf16(q), torch.from_numpy(lens).to(DEV)
+    S0 = ksa.ksa_build_block_summaries(to_dev_bf16(K_old), Ld, bs)
+    Kn = to_dev_bf16(K_new)
+    S_a = S0.clone()
+    ksa.ksa_build_block_summaries(Kn, Ld, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S_a)
+    idx_a, cnt_a = ksa.ksa_select_blocks(qd, S_a, Ld, bs, T, k)
+    S_b = S0.clone()
+    st = status_tensor()
+    idx_b, cnt_b = ksa.ksa_decode_select_blocks(qd, Kn, S_b, Ld, bs, k, dev_status=st)
+    assert torch.equal(S_a, S_b)
+    assert torch.equal(idx_a, idx_b) and torch.equal(cnt_a, cnt_b)
+    ref_idx, ref_cnt = oracle.select_blocks(q, K_new, lens, bs, k)
+    assert np.array_equal(idx_b.cpu().numpy(), ref_idx)
+    assert np.array_equal(cnt_b.cpu().numpy(), ref_cnt)
+    assert st.item() == 0
+
+
+def test_select_many_rows_persistent_units(ksa, oracle):
+    """More (row, chunk) units than resident CTAs: every CTA cycles its
+    two-buffer ring several times."""
+    rng = np.random.default_rng(950)
+    B, Hq, Hkv, D, bs, k = 48, 16, 8, 128, 16, 16
+    T = 200 * bs
+    lens = rng.integers(10, T + 1, size=B).astype(np.int32)
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    for b in range(B):
+        K[b], _ = gap_fix_row(oracle, q[b], K[b], int(lens[b]), bs, k)
+    qd, Kd, Ld = to_dev_bf16(q), to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    S = ksa.ksa_build_block_summaries(Kd, Ld, bs)
+    ws = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
+                     dtype=torch.uint8, device=DEV)
+    ref_idx, ref_cnt = oracle.select_blocks(q, K, lens, bs, k)
+    for _ in range(2):  # the workspace semaphores must come back to zero
+        idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k, workspace=ws)
+        assert np.array_equal(idx.cpu().numpy(), ref_idx)
+        assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
