@@ -291,7 +291,11 @@ def run_block(args, dist, dev, kind):
         ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt, tokens_per_idx=bs,
                                    out=out, workspace=ws_att, stream=stream)
 
-    launches_per_step = 1 if kind == "dense" else 2
+    # selection: a scoring launch (when some row can hold more than k blocks)
+    # and a ranking launch; then the attention launch
+    nb_max = -(-T // bs)
+    sel_launches = 2 if nb_max > k else 1
+    launches_per_step = 1 if kind == "dense" else sel_launches + 1
     for i in range(args.warmup):
         step(i)
     # per-kernel events on a sample of the timed steps

@@ -5,20 +5,31 @@
 // (the source gives no formula): the dot product of the block mean with the
 // sum of the kv-group's query heads, one selection per kv-head.
 //
-// One CTA per (row b, kv-head g, chunk of up to 64 blocks).  The CTA pulls its
-// chunk of fp32 summaries (<= 32 KB, contiguous) into shared memory with one
-// TMA bulk copy, so the whole chunk is in flight at once, forms the group
-// query sum meanwhile, scores the blocks (8 lanes per summary row, warp
-// shuffles) and stores order-preserving uint32 score keys in the workspace.
-// The row's chunks count themselves on a semaphore; the CTA finishing last
-// stages the row's keys in shared memory and runs an exact radix select
-// (k-th largest key; ties at the threshold go to the lower block index),
-// writes the winners in ascending block order, and resets the semaphore.
+// Two launches:
+//  1. scoring, persistent.  The summaries of every (row b, kv-head g) are cut
+//     into pieces of 8 KB (2048 / D consecutive blocks, D fp32 each,
+//     contiguous); each row is padded to the same number of pieces and the
+//     grid's warps take equal contiguous slices of the flat piece sequence, so
+//     a warp streams one region front to back and forms each row's group
+//     query sum once.  A warp pulls a whole piece into registers with 16-byte
+//     loads (all in flight at once), then scores it -- 8 lanes per summary
+//     row, warp shuffles -- and stores order-preserving uint32 keys in the
+//     workspace.  No shared memory, no barriers.  Pieces of rows with at most
+//     k blocks are skipped: nothing is read.
+//  2. ranking.  Rows of up to 1024 blocks: one warp per (row, kv-head) holds
+//     the row's keys (just written, in L2) in registers and runs an exact
+//     radix select for the k-th largest key (ties at the threshold go to the
+//     lower block); ballots place the winners in ascending block order.
+//     Longer rows: one CTA per row, keys staged in shared memory, the same
+//     selection block-wide.  Rows with at most k blocks keep every block.
 //
-// With a key cache given (the fused decode-step entry point), the CTA whose
-// chunk holds a row's last block first recomputes that block's mean from the
-// keys -- the per-step maintenance of the block representation -- while its
-// chunk is in flight, stores it in the summaries and scores the fresh value.
+// With a key cache given (the fused decode-step entry point), the last block
+// of every row is first re-averaged from the keys -- the per-step maintenance
+// of the block representation: by the warp whose piece holds it, before it
+// reads the piece (so the fresh value is scored), or by the ranking warp or
+// CTA for rows whose blocks are all kept.
+#include <string.h>
+
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
 
@@ -26,217 +37,401 @@ namespace ksa {
 
 namespace {
 
-constexpr int kSelThreads = 256;
-constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSelRows = 64;  // summary rows per CTA (32 KB at D = 128: many CTAs resident)
+constexpr int kPieceBytes = 8192;  // one piece: 2048 / D summary rows
+constexpr int kScThreads = 256;
+constexpr int kRankWarpThreads = 128;
+constexpr int kRankThreads = 256;
 
-struct SelDev {
+struct ScoreDev {
   SelectArgs a;
-  const uint16_t *K;  // non-null: refresh each row's last-block summary from K first
-  int chunks;      // CTAs per (row, kv-head)
-  uint32_t *keys;  // workspace [B*Hkv, nb_max]
-  int32_t *sem;    // workspace [B*Hkv], zero between calls
+  const uint16_t *K;  // non-null: refresh the last block of each scored row from K
+  uint32_t *keys;     // workspace [B*Hkv, nb_max]
+  int prow;           // summary rows per piece
+  int pieces;         // pieces per row: ceil(nb_max / prow)
+  long long units;    // rows * pieces
+  int N;              // CTAs in the grid
 };
 
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
-                                         uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
+struct Piece {
+  int row, b, g, L, nb, j0, n;  // blocks [j0, j0 + n) of the row; n == 0: nothing to score
+};
+
+// `report`: flag an out-of-range sequence length in the status word (once per row).
+__device__ __forceinline__ Piece piece_of(const ScoreDev &p, long long u, bool report = false) {
+  Piece x;
+  x.row = static_cast<int>(u / p.pieces);
+  const int piece = static_cast<int>(u - static_cast<long long>(x.row) * p.pieces);
+  x.b = x.row / p.a.Hkv;
+  x.g = x.row - x.b * p.a.Hkv;
+  x.L = clamp_len(p.a.seq_lens[x.b], p.a.T, (report && piece == 0) ? p.a.status : nullptr);
+  x.nb = (x.L + p.a.bs - 1) / p.a.bs;
+  x.j0 = piece * p.prow;
+  x.n = (x.nb > p.a.k && x.j0 < x.nb) ? min(p.prow, x.nb - x.j0) : 0;
+  return x;
+}
+
+// Re-averages block nb-1 of `row` from K and stores it in the summaries.
+// Lanes l < D/8 get dims [8 (l % (D/8)), +8) in mean[] and return true.
+// One whole warp.
+template <int D>
+__device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const uint16_t *K,
+                                                   int row, int L, int nb, float (&mean)[8]) {
+  const int nb_max = (a.T + a.bs - 1) / a.bs;
+  const int jl = nb - 1;
+  const uint16_t *rows = K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
+  const bool mine = warp_block_mean<D>(rows, L - jl * a.bs, mean);
+  if (mine) {
+    const int c8 = ((threadIdx.x & 31) % (D / 8)) * 8;
+    float *dst = a.S + (static_cast<size_t>(row) * nb_max + jl) * D + c8;
+    reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+    reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+  }
+  return mine;
+}
+
+// Exact top-k of one row's nb (k < nb <= 32 KPL) score keys by one warp, the
+// keys held in registers: lane l holds blocks l, l + 32, l + 64, ... so that
+// (slot, lane) order is block order.  Radix select for the k-th largest key
+// tau, 8 bits a pass from the highest bit in which the row's keys differ (the
+// bits above are common to all): a 256-bin shared-memory histogram of the
+// keys that match the digits fixed so far, then the bin where the count from
+// the top reaches the number still to take.  Every key above tau is kept, and
+// of the keys equal to tau the lowest-index ones, k in all; ballots give each
+// winner its place, so out[0..k) comes out in ascending block order.
+// `hist`: 256 words of this warp's shared memory, 16-byte aligned.
+template <int KPL>
+__device__ __forceinline__ void warp_topk(const uint32_t *krow, int nb, int k, int32_t *out,
+                                          uint32_t *hist) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
+  uint32_t key[KPL];
+  uint32_t live = 0u;  // bit e: block lane + 32 e exists
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const bool ok = lane + 32 * e < nb;
+    key[e] = ok ? __ldcg(krow + lane + 32 * e) : 0u;
+    live |= ok ? (1u << e) : 0u;
+    if (ok) {
+      kmin = min(kmin, key[e]);
+      kmax = max(kmax, key[e]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  uint32_t tau = kmin;                            // every key equal: tau is that key
+  uint32_t remaining = static_cast<uint32_t>(k);  // keys still to take at or below tau
+  if (kmin != kmax) {
+    const int hb = 31 - __clz(kmin ^ kmax);  // highest bit in which keys differ
+    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);  // bits fixed so far
+    uint32_t prefix = kmin & pmask;
+    for (int shift = hb - 7;; shift -= 8) {
+      const int sh = shift > 0 ? shift : 0;
+      reinterpret_cast<uint4 *>(hist)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4 *>(hist)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) {
+        if (((live >> e) & 1u) && (key[e] & pmask) == prefix)
+          atomicAdd(&hist[(key[e] >> sh) & 255u], 1u);
+      }
+      __syncwarp();
+      // lane l owns bins [8l, 8l + 8); counts from the top bin down
+      const uint4 h0 = reinterpret_cast<const uint4 *>(hist)[2 * lane];
+      const uint4 h1 = reinterpret_cast<const uint4 *>(hist)[2 * lane + 1];
+      const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      const uint32_t tot = c[0] + c[1] + c[2] + c[3] + c[4] + c[5] + c[6] + c[7];
+      uint32_t incl = tot;  // keys in the bins of lanes >= this lane
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl += y;
+      }
+      uint32_t run = incl - tot, digit = 0u, above = 0u;
+      bool found = false;
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        const uint32_t before = run;
+        run += c[j];
+        if (before < remaining && run >= remaining) {
+          found = true;
+          digit = static_cast<uint32_t>(lane * 8 + j);
+          above = before;
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, found)) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      remaining -= above;
+      prefix = (prefix & ~(255u << sh)) | (digit << sh);
+      pmask |= 255u << sh;
+      __syncwarp();  // the bins are read before the next pass clears them
+      if (sh == 0) break;
+    }
+    tau = prefix;
+  }
+  const uint32_t take_eq = remaining;  // k minus the keys above tau
+  uint32_t base = 0u, eq_seen = 0u;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const bool ok = (live >> e) & 1u;
+    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    const bool sel = gt || (eq && eq_seen + __popc(eb & lt) < take_eq);
+    eq_seen += __popc(eb);
+    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[base + __popc(sb & lt)] = lane + 32 * e;
+    base += __popc(sb);
+  }
+}
+
+// A row with at most k blocks keeps them all (and -1 pads the list).
+template <int D>
+__device__ __forceinline__ void keep_all_blocks(const ScoreDev &p, int row, int L, int nb) {
+  const int lane = threadIdx.x & 31;
+  const SelectArgs &a = p.a;
+  int32_t *out = a.block_idx + static_cast<size_t>(row) * a.k;
+  for (int i = lane; i < a.k; i += 32) out[i] = i < nb ? i : -1;
+  if (lane == 0) a.num_sel[row] = nb;
+  if (p.K != nullptr && nb > 0) {
+    float mean[8];
+    refresh_last_block<D>(a, p.K, row, L, nb, mean);  // the step's maintenance still runs
+  }
+}
+
+// Group query sum of kv-head g of batch row b over this lane's columns
+// (float4 chunks sub + 8 j of a summary row), summed over the heads in order.
+template <int D>
+__device__ __forceinline__ void load_qsum(const SelectArgs &a, int b, int g, int sub,
+                                          float4 (&qv)[D / 32]) {
+  constexpr int PER = D / 32;
+  const int G = a.Hq / a.Hkv;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) qv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint16_t *qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * D;
+#pragma unroll 4
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const uint32_t *q2 = reinterpret_cast<const uint32_t *>(
+          qg + static_cast<size_t>(h) * D + 4 * (sub + 8 * j));
+      const uint32_t w0 = __ldg(q2), w1 = __ldg(q2 + 1);
+      qv[j].x += bf16_lo(w0);
+      qv[j].y += bf16_hi(w0);
+      qv[j].z += bf16_lo(w1);
+      qv[j].w += bf16_hi(w1);
+    }
+  }
+}
+
+// Scores piece x (x.n > 0) against the group query sum qv: the whole piece is
+// pulled into registers at once (lane (r, sub) holds chunks sub + 8 j of rows
+// 4 it + r), each summary row is reduced over its 8 lanes, and the keys are
+// stored.  With a key cache given, the piece holding the row's last block
+// first re-averages that block, so the fresh value is the one scored.
+template <int D>
+__device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
+                                            const float4 (&qv)[D / 32], uint32_t &bad) {
+  constexpr int R = kPieceBytes / (D * 4);
+  constexpr int PER = D / 32;
+  constexpr int IT = R / 4;
+  const SelectArgs &a = p.a;
+  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int nb_max = (a.T + a.bs - 1) / a.bs;
+  if (p.K != nullptr && x.j0 + x.n == x.nb) {
+    float mean[8];
+    refresh_last_block<D>(a, p.K, x.row, x.L, x.nb, mean);
+    __syncwarp();  // the fresh summary is visible to the whole warp's loads below
+  }
+  const float4 *src =
+      reinterpret_cast<const float4 *>(a.S + (static_cast<size_t>(x.row) * nb_max + x.j0) * D);
+  float4 v[IT][PER];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int jr = it * 4 + (lane >> 3);
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+      v[it][j] = jr < x.n ? __ldcg(src + jr * (D / 4) + sub + 8 * j)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  uint32_t *krow = p.keys + static_cast<size_t>(x.row) * nb_max + x.j0;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int jr = it * 4 + (lane >> 3);
+    float sc = 0.f;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      sc = fmaf(qv[j].x, v[it][j].x, sc);
+      sc = fmaf(qv[j].y, v[it][j].y, sc);
+      sc = fmaf(qv[j].z, v[it][j].z, sc);
+      sc = fmaf(qv[j].w, v[it][j].w, sc);
+    }
+    sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+    sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+    sc += __shfl_xor_sync(0xffffffffu, sc, 4);
+    if (jr < x.n && sub == 0) {
+      bool nan;
+      krow[jr] = score_key(sc, nan);
+      bad |= nan ? KSA_FLAG_NONFINITE_SCORE : 0u;
+    }
+  }
+}
+
+// Scoring.  The grid's warps take equal contiguous slices of the flat piece
+// sequence: a warp streams one region of the summaries front to back (the
+// pattern the DRAM serves best, measured against round-robin and
+// counter-driven orders) and forms each row's group query sum once.
+template <int D>
+__global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev p) {
+  constexpr int kWarps = kScThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane & 7;
+  pdl_wait();
+  pdl_launch_dependents();
+  uint32_t bad = 0u;
+  int qrow = -1;  // row whose group query sum qv holds
+  float4 qv[D / 32];
+  const long long NW = static_cast<long long>(p.N) * kWarps;
+  const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  const long long s0 = gw * p.units / NW, s1 = (gw + 1) * p.units / NW;
+  for (long long u = s0; u < s1; ++u) {  // warp-uniform control flow throughout
+    const Piece x = piece_of(p, u);
+    if (x.n == 0) continue;
+    if (x.row != qrow) {
+      qrow = x.row;
+      load_qsum<D>(p.a, x.b, x.g, sub, qv);
+    }
+    score_piece<D>(p, x, qv, bad);
+  }
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  if (bad != 0u && lane == 0) flag_status(p.a.status, bad);
+}
+
+// Ranking, one warp per (row, kv-head), for rows of at most 32 KPL blocks:
+// the row's keys (just written, in L2) go into registers and warp_topk picks
+// the k best.  Rows with at most k blocks keep every block.
+template <int D, int KPL>
+__global__ void __launch_bounds__(kRankWarpThreads) rank_rows_kernel(const ScoreDev p) {
+  constexpr int kWarps = kRankWarpThreads / 32;
+  __shared__ __align__(16) uint32_t s_hist[kWarps][256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
+  const SelectArgs &a = p.a;
+  const int row = blockIdx.x * kWarps + warp;
+  if (row >= a.B * a.Hkv) return;
+  const int nb_max = (a.T + a.bs - 1) / a.bs;
+  const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, lane == 0 ? a.status : nullptr);
+  const int nb = (L + a.bs - 1) / a.bs;
+  if (nb <= a.k) {
+    keep_all_blocks<D>(p, row, L, nb);
+    return;
+  }
+  warp_topk<KPL>(p.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
+                 a.block_idx + static_cast<size_t>(row) * a.k, s_hist[warp]);
+  if (lane == 0) a.num_sel[row] = a.k;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(const SelDev p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  float *sbuf = reinterpret_cast<float *>(smem_raw);  // chunk summaries, later the row's keys
-  __shared__ uint64_t bar;
-  __shared__ __align__(16) float qsum[D];
-  __shared__ __align__(16) float fresh[D];
+__global__ void __launch_bounds__(kRankThreads) rank_blocks_kernel(const ScoreDev p) {
+  extern __shared__ __align__(16) uint32_t kb[];  // the row's keys
   __shared__ uint32_t hist[256];
   __shared__ uint32_t info[4];
   __shared__ uint32_t scratch[33];
-  __shared__ int is_last;
-  __shared__ int timed_out;
 
   const SelectArgs &a = p.a;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = blockIdx.x / p.chunks, chunk = blockIdx.x % p.chunks;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = blockIdx.x;
   pdl_wait();
   pdl_launch_dependents();
-  const int b = row / a.Hkv, g = row % a.Hkv;
-  const int G = a.Hq / a.Hkv;
+  const int b = row / a.Hkv;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
-  const int L = clamp_len(a.seq_lens[b], a.T, (chunk == 0 && tid == 0) ? a.status : nullptr);
+  const int L = clamp_len(a.seq_lens[b], a.T, tid == 0 ? a.status : nullptr);
   const int nb = (L + a.bs - 1) / a.bs;
   const int k = a.k;
   int32_t *out = a.block_idx + static_cast<size_t>(row) * k;
 
   if (nb <= k) {  // every block is kept; no summary is read
-    if (chunk == 0) {
-      for (int i = tid; i < k; i += kSelThreads) out[i] = i < nb ? i : -1;
-      if (tid == 0) a.num_sel[row] = nb;
-      if (p.K != nullptr && nb > 0 && warp == 0) {
-        // fused maintenance still keeps the last block's mean current
-        float mean[8];
-        const int jl = nb - 1;
-        const uint16_t *rows =
-            p.K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
-        if (warp_block_mean<D>(rows, L - jl * a.bs, mean)) {
-          float *dst = a.S + (static_cast<size_t>(row) * nb_max + jl) * D + (lane % (D / 8)) * 8;
-          reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
-          reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
-        }
-      }
+    for (int i = tid; i < k; i += kRankThreads) out[i] = i < nb ? i : -1;
+    if (tid == 0) a.num_sel[row] = nb;
+    if (p.K != nullptr && nb > 0 && warp == 0) {
+      float mean[8];
+      refresh_last_block<D>(a, p.K, row, L, nb, mean);  // the step's maintenance still runs
     }
     return;
   }
-  const int j0 = static_cast<int>(static_cast<long long>(chunk) * nb / p.chunks);
-  const int j1 = static_cast<int>(static_cast<long long>(chunk + 1) * nb / p.chunks);
-  const int n = j1 - j0;
-  if (tid == 0) {
-    mbar_init(&bar, 1u);
-    timed_out = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0 && n > 0) {
-    const uint32_t bytes = static_cast<uint32_t>(n) * D * 4u;
-    mbar_arrive_expect_tx(&bar, bytes);
-    bulk_g2s(sbuf, a.S + (static_cast<size_t>(row) * nb_max + j0) * D, bytes, &bar);
-  }
-  // group query sum while the chunk is in flight
-  for (int d = tid; d < D; d += kSelThreads) {
-    const uint16_t *qp = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * D + d;
-    float s = 0.f;
-    for (int h = 0; h < G; ++h) s += bf16_bits_to_f32(qp[static_cast<size_t>(h) * D]);
-    qsum[d] = s;
-  }
-  // fused maintenance: the chunk holding the row's last block refreshes its mean
-  const bool refresh = p.K != nullptr && n > 0 && j1 == nb;
-  if (refresh && warp == 0) {
-    float mean[8];
-    const int jl = nb - 1;
-    const uint16_t *rows =
-        p.K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
-    if (warp_block_mean<D>(rows, L - jl * a.bs, mean)) {
-      const int c8 = (lane % (D / 8)) * 8;
-      float *dst = a.S + (static_cast<size_t>(row) * nb_max + jl) * D + c8;
-      reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
-      reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) fresh[c8 + i] = mean[i];
-    }
-  }
-  __syncthreads();
-
-  uint32_t bad = 0u;
-  if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar, 0u))) {
-    bad |= KSA_FLAG_WAIT_TIMEOUT;
-    timed_out = 1;
-  }
-  if (refresh && bad == 0u) {  // after the copy landed: overwrite the stale summary
-    for (int d = tid; d < D; d += kSelThreads) sbuf[static_cast<size_t>(n - 1) * D + d] = fresh[d];
-  }
-  __syncthreads();
-  if (n > 0 && bad == 0u) {
-    constexpr int PER = D / 32;  // float4 chunks per lane: chunk (sub + 8*i) of the row
-    const int sub = lane & 7;
-    float4 qv[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) qv[i] = reinterpret_cast<const float4 *>(qsum)[sub + 8 * i];
-    uint32_t *krow = p.keys + static_cast<size_t>(row) * nb_max;
-    // warp-uniform trip count: every lane reaches the full-mask shuffles
-    for (int jw = warp * 4; jw < n; jw += kSelWarps * 4) {
-      const int jr = jw + (lane >> 3);
-      const bool live = jr < n;
-      const float4 *srow = reinterpret_cast<const float4 *>(sbuf + static_cast<size_t>(jr) * D);
-      float s = 0.f;
-      if (live) {
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const float4 v = srow[sub + 8 * i];
-          s = fmaf(qv[i].x, v.x, s);
-          s = fmaf(qv[i].y, v.y, s);
-          s = fmaf(qv[i].z, v.z, s);
-          s = fmaf(qv[i].w, v.w, s);
-        }
-      }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if (live && sub == 0) {
-        bool nan;
-        krow[j0 + jr] = score_key(s, nan);
-        bad |= nan ? KSA_FLAG_NONFINITE_SCORE : 0u;
-      }
-    }
-  }
-  flag_status(a.status, bad);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(&p.sem[row], 1) == p.chunks - 1) ? 1 : 0;
-  __syncthreads();
-  if (timed_out) {  // block-uniform: read after the barrier above
-    if (tid == 0) mbar_wait(&bar, 0u);  // let the copy land before the smem is reused
-    __syncthreads();
-  }
-  if (!is_last) return;
-
-  // ---- last chunk of the row: exact top-k over the row's keys
-  __threadfence();
-  uint32_t *kb = reinterpret_cast<uint32_t *>(sbuf);
   const uint32_t *krow = p.keys + static_cast<size_t>(row) * nb_max;
-  for (int j = tid; j < nb; j += kSelThreads) kb[j] = __ldcg(krow + j);
+  for (int j = tid; j < nb; j += kRankThreads) kb[j] = krow[j];
   __syncthreads();
   uint32_t tau, n_gt, n_eq;
-  radix_select_desc<kSelThreads>(kb, nb, k, 32, hist, info, tau, n_gt, n_eq);
-  select_ascending<kSelThreads>(kb, nb, tau, n_gt, n_eq, k, out, scratch, [](int) {});
-  if (tid == 0) {
-    a.num_sel[row] = k;
-    p.sem[row] = 0;  // ready for the next call
+  radix_select_desc<kRankThreads>(kb, nb, k, 32, hist, info, tau, n_gt, n_eq);
+  select_ascending<kRankThreads>(kb, nb, tau, n_gt, n_eq, k, out, scratch, [](int) {});
+  if (tid == 0) a.num_sel[row] = k;
+}
+
+template <int D>
+cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) {
+  ScoreDev p = p0;
+  const SelectArgs &a = p.a;
+  const int nb_max = (a.T + a.bs - 1) / a.bs;
+  const int rows = a.B * a.Hkv;
+  cudaError_t err;
+  if (nb_max > a.k) {  // otherwise no row has a block to score
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_blocks_kernel<D>,
+                                                        kScThreads, 0);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    constexpr int kWarps = kScThreads / 32;
+    long long n = static_cast<long long>(num_sms) * per_sm;
+    const long long need = (p.units + kWarps - 1) / kWarps;
+    if (n > need) n = need;
+    p.N = static_cast<int>(n);
+    err = launch_pdl(score_blocks_kernel<D>, dim3(static_cast<unsigned>(p.N)), dim3(kScThreads),
+                     0, stream, p);
+    if (err != cudaSuccess) return err;
   }
+  // rows of up to 1024 blocks: one warp per row; longer rows: one CTA per row
+  constexpr int kRw = kRankWarpThreads / 32;
+  const dim3 wgrid(static_cast<unsigned>((rows + kRw - 1) / kRw)), wblock(kRankWarpThreads);
+  if (nb_max <= 128) return launch_pdl(rank_rows_kernel<D, 4>, wgrid, wblock, 0, stream, p);
+  if (nb_max <= 256) return launch_pdl(rank_rows_kernel<D, 8>, wgrid, wblock, 0, stream, p);
+  if (nb_max <= 512) return launch_pdl(rank_rows_kernel<D, 16>, wgrid, wblock, 0, stream, p);
+  if (nb_max <= 1024) return launch_pdl(rank_rows_kernel<D, 32>, wgrid, wblock, 0, stream, p);
+  const size_t rsmem = static_cast<size_t>(nb_max) * sizeof(uint32_t);
+  err = cudaFuncSetAttribute(rank_blocks_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(rsmem));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(rank_blocks_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(kRankThreads),
+                    rsmem, stream, p);
 }
 
 }  // namespace
 
+// workspace: a leading region of one word per row plus two (reserved: zero)
+// + score keys [B*Hkv, nb_max]
 size_t select_workspace_bytes(int B, int Hkv, int T, int bs) {
   const size_t rows = static_cast<size_t>(B) * Hkv;
   const size_t nb_max = static_cast<size_t>((T + bs - 1) / bs);
-  const size_t sems = (rows * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  const size_t sems = ((rows + 2) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
   const size_t keys = (rows * nb_max * sizeof(uint32_t) + 255) & ~static_cast<size_t>(255);
   return sems + keys;
 }
 
 cudaError_t launch_select_blocks(const SelectArgs &a, const uint16_t *K, void *ws, int num_sms,
                                  cudaStream_t stream) {
-  (void)num_sms;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
-  SelDev p;
+  const size_t rows = static_cast<size_t>(a.B) * a.Hkv;
+  const size_t sems = ((rows + 2) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  ScoreDev p;
+  memset(&p, 0, sizeof(p));
   p.a = a;
   p.K = K;
-  p.chunks = (nb_max + kSelRows - 1) / kSelRows;
-  const size_t rows = static_cast<size_t>(a.B) * a.Hkv;
-  const size_t sems = (rows * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
-  p.sem = static_cast<int32_t *>(ws);
   p.keys = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + sems);
-  size_t smem = static_cast<size_t>(kSelRows) * a.D * sizeof(float);
-  if (static_cast<size_t>(nb_max) * sizeof(uint32_t) > smem)
-    smem = static_cast<size_t>(nb_max) * sizeof(uint32_t);
-  const unsigned grid = static_cast<unsigned>(rows * p.chunks);
-  cudaError_t err;
-  if (a.D == 128) {
-    err = cudaFuncSetAttribute(select_blocks_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    return launch_pdl(select_blocks_kernel<128>, dim3(grid), dim3(kSelThreads), smem, stream, p);
-  } else {
-    err = cudaFuncSetAttribute(select_blocks_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    return launch_pdl(select_blocks_kernel<64>, dim3(grid), dim3(kSelThreads), smem, stream, p);
-  }
+  p.prow = kPieceBytes / (a.D * static_cast<int>(sizeof(float)));
+  p.pieces = (nb_max + p.prow - 1) / p.prow;
+  p.units = static_cast<long long>(rows) * p.pieces;
+  p.N = 1;
+  return a.D == 128 ? launch_select<128>(p, num_sms, stream) : launch_select<64>(p, num_sms, stream);
 }
 
 }  // namespace ksa

@@ -106,12 +106,15 @@ def test_select_blocks_planted_gap(ksa, oracle, D, bs, k):
     _select_case(ksa, oracle, rng, B, Hq, Hkv, D, T, bs, k, lens)
 
 
-def test_select_blocks_exact_ties(ksa, oracle):
+@pytest.mark.parametrize("nblk", [256, 700, 1100])
+def test_select_blocks_exact_ties(ksa, oracle, nblk):
     """Dyadic inputs, full blocks: every score is exact in fp32, many tie
-    exactly, and both sides must break ties toward the lower block."""
-    rng = np.random.default_rng(210)
+    exactly, and both sides must break ties toward the lower block.  Rows of
+    up to 1024 blocks are ranked inside the scoring launch, longer ones by the
+    separate ranking launch: 700 and 1100 blocks take one path each."""
+    rng = np.random.default_rng(210 + nblk)
     B, Hq, Hkv, D, bs = 2, 4, 2, 128, 16
-    T = 256 * bs
+    T = nblk * bs
     lens = np.array([T, 100 * bs], np.int32)
     q = bf16_bits(np.round(rng.standard_normal((B, Hq, D))) * 0.25)
     K = bf16_bits(np.clip(np.round(rng.standard_normal((B, Hkv, T, D)) * 0.5), -2, 2) * 0.25)
@@ -420,13 +423,14 @@ def test_long_pipelines(ksa, oracle, mode):
         assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, 1, shared=True) == 0
 
 
-@pytest.mark.parametrize("D,bs,k", [(128, 16, 8), (64, 32, 6)])
-def test_decode_select_fuses_last_block_refresh(ksa, oracle, D, bs, k):
+@pytest.mark.parametrize("D,bs,k,nblk", [(128, 16, 8, 40), (64, 32, 6, 40), (64, 16, 12, 1100)])
+def test_decode_select_fuses_last_block_refresh(ksa, oracle, D, bs, k, nblk):
     """ksa_decode_select_blocks == LAST_BLOCK refresh followed by selection:
-    the same summaries bit for bit, the same blocks, and the oracle's blocks."""
-    rng = np.random.default_rng(900 + D)
+    the same summaries bit for bit, the same blocks, and the oracle's blocks
+    (1100 blocks: rows too long to rank inside the scoring launch)."""
+    rng = np.random.default_rng(900 + D + nblk)
     B, Hq, Hkv = 4, 8, 2
-    T = 40 * bs + 9
+    T = nblk * bs + 9
     lens = np.array([T, 3 * bs + 1, 5, 20 * bs], np.int32)  # rows 1 and 2 keep every block
     q = rand_bits(rng, (B, Hq, D))
     K_new = rand_bits(rng, (B, Hkv, T, D))
@@ -454,8 +458,8 @@ def test_decode_select_fuses_last_block_refresh(ksa, oracle, D, bs, k):
 
 
 def test_select_many_rows_persistent_units(ksa, oracle):
-    """More (row, chunk) units than resident CTAs: every CTA cycles its
-    two-buffer ring several times."""
+    """Ragged rows split between scoring warps: each row is ranked by the warp
+    that completes it, and the per-row counters come back to zero."""
     rng = np.random.default_rng(950)
     B, Hq, Hkv, D, bs, k = 48, 16, 8, 128, 16, 16
     T = 200 * bs
