@@ -42,6 +42,7 @@ constexpr uint32_t kFullMask = kStageTok >= 32 ? 0xffffffffu : ((1u << kStageTok
 constexpr int kConsumers = 4;
 constexpr int kAttnThreads = (kConsumers + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMergeParts = 4;  // split-row partials combined per round of loads
 
 enum { kModeDense = 0, kModeTma = 1, kModeCp = 2 };
 
@@ -127,6 +128,75 @@ __device__ __forceinline__ void store_out(const AttnArgs &a, size_t oi, float v)
     a.out_f32[oi] = v;
   else
     a.out_bf16[oi] = f32_to_bf16_bits(v);
+}
+
+// Merges the partials (m, l, o per head) that the CTAs sharing row r left in
+// the workspace and writes the row's output and lse.  The 128 consumer
+// threads take two output elements each per round and issue every load for
+// them (up to kMergeParts partials) before combining, so a row split between a
+// few CTAs costs one round trip to L2.
+template <int D>
+__device__ __forceinline__ void merge_partials(const AttnDev &p, int r, int tid) {
+  const AttnArgs &a = p.a;
+  const int G = a.Hq / a.Hkv;
+  const int SL = p.slot;
+  const int b = r / a.Hkv, g = r % a.Hkv;
+  const long long rv0 = static_cast<long long>(r) * p.V;
+  const int c_first = cta_of(rv0, p.W, p.N);
+  const int c_last = cta_of(rv0 + p.V - 1, p.W, p.N);
+  const size_t obase = (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G);
+  constexpr int NT = kConsumers * 32;
+  for (int e0 = tid; e0 < G * D; e0 += 2 * NT) {
+    float M[2] = {-INFINITY, -INFINITY}, o[2] = {0.f, 0.f}, l[2] = {0.f, 0.f};
+    for (int cq0 = c_first; cq0 <= c_last; cq0 += kMergeParts) {
+      float mv[2][kMergeParts], lv[2][kMergeParts], ov[2][kMergeParts];
+#pragma unroll
+      for (int i = 0; i < kMergeParts; ++i) {
+        const int cq = cq0 + i;
+        const float *sl = nullptr;
+        if (cq <= c_last) {
+          const int wq = (r == static_cast<int>(cta_start(cq, p.W, p.N) / p.V)) ? 0 : 1;
+          sl = p.part + (static_cast<size_t>(cq) * 2 + wq) * SL;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int e = e0 + h * NT;
+          const bool ok = sl != nullptr && e < G * D;
+          const int hh = e / D, d = e % D;
+          mv[h][i] = ok ? __ldcg(sl + hh) : -INFINITY;
+          lv[h][i] = ok ? __ldcg(sl + G + hh) : 0.f;
+          ov[h][i] = ok ? __ldcg(sl + 2 * G + hh * D + d) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float Mn = M[h];
+#pragma unroll
+        for (int i = 0; i < kMergeParts; ++i) Mn = fmaxf(Mn, mv[h][i]);
+        const float base = (Mn == -INFINITY) ? 0.f : Mn;
+        const float sc = fast_exp2(M[h] - base);  // rescale what was summed so far
+        o[h] *= sc;
+        l[h] *= sc;
+#pragma unroll
+        for (int i = 0; i < kMergeParts; ++i) {
+          const float f = fast_exp2(mv[h][i] - base);
+          o[h] += f * ov[h][i];
+          l[h] += f * lv[h][i];
+        }
+        M[h] = Mn;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e = e0 + h * NT;
+      if (e < G * D) {
+        const int hh = e / D, d = e % D;
+        store_out(a, (obase + hh) * D + d, l[h] > 0.f ? o[h] / l[h] : 0.f);
+        if (d == 0 && a.lse != nullptr)
+          a.lse[obase + hh] = l[h] > 0.f ? (M[h] + log2f(l[h])) * kLn2 : -INFINITY;
+      }
+    }
+  }
 }
 
 template <int D, int MODE>
@@ -219,7 +289,10 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
             } else {
               const int e = (tpi >= kStageTok) ? j / spe : j * nseg + u;
               const int part = (tpi >= kStageTok) ? j % spe : 0;
-              const int id = e < ri.n_idx ? __ldg(ri.list + e) : -1;
+              // read the entry without waiting for the count (any e < cap is in
+              // bounds): one dependent round trip fewer per row
+              const int id_any = e < a.cap ? __ldg(ri.list + e) : -1;
+              const int id = e < ri.n_idx ? id_any : -1;
               ok = e < ri.n_idx && id >= 0;
               t0[u] = static_cast<long long>(id) * tpi + static_cast<long long>(part) * kStageTok;
               if (e < ri.n_idx && (id < 0 || (part == 0 && t0[u] >= ri.L)))
@@ -271,8 +344,11 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         int wbase = 0, cur = -1, nxt = -1;
         if (ja < jb) {
           wbase = (ja * eps) & ~31;
-          cur = (wbase + lane < ri.n_idx) ? ri.list[wbase + lane] : -1;
-          nxt = (wbase + 32 + lane < ri.n_idx) ? ri.list[wbase + 32 + lane] : -1;
+          // entries are read before the count is known (any index < cap is in bounds)
+          const int c0 = (wbase + lane < a.cap) ? ri.list[wbase + lane] : -1;
+          const int c1 = (wbase + 32 + lane < a.cap) ? ri.list[wbase + 32 + lane] : -1;
+          cur = (wbase + lane < ri.n_idx) ? c0 : -1;
+          nxt = (wbase + 32 + lane < ri.n_idx) ? c1 : -1;
         }
         for (int j = ja; j < jb; ++j, ++i) {
           const int buf = i % NS;
@@ -520,35 +596,16 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         }
       }
       if (!whole) {
-        __threadfence();
+        __threadfence();  // this thread's partial stores before the count
         consumer_bar();
         if (tid == 0) {
           const int old = atomicAdd(&p.sem[r], 1);
           *last_flag = (old == c_last - c_first) ? 1 : 0;
         }
         consumer_bar();
-        if (*last_flag) {
+        if (*last_flag) {  // this CTA completes the row: merge the partials
           __threadfence();
-          for (int e = tid; e < G * D; e += kConsumers * 32) {
-            const int hh = e / D, d = e % D;
-            float M = -INFINITY;
-            for (int cq = c_first; cq <= c_last; ++cq) {
-              const int wq = (r == static_cast<int>(cta_start(cq, p.W, p.N) / p.V)) ? 0 : 1;
-              M = fmaxf(M, __ldcg(p.part + (static_cast<size_t>(cq) * 2 + wq) * SL + hh));
-            }
-            const float base = (M == -INFINITY) ? 0.f : M;
-            float o = 0.f, l = 0.f;
-            for (int cq = c_first; cq <= c_last; ++cq) {
-              const int wq = (r == static_cast<int>(cta_start(cq, p.W, p.N) / p.V)) ? 0 : 1;
-              const float *sl = p.part + (static_cast<size_t>(cq) * 2 + wq) * SL;
-              const float f = fast_exp2(__ldcg(sl + hh) - base);
-              o += f * __ldcg(sl + 2 * G + hh * D + d);
-              l += f * __ldcg(sl + G + hh);
-            }
-            store_out(a, (obase + hh) * D + d, l > 0.f ? o / l : 0.f);
-            if (d == 0 && a.lse != nullptr)
-              a.lse[obase + hh] = l > 0.f ? (M + log2f(l)) * kLn2 : -INFINITY;
-          }
+          merge_partials<D>(p, r, tid);
           if (tid == 0) p.sem[r] = 0;  // ready for the next call
         }
       }
@@ -589,8 +646,10 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   if (n > p.W) n = p.W;
   if (n < 1) n = 1;
   p.N = static_cast<int>(n);
-  return launch_pdl(sparse_decode_attn_kernel<D, MODE>, dim3(p.N), dim3(kAttnThreads), smem,
-                    stream, km, vm, p);
+  // programmatic: the CTAs take their places and set up while the grid in
+  // front (normally the small ranking launch) finishes
+  return launch_programmatic(sparse_decode_attn_kernel<D, MODE>, dim3(p.N), dim3(kAttnThreads),
+                             smem, stream, km, vm, p);
 }
 
 }  // namespace
