@@ -20,8 +20,8 @@
 //     the row's keys (just written, in L2) in registers and runs an exact
 //     radix select for the k-th largest key (ties at the threshold go to the
 //     lower block); ballots place the winners in ascending block order.
-//     Longer rows: one CTA per row, keys staged in shared memory, the same
-//     selection block-wide.  Rows with at most k blocks keep every block.
+//     Longer rows: one CTA per row, keys in registers, the same selection
+//     block-wide.  Rows with at most k blocks keep every block.
 //
 // With a key cache given (the fused decode-step entry point), the last block
 // of every row is first re-averaged from the keys -- the per-step maintenance
@@ -331,40 +331,146 @@ __global__ void __launch_bounds__(kRankWarpThreads) rank_rows_kernel(const Score
   if (lane == 0) a.num_sel[row] = a.k;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRankThreads) rank_blocks_kernel(const ScoreDev p) {
-  extern __shared__ __align__(16) uint32_t kb[];  // the row's keys
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t info[4];
-  __shared__ uint32_t scratch[33];
-
-  const SelectArgs &a = p.a;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = blockIdx.x;
+// Ranking for rows of more than 1024 blocks (up to 256 KPL): one CTA of
+// kRankThreads per (row, kv-head), keys in registers (thread t holds blocks
+// t, t + NT, ... so that (slot, thread) order is block order).  The same exact
+// radix select as warp_topk, block-wide: per pass, per-warp 256-bin shared
+// histograms (fewer same-address atomics), summed by warp 0, which finds the
+// digit.  Output: per slot, ballots and one exchange of per-warp counts give
+// every winner its place, ascending.
+template <int D, int KPL>
+__global__ void __launch_bounds__(kRankThreads) rank_long_kernel(const ScoreDev p) {
+  constexpr int NT = kRankThreads, NW = NT / 32;
+  __shared__ __align__(16) uint32_t hist[NW][256];
+  __shared__ uint32_t red[2][NW];
+  __shared__ uint32_t xinfo[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
   pdl_wait();
   pdl_launch_dependents();
-  const int b = row / a.Hkv;
+  const SelectArgs &a = p.a;
+  const int row = blockIdx.x;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
-  const int L = clamp_len(a.seq_lens[b], a.T, tid == 0 ? a.status : nullptr);
+  const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, tid == 0 ? a.status : nullptr);
   const int nb = (L + a.bs - 1) / a.bs;
   const int k = a.k;
-  int32_t *out = a.block_idx + static_cast<size_t>(row) * k;
-
-  if (nb <= k) {  // every block is kept; no summary is read
-    for (int i = tid; i < k; i += kRankThreads) out[i] = i < nb ? i : -1;
-    if (tid == 0) a.num_sel[row] = nb;
-    if (p.K != nullptr && nb > 0 && warp == 0) {
-      float mean[8];
-      refresh_last_block<D>(a, p.K, row, L, nb, mean);  // the step's maintenance still runs
-    }
+  if (nb <= k) {
+    if (warp == 0) keep_all_blocks<D>(p, row, L, nb);
     return;
   }
+  int32_t *out = a.block_idx + static_cast<size_t>(row) * k;
   const uint32_t *krow = p.keys + static_cast<size_t>(row) * nb_max;
-  for (int j = tid; j < nb; j += kRankThreads) kb[j] = krow[j];
+  uint32_t key[KPL];
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = tid + NT * e;
+    key[e] = j < nb ? __ldcg(krow + j) : 0u;
+    if (j < nb) {
+      kmin = min(kmin, key[e]);
+      kmax = max(kmax, key[e]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    red[0][warp] = kmin;
+    red[1][warp] = kmax;
+  }
   __syncthreads();
-  uint32_t tau, n_gt, n_eq;
-  radix_select_desc<kRankThreads>(kb, nb, k, 32, hist, info, tau, n_gt, n_eq);
-  select_ascending<kRankThreads>(kb, nb, tau, n_gt, n_eq, k, out, scratch, [](int) {});
+  kmin = red[0][0];
+  kmax = red[1][0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    kmin = min(kmin, red[0][w]);
+    kmax = max(kmax, red[1][w]);
+  }
+  uint32_t tau = kmin;
+  uint32_t remaining = static_cast<uint32_t>(k);  // keys still to take at or below tau
+  if (kmin != kmax) {
+    const int hb = 31 - __clz(kmin ^ kmax);
+    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
+    uint32_t prefix = kmin & pmask;
+    for (int shift = hb - 7;; shift -= 8) {
+      const int sh = shift > 0 ? shift : 0;
+      for (int i = tid; i < NW * 256; i += NT) (&hist[0][0])[i] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) {
+        if (tid + NT * e < nb && (key[e] & pmask) == prefix)
+          atomicAdd(&hist[warp][(key[e] >> sh) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {  // lane l owns bins [8l, 8l + 8); counts from the top bin down
+        uint32_t c[8];
+        uint32_t tot = 0u;
+#pragma unroll
+        for (int jb = 0; jb < 8; ++jb) {
+          uint32_t v = 0u;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) v += hist[w][lane * 8 + jb];
+          c[jb] = v;
+          tot += v;
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+          if (lane + off < 32) incl += y;
+        }
+        uint32_t run = incl - tot;
+#pragma unroll
+        for (int jb = 7; jb >= 0; --jb) {
+          const uint32_t before = run;
+          run += c[jb];
+          if (before < remaining && run >= remaining) {
+            xinfo[0] = static_cast<uint32_t>(lane * 8 + jb);
+            xinfo[1] = before;
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t digit = xinfo[0];
+      remaining -= xinfo[1];
+      prefix = (prefix & ~(255u << sh)) | (digit << sh);
+      pmask |= 255u << sh;
+      __syncthreads();  // xinfo and the bins are read before the next pass
+      if (sh == 0) break;
+    }
+    tau = prefix;
+  }
+  const uint32_t take_eq = remaining;
+  uint32_t base = 0u, eq_seen = 0u;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = tid + NT * e;
+    const bool ok = j < nb;
+    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) red[0][warp] = __popc(eb);
+    __syncthreads();
+    uint32_t eq_below = 0u, eq_tot = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t v = red[0][w];
+      eq_below += w < warp ? v : 0u;
+      eq_tot += v;
+    }
+    const bool sel = gt || (eq && eq_seen + eq_below + __popc(eb & lt) < take_eq);
+    eq_seen += eq_tot;
+    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) red[1][warp] = __popc(sb);
+    __syncthreads();
+    uint32_t sel_below = 0u, sel_tot = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t v = red[1][w];
+      sel_below += w < warp ? v : 0u;
+      sel_tot += v;
+    }
+    if (sel) out[base + sel_below + __popc(sb & lt)] = j;
+    base += sel_tot;
+  }
   if (tid == 0) a.num_sel[row] = k;
 }
 
@@ -397,12 +503,12 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
   if (nb_max <= 256) return launch_pdl(rank_rows_kernel<D, 8>, wgrid, wblock, 0, stream, p);
   if (nb_max <= 512) return launch_pdl(rank_rows_kernel<D, 16>, wgrid, wblock, 0, stream, p);
   if (nb_max <= 1024) return launch_pdl(rank_rows_kernel<D, 32>, wgrid, wblock, 0, stream, p);
-  const size_t rsmem = static_cast<size_t>(nb_max) * sizeof(uint32_t);
-  err = cudaFuncSetAttribute(rank_blocks_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(rsmem));
-  if (err != cudaSuccess) return err;
-  return launch_pdl(rank_blocks_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(kRankThreads),
-                    rsmem, stream, p);
+  // longer rows (nb_max <= 16384 is checked by the API): one CTA per row
+  const dim3 rgrid(static_cast<unsigned>(rows)), rblock(kRankThreads);
+  if (nb_max <= 8 * kRankThreads) return launch_pdl(rank_long_kernel<D, 8>, rgrid, rblock, 0, stream, p);
+  if (nb_max <= 16 * kRankThreads) return launch_pdl(rank_long_kernel<D, 16>, rgrid, rblock, 0, stream, p);
+  if (nb_max <= 32 * kRankThreads) return launch_pdl(rank_long_kernel<D, 32>, rgrid, rblock, 0, stream, p);
+  return launch_pdl(rank_long_kernel<D, 64>, rgrid, rblock, 0, stream, p);
 }
 
 }  // namespace
