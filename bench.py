@@ -314,11 +314,11 @@ def run_block(args, dist, dev, kind):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             q = qs[i % nq]
             ev[0].record(stream)
-            if kind == "dense":
-                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out,
-                                           workspace=ws_att, stream=stream)
+            if kind == "dense":  # no selection: ev[1]..ev[2] is empty
                 ev[1].record(stream)
                 ev[2].record(stream)
+                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out,
+                                           workspace=ws_att, stream=stream)
             else:
                 ev[1].record(stream)
                 ksa.ksa_decode_select_blocks(q, inp.K, S, inp.seq_lens, bs, k, block_idx=idx,
@@ -347,7 +347,8 @@ def run_block(args, dist, dev, kind):
     res = {
         "ms_per_step": ms / args.steps,
         "value": value,
-        "kernels_ms": {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att},
+        "kernels_ms": ({"sparse_decode_attn": t_att} if kind == "dense" else
+                       {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att}),
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                      "frac": attn_gbs / peak,
                      "traffic": stored_traffic("sparse_decode_attn", args.workload),
@@ -355,8 +356,9 @@ def run_block(args, dist, dev, kind):
                      "bytes_per_launch": attn_b},
         "step_hbm": {"bytes_per_step": total_b, "gbs": total_b / per_step_s / 1e9,
                      "frac": total_b / per_step_s / 1e9 / peak},
-        "select_hbm": {"bytes_per_launch": summ_b,
-                       "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None},
+        "select_hbm": (None if kind == "dense" else
+                       {"bytes_per_launch": summ_b,
+                        "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None}),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "config": {"workload": shape.name, "batch_per_gpu": B, "num_q_heads": Hq,
