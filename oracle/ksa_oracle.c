@@ -30,7 +30,10 @@
  *  (R7) softmax scale defaults to 1/sqrt(D);
  *  (R8) LessIsMore voted tokens are drawn from outside the recency window, so
  *       voted + window is exactly the budget;
- *  (R9) per-head selection ranks raw q.k (softmax is monotone per head).
+ *  (R9) per-head selection ranks raw q.k (softmax is monotone per head);
+ *  (R10) bf16 block summaries are a storage format of the block mean: each
+ *        mean is replaced by the nearest bf16 value (ties to even) and the
+ *        scores read the stored values.
  *
  * Inputs: bf16 values arrive as their 16-bit patterns and are widened to fp64
  * exactly.  All arrays are dense row-major.  Threads: OpenMP over independent
@@ -106,6 +109,41 @@ void ksa_oracle_block_summaries(int B, int Hkv, int T, int D, int bs,
   }
 }
 
+/*
+ * Optional bf16 storage of the summaries (R10).  A bf16 number is a binary32
+ * whose low 16 bits are zero: sign, 8 exponent bits, 7 stored mantissa bits.
+ * In the binade [2^(e-1), 2^e) the bf16 numbers are the multiples of
+ * 2^(e-8); below 2^-126 the spacing stays 2^-133 (subnormals).  The value is
+ * scaled onto that grid (exact), rounded to the nearest integer with ties to
+ * the even one, and scaled back; results above the largest bf16 become
+ * infinity.  Returns the 16-bit pattern.
+ */
+uint16_t ksa_oracle_round_bf16(double x) {
+  if (isnan(x)) return 0x7FC0;
+  const uint16_t sign = signbit(x) ? 0x8000 : 0;
+  const double a = fabs(x);
+  if (a == 0.0) return sign;
+  if (isinf(a)) return (uint16_t)(sign | 0x7F80);
+  int e;
+  frexp(a, &e); /* a = f * 2^e with 0.5 <= f < 1 */
+  int q = e - 8;
+  if (q < -133) q = -133;
+  const double m = ldexp(a, -q); /* a in units of the grid spacing, exact */
+  double r = floor(m);
+  const double frac = m - r;
+  if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+  const double v = ldexp(r, q);
+  if (v > 3.3895313892515355e38) return (uint16_t)(sign | 0x7F80); /* above the largest bf16 */
+  const float f = (float)v; /* exact: v has at most 9 significant bits */
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  return (uint16_t)(sign | (uint16_t)(u >> 16));
+}
+
+void ksa_oracle_round_bf16_array(size_t n, const double *in, uint16_t *out) {
+  for (size_t i = 0; i < n; ++i) out[i] = ksa_oracle_round_bf16(in[i]);
+}
+
 /* ---- (A2) block scores -------------------------------------------------- */
 /*
  * Kinetics section 5: score every block against the query (R1, R2):
@@ -172,19 +210,24 @@ int ksa_oracle_topk(int n, const double *s, int k, int32_t *out) {
 
 /*
  * (A1 -> A2 -> A3) composed: block ids per (b, g), ascending, -1 padded.
+ * summary_bf16 != 0: the summaries are stored as bf16 (R10) before scoring.
  *   block_idx: [B, Hkv, k];  num_sel: [B, Hkv];
  *   scores_out (nullable): [B, Hkv, ceil(T/bs)].
  */
-void ksa_oracle_select_blocks(int B, int Hq, int Hkv, int D, int T, int bs,
-                              const uint16_t *q, const uint16_t *K,
-                              const int32_t *seq_lens, int k,
-                              int32_t *block_idx, int32_t *num_sel,
-                              double *scores_out) {
+void ksa_oracle_select_blocks_ex(int B, int Hq, int Hkv, int D, int T, int bs,
+                                 const uint16_t *q, const uint16_t *K,
+                                 const int32_t *seq_lens, int k, int summary_bf16,
+                                 int32_t *block_idx, int32_t *num_sel,
+                                 double *scores_out) {
   const int nb_max = num_blocks(T, bs);
-  double *S = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb_max * D);
+  const size_t n_sum = (size_t)B * Hkv * nb_max * D;
+  double *S = (double *)malloc(sizeof(double) * n_sum);
   double *s = scores_out ? scores_out
                          : (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb_max);
   ksa_oracle_block_summaries(B, Hkv, T, D, bs, K, seq_lens, S);
+  if (summary_bf16) {
+    for (size_t i = 0; i < n_sum; ++i) S[i] = bf16_to_f64(ksa_oracle_round_bf16(S[i]));
+  }
   ksa_oracle_block_scores(B, Hq, Hkv, D, nb_max, bs, q, S, seq_lens, s);
 #pragma omp parallel for collapse(2) schedule(dynamic)
   for (int b = 0; b < B; ++b) {
@@ -198,6 +241,15 @@ void ksa_oracle_select_blocks(int B, int Hq, int Hkv, int D, int T, int bs,
   }
   free(S);
   if (!scores_out) free(s);
+}
+
+void ksa_oracle_select_blocks(int B, int Hq, int Hkv, int D, int T, int bs,
+                              const uint16_t *q, const uint16_t *K,
+                              const int32_t *seq_lens, int k,
+                              int32_t *block_idx, int32_t *num_sel,
+                              double *scores_out) {
+  ksa_oracle_select_blocks_ex(B, Hq, Hkv, D, T, bs, q, K, seq_lens, k, 0, block_idx,
+                              num_sel, scores_out);
 }
 
 /* ---- (A4/A5/A7/A8) attention over a selected token set ------------------ */

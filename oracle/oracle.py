@@ -49,6 +49,11 @@ class Oracle:
         L.ksa_oracle_topk.restype = c_int
         L.ksa_oracle_select_blocks.argtypes = ([c_int] * 6 + [_u16p, _u16p, _i32p, c_int,
                                                 _i32p, _i32p, nullable_f64])
+        L.ksa_oracle_select_blocks_ex.argtypes = ([c_int] * 6 + [_u16p, _u16p, _i32p, c_int,
+                                                   c_int, _i32p, _i32p, nullable_f64])
+        L.ksa_oracle_round_bf16.argtypes = [c_double]
+        L.ksa_oracle_round_bf16.restype = ctypes.c_uint16
+        L.ksa_oracle_round_bf16_array.argtypes = [ctypes.c_size_t, _f64p, _u16p]
         L.ksa_oracle_attention.argtypes = ([c_int] * 5 + [_u16p, _u16p, _u16p, _i32p,
                                            ctypes.c_void_p, ctypes.c_void_p, c_int, c_int,
                                            c_int, c_double, _f64p, nullable_f64,
@@ -77,6 +82,17 @@ class Oracle:
                                             np.ascontiguousarray(seq_lens, np.int32), S)
         return S
 
+    def round_bf16(self, x) -> np.ndarray:
+        """Nearest bf16 (ties to even) of fp64 values -> uint16 bit patterns, same shape."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty(x.shape, np.uint16)
+        self.lib.ksa_oracle_round_bf16_array(x.size, x.reshape(-1), out.reshape(-1))
+        return out
+
+    def block_summaries_bf16(self, K: np.ndarray, seq_lens: np.ndarray, bs: int) -> np.ndarray:
+        """The block means stored as bf16 -> uint16 bits [B,Hkv,ceil(T/bs),D]."""
+        return self.round_bf16(self.block_summaries(K, seq_lens, bs))
+
     # -- A2 -----------------------------------------------------------------
     def block_scores(self, q: np.ndarray, S: np.ndarray, seq_lens: np.ndarray,
                      bs: int) -> np.ndarray:
@@ -98,8 +114,10 @@ class Oracle:
         m = self.lib.ksa_oracle_topk(s.shape[0], s, k, out)
         return out[:m].copy()
 
-    def select_blocks(self, q, K, seq_lens, bs: int, k: int, want_scores: bool = False):
-        """A1+A2+A3: (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv][, scores])."""
+    def select_blocks(self, q, K, seq_lens, bs: int, k: int, want_scores: bool = False,
+                      summary_bf16: bool = False):
+        """A1+A2+A3: (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv][, scores]).
+        summary_bf16: the block means are stored as bf16 before scoring."""
         q = np.ascontiguousarray(q, dtype=np.uint16)
         K = np.ascontiguousarray(K, dtype=np.uint16)
         B, Hq, D = q.shape
@@ -107,9 +125,9 @@ class Oracle:
         idx = np.empty((B, Hkv, k), np.int32)
         cnt = np.empty((B, Hkv), np.int32)
         scores = np.empty((B, Hkv, -(-T // bs)), np.float64) if want_scores else None
-        self.lib.ksa_oracle_select_blocks(
-            B, Hq, Hkv, D, T, bs, q, K, np.ascontiguousarray(seq_lens, np.int32), k, idx,
-            cnt, scores.ctypes.data if want_scores else None)
+        self.lib.ksa_oracle_select_blocks_ex(
+            B, Hq, Hkv, D, T, bs, q, K, np.ascontiguousarray(seq_lens, np.int32), k,
+            int(summary_bf16), idx, cnt, scores.ctypes.data if want_scores else None)
         return (idx, cnt, scores) if want_scores else (idx, cnt)
 
     # -- A4/A5/A7/A8 --------------------------------------------------------

@@ -498,3 +498,83 @@ def test_unified_window_excluded_from_voted_part(oracle):
                                      20, 10)
     assert cnt[0] == 20
     assert list(idx[0]) == list(range(10)) + list(range(40, 50))
+
+
+# ---------------------------------------------------------------------------
+# bf16 storage of the block summaries (the nearest bf16, ties to even)
+
+
+@pytest.mark.parametrize("x,bits", [
+    (1.0, 0x3F80),
+    (1.0 + 2.0 ** -8, 0x3F80),              # midway between 1 and 1 + 2^-7: the even one (1)
+    (1.0 + 3 * 2.0 ** -8, 0x3F82),          # midway between 0x3F81 and 0x3F82: the even one
+    (1.0 + 2.0 ** -8 + 2.0 ** -30, 0x3F81), # just past the midpoint: up
+    (-2.5, 0xC020),
+    (0.0, 0x0000),
+    (-0.0, 0x8000),
+    ((2.0 - 2.0 ** -7) * 2.0 ** 127, 0x7F7F),  # the largest bf16
+    (2.0 ** 128, 0x7F80),                    # past it: infinity
+    (2.0 ** -133, 0x0001),                   # the smallest subnormal bf16
+    (2.0 ** -134, 0x0000),                   # half of it: ties to even (zero)
+    (3 * 2.0 ** -135, 0x0001),               # three quarters of it: up
+])
+def test_round_bf16_format_values(oracle, x, bits):
+    """Bit patterns worked out from the bf16 format (1 sign, 8 exponent, 7 mantissa bits)."""
+    assert int(oracle.round_bf16(np.array([x]))[0]) == bits
+
+
+def test_round_bf16_matches_torch_on_binary32(oracle):
+    """For binary32 inputs the nearest-even bf16 is torch's float32 -> bfloat16 conversion."""
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-40, 40, 20000))).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.round_bf16(x.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+def test_round_bf16_is_nearest_on_doubles(oracle):
+    """Brute force on doubles: no neighbouring bf16 is closer; a tie picks the even pattern."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal(5000) * np.exp2(rng.integers(-20, 20, 5000).astype(np.float64))
+    got = oracle.round_bf16(x)
+    for xi, bi in zip(x, got):
+        b = int(bi)
+        mag = b & 0x7FFF
+        v = float(bf16_value(np.array([b], np.uint16))[0])
+        for nb in (mag - 1, mag + 1):
+            if 0 <= nb < 0x7F80:
+                vn = float(bf16_value(np.array([(b & 0x8000) | nb], np.uint16))[0])
+                assert abs(xi - v) <= abs(xi - vn)
+                if abs(xi - v) == abs(xi - vn):
+                    assert mag % 2 == 0
+
+
+def test_select_blocks_bf16_storage_tie(oracle):
+    """Block 1's mean (1 + 2^-8 in the only non-zero column) beats block 0's mean
+    (exactly 1) in fp64, but both store as bf16 1.0: the tie goes to block 0."""
+    D, bs = 64, 2
+    K = np.zeros((1, 1, 4, D), np.float32)
+    K[0, 0, 0:2, 0] = 1.0
+    K[0, 0, 2, 0] = 1.0
+    K[0, 0, 3, 0] = 1.0 + 2.0 ** -7
+    q = np.zeros((1, 1, D), np.float32)
+    q[0, 0, 0] = 1.0
+    lens = np.array([4], np.int32)
+    idx64, _ = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, 1)
+    idx16, _ = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, 1, summary_bf16=True)
+    assert idx64[0, 0, 0] == 1 and idx16[0, 0, 0] == 0
+
+
+def test_select_blocks_bf16_storage_exact_means(oracle):
+    """Keys on a 1/4 grid in [-2, 2] with blocks of 4 give means on a 1/16 grid, all exact
+    in bf16: the stored summaries change nothing."""
+    rng = np.random.default_rng(33)
+    B, Hq, Hkv, D, T, bs = 2, 4, 2, 64, 160, 4
+    K = np.clip(np.round(rng.standard_normal((B, Hkv, T, D)) * 4) / 4, -2, 2).astype(np.float32)
+    q = np.round(rng.standard_normal((B, Hq, D)) * 4).astype(np.float32) / 4
+    lens = np.array([T, 97], np.int32)
+    S = oracle.block_summaries(bf16_bits(K), lens, bs)
+    assert np.array_equal(bf16_value(oracle.round_bf16(S)), S)
+    a = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, 7)
+    b = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, 7, summary_bf16=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
