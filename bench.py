@@ -53,6 +53,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--batch", type=int, default=0,
                    help="override the per-GPU batch (small profiling cases only)")
+    p.add_argument("--summaries", choices=["f32", "bf16"], default="f32",
+                   help="storage type of the block summaries (block workloads)")
     return p.parse_args()
 
 
@@ -159,9 +161,10 @@ def query_sets(shape, count, device):
     return synth.make_queries(shape, 5000, count, device, group_noise=noise)
 
 
-def algorithmic_bytes(shape, seq_lens, kind: str):
+def algorithmic_bytes(shape, seq_lens, kind: str, summary_bytes: int = 4):
     """Per step: summaries read (when k < NB_b) + selected K/V + q + out (fp32).
-    Also returns the attention kernel's share (selected K/V + q + out)."""
+    Also returns the attention kernel's share (selected K/V + q + out).
+    summary_bytes: 4 for fp32-stored summaries, 2 for bf16."""
     bs, Hkv, Hq, D = shape.block_size, shape.num_kv_heads, shape.num_q_heads, shape.head_dim
     k = shape.k_blocks
     summ = kv = 0
@@ -171,7 +174,7 @@ def algorithmic_bytes(shape, seq_lens, kind: str):
             kv += Hkv * int(L) * D * 2 * 2
             continue
         if k < nb:
-            summ += Hkv * nb * D * 4
+            summ += Hkv * nb * D * summary_bytes
         kv += Hkv * min(k * bs, int(L)) * D * 2 * 2
     qo = len(seq_lens) * Hq * D * (2 + 4)
     return summ + kv + qo, kv + qo, summ
@@ -270,7 +273,8 @@ def run_block(args, dist, dev, kind):
     k = shape.k_blocks
     nq = 16
     qs = query_sets(shape, nq, dev)
-    S = ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs)  # prefill, untimed
+    sdt = torch.bfloat16 if args.summaries == "bf16" else torch.float32
+    S = ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, summary_dtype=sdt)  # prefill, untimed
     ws_sel = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
                          dtype=torch.uint8, device=dev)
     ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
@@ -340,7 +344,7 @@ def run_block(args, dist, dev, kind):
     t_sel = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
     t_att = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
     lens = inp.seq_lens.cpu().tolist()
-    total_b, attn_b, summ_b = algorithmic_bytes(shape, lens, kind)
+    total_b, attn_b, summ_b = algorithmic_bytes(shape, lens, kind, S.element_size())
     per_step_s = ms / 1e3 / args.steps
     peak, peak_kind = measured_peak()
     attn_gbs = attn_b / (t_att * 1e-3) / 1e9
@@ -364,6 +368,7 @@ def run_block(args, dist, dev, kind):
         "config": {"workload": shape.name, "batch_per_gpu": B, "num_q_heads": Hq,
                    "num_kv_heads": Hkv, "head_dim": D, "capacity": T, "block_size": bs,
                    "k_blocks": k if kind != "dense" else "all",
+                   "summaries": "bf16" if S.dtype == torch.bfloat16 else "f32",
                    "l2": "inputs larger than L2: K/V cache %.1f GB, %.0f MB read per step, %d "
                          "rotating query sets" % (2 * inp.K.numel() * 2 / 1e9, total_b / 1e6, nq),
                    "step": ("dense attention" if kind == "dense" else

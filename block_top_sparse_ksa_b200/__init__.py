@@ -25,7 +25,9 @@ __all__ = [
     "ksa_select_blocks_workspace", "ksa_sparse_decode_attn_workspace",
     "ksa_sparse_decode_attn_noalloc", "ksa_decode_select_blocks",
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
-    "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "OUT_F32", "OUT_BF16", "FLAG_SEQ_LEN_CLAMPED",
+    "ksa_build_block_summaries_ex", "ksa_select_blocks_ex", "ksa_decode_select_blocks_ex",
+    "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
+    "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
 ]
 
@@ -33,6 +35,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libksa.so")
 
 SUMMARY_ALL, SUMMARY_LAST_BLOCK = 0, 1
+SUMMARIES_F32, SUMMARIES_BF16 = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 FLAG_SEQ_LEN_CLAMPED, FLAG_INDEX_SKIPPED, FLAG_NONFINITE_SCORE, FLAG_WAIT_TIMEOUT = 1, 2, 4, 8
 _STATUS = {0: "KSA_OK", 1: "KSA_ERR_INVALID_ARG", 2: "KSA_ERR_UNSUPPORTED",
@@ -56,6 +59,12 @@ class Shape(ctypes.Structure):
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
     "ksa_build_block_summaries": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _i32, _vp, _vp, _vp]),
+    "ksa_build_block_summaries_ex": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _i32, _i32, _vp,
+                                            _vp, _vp]),
+    "ksa_select_blocks_ex": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _i32, _vp, _i32, _vp, _vp,
+                                    _vp, _sz, _vp, _vp]),
+    "ksa_decode_select_blocks_ex": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _i32,
+                                           _vp, _vp, _vp, _sz, _vp, _vp]),
     "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]),
@@ -144,22 +153,36 @@ def _shape(B, Hq, Hkv, D, T, bs=16) -> Shape:
 # entry points (same names as the C ABI)
 
 
+def _summary_dtype(summaries: torch.Tensor) -> int:
+    """KSA_SUMMARIES_* code of a summaries tensor (fp32 or bf16)."""
+    if summaries.dtype == torch.float32:
+        return SUMMARIES_F32
+    if summaries.dtype == torch.bfloat16:
+        return SUMMARIES_BF16
+    raise TypeError(f"summaries must be float32 or bfloat16, not {summaries.dtype}")
+
+
 def ksa_build_block_summaries(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
                               mode: int = SUMMARY_ALL, summaries: Optional[torch.Tensor] = None,
-                              dev_status: Optional[torch.Tensor] = None,
-                              stream=None) -> torch.Tensor:
-    """Block mean keys S [B, Hkv, ceil(T/bs), D] fp32 (all blocks, or the last one)."""
+                              dev_status: Optional[torch.Tensor] = None, stream=None,
+                              summary_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """Block mean keys S [B, Hkv, ceil(T/bs), D] (all blocks, or the last one), stored as
+    fp32 or bf16: the given tensor's dtype, else `summary_dtype`."""
     _dev(K, "K", torch.bfloat16)
     _dev(seq_lens, "seq_lens", torch.int32)
     B, Hkv, T, D = K.shape
     nb = -(-T // block_size)
     if summaries is None:
-        summaries = torch.empty((B, Hkv, nb, D), dtype=torch.float32, device=K.device)
-    _dev(summaries, "summaries", torch.float32)
+        summaries = torch.empty((B, Hkv, nb, D), dtype=summary_dtype, device=K.device)
+    _dev(summaries, "summaries", summaries.dtype)
     sh = _shape(B, Hkv, Hkv, D, T, block_size)
-    _check(lib().ksa_build_block_summaries(ctypes.byref(sh), _ptr(K), _ptr(seq_lens), int(mode),
-                                           _ptr(summaries), _ptr(dev_status), _stream(stream)))
+    _check(lib().ksa_build_block_summaries_ex(
+        ctypes.byref(sh), _ptr(K), _ptr(seq_lens), int(mode), _summary_dtype(summaries),
+        _ptr(summaries), _ptr(dev_status), _stream(stream)))
     return summaries
+
+
+ksa_build_block_summaries_ex = ksa_build_block_summaries
 
 
 def _workspace(ws: Optional[torch.Tensor], need: int, device) -> torch.Tensor:
@@ -182,9 +205,10 @@ def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.
                       num_sel: Optional[torch.Tensor] = None,
                       workspace: Optional[torch.Tensor] = None,
                       dev_status: Optional[torch.Tensor] = None, stream=None):
-    """Top-k blocks per (row, kv-head): (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv])."""
+    """Top-k blocks per (row, kv-head): (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv]).
+    The summaries' dtype (fp32 or bf16) selects their storage type."""
     _dev(q, "q", torch.bfloat16)
-    _dev(summaries, "summaries", torch.float32)
+    _dev(summaries, "summaries", summaries.dtype)
     _dev(seq_lens, "seq_lens", torch.int32)
     B, Hq, D = q.shape
     Hkv = summaries.shape[1]
@@ -195,11 +219,15 @@ def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.
     sh = _shape(B, Hq, Hkv, D, capacity, block_size)
     ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
                     q.device)
-    _check(lib().ksa_select_blocks(ctypes.byref(sh), _ptr(q), _ptr(summaries), _ptr(seq_lens),
-                                   int(k_blocks), _ptr(block_idx), _ptr(num_sel), _ptr(ws),
-                                   ws.numel() * ws.element_size(), _ptr(dev_status),
-                                   _stream(stream)))
+    _check(lib().ksa_select_blocks_ex(ctypes.byref(sh), _ptr(q), _ptr(summaries),
+                                      _summary_dtype(summaries), _ptr(seq_lens), int(k_blocks),
+                                      _ptr(block_idx), _ptr(num_sel), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _ptr(dev_status),
+                                      _stream(stream)))
     return block_idx, num_sel
+
+
+ksa_select_blocks_ex = ksa_select_blocks
 
 
 def ksa_decode_select_blocks(q: torch.Tensor, K: torch.Tensor, summaries: torch.Tensor,
@@ -211,7 +239,7 @@ def ksa_decode_select_blocks(q: torch.Tensor, K: torch.Tensor, summaries: torch.
     """Refresh every row's last-block summary from K, then select (one launch)."""
     _dev(q, "q", torch.bfloat16)
     _dev(K, "K", torch.bfloat16)
-    _dev(summaries, "summaries", torch.float32)
+    _dev(summaries, "summaries", summaries.dtype)
     _dev(seq_lens, "seq_lens", torch.int32)
     B, Hq, D = q.shape
     _, Hkv, T, _ = K.shape
@@ -222,11 +250,14 @@ def ksa_decode_select_blocks(q: torch.Tensor, K: torch.Tensor, summaries: torch.
     sh = _shape(B, Hq, Hkv, D, T, block_size)
     ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
                     q.device)
-    _check(lib().ksa_decode_select_blocks(
-        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(summaries), _ptr(seq_lens), int(k_blocks),
-        _ptr(block_idx), _ptr(num_sel), _ptr(ws), ws.numel() * ws.element_size(),
-        _ptr(dev_status), _stream(stream)))
+    _check(lib().ksa_decode_select_blocks_ex(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(summaries), _summary_dtype(summaries),
+        _ptr(seq_lens), int(k_blocks), _ptr(block_idx), _ptr(num_sel), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
     return block_idx, num_sel
+
+
+ksa_decode_select_blocks_ex = ksa_decode_select_blocks
 
 
 def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,

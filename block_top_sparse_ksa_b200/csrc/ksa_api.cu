@@ -120,21 +120,25 @@ bool encode_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int
 
 extern "C" {
 
-ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
-                                     const int32_t *seq_lens, int32_t mode, float *summaries,
-                                     uint32_t *dev_status, void *stream) {
+ksa_status ksa_build_block_summaries_ex(const ksa_shape *shape, const uint16_t *K,
+                                        const int32_t *seq_lens, int32_t mode,
+                                        int32_t summary_dtype, void *summaries,
+                                        uint32_t *dev_status, void *stream) {
   ksa_status st = check_shape(shape, true);
   if (st != KSA_OK) return st;
   if (K == nullptr || seq_lens == nullptr || summaries == nullptr)
     return fail(KSA_ERR_INVALID_ARG, "K, seq_lens and summaries must be non-NULL");
   if (mode != KSA_SUMMARY_ALL && mode != KSA_SUMMARY_LAST_BLOCK)
     return fail(KSA_ERR_INVALID_ARG, "mode %d is neither ALL nor LAST_BLOCK", mode);
+  if (summary_dtype != KSA_SUMMARIES_F32 && summary_dtype != KSA_SUMMARIES_BF16)
+    return fail(KSA_ERR_INVALID_ARG, "summary_dtype %d is neither F32 nor BF16", summary_dtype);
   if (!aligned(K, 16) || !aligned(summaries, 16) || !aligned(seq_lens, 4))
     return fail(KSA_ERR_INVALID_ARG, "K and summaries must be 16-byte aligned");
   ksa::SummaryArgs a;
   a.K = K;
   a.seq_lens = seq_lens;
   a.S = summaries;
+  a.sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
   a.status = dev_status;
   a.B = shape->batch;
   a.Hkv = shape->num_kv_heads;
@@ -146,6 +150,13 @@ ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
                      "ksa_build_block_summaries launch");
 }
 
+ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
+                                     const int32_t *seq_lens, int32_t mode, float *summaries,
+                                     uint32_t *dev_status, void *stream) {
+  return ksa_build_block_summaries_ex(shape, K, seq_lens, mode, KSA_SUMMARIES_F32, summaries,
+                                      dev_status, stream);
+}
+
 size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks) {
   (void)k_blocks;
   if (check_shape(shape, true) != KSA_OK) return 0;
@@ -153,15 +164,20 @@ size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks) {
                                      shape->block_size);
 }
 
-ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const float *summaries,
-                             const int32_t *seq_lens, int32_t k_blocks, int32_t *block_idx,
-                             int32_t *num_sel, void *ws, size_t ws_bytes, uint32_t *dev_status,
-                             void *stream) {
+namespace {
+
+// Shared by the selection entry points; K non-NULL fuses the last-block refresh.
+ksa_status select_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                         void *summaries, int32_t summary_dtype, const int32_t *seq_lens,
+                         int32_t k_blocks, int32_t *block_idx, int32_t *num_sel, void *ws,
+                         size_t ws_bytes, uint32_t *dev_status, void *stream, const char *what) {
   ksa_status st = check_shape(shape, true);
   if (st != KSA_OK) return st;
   if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
       num_sel == nullptr)
     return fail(KSA_ERR_INVALID_ARG, "q, summaries, seq_lens, block_idx, num_sel must be non-NULL");
+  if (summary_dtype != KSA_SUMMARIES_F32 && summary_dtype != KSA_SUMMARIES_BF16)
+    return fail(KSA_ERR_INVALID_ARG, "summary_dtype %d is neither F32 nor BF16", summary_dtype);
   if (k_blocks < 1) return fail(KSA_ERR_INVALID_ARG, "k_blocks must be >= 1 (got %d)", k_blocks);
   const int nb_max = (shape->capacity + shape->block_size - 1) / shape->block_size;
   if (nb_max > 16384)
@@ -175,7 +191,8 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const fl
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   ksa::SelectArgs a;
   a.q = q;
-  a.S = const_cast<float *>(summaries);  // read only: no K is given, so nothing is refreshed
+  a.S = summaries;  // written only when K is given (the fused refresh)
+  a.sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
   a.seq_lens = seq_lens;
   a.block_idx = block_idx;
   a.num_sel = num_sel;
@@ -188,51 +205,48 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const fl
   a.bs = shape->block_size;
   a.k = k_blocks;
   return cuda_status(
-      ksa::launch_select_blocks(a, nullptr, ws, device_sm_count(),
-                                static_cast<cudaStream_t>(stream)),
-      "ksa_select_blocks launch");
+      ksa::launch_select_blocks(a, K, ws, device_sm_count(), static_cast<cudaStream_t>(stream)),
+      what);
+}
+
+}  // namespace
+
+ksa_status ksa_select_blocks_ex(const ksa_shape *shape, const uint16_t *q, const void *summaries,
+                                int32_t summary_dtype, const int32_t *seq_lens, int32_t k_blocks,
+                                int32_t *block_idx, int32_t *num_sel, void *ws, size_t ws_bytes,
+                                uint32_t *dev_status, void *stream) {
+  // read only: no K is given, so nothing is refreshed
+  return select_common(shape, q, nullptr, const_cast<void *>(summaries), summary_dtype, seq_lens,
+                       k_blocks, block_idx, num_sel, ws, ws_bytes, dev_status, stream,
+                       "ksa_select_blocks launch");
+}
+
+ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q, const float *summaries,
+                             const int32_t *seq_lens, int32_t k_blocks, int32_t *block_idx,
+                             int32_t *num_sel, void *ws, size_t ws_bytes, uint32_t *dev_status,
+                             void *stream) {
+  return ksa_select_blocks_ex(shape, q, summaries, KSA_SUMMARIES_F32, seq_lens, k_blocks,
+                              block_idx, num_sel, ws, ws_bytes, dev_status, stream);
+}
+
+ksa_status ksa_decode_select_blocks_ex(const ksa_shape *shape, const uint16_t *q,
+                                       const uint16_t *K, void *summaries, int32_t summary_dtype,
+                                       const int32_t *seq_lens, int32_t k_blocks,
+                                       int32_t *block_idx, int32_t *num_sel, void *ws,
+                                       size_t ws_bytes, uint32_t *dev_status, void *stream) {
+  if (K == nullptr) return fail(KSA_ERR_INVALID_ARG, "K must be non-NULL");
+  if (!aligned(K, 16)) return fail(KSA_ERR_INVALID_ARG, "K must be 16-byte aligned");
+  return select_common(shape, q, K, summaries, summary_dtype, seq_lens, k_blocks, block_idx,
+                       num_sel, ws, ws_bytes, dev_status, stream, "ksa_decode_select_blocks launch");
 }
 
 ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
                                     float *summaries, const int32_t *seq_lens, int32_t k_blocks,
                                     int32_t *block_idx, int32_t *num_sel, void *ws,
                                     size_t ws_bytes, uint32_t *dev_status, void *stream) {
-  if (K == nullptr) return fail(KSA_ERR_INVALID_ARG, "K must be non-NULL");
-  if (!aligned(K, 16)) return fail(KSA_ERR_INVALID_ARG, "K must be 16-byte aligned");
-  // same validation as the selection alone
-  ksa_status st = check_shape(shape, true);
-  if (st != KSA_OK) return st;
-  if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
-      num_sel == nullptr)
-    return fail(KSA_ERR_INVALID_ARG, "q, summaries, seq_lens, block_idx, num_sel must be non-NULL");
-  if (k_blocks < 1) return fail(KSA_ERR_INVALID_ARG, "k_blocks must be >= 1 (got %d)", k_blocks);
-  const int nb_max = (shape->capacity + shape->block_size - 1) / shape->block_size;
-  if (nb_max > 16384)
-    return fail(KSA_ERR_UNSUPPORTED, "ceil(capacity/block_size) = %d exceeds 16384", nb_max);
-  if (!aligned(summaries, 16) || !aligned(q, 4))
-    return fail(KSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
-  const size_t need = ksa::select_workspace_bytes(shape->batch, shape->num_kv_heads,
-                                                  shape->capacity, shape->block_size);
-  if (ws == nullptr || ws_bytes < need)
-    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
-  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  ksa::SelectArgs a;
-  a.q = q;
-  a.S = summaries;
-  a.seq_lens = seq_lens;
-  a.block_idx = block_idx;
-  a.num_sel = num_sel;
-  a.status = dev_status;
-  a.B = shape->batch;
-  a.Hq = shape->num_q_heads;
-  a.Hkv = shape->num_kv_heads;
-  a.D = shape->head_dim;
-  a.T = shape->capacity;
-  a.bs = shape->block_size;
-  a.k = k_blocks;
-  return cuda_status(ksa::launch_select_blocks(a, K, ws, device_sm_count(),
-                                               static_cast<cudaStream_t>(stream)),
-                     "ksa_decode_select_blocks launch");
+  return ksa_decode_select_blocks_ex(shape, q, K, summaries, KSA_SUMMARIES_F32, seq_lens,
+                                     k_blocks, block_idx, num_sel, ws, ws_bytes, dev_status,
+                                     stream);
 }
 
 size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape, int32_t idx_capacity,

@@ -303,6 +303,22 @@ __device__ __forceinline__ bool warp_block_mean(const uint16_t *rows, int n, flo
   return rp == 0;
 }
 
+// Stores dims [c8, c8 + 8) of a block mean at element offset `row` of the
+// summaries: fp32, or (sbf16) bf16 rounded to nearest even.  Every writer of
+// summaries goes through here, so all of them store the same bits.
+__device__ __forceinline__ void store_mean8(void *S, int sbf16, size_t row, int c8,
+                                            const float (&m)[8]) {
+  if (sbf16) {
+    *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(S) + row + c8) =
+        make_uint4(pack_bf16x2(m[0], m[1]), pack_bf16x2(m[2], m[3]), pack_bf16x2(m[4], m[5]),
+                   pack_bf16x2(m[6], m[7]));
+  } else {
+    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(S) + row + c8);
+    dst[0] = make_float4(m[0], m[1], m[2], m[3]);
+    dst[1] = make_float4(m[4], m[5], m[6], m[7]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // block-wide helpers
 

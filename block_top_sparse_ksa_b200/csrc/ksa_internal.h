@@ -15,7 +15,8 @@ namespace ksa {
 struct SummaryArgs {
   const uint16_t *K;
   const int32_t *seq_lens;
-  float *S;
+  void *S;    // fp32 or bf16 [B, Hkv, ceil(T/bs), D]
+  int sbf16;  // summaries stored as bf16
   uint32_t *status;
   int B, Hkv, T, D, bs, mode;
 };
@@ -23,7 +24,8 @@ cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream);
 
 struct SelectArgs {
   const uint16_t *q;
-  float *S;  // read; written only by the fused last-block refresh
+  void *S;    // fp32 or bf16; read; written only by the fused last-block refresh
+  int sbf16;  // summaries stored as bf16
   const int32_t *seq_lens;
   int32_t *block_idx;
   int32_t *num_sel;

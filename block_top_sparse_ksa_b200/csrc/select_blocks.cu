@@ -7,9 +7,9 @@
 //
 // Two launches:
 //  1. scoring, persistent.  The summaries of every (row b, kv-head g) are cut
-//     into pieces of 8 KB (2048 / D consecutive blocks, D fp32 each,
-//     contiguous); each row is padded to the same number of pieces and the
-//     grid's warps take equal contiguous slices of the flat piece sequence, so
+//     into pieces of 8 KB (2048 / D consecutive blocks of D fp32, or 4096 / D
+//     of D bf16, contiguous); each row is padded to the same number of pieces
+//     and the grid's warps take equal contiguous slices of the flat piece sequence, so
 //     a warp streams one region front to back and forms each row's group
 //     query sum once.  A warp pulls a whole piece into registers with 16-byte
 //     loads (all in flight at once), then scores it -- 8 lanes per summary
@@ -37,7 +37,7 @@ namespace ksa {
 
 namespace {
 
-constexpr int kPieceBytes = 8192;  // one piece: 2048 / D summary rows
+constexpr int kPieceBytes = 8192;  // one piece: 2048 / D fp32 or 4096 / D bf16 summary rows
 constexpr int kScThreads = 256;
 constexpr int kRankWarpThreads = 128;
 constexpr int kRankThreads = 256;
@@ -80,12 +80,9 @@ __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const ui
   const int jl = nb - 1;
   const uint16_t *rows = K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
   const bool mine = warp_block_mean<D>(rows, L - jl * a.bs, mean);
-  if (mine) {
-    const int c8 = ((threadIdx.x & 31) % (D / 8)) * 8;
-    float *dst = a.S + (static_cast<size_t>(row) * nb_max + jl) * D + c8;
-    reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
-    reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
-  }
+  if (mine)
+    store_mean8(a.S, a.sbf16, (static_cast<size_t>(row) * nb_max + jl) * D,
+                ((threadIdx.x & 31) % (D / 8)) * 8, mean);
   return mine;
 }
 
@@ -199,22 +196,26 @@ __device__ __forceinline__ void keep_all_blocks(const ScoreDev &p, int row, int 
   }
 }
 
-// Group query sum of kv-head g of batch row b over this lane's columns
-// (float4 chunks sub + 8 j of a summary row), summed over the heads in order.
-template <int D>
+// Group query sum of kv-head g of batch row b over this lane's columns,
+// summed over the heads in order.  The lane reads 16-byte chunks sub + 8 j of
+// a summary row: 4 fp32 dims each (qv[j]), or with bf16 summaries 8 dims each
+// (qv[2j], qv[2j+1]).  Either way qv covers D/8 dims in D/32 float4.
+template <int D, bool SBF>
 __device__ __forceinline__ void load_qsum(const SelectArgs &a, int b, int g, int sub,
                                           float4 (&qv)[D / 32]) {
-  constexpr int PER = D / 32;
+  constexpr int NQ = D / 32;
   const int G = a.Hq / a.Hkv;
 #pragma unroll
-  for (int j = 0; j < PER; ++j) qv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < NQ; ++j) qv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
   const uint16_t *qg = a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G) * D;
 #pragma unroll 4
   for (int h = 0; h < G; ++h) {
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const uint32_t *q2 = reinterpret_cast<const uint32_t *>(
-          qg + static_cast<size_t>(h) * D + 4 * (sub + 8 * j));
+    for (int j = 0; j < NQ; ++j) {
+      // dims 4 c .. 4 c + 3 with c the 4-dim group of qv[j]
+      const int c4 = SBF ? 2 * (sub + 8 * (j >> 1)) + (j & 1) : sub + 8 * j;
+      const uint32_t *q2 =
+          reinterpret_cast<const uint32_t *>(qg + static_cast<size_t>(h) * D + 4 * c4);
       const uint32_t w0 = __ldg(q2), w1 = __ldg(q2 + 1);
       qv[j].x += bf16_lo(w0);
       qv[j].y += bf16_hi(w0);
@@ -224,16 +225,17 @@ __device__ __forceinline__ void load_qsum(const SelectArgs &a, int b, int g, int
   }
 }
 
-// Scores piece x (x.n > 0) against the group query sum qv: the whole piece is
-// pulled into registers at once (lane (r, sub) holds chunks sub + 8 j of rows
-// 4 it + r), each summary row is reduced over its 8 lanes, and the keys are
-// stored.  With a key cache given, the piece holding the row's last block
-// first re-averages that block, so the fresh value is the one scored.
-template <int D>
+// Scores piece x (x.n > 0) against the group query sum qv: the whole 8 KB
+// piece is pulled into registers at once (lane (r, sub) holds chunks sub + 8 j
+// of rows 4 it + r), each summary row is reduced over its 8 lanes, and the
+// keys are stored.  With a key cache given, the piece holding the row's last
+// block first re-averages that block, so the fresh value is the one scored.
+template <int D, bool SBF>
 __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
                                             const float4 (&qv)[D / 32], uint32_t &bad) {
-  constexpr int R = kPieceBytes / (D * 4);
-  constexpr int PER = D / 32;
+  constexpr int RB = D * (SBF ? 2 : 4);  // bytes per summary row
+  constexpr int R = kPieceBytes / RB;     // rows per piece
+  constexpr int PER = RB / 16 / 8;        // 16-byte chunks per lane and row
   constexpr int IT = R / 4;
   const SelectArgs &a = p.a;
   const int lane = threadIdx.x & 31, sub = lane & 7;
@@ -243,16 +245,15 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
     refresh_last_block<D>(a, p.K, x.row, x.L, x.nb, mean);
     __syncwarp();  // the fresh summary is visible to the whole warp's loads below
   }
-  const float4 *src =
-      reinterpret_cast<const float4 *>(a.S + (static_cast<size_t>(x.row) * nb_max + x.j0) * D);
-  float4 v[IT][PER];
+  const uint4 *src = reinterpret_cast<const uint4 *>(
+      static_cast<const uint8_t *>(a.S) + (static_cast<size_t>(x.row) * nb_max + x.j0) * RB);
+  uint4 v[IT][PER];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const int jr = it * 4 + (lane >> 3);
 #pragma unroll
     for (int j = 0; j < PER; ++j)
-      v[it][j] = jr < x.n ? __ldcg(src + jr * (D / 4) + sub + 8 * j)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[it][j] = jr < x.n ? __ldcg(src + jr * (RB / 16) + sub + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
   }
   uint32_t *krow = p.keys + static_cast<size_t>(x.row) * nb_max + x.j0;
 #pragma unroll
@@ -261,10 +262,23 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
     float sc = 0.f;
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
-      sc = fmaf(qv[j].x, v[it][j].x, sc);
-      sc = fmaf(qv[j].y, v[it][j].y, sc);
-      sc = fmaf(qv[j].z, v[it][j].z, sc);
-      sc = fmaf(qv[j].w, v[it][j].w, sc);
+      const uint4 w = v[it][j];
+      if (SBF) {
+        const float4 qa = qv[2 * j], qb = qv[2 * j + 1];
+        sc = fmaf(qa.x, bf16_lo(w.x), sc);
+        sc = fmaf(qa.y, bf16_hi(w.x), sc);
+        sc = fmaf(qa.z, bf16_lo(w.y), sc);
+        sc = fmaf(qa.w, bf16_hi(w.y), sc);
+        sc = fmaf(qb.x, bf16_lo(w.z), sc);
+        sc = fmaf(qb.y, bf16_hi(w.z), sc);
+        sc = fmaf(qb.z, bf16_lo(w.w), sc);
+        sc = fmaf(qb.w, bf16_hi(w.w), sc);
+      } else {
+        sc = fmaf(qv[j].x, __uint_as_float(w.x), sc);
+        sc = fmaf(qv[j].y, __uint_as_float(w.y), sc);
+        sc = fmaf(qv[j].z, __uint_as_float(w.z), sc);
+        sc = fmaf(qv[j].w, __uint_as_float(w.w), sc);
+      }
     }
     sc += __shfl_xor_sync(0xffffffffu, sc, 1);
     sc += __shfl_xor_sync(0xffffffffu, sc, 2);
@@ -281,7 +295,7 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
 // sequence: a warp streams one region of the summaries front to back (the
 // pattern the DRAM serves best, measured against round-robin and
 // counter-driven orders) and forms each row's group query sum once.
-template <int D>
+template <int D, bool SBF>
 __global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev p) {
   constexpr int kWarps = kScThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane & 7;
@@ -298,9 +312,9 @@ __global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev
     if (x.n == 0) continue;
     if (x.row != qrow) {
       qrow = x.row;
-      load_qsum<D>(p.a, x.b, x.g, sub, qv);
+      load_qsum<D, SBF>(p.a, x.b, x.g, sub, qv);
     }
-    score_piece<D>(p, x, qv, bad);
+    score_piece<D, SBF>(p, x, qv, bad);
   }
   bad = __reduce_or_sync(0xffffffffu, bad);
   if (bad != 0u && lane == 0) flag_status(p.a.status, bad);
@@ -482,9 +496,9 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
   const int rows = a.B * a.Hkv;
   cudaError_t err;
   if (nb_max > a.k) {  // otherwise no row has a block to score
+    const auto kern = a.sbf16 ? score_blocks_kernel<D, true> : score_blocks_kernel<D, false>;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_blocks_kernel<D>,
-                                                        kScThreads, 0);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kScThreads, 0);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     constexpr int kWarps = kScThreads / 32;
@@ -492,8 +506,7 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
     const long long need = (p.units + kWarps - 1) / kWarps;
     if (n > need) n = need;
     p.N = static_cast<int>(n);
-    err = launch_pdl(score_blocks_kernel<D>, dim3(static_cast<unsigned>(p.N)), dim3(kScThreads),
-                     0, stream, p);
+    err = launch_pdl(kern, dim3(static_cast<unsigned>(p.N)), dim3(kScThreads), 0, stream, p);
     if (err != cudaSuccess) return err;
   }
   // rows of up to 1024 blocks: one warp per row; longer rows: one CTA per row
@@ -533,7 +546,7 @@ cudaError_t launch_select_blocks(const SelectArgs &a, const uint16_t *K, void *w
   p.a = a;
   p.K = K;
   p.keys = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + sems);
-  p.prow = kPieceBytes / (a.D * static_cast<int>(sizeof(float)));
+  p.prow = kPieceBytes / (a.D * (a.sbf16 ? 2 : 4));
   p.pieces = (nb_max + p.prow - 1) / p.prow;
   p.units = static_cast<long long>(rows) * p.pieces;
   p.N = 1;

@@ -8,7 +8,8 @@
 // rows l / (D/8), l / (D/8) + 32/(D/8), ... so every warp-wide load covers
 // 2 (D = 128) or 4 (D = 64) whole key rows and all of a block's loads are
 // independent (in flight together).  Partial sums meet through warp shuffles;
-// then one IEEE division by n_j, in fp32.
+// then one IEEE division by n_j, in fp32, and the mean is stored as fp32 or
+// as bf16 rounded to nearest even.
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
 
@@ -44,11 +45,9 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
     float mean[8];
     const uint16_t *rows =
         a.K + (static_cast<size_t>(bg) * a.T + static_cast<size_t>(j) * a.bs) * D;
-    if (warp_block_mean<D>(rows, n, mean)) {
-      float *dst = a.S + (static_cast<size_t>(bg) * nb_max + j) * D + (lane % (D / 8)) * 8;
-      reinterpret_cast<float4 *>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
-      reinterpret_cast<float4 *>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
-    }
+    if (warp_block_mean<D>(rows, n, mean))
+      store_mean8(a.S, a.sbf16, (static_cast<size_t>(bg) * nb_max + j) * D, (lane % (D / 8)) * 8,
+                  mean);
   }
 }
 

@@ -67,6 +67,8 @@ typedef struct {
 } ksa_shape;
 
 enum { KSA_SUMMARY_ALL = 0, KSA_SUMMARY_LAST_BLOCK = 1 };
+/* Storage type of the block summaries (the *_ex entry points). */
+enum { KSA_SUMMARIES_F32 = 0, KSA_SUMMARIES_BF16 = 1 };
 enum { KSA_OUT_F32 = 0, KSA_OUT_BF16 = 1 };
 
 enum {
@@ -128,6 +130,36 @@ ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q,
                                     const int32_t *seq_lens, int32_t k_blocks,
                                     int32_t *block_idx, int32_t *num_sel, void *ws,
                                     size_t ws_bytes, uint32_t *dev_status, void *stream);
+
+/*
+ * The same three calls with the summaries stored as bf16 or fp32
+ * (summary_dtype: KSA_SUMMARIES_F32 or KSA_SUMMARIES_BF16).  With bf16 each
+ * block mean is computed in fp32 as above and stored rounded to the nearest
+ * bf16 (ties to even): half the bytes for the maintenance writes and, above
+ * all, for the scoring reads, which dominate at long context and small budget
+ * [KIN s.5 names the block mean; the storage precision is this library's
+ * option, not the source's].  Scores are accumulated in fp32 from the stored
+ * values, so blocks whose scores differ by less than the rounding of their
+ * means may rank differently than with fp32 summaries.
+ *   summaries: [B, Hkv, ceil(T/bs), D] of the given type, 16-byte aligned.
+ * Every other argument, limit and error as the fp32 calls, which are these
+ * with KSA_SUMMARIES_F32.  An unknown summary_dtype is KSA_ERR_INVALID_ARG.
+ */
+ksa_status ksa_build_block_summaries_ex(const ksa_shape *shape, const uint16_t *K,
+                                        const int32_t *seq_lens, int32_t mode,
+                                        int32_t summary_dtype, void *summaries,
+                                        uint32_t *dev_status, void *stream);
+ksa_status ksa_select_blocks_ex(const ksa_shape *shape, const uint16_t *q,
+                                const void *summaries, int32_t summary_dtype,
+                                const int32_t *seq_lens, int32_t k_blocks,
+                                int32_t *block_idx, int32_t *num_sel, void *ws,
+                                size_t ws_bytes, uint32_t *dev_status, void *stream);
+ksa_status ksa_decode_select_blocks_ex(const ksa_shape *shape, const uint16_t *q,
+                                       const uint16_t *K, void *summaries,
+                                       int32_t summary_dtype, const int32_t *seq_lens,
+                                       int32_t k_blocks, int32_t *block_idx,
+                                       int32_t *num_sel, void *ws, size_t ws_bytes,
+                                       uint32_t *dev_status, void *stream);
 
 /*
  * Sparse decode attention over a selected token set [KIN s.5; LIM s.5

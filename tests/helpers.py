@@ -21,14 +21,22 @@ REL_TOL = 1e-2
 LSE_TOL = 1e-4
 
 
+def _row_scores(oracle, q_row, K, lens, bs, summary_bf16):
+    S = oracle.block_summaries(K[None], lens, bs)
+    if summary_bf16:  # the scores the bf16-stored means give
+        S = bf16_value(oracle.round_bf16(S))
+    return oracle.block_scores(q_row[None], S, lens, bs)[0]  # [Hkv, nb]
+
+
 def gap_fix_row(oracle, q_row: np.ndarray, K_row: np.ndarray, L: int, bs: int, k: int,
-                delta: float = DELTA, max_iter: int = 20):
+                delta: float = DELTA, max_iter: int = 20, summary_bf16: bool = False):
     """Plant a score gap >= delta at the top-k boundary of every kv-head of one row.
 
     q_row: uint16 [Hq, D] bits; K_row: uint16 [Hkv, T, D] bits (edited copy returned).
     Selected blocks that sit within delta of the best unselected score have all
     their valid keys moved along the group's query-sum direction until the
-    boundary gap is at least delta.  Returns (K_row, number of blocks moved)."""
+    boundary gap is at least delta (scored from bf16-stored means when
+    summary_bf16).  Returns (K_row, number of blocks moved)."""
     K = K_row.copy()
     Hq, D = q_row.shape
     Hkv, T, _ = K.shape
@@ -37,8 +45,7 @@ def gap_fix_row(oracle, q_row: np.ndarray, K_row: np.ndarray, L: int, bs: int, k
     lens = np.array([L], np.int32)
     moved = 0
     for _ in range(max_iter):
-        S = oracle.block_summaries(K[None], lens, bs)
-        s = oracle.block_scores(q_row[None], S, lens, bs)[0]  # [Hkv, nb]
+        s = _row_scores(oracle, q_row, K, lens, bs, summary_bf16)
         nb = -(-L // bs)
         if nb <= k:
             return K, moved
@@ -65,10 +72,9 @@ def gap_fix_row(oracle, q_row: np.ndarray, K_row: np.ndarray, L: int, bs: int, k
     raise AssertionError("could not plant the score gap")
 
 
-def min_boundary_gap(oracle, q_row, K_row, L, bs, k) -> float:
+def min_boundary_gap(oracle, q_row, K_row, L, bs, k, summary_bf16: bool = False) -> float:
     lens = np.array([L], np.int32)
-    S = oracle.block_summaries(K_row[None], lens, bs)
-    s = oracle.block_scores(q_row[None], S, lens, bs)[0]
+    s = _row_scores(oracle, q_row, K_row, lens, bs, summary_bf16)
     nb = -(-L // bs)
     if nb <= k:
         return np.inf

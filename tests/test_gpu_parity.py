@@ -273,7 +273,8 @@ def test_seq_len_out_of_range_is_clamped_and_flagged(ksa, oracle):
 
 @pytest.mark.parametrize("L,P,budget,R", [(300, 50, 64, 16), (1500, 400, 300, 75),
                                            (2500, 2600, 500, 125), (900, 120, 900, 225),
-                                           (4100, 1000, 1000, 1000), (5000, 800, 1200, 0)])
+                                           (4100, 1000, 1000, 1000), (5000, 800, 1200, 0),
+                                           (30000, 3000, 4000, 1000)])
 def test_unified_select_exact(ksa, oracle, L, P, budget, R):
     rng = np.random.default_rng(700 + L)
     B, Hq, Hkv, D = 3, 16, 4, 128
@@ -449,7 +450,7 @@ def test_decode_select_fuses_last_block_refresh(ksa, oracle, D, bs, k, nblk):
     S_b = S0.clone()
     st = status_tensor()
     idx_b, cnt_b = ksa.ksa_decode_select_blocks(qd, Kn, S_b, Ld, bs, k, dev_status=st)
-    assert torch.equal(S_a, S_b)
+    assert torch.equal(S_a.view(torch.int32), S_b.view(torch.int32))  # bits (see above)
     assert torch.equal(idx_a, idx_b) and torch.equal(cnt_a, cnt_b)
     ref_idx, ref_cnt = oracle.select_blocks(q, K_new, lens, bs, k)
     assert np.array_equal(idx_b.cpu().numpy(), ref_idx)
@@ -477,3 +478,71 @@ def test_select_many_rows_persistent_units(ksa, oracle):
         idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k, workspace=ws)
         assert np.array_equal(idx.cpu().numpy(), ref_idx)
         assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+
+
+# ---------------------------------------------------------------------------
+# bf16-stored block summaries
+
+DELTA_BF16 = 0.05  # one bf16 unit in one stored mean moves a score by at most ~0.02 here
+
+
+@pytest.mark.parametrize("D,bs", [(128, 16), (64, 32)])
+def test_summaries_bf16_storage(ksa, oracle, D, bs):
+    """bf16 storage = the fp32 mean rounded to nearest even, bit for bit; and within one
+    bf16 unit of the oracle's rounding of the exact mean.  LAST_BLOCK writes one block."""
+    rng = np.random.default_rng(1100 + D)
+    B, Hkv, T = 3, 2, 9 * bs + 3
+    K = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([T, 1, 2 * bs + 5], np.int32)
+    Kd, Ld = to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    S32 = ksa.ksa_build_block_summaries(Kd, Ld, bs)
+    S16 = ksa.ksa_build_block_summaries(Kd, Ld, bs, summary_dtype=torch.bfloat16)
+    assert S16.dtype == torch.bfloat16
+    ref = oracle.block_summaries_bf16(K, lens, bs).astype(np.int32)
+    got = S16.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.int32)
+    want = S32.to(torch.bfloat16).view(torch.int16).cpu().numpy().view(np.uint16).astype(np.int32)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        assert np.array_equal(got[b, :, :nb], want[b, :, :nb])
+        assert np.abs(got[b, :, :nb] - ref[b, :, :nb]).max() <= 1
+    S2 = torch.full_like(S16, float("nan"))
+    ksa.ksa_build_block_summaries(Kd, Ld, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S2)
+    S2 = S2.float().cpu().numpy()
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        np.testing.assert_array_equal(S2[b, :, nb - 1], S16[b, :, nb - 1].float().cpu().numpy())
+        assert np.all(np.isnan(S2[b, :, :nb - 1])) and np.all(np.isnan(S2[b, :, nb:]))
+
+
+@pytest.mark.parametrize("D,bs,k,nblk", [(128, 16, 8, 40), (64, 32, 6, 300), (128, 16, 32, 1100)])
+def test_select_blocks_bf16_summaries(ksa, oracle, D, bs, k, nblk):
+    """Selection from bf16-stored summaries: the oracle's blocks for bf16-stored means,
+    with a planted gap; the fused decode-step form refreshes the last block in bf16."""
+    rng = np.random.default_rng(1200 + nblk)
+    B, Hq, Hkv = 3, 8, 2
+    T = nblk * bs + 7
+    lens = np.array([T, 13 * bs + 1, 3 * bs], np.int32)
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    for b in range(B):
+        K[b], _ = gap_fix_row(oracle, q[b], K[b], int(lens[b]), bs, k, delta=DELTA_BF16,
+                              summary_bf16=True)
+        assert min_boundary_gap(oracle, q[b], K[b], int(lens[b]), bs, k,
+                                summary_bf16=True) >= DELTA_BF16
+    qd, Kd, Ld = to_dev_bf16(q), to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    st = status_tensor()
+    S = ksa.ksa_build_block_summaries(Kd, Ld, bs, summary_dtype=torch.bfloat16, dev_status=st)
+    idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k, dev_status=st)
+    ref_idx, ref_cnt = oracle.select_blocks(q, K, lens, bs, k, summary_bf16=True)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    # fused form: stale last blocks in the summaries, refreshed (in bf16) by the call
+    S_old = S.clone()
+    for b in range(B):
+        jl = (lens[b] - 1) // bs
+        S_old[b, :, jl] = 0
+    idx2, cnt2 = ksa.ksa_decode_select_blocks(qd, Kd, S_old, Ld, bs, k, dev_status=st)
+    # bit patterns: blocks past a row's end hold unwritten memory, possibly NaN patterns
+    assert torch.equal(S_old.view(torch.int16), S.view(torch.int16))
+    assert torch.equal(idx2, idx) and torch.equal(cnt2, cnt)
+    assert st.item() == 0
