@@ -144,6 +144,35 @@ void ksa_oracle_round_bf16_array(size_t n, const double *in, uint16_t *out) {
   for (size_t i = 0; i < n; ++i) out[i] = ksa_oracle_round_bf16(in[i]);
 }
 
+/*
+ * Paged KV cache (Kinetics section 5 integrates block top-k with paging: a
+ * page holds one block).  Pages are [num_pages, Hkv, bs, D]; block_table
+ * [B, max_blocks] names the page of logical block j of row b.  The logical
+ * cache [B, Hkv, T = max_blocks*bs, D] is, for every t < L_b,
+ *   K[b, g, t, :] = pages[block_table[b, t/bs], g, t % bs, :];
+ * slots t >= L_b, and blocks whose page id is outside [0, num_pages), are
+ * written as zero bits.  Every computation on a paged cache is the same
+ * computation on this gathered cache.
+ */
+void ksa_oracle_gather_pages(int B, int Hkv, int D, int bs, int max_blocks, int num_pages,
+                             const uint16_t *pages, const int32_t *block_table,
+                             const int32_t *seq_lens, uint16_t *K) {
+  const int T = max_blocks * bs;
+  memset(K, 0, sizeof(uint16_t) * (size_t)B * Hkv * T * D);
+  for (int b = 0; b < B; ++b) {
+    int L = seq_lens[b];
+    if (L > T) L = T;
+    for (int t = 0; t < L; ++t) {
+      const int page = block_table[(size_t)b * max_blocks + t / bs];
+      if (page < 0 || page >= num_pages) continue;
+      for (int g = 0; g < Hkv; ++g) {
+        const uint16_t *src = pages + (((size_t)page * Hkv + g) * bs + t % bs) * D;
+        memcpy(K + (((size_t)b * Hkv + g) * T + t) * D, src, sizeof(uint16_t) * (size_t)D);
+      }
+    }
+  }
+}
+
 /* ---- (A2) block scores -------------------------------------------------- */
 /*
  * Kinetics section 5: score every block against the query (R1, R2):

@@ -51,6 +51,7 @@ class Oracle:
                                                 _i32p, _i32p, nullable_f64])
         L.ksa_oracle_select_blocks_ex.argtypes = ([c_int] * 6 + [_u16p, _u16p, _i32p, c_int,
                                                    c_int, _i32p, _i32p, nullable_f64])
+        L.ksa_oracle_gather_pages.argtypes = [c_int] * 6 + [_u16p, _i32p, _i32p, _u16p]
         L.ksa_oracle_round_bf16.argtypes = [c_double]
         L.ksa_oracle_round_bf16.restype = ctypes.c_uint16
         L.ksa_oracle_round_bf16_array.argtypes = [ctypes.c_size_t, _f64p, _u16p]
@@ -81,6 +82,19 @@ class Oracle:
         self.lib.ksa_oracle_block_summaries(B, Hkv, T, D, bs, K,
                                             np.ascontiguousarray(seq_lens, np.int32), S)
         return S
+
+    def gather_pages(self, pages: np.ndarray, block_table: np.ndarray,
+                     seq_lens: np.ndarray) -> np.ndarray:
+        """Logical cache of a paged one: pages uint16 [P,Hkv,bs,D], block_table int32
+        [B,max_blocks] -> uint16 [B,Hkv,max_blocks*bs,D] (zero past L_b and for bad pages)."""
+        pages = np.ascontiguousarray(pages, dtype=np.uint16)
+        tbl = np.ascontiguousarray(block_table, dtype=np.int32)
+        P, Hkv, bs, D = pages.shape
+        B, mb = tbl.shape
+        K = np.empty((B, Hkv, mb * bs, D), np.uint16)
+        self.lib.ksa_oracle_gather_pages(B, Hkv, D, bs, mb, P, pages, tbl,
+                                         np.ascontiguousarray(seq_lens, np.int32), K)
+        return K
 
     def round_bf16(self, x) -> np.ndarray:
         """Nearest bf16 (ties to even) of fp64 values -> uint16 bit patterns, same shape."""

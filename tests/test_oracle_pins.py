@@ -578,3 +578,46 @@ def test_select_blocks_bf16_storage_exact_means(oracle):
     a = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, 7)
     b = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, 7, summary_bf16=True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------------------
+# paged KV cache: the logical cache the pages and the block table describe
+
+
+def test_gather_pages_identity_table(oracle):
+    """Pages laid out in row order with the identity table are the contiguous cache."""
+    rng = np.random.default_rng(41)
+    B, Hkv, D, bs, mb = 2, 3, 64, 16, 5
+    K = rng.integers(0, 1 << 16, size=(B, Hkv, mb * bs, D), dtype=np.uint16)
+    lens = np.array([mb * bs, 37], np.int32)
+    # page b*mb + j holds block j of row b, all kv-heads
+    pages = K.reshape(B, Hkv, mb, bs, D).transpose(0, 2, 1, 3, 4).reshape(B * mb, Hkv, bs, D)
+    tbl = np.arange(B * mb, dtype=np.int32).reshape(B, mb)
+    got = oracle.gather_pages(pages, tbl, lens)
+    for b in range(B):
+        assert np.array_equal(got[b, :, :lens[b]], K[b, :, :lens[b]])
+        assert not got[b, :, lens[b]:].any()
+
+
+def test_gather_pages_scatter_roundtrip_and_bad_pages(oracle):
+    """A random page placement reproduces the cache it was scattered from; a block whose
+    page id is out of range reads as zeros."""
+    rng = np.random.default_rng(42)
+    B, Hkv, D, bs, mb, P = 3, 2, 64, 32, 4, 20
+    K = rng.integers(0, 1 << 16, size=(B, Hkv, mb * bs, D), dtype=np.uint16)
+    lens = np.array([mb * bs, 70, 1], np.int32)
+    tbl = rng.permutation(P)[:B * mb].astype(np.int32).reshape(B, mb)
+    pages = rng.integers(0, 1 << 16, size=(P, Hkv, bs, D), dtype=np.uint16)
+    for b in range(B):
+        for j in range(mb):
+            for g in range(Hkv):
+                pages[tbl[b, j], g] = K[b, g, j * bs:(j + 1) * bs]
+    got = oracle.gather_pages(pages, tbl, lens)
+    for b in range(B):
+        assert np.array_equal(got[b, :, :lens[b]], K[b, :, :lens[b]])
+    tbl2 = tbl.copy()
+    tbl2[0, 1] = P          # out of range
+    tbl2[0, 2] = -1         # negative
+    got2 = oracle.gather_pages(pages, tbl2, lens)
+    assert not got2[0, :, bs:3 * bs].any()
+    assert np.array_equal(got2[0, :, :bs], K[0, :, :bs])
