@@ -26,6 +26,8 @@ __all__ = [
     "ksa_sparse_decode_attn_noalloc", "ksa_decode_select_blocks",
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
     "ksa_build_block_summaries_ex", "ksa_select_blocks_ex", "ksa_decode_select_blocks_ex",
+    "ksa_build_block_summaries_paged", "ksa_decode_select_blocks_paged",
+    "ksa_sparse_decode_attn_paged", "Pages",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -56,6 +58,12 @@ class Shape(ctypes.Structure):
                 ("capacity", ctypes.c_int32), ("block_size", ctypes.c_int32)]
 
 
+class Pages(ctypes.Structure):
+    """ksa_pages: the block table of a paged K/V cache (page = block)."""
+    _fields_ = [("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
+
+
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
     "ksa_build_block_summaries": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _i32, _vp, _vp, _vp]),
@@ -65,6 +73,14 @@ _SIGS = {
                                     _vp, _sz, _vp, _vp]),
     "ksa_decode_select_blocks_ex": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _i32,
                                            _vp, _vp, _vp, _sz, _vp, _vp]),
+    "ksa_build_block_summaries_paged": (_i32, [ctypes.POINTER(Shape), _vp, ctypes.POINTER(Pages),
+                                               _vp, _i32, _i32, _vp, _vp, _vp]),
+    "ksa_decode_select_blocks_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp,
+                                              ctypes.POINTER(Pages), _vp, _i32, _vp, _i32, _vp,
+                                              _vp, _vp, _sz, _vp, _vp]),
+    "ksa_sparse_decode_attn_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp,
+                                            ctypes.POINTER(Pages), _vp, _vp, _vp, _i32, _i32,
+                                            _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]),
@@ -373,3 +389,105 @@ def ksa_unified_select(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor,
         int(token_budget), int(recent_tokens), _ptr(token_idx), _ptr(num_sel), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
     return token_idx, num_sel
+
+
+# ---------------------------------------------------------------------------
+# paged K/V cache: pools [num_pages, Hkv, block_size, D] bf16 and a block table
+# [B, max_blocks] int32 naming the page of each logical block
+
+
+def _pages(block_table: torch.Tensor, num_pages: int) -> Pages:
+    _dev(block_table, "block_table", torch.int32)
+    return Pages(ctypes.c_void_p(block_table.data_ptr()), int(block_table.shape[1]),
+                 int(num_pages))
+
+
+def ksa_build_block_summaries_paged(K_pages: torch.Tensor, block_table: torch.Tensor,
+                                    seq_lens: torch.Tensor, mode: int = SUMMARY_ALL,
+                                    summaries: Optional[torch.Tensor] = None,
+                                    dev_status: Optional[torch.Tensor] = None, stream=None,
+                                    summary_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """ksa_build_block_summaries on a paged key cache; the page size is the block size."""
+    _dev(K_pages, "K_pages", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    P, Hkv, bs, D = K_pages.shape
+    B, mb = block_table.shape
+    if summaries is None:
+        summaries = torch.empty((B, Hkv, mb, D), dtype=summary_dtype, device=K_pages.device)
+    _dev(summaries, "summaries", summaries.dtype)
+    sh = _shape(B, Hkv, Hkv, D, mb * bs, bs)
+    pg = _pages(block_table, P)
+    _check(lib().ksa_build_block_summaries_paged(
+        ctypes.byref(sh), _ptr(K_pages), ctypes.byref(pg), _ptr(seq_lens), int(mode),
+        _summary_dtype(summaries), _ptr(summaries), _ptr(dev_status), _stream(stream)))
+    return summaries
+
+
+def ksa_decode_select_blocks_paged(q: torch.Tensor, K_pages: torch.Tensor,
+                                   block_table: torch.Tensor, summaries: torch.Tensor,
+                                   seq_lens: torch.Tensor, k_blocks: int,
+                                   block_idx: Optional[torch.Tensor] = None,
+                                   num_sel: Optional[torch.Tensor] = None,
+                                   workspace: Optional[torch.Tensor] = None,
+                                   dev_status: Optional[torch.Tensor] = None, stream=None):
+    """ksa_decode_select_blocks on a paged key cache."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K_pages, "K_pages", torch.bfloat16)
+    _dev(summaries, "summaries", summaries.dtype)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    P, Hkv, bs, _ = K_pages.shape
+    mb = block_table.shape[1]
+    if block_idx is None:
+        block_idx = torch.empty((B, Hkv, k_blocks), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    sh = _shape(B, Hq, Hkv, D, mb * bs, bs)
+    pg = _pages(block_table, P)
+    ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
+                    q.device)
+    _check(lib().ksa_decode_select_blocks_paged(
+        ctypes.byref(sh), _ptr(q), _ptr(K_pages), ctypes.byref(pg), _ptr(summaries),
+        _summary_dtype(summaries), _ptr(seq_lens), int(k_blocks), _ptr(block_idx), _ptr(num_sel),
+        _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+    return block_idx, num_sel
+
+
+def ksa_sparse_decode_attn_paged(q: torch.Tensor, K_pages: torch.Tensor, V_pages: torch.Tensor,
+                                 block_table: torch.Tensor, seq_lens: torch.Tensor,
+                                 idx: Optional[torch.Tensor] = None,
+                                 num_idx: Optional[torch.Tensor] = None, tokens_per_idx: int = 1,
+                                 idx_shared: bool = False, scale: float = 0.0,
+                                 out_dtype: int = OUT_F32, out: Optional[torch.Tensor] = None,
+                                 lse: Optional[torch.Tensor] = None,
+                                 workspace: Optional[torch.Tensor] = None,
+                                 dev_status: Optional[torch.Tensor] = None, stream=None):
+    """ksa_sparse_decode_attn on a paged K/V cache: (out, lse)."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K_pages, "K_pages", torch.bfloat16)
+    _dev(V_pages, "V_pages", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    P, Hkv, bs, _ = K_pages.shape
+    mb = block_table.shape[1]
+    odt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=odt, device=q.device)
+    _dev(out, "out", odt)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32)
+    cap = 0
+    if idx is not None:
+        _dev(idx, "idx", torch.int32)
+        _dev(num_idx, "num_idx", torch.int32)
+        cap = idx.shape[-1]
+    sh = _shape(B, Hq, Hkv, D, mb * bs, bs)
+    pg = _pages(block_table, P)
+    ws = _workspace(workspace, lib().ksa_sparse_decode_attn_workspace(
+        ctypes.byref(sh), int(cap), int(tokens_per_idx)), q.device)
+    _check(lib().ksa_sparse_decode_attn_paged(
+        ctypes.byref(sh), _ptr(q), _ptr(K_pages), _ptr(V_pages), ctypes.byref(pg),
+        _ptr(seq_lens), _ptr(idx), _ptr(num_idx), int(cap), int(tokens_per_idx),
+        int(bool(idx_shared)), float(scale), int(out_dtype), _ptr(out), _ptr(lse), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+    return out, lse

@@ -275,13 +275,14 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
           }
           if (r > r_last) break;
           const int j = ja + (i - row_base);
-          long long t0[kTiles];
+          long long t0[kTiles], yr[kTiles];
           int nv[kTiles];
           uint32_t mask = 0u, bytes = 0u;
 #pragma unroll
           for (int u = 0; u < kTiles; ++u) {  // nseg <= kTiles segments
             nv[u] = 0;
             t0[u] = 0;
+            yr[u] = 0;
             if (u >= nseg) continue;
             bool ok = true;
             if (MODE == kModeDense) {
@@ -300,6 +301,13 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
             }
             const long long left = ri.L - t0[u];
             nv[u] = (!ok || left <= 0) ? 0 : (left < seg ? static_cast<int>(left) : seg);
+            if (nv[u] > 0) {  // the segment's first K/V row (its page, when paged)
+              yr[u] = kv_row(a.kv, r / a.Hkv, r % a.Hkv, a.Hkv, a.T, t0[u]);
+              if (yr[u] < 0) {
+                nv[u] = 0;
+                skipped = KSA_FLAG_INDEX_SKIPPED;
+              }
+            }
             if (nv[u] > 0) {
               mask |= (nv[u] >= 32 ? 0xffffffffu : ((1u << nv[u]) - 1u)) << (u * seg);
               bytes += static_cast<uint32_t>(seg) * 128u * C::kHalves * 2u;
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
 #pragma unroll
           for (int u = 0; u < kTiles; ++u) {
             if (nv[u] <= 0) continue;
-            const int yrow = static_cast<int>(static_cast<long long>(r) * a.T + t0[u]);
+            const int yrow = static_cast<int>(yr[u]);
 #pragma unroll
             for (int h = 0; h < C::kHalves; ++h) {
               tma_load_2d(sK + h * C::kHalfBytes + u * seg * 128, &kmap, h * 64, yrow, &full[lane]);
@@ -373,13 +381,20 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
           const int e = j * eps + lane / tpi;
           const int id = __shfl_sync(0xffffffffu, cur, (e - wbase) & 31);
           bool valid = false;
-          long long t = 0;
+          long long trow = 0;  // the token's K/V row
           if (lane < kStageTok && e < ri.n_idx) {
-            t = static_cast<long long>(id) * tpi + (lane % tpi);
+            const long long t = static_cast<long long>(id) * tpi + (lane % tpi);
             valid = id >= 0 && t < ri.L;
             if (!valid && (lane % tpi) == 0 &&
                 (id < 0 || static_cast<long long>(id) * tpi >= ri.L))
               skipped = KSA_FLAG_INDEX_SKIPPED;
+            if (valid) {
+              trow = kv_row(a.kv, r / a.Hkv, r % a.Hkv, a.Hkv, a.T, t);
+              if (trow < 0) {  // its page id names no page
+                valid = false;
+                skipped = KSA_FLAG_INDEX_SKIPPED;
+              }
+            }
           }
           const uint32_t mask = __ballot_sync(0xffffffffu, valid);
           constexpr int CH = D / 8;     // 16-byte chunks per row
@@ -388,9 +403,9 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
           for (int q0 = 0; q0 < kStageTok; q0 += RPW) {
             const int u = q0 + lane / CH;
             const int uv = __shfl_sync(0xffffffffu, static_cast<int>(valid), u);
-            const long long ut = __shfl_sync(0xffffffffu, t, u);
+            const long long ur = __shfl_sync(0xffffffffu, trow, u);
             if (uv) {
-              const size_t src = (static_cast<size_t>(r) * a.T + ut) * D + my_c * 8;
+              const size_t src = static_cast<size_t>(ur) * D + my_c * 8;
               const uint32_t off = (my_c >> 3) * C::kHalfBytes + swz128(u, my_c & 7);
               cp_async_16(sK + off, a.K + src);
               cp_async_16(sV + off, a.V + src);
@@ -670,7 +685,9 @@ cudaError_t launch_sparse_decode_attn(const AttnArgs &a, void *ws, int num_sms,
   memset(&vm, 0, sizeof vm);
   if (mode != kModeCp) {
     const int box_rows = (mode == kModeDense || a.tpi >= kStageTok) ? kStageTok : a.tpi;
-    const uint64_t rows = static_cast<uint64_t>(a.B) * a.Hkv * a.T;
+    const uint64_t rows = a.kv.table != nullptr
+                              ? static_cast<uint64_t>(a.kv.num_pages) * a.Hkv * a.kv.bs
+                              : static_cast<uint64_t>(a.B) * a.Hkv * a.T;
     if (!encode_kv_tensor_map(&km, a.K, rows, a.D, box_rows) ||
         !encode_kv_tensor_map(&vm, a.V, rows, a.D, box_rows))
       return cudaErrorInvalidValue;

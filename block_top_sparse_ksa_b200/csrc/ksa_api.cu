@@ -120,10 +120,32 @@ bool encode_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int
 
 extern "C" {
 
-ksa_status ksa_build_block_summaries_ex(const ksa_shape *shape, const uint16_t *K,
-                                        const int32_t *seq_lens, int32_t mode,
-                                        int32_t summary_dtype, void *summaries,
-                                        uint32_t *dev_status, void *stream) {
+namespace {
+
+// Validates the page pool of a paged cache and fills the kernels' layout.
+ksa_status check_pages(const ksa_shape *shape, const ksa_pages *pages, ksa::KvLayout *kv) {
+  if (pages == nullptr || pages->block_table == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "pages and pages->block_table must be non-NULL");
+  if (pages->max_blocks < 1 || pages->num_pages < 1)
+    return fail(KSA_ERR_INVALID_ARG, "max_blocks and num_pages must be >= 1");
+  if (static_cast<long long>(pages->max_blocks) * shape->block_size != shape->capacity)
+    return fail(KSA_ERR_INVALID_ARG, "capacity %d must equal max_blocks * block_size (%d * %d)",
+                shape->capacity, pages->max_blocks, shape->block_size);
+  if (static_cast<long long>(pages->num_pages) * shape->num_kv_heads * shape->block_size >=
+      (1LL << 31))
+    return fail(KSA_ERR_UNSUPPORTED, "num_pages * num_kv_heads * block_size must be < 2^31");
+  if (!aligned(pages->block_table, 4))
+    return fail(KSA_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+  kv->table = pages->block_table;
+  kv->max_blocks = pages->max_blocks;
+  kv->num_pages = pages->num_pages;
+  kv->bs = shape->block_size;
+  return KSA_OK;
+}
+
+ksa_status summaries_common(const ksa_shape *shape, const uint16_t *K, const ksa_pages *pages,
+                            const int32_t *seq_lens, int32_t mode, int32_t summary_dtype,
+                            void *summaries, uint32_t *dev_status, void *stream) {
   ksa_status st = check_shape(shape, true);
   if (st != KSA_OK) return st;
   if (K == nullptr || seq_lens == nullptr || summaries == nullptr)
@@ -135,6 +157,7 @@ ksa_status ksa_build_block_summaries_ex(const ksa_shape *shape, const uint16_t *
   if (!aligned(K, 16) || !aligned(summaries, 16) || !aligned(seq_lens, 4))
     return fail(KSA_ERR_INVALID_ARG, "K and summaries must be 16-byte aligned");
   ksa::SummaryArgs a;
+  if (pages != nullptr && (st = check_pages(shape, pages, &a.kv)) != KSA_OK) return st;
   a.K = K;
   a.seq_lens = seq_lens;
   a.S = summaries;
@@ -148,6 +171,25 @@ ksa_status ksa_build_block_summaries_ex(const ksa_shape *shape, const uint16_t *
   a.mode = mode;
   return cuda_status(ksa::launch_block_summaries(a, static_cast<cudaStream_t>(stream)),
                      "ksa_build_block_summaries launch");
+}
+
+}  // namespace
+
+ksa_status ksa_build_block_summaries_ex(const ksa_shape *shape, const uint16_t *K,
+                                        const int32_t *seq_lens, int32_t mode,
+                                        int32_t summary_dtype, void *summaries,
+                                        uint32_t *dev_status, void *stream) {
+  return summaries_common(shape, K, nullptr, seq_lens, mode, summary_dtype, summaries,
+                          dev_status, stream);
+}
+
+ksa_status ksa_build_block_summaries_paged(const ksa_shape *shape, const uint16_t *K_pages,
+                                           const ksa_pages *pages, const int32_t *seq_lens,
+                                           int32_t mode, int32_t summary_dtype, void *summaries,
+                                           uint32_t *dev_status, void *stream) {
+  if (pages == nullptr) return fail(KSA_ERR_INVALID_ARG, "pages must be non-NULL");
+  return summaries_common(shape, K_pages, pages, seq_lens, mode, summary_dtype, summaries,
+                          dev_status, stream);
 }
 
 ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,
@@ -168,7 +210,8 @@ namespace {
 
 // Shared by the selection entry points; K non-NULL fuses the last-block refresh.
 ksa_status select_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
-                         void *summaries, int32_t summary_dtype, const int32_t *seq_lens,
+                         const ksa_pages *pages, void *summaries, int32_t summary_dtype,
+                         const int32_t *seq_lens,
                          int32_t k_blocks, int32_t *block_idx, int32_t *num_sel, void *ws,
                          size_t ws_bytes, uint32_t *dev_status, void *stream, const char *what) {
   ksa_status st = check_shape(shape, true);
@@ -190,6 +233,7 @@ ksa_status select_common(const ksa_shape *shape, const uint16_t *q, const uint16
     return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   ksa::SelectArgs a;
+  if (pages != nullptr && (st = check_pages(shape, pages, &a.kv)) != KSA_OK) return st;
   a.q = q;
   a.S = summaries;  // written only when K is given (the fused refresh)
   a.sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
@@ -216,7 +260,8 @@ ksa_status ksa_select_blocks_ex(const ksa_shape *shape, const uint16_t *q, const
                                 int32_t *block_idx, int32_t *num_sel, void *ws, size_t ws_bytes,
                                 uint32_t *dev_status, void *stream) {
   // read only: no K is given, so nothing is refreshed
-  return select_common(shape, q, nullptr, const_cast<void *>(summaries), summary_dtype, seq_lens,
+  return select_common(shape, q, nullptr, nullptr, const_cast<void *>(summaries), summary_dtype,
+                       seq_lens,
                        k_blocks, block_idx, num_sel, ws, ws_bytes, dev_status, stream,
                        "ksa_select_blocks launch");
 }
@@ -236,8 +281,23 @@ ksa_status ksa_decode_select_blocks_ex(const ksa_shape *shape, const uint16_t *q
                                        size_t ws_bytes, uint32_t *dev_status, void *stream) {
   if (K == nullptr) return fail(KSA_ERR_INVALID_ARG, "K must be non-NULL");
   if (!aligned(K, 16)) return fail(KSA_ERR_INVALID_ARG, "K must be 16-byte aligned");
-  return select_common(shape, q, K, summaries, summary_dtype, seq_lens, k_blocks, block_idx,
-                       num_sel, ws, ws_bytes, dev_status, stream, "ksa_decode_select_blocks launch");
+  return select_common(shape, q, K, nullptr, summaries, summary_dtype, seq_lens, k_blocks,
+                       block_idx, num_sel, ws, ws_bytes, dev_status, stream,
+                       "ksa_decode_select_blocks launch");
+}
+
+ksa_status ksa_decode_select_blocks_paged(const ksa_shape *shape, const uint16_t *q,
+                                          const uint16_t *K_pages, const ksa_pages *pages,
+                                          void *summaries, int32_t summary_dtype,
+                                          const int32_t *seq_lens, int32_t k_blocks,
+                                          int32_t *block_idx, int32_t *num_sel, void *ws,
+                                          size_t ws_bytes, uint32_t *dev_status, void *stream) {
+  if (K_pages == nullptr || pages == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "K_pages and pages must be non-NULL");
+  if (!aligned(K_pages, 16)) return fail(KSA_ERR_INVALID_ARG, "K_pages must be 16-byte aligned");
+  return select_common(shape, q, K_pages, pages, summaries, summary_dtype, seq_lens, k_blocks,
+                       block_idx, num_sel, ws, ws_bytes, dev_status, stream,
+                       "ksa_decode_select_blocks_paged launch");
 }
 
 ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
@@ -258,13 +318,15 @@ size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape, int32_t idx_capa
                                    shape->head_dim, device_sm_count());
 }
 
-ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
-                                  const uint16_t *V, const int32_t *seq_lens, const int32_t *idx,
-                                  const int32_t *num_idx, int32_t idx_capacity,
-                                  int32_t tokens_per_idx, int32_t idx_shared, float scale,
-                                  int32_t out_dtype, void *out, float *lse, void *ws,
-                                  size_t ws_bytes, uint32_t *dev_status, void *stream) {
-  ksa_status st = check_shape(shape, false);
+namespace {
+
+ksa_status attn_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                       const uint16_t *V, const ksa_pages *pages, const int32_t *seq_lens,
+                       const int32_t *idx, const int32_t *num_idx, int32_t idx_capacity,
+                       int32_t tokens_per_idx, int32_t idx_shared, float scale, int32_t out_dtype,
+                       void *out, float *lse, void *ws, size_t ws_bytes, uint32_t *dev_status,
+                       void *stream) {
+  ksa_status st = check_shape(shape, pages != nullptr);
   if (st != KSA_OK) return st;
   if (q == nullptr || K == nullptr || V == nullptr || seq_lens == nullptr || out == nullptr)
     return fail(KSA_ERR_INVALID_ARG, "q, K, V, seq_lens and out must be non-NULL");
@@ -297,6 +359,7 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, con
     return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   ksa::AttnArgs a;
+  if (pages != nullptr && (st = check_pages(shape, pages, &a.kv)) != KSA_OK) return st;
   a.q = q;
   a.K = K;
   a.V = V;
@@ -320,6 +383,33 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, con
   return cuda_status(
       ksa::launch_sparse_decode_attn(a, ws, sms, static_cast<cudaStream_t>(stream)),
       "ksa_sparse_decode_attn launch");
+}
+
+}  // namespace
+
+ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                                  const uint16_t *V, const int32_t *seq_lens, const int32_t *idx,
+                                  const int32_t *num_idx, int32_t idx_capacity,
+                                  int32_t tokens_per_idx, int32_t idx_shared, float scale,
+                                  int32_t out_dtype, void *out, float *lse, void *ws,
+                                  size_t ws_bytes, uint32_t *dev_status, void *stream) {
+  return attn_common(shape, q, K, V, nullptr, seq_lens, idx, num_idx, idx_capacity,
+                     tokens_per_idx, idx_shared, scale, out_dtype, out, lse, ws, ws_bytes,
+                     dev_status, stream);
+}
+
+ksa_status ksa_sparse_decode_attn_paged(const ksa_shape *shape, const uint16_t *q,
+                                        const uint16_t *K_pages, const uint16_t *V_pages,
+                                        const ksa_pages *pages, const int32_t *seq_lens,
+                                        const int32_t *idx, const int32_t *num_idx,
+                                        int32_t idx_capacity, int32_t tokens_per_idx,
+                                        int32_t idx_shared, float scale, int32_t out_dtype,
+                                        void *out, float *lse, void *ws, size_t ws_bytes,
+                                        uint32_t *dev_status, void *stream) {
+  if (pages == nullptr) return fail(KSA_ERR_INVALID_ARG, "pages must be non-NULL");
+  return attn_common(shape, q, K_pages, V_pages, pages, seq_lens, idx, num_idx, idx_capacity,
+                     tokens_per_idx, idx_shared, scale, out_dtype, out, lse, ws, ws_bytes,
+                     dev_status, stream);
 }
 
 size_t ksa_unified_select_workspace(const ksa_shape *shape, int32_t per_head_topk,

@@ -12,6 +12,28 @@
 
 namespace ksa {
 
+// Where the K/V rows of (row b, kv-head g, token t) live: a contiguous cache
+// [B, Hkv, T, D] (table == nullptr), or a paged one [num_pages, Hkv, bs, D]
+// whose block_table [B, max_blocks] names the page of logical block t / bs.
+struct KvLayout {
+  const int32_t *table = nullptr;
+  int max_blocks = 0;
+  int num_pages = 0;
+  int bs = 0;
+};
+
+#ifdef __CUDACC__
+// Row (in units of D elements) holding token t of (b, g); -1 when the block's
+// page id is outside [0, num_pages) (nothing may be read for it).
+__device__ __forceinline__ long long kv_row(const KvLayout &kv, int b, int g, int Hkv, int T,
+                                            long long t) {
+  if (kv.table == nullptr) return (static_cast<long long>(b) * Hkv + g) * T + t;
+  const int page = __ldg(kv.table + static_cast<size_t>(b) * kv.max_blocks + t / kv.bs);
+  if (page < 0 || page >= kv.num_pages) return -1;
+  return (static_cast<long long>(page) * Hkv + g) * kv.bs + t % kv.bs;
+}
+#endif
+
 struct SummaryArgs {
   const uint16_t *K;
   const int32_t *seq_lens;
@@ -19,6 +41,7 @@ struct SummaryArgs {
   int sbf16;  // summaries stored as bf16
   uint32_t *status;
   int B, Hkv, T, D, bs, mode;
+  KvLayout kv;
 };
 cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream);
 
@@ -31,6 +54,7 @@ struct SelectArgs {
   int32_t *num_sel;
   uint32_t *status;
   int B, Hq, Hkv, D, T, bs, k;
+  KvLayout kv;  // of the key cache given for the fused refresh
 };
 // workspace: semaphores [B*Hkv] (zero between calls) + score keys [B*Hkv, ceil(T/bs)]
 size_t select_workspace_bytes(int B, int Hkv, int T, int bs);
@@ -50,6 +74,7 @@ struct AttnArgs {
   int B, Hq, Hkv, D, T;
   int cap, tpi, shared;
   float scale;
+  KvLayout kv;
 };
 // Resident CTAs per SM the attention workspace is sized for (the launch never exceeds it).
 constexpr int kAttnMaxCtasPerSm = 4;

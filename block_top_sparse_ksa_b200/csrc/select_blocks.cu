@@ -78,8 +78,18 @@ __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const ui
                                                    int row, int L, int nb, float (&mean)[8]) {
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   const int jl = nb - 1;
-  const uint16_t *rows = K + (static_cast<size_t>(row) * a.T + static_cast<size_t>(jl) * a.bs) * D;
-  const bool mine = warp_block_mean<D>(rows, L - jl * a.bs, mean);
+  const int b = row / a.Hkv;
+  const long long row0 = kv_row(a.kv, b, row - b * a.Hkv, a.Hkv, a.T,
+                                static_cast<long long>(jl) * a.bs);
+  bool mine;
+  if (row0 < 0) {  // a page id that names no page: flagged, the block reads as zeros
+    if ((threadIdx.x & 31) == 0) flag_status(a.status, KSA_FLAG_INDEX_SKIPPED);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mean[i] = 0.f;
+    mine = (threadIdx.x & 31) < D / 8;
+  } else {
+    mine = warp_block_mean<D>(K + static_cast<size_t>(row0) * D, L - jl * a.bs, mean);
+  }
   if (mine)
     store_mean8(a.S, a.sbf16, (static_cast<size_t>(row) * nb_max + jl) * D,
                 ((threadIdx.x & 31) % (D / 8)) * 8, mean);

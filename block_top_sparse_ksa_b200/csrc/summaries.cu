@@ -43,9 +43,18 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
     }
     const int n = min(a.bs, L - j * a.bs);
     float mean[8];
-    const uint16_t *rows =
-        a.K + (static_cast<size_t>(bg) * a.T + static_cast<size_t>(j) * a.bs) * D;
-    if (warp_block_mean<D>(rows, n, mean))
+    const long long row0 = kv_row(a.kv, b, static_cast<int>(bg - static_cast<long long>(b) * a.Hkv),
+                                  a.Hkv, a.T, static_cast<long long>(j) * a.bs);
+    bool mine;
+    if (row0 < 0) {  // a page id that names no page: flagged, the block reads as zeros
+      if (lane == 0) flag_status(a.status, KSA_FLAG_INDEX_SKIPPED);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mean[i] = 0.f;
+      mine = lane < D / 8;
+    } else {
+      mine = warp_block_mean<D>(a.K + static_cast<size_t>(row0) * D, n, mean);
+    }
+    if (mine)
       store_mean8(a.S, a.sbf16, (static_cast<size_t>(bg) * nb_max + j) * D, (lane % (D / 8)) * 8,
                   mean);
   }

@@ -162,6 +162,35 @@ ksa_status ksa_decode_select_blocks_ex(const ksa_shape *shape, const uint16_t *q
                                        uint32_t *dev_status, void *stream);
 
 /*
+ * Paged KV cache [KIN s.5 pairs block top-k with paged attention; here a page
+ * holds one block].  K and V are a pool of pages [num_pages, Hkv, block_size, D]
+ * bf16; block_table[b * max_blocks + j] is the page of logical block j of row
+ * b, so token t of row b, kv-head g is pages[block_table[b, t / bs], g, t % bs].
+ * The logical capacity T (shape->capacity) must equal max_blocks * block_size.
+ * The block table is device data: a page id outside [0, num_pages) is never
+ * read; it sets KSA_FLAG_INDEX_SKIPPED, its block summarises to zeros, and its
+ * tokens are left out of attention.
+ */
+typedef struct {
+  const int32_t *block_table; /* [B, max_blocks] int32, device */
+  int32_t max_blocks;         /* entries per row of the table */
+  int32_t num_pages;          /* pages in the K and V pools */
+} ksa_pages;
+
+/* ksa_build_block_summaries_ex on a paged key cache (K_pages, pages). */
+ksa_status ksa_build_block_summaries_paged(const ksa_shape *shape, const uint16_t *K_pages,
+                                           const ksa_pages *pages, const int32_t *seq_lens,
+                                           int32_t mode, int32_t summary_dtype, void *summaries,
+                                           uint32_t *dev_status, void *stream);
+/* ksa_decode_select_blocks_ex on a paged key cache (the last-block refresh reads pages). */
+ksa_status ksa_decode_select_blocks_paged(const ksa_shape *shape, const uint16_t *q,
+                                          const uint16_t *K_pages, const ksa_pages *pages,
+                                          void *summaries, int32_t summary_dtype,
+                                          const int32_t *seq_lens, int32_t k_blocks,
+                                          int32_t *block_idx, int32_t *num_sel, void *ws,
+                                          size_t ws_bytes, uint32_t *dev_status, void *stream);
+
+/*
  * Sparse decode attention over a selected token set [KIN s.5; LIM s.5
  * "sparse attention layer", GQA kernel sharing one KV set per group].
  * For query head h of row b (kv-head g = h / G) and selected tokens T_sel:
@@ -194,6 +223,21 @@ ksa_status ksa_sparse_decode_attn(const ksa_shape *shape, const uint16_t *q,
                                   float scale, int32_t out_dtype, void *out,
                                   float *lse, void *ws, size_t ws_bytes,
                                   uint32_t *dev_status, void *stream);
+
+/*
+ * ksa_sparse_decode_attn on a paged K/V cache (K_pages, V_pages share the
+ * block table in `pages`; see "Paged KV cache" above).  shape->block_size is
+ * the page size and must be 16, 32 or 64; the workspace is the same as for
+ * ksa_sparse_decode_attn.
+ */
+ksa_status ksa_sparse_decode_attn_paged(const ksa_shape *shape, const uint16_t *q,
+                                        const uint16_t *K_pages, const uint16_t *V_pages,
+                                        const ksa_pages *pages, const int32_t *seq_lens,
+                                        const int32_t *idx, const int32_t *num_idx,
+                                        int32_t idx_capacity, int32_t tokens_per_idx,
+                                        int32_t idx_shared, float scale, int32_t out_dtype,
+                                        void *out, float *lse, void *ws, size_t ws_bytes,
+                                        uint32_t *dev_status, void *stream);
 
 /*
  * ksa_sparse_decode_attn without a workspace argument: the same computation,

@@ -546,3 +546,127 @@ def test_select_blocks_bf16_summaries(ksa, oracle, D, bs, k, nblk):
     assert torch.equal(S_old.view(torch.int16), S.view(torch.int16))
     assert torch.equal(idx2, idx) and torch.equal(cnt2, cnt)
     assert st.item() == 0
+
+
+# ---------------------------------------------------------------------------
+# paged K/V cache (page = block)
+
+
+def _paged_case(rng, B, Hkv, D, bs, mb, extra_pages):
+    """A page pool larger than needed, blocks placed on random distinct pages."""
+    P = B * mb + extra_pages
+    K_pages = rand_bits(rng, (P, Hkv, bs, D))
+    V_pages = rand_bits(rng, (P, Hkv, bs, D))
+    tbl = rng.permutation(P)[:B * mb].astype(np.int32).reshape(B, mb)
+    return K_pages, V_pages, tbl
+
+
+def _scatter(K, tbl, pages, bs):
+    for b in range(K.shape[0]):
+        for j in range(tbl.shape[1]):
+            pages[tbl[b, j]] = K[b, :, j * bs:(j + 1) * bs]
+
+
+@pytest.mark.parametrize("D,bs,k", [(128, 16, 8), (64, 32, 5)])
+def test_paged_kv_matches_gathered_cache(ksa, oracle, D, bs, k):
+    """Every paged entry point equals its contiguous form on the gathered cache, bit for bit,
+    and the oracle on it: summaries, the fused decode selection, and attention over block
+    lists, token lists and the dense set."""
+    rng = np.random.default_rng(1300 + D)
+    B, Hq, Hkv, mb = 3, 8, 2, 40
+    T = mb * bs
+    lens = np.array([T, 13 * bs + 1, 5], np.int32)
+    K_pages, V_pages, tbl = _paged_case(rng, B, Hkv, D, bs, mb, extra_pages=17)
+    q = rand_bits(rng, (B, Hq, D))
+    K = oracle.gather_pages(K_pages, tbl, lens)
+    for b in range(B):  # plant the score gap on the logical cache, then write it back
+        K[b], _ = gap_fix_row(oracle, q[b], K[b], int(lens[b]), bs, k)
+    _scatter(K, tbl, K_pages, bs)
+    K = oracle.gather_pages(K_pages, tbl, lens)
+    V = oracle.gather_pages(V_pages, tbl, lens)
+    qd, Ld = to_dev_bf16(q), torch.from_numpy(lens).to(DEV)
+    Kp, Vp = to_dev_bf16(K_pages), to_dev_bf16(V_pages)
+    Kc, Vc = to_dev_bf16(K), to_dev_bf16(V)
+    td = torch.from_numpy(tbl).to(DEV)
+    st = status_tensor()
+    S_p = ksa.ksa_build_block_summaries_paged(Kp, td, Ld, dev_status=st)
+    S_c = ksa.ksa_build_block_summaries(Kc, Ld, bs)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        assert torch.equal(S_p[b, :, :nb], S_c[b, :, :nb])
+    # fused decode selection from stale last blocks
+    S_old = S_p.clone()
+    for b in range(B):
+        S_old[b, :, (lens[b] - 1) // bs] = 0.0
+    idx, cnt = ksa.ksa_decode_select_blocks_paged(qd, Kp, td, S_old, Ld, k, dev_status=st)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        assert torch.equal(S_old[b, :, :nb], S_p[b, :, :nb])
+    ref_idx, ref_cnt = oracle.select_blocks(q, K, lens, bs, k)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    # attention: block list
+    out_p, _ = ksa.ksa_sparse_decode_attn_paged(qd, Kp, Vp, td, Ld, idx, cnt, tokens_per_idx=bs,
+                                                dev_status=st)
+    out_c, _ = ksa.ksa_sparse_decode_attn(qd, Kc, Vc, Ld, idx, cnt, tokens_per_idx=bs)
+    assert torch.equal(out_p, out_c)
+    ref, _, _ = oracle.attention(q, K, V, lens, ref_idx, ref_cnt, bs)
+    assert_out_close(out_p.cpu().numpy(), ref)
+    # token list shared by the kv-heads, and the dense set
+    lst = np.full((B, 64), -1, np.int32)
+    n_t = np.zeros((B,), np.int32)
+    for b in range(B):
+        pick = np.sort(rng.choice(int(lens[b]), size=min(64, int(lens[b])), replace=False))
+        lst[b, :len(pick)] = pick
+        n_t[b] = len(pick)
+    lst_d, n_d = torch.from_numpy(lst).to(DEV), torch.from_numpy(n_t).to(DEV)
+    out_p, _ = ksa.ksa_sparse_decode_attn_paged(qd, Kp, Vp, td, Ld, lst_d, n_d, tokens_per_idx=1,
+                                                idx_shared=True, dev_status=st)
+    out_c, _ = ksa.ksa_sparse_decode_attn(qd, Kc, Vc, Ld, lst_d, n_d, tokens_per_idx=1,
+                                          idx_shared=True)
+    assert torch.equal(out_p, out_c)
+    out_p, _ = ksa.ksa_sparse_decode_attn_paged(qd, Kp, Vp, td, Ld, dev_status=st)
+    out_c, _ = ksa.ksa_sparse_decode_attn(qd, Kc, Vc, Ld)
+    assert torch.equal(out_p, out_c)
+    ref, _, _ = oracle.attention(q, K, V, lens)
+    assert_out_close(out_p.cpu().numpy(), ref)
+    assert st.item() == 0
+
+
+def test_paged_kv_bad_page_ids_are_flagged_not_read(ksa, oracle):
+    """A block whose page id is outside the pool is never read: its summary is zero, its
+    tokens are left out of attention, and the status word says so."""
+    rng = np.random.default_rng(1400)
+    B, Hq, Hkv, D, bs, mb, k = 2, 4, 2, 128, 16, 12, 4
+    lens = np.array([mb * bs, 7 * bs], np.int32)
+    K_pages, V_pages, tbl = _paged_case(rng, B, Hkv, D, bs, mb, extra_pages=3)
+    P = K_pages.shape[0]
+    bad = tbl.copy()
+    bad[0, 3] = P          # one past the pool
+    bad[1, 6] = -5         # negative: the last block of row 1
+    qd, Ld = to_dev_bf16(rand_bits(rng, (B, Hq, D))), torch.from_numpy(lens).to(DEV)
+    Kp, Vp, td = to_dev_bf16(K_pages), to_dev_bf16(V_pages), torch.from_numpy(bad).to(DEV)
+    st = status_tensor()
+    S = ksa.ksa_build_block_summaries_paged(Kp, td, Ld, dev_status=st)
+    assert st.item() & ksa.FLAG_INDEX_SKIPPED
+    assert not S[0, :, 3].any() and not S[1, :, 6].any()
+    st.zero_()
+    idx, cnt = ksa.ksa_decode_select_blocks_paged(qd, Kp, td, S, Ld, k, dev_status=st)
+    assert st.item() & ksa.FLAG_INDEX_SKIPPED  # the refresh of row 1's last block
+    st.zero_()
+    all_idx = torch.arange(mb, dtype=torch.int32, device=DEV).repeat(B, Hkv, 1)
+    all_cnt = torch.tensor([[mb] * Hkv, [7] * Hkv], dtype=torch.int32, device=DEV)
+    out, lse = ksa.ksa_sparse_decode_attn_paged(qd, Kp, Vp, td, Ld, all_idx, all_cnt,
+                                                tokens_per_idx=bs,
+                                                lse=torch.empty((B, Hq), device=DEV),
+                                                dev_status=st)
+    assert st.item() & ksa.FLAG_INDEX_SKIPPED
+    assert torch.isfinite(out).all()
+    # the same attention over a table whose bad blocks are simply not selected
+    keep = [j for j in range(mb) if j != 3]
+    sel = torch.tensor(keep + [-1], dtype=torch.int32, device=DEV).repeat(1, Hkv, 1)
+    cnt0 = torch.tensor([[len(keep)] * Hkv], dtype=torch.int32, device=DEV)
+    out0, _ = ksa.ksa_sparse_decode_attn_paged(qd[:1], Kp, Vp, td[:1], Ld[:1], sel, cnt0,
+                                               tokens_per_idx=bs)
+    # (another batch splits the work differently, so fp32 sums differ in the last bits)
+    torch.testing.assert_close(out[:1], out0, atol=1e-5, rtol=1e-5)
