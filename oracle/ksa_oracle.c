@@ -281,6 +281,25 @@ void ksa_oracle_select_blocks(int B, int Hq, int Hkv, int D, int T, int bs,
                               num_sel, scores_out);
 }
 
+/*
+ * Kinetics section 5 compares block top-k with local attention, a fixed
+ * pattern that attends only to the nearest tokens.  As a block selection:
+ * every (b, g) keeps its last min(k, NB_b) blocks, NB_b - min(k, NB_b) ..
+ * NB_b - 1, ascending and -1 padded.
+ */
+void ksa_oracle_select_window(int B, int Hkv, int bs, const int32_t *seq_lens, int k,
+                              int32_t *block_idx, int32_t *num_sel) {
+  for (int b = 0; b < B; ++b) {
+    const int nb = num_blocks(seq_lens[b], bs);
+    const int n = k < nb ? k : nb;
+    for (int g = 0; g < Hkv; ++g) {
+      int32_t *row = block_idx + ((size_t)b * Hkv + g) * k;
+      for (int i = 0; i < k; ++i) row[i] = i < n ? nb - n + i : -1;
+      num_sel[b * Hkv + g] = n;
+    }
+  }
+}
+
 /* ---- (A4/A5/A7/A8) attention over a selected token set ------------------ */
 /*
  * Kinetics section 5 and LessIsMore section 5 "sparse attention layer":

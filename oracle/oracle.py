@@ -51,6 +51,7 @@ class Oracle:
                                                 _i32p, _i32p, nullable_f64])
         L.ksa_oracle_select_blocks_ex.argtypes = ([c_int] * 6 + [_u16p, _u16p, _i32p, c_int,
                                                    c_int, _i32p, _i32p, nullable_f64])
+        L.ksa_oracle_select_window.argtypes = [c_int] * 3 + [_i32p, c_int, _i32p, _i32p]
         L.ksa_oracle_gather_pages.argtypes = [c_int] * 6 + [_u16p, _i32p, _i32p, _u16p]
         L.ksa_oracle_round_bf16.argtypes = [c_double]
         L.ksa_oracle_round_bf16.restype = ctypes.c_uint16
@@ -143,6 +144,15 @@ class Oracle:
             B, Hq, Hkv, D, T, bs, q, K, np.ascontiguousarray(seq_lens, np.int32), k,
             int(summary_bf16), idx, cnt, scores.ctypes.data if want_scores else None)
         return (idx, cnt, scores) if want_scores else (idx, cnt)
+
+    def select_window(self, seq_lens, num_kv_heads: int, bs: int, k: int):
+        """Local attention as a block selection: the last min(k, NB_b) blocks, ascending."""
+        lens = np.ascontiguousarray(seq_lens, np.int32)
+        B = lens.shape[0]
+        idx = np.empty((B, num_kv_heads, k), np.int32)
+        cnt = np.empty((B, num_kv_heads), np.int32)
+        self.lib.ksa_oracle_select_window(B, num_kv_heads, bs, lens, k, idx, cnt)
+        return idx, cnt
 
     # -- A4/A5/A7/A8 --------------------------------------------------------
     def attention(self, q, K, V, seq_lens, idx=None, num_idx=None, tokens_per_idx: int = 1,

@@ -621,3 +621,25 @@ def test_gather_pages_scatter_roundtrip_and_bad_pages(oracle):
     got2 = oracle.gather_pages(pages, tbl2, lens)
     assert not got2[0, :, bs:3 * bs].any()
     assert np.array_equal(got2[0, :, :bs], K[0, :, :bs])
+
+
+def test_select_window_is_topk_of_a_recency_score(oracle):
+    """Local attention as a block selection equals block top-k when the scores grow with
+    the block index: keys of block j are j * c * u, with u the group's query direction."""
+    rng = np.random.default_rng(51)
+    B, Hq, Hkv, D, bs, nbk = 3, 4, 2, 64, 16, 12
+    G = Hq // Hkv
+    T = nbk * bs
+    lens = np.array([T, 5 * bs + 3, 2 * bs], np.int32)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float32)
+    K = np.zeros((B, Hkv, T, D), np.float32)
+    for b in range(B):
+        for g in range(Hkv):
+            u = q[b, g * G:(g + 1) * G].sum(0)
+            u /= np.linalg.norm(u)
+            for j in range(nbk):
+                K[b, g, j * bs:(j + 1) * bs] = (j + 1) * 0.25 * u
+    for k in (1, 4, 12):
+        want = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, k)
+        got = oracle.select_window(lens, Hkv, bs, k)
+        assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
