@@ -27,7 +27,7 @@ __all__ = [
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
     "ksa_build_block_summaries_ex", "ksa_select_blocks_ex", "ksa_decode_select_blocks_ex",
     "ksa_build_block_summaries_paged", "ksa_decode_select_blocks_paged",
-    "ksa_sparse_decode_attn_paged", "Pages",
+    "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -81,6 +81,7 @@ _SIGS = {
     "ksa_sparse_decode_attn_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp,
                                             ctypes.POINTER(Pages), _vp, _vp, _vp, _i32, _i32,
                                             _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "ksa_select_window": (_i32, [ctypes.POINTER(Shape), _vp, _i32, _vp, _vp, _vp, _vp]),
     "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]),
@@ -491,3 +492,23 @@ def ksa_sparse_decode_attn_paged(q: torch.Tensor, K_pages: torch.Tensor, V_pages
         int(bool(idx_shared)), float(scale), int(out_dtype), _ptr(out), _ptr(lse), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
     return out, lse
+
+
+def ksa_select_window(seq_lens: torch.Tensor, num_kv_heads: int, block_size: int, capacity: int,
+                      k_blocks: int, block_idx: Optional[torch.Tensor] = None,
+                      num_sel: Optional[torch.Tensor] = None,
+                      dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Local attention as a block selection: (block_idx [B,Hkv,k] ascending -1 padded,
+    num_sel [B,Hkv]) = each row's last min(k, NB_b) blocks."""
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B = seq_lens.shape[0]
+    if block_idx is None:
+        block_idx = torch.empty((B, num_kv_heads, k_blocks), dtype=torch.int32,
+                                device=seq_lens.device)
+    if num_sel is None:
+        num_sel = torch.empty((B, num_kv_heads), dtype=torch.int32, device=seq_lens.device)
+    sh = _shape(B, num_kv_heads, num_kv_heads, 64, capacity, block_size)
+    _check(lib().ksa_select_window(ctypes.byref(sh), _ptr(seq_lens), int(k_blocks),
+                                   _ptr(block_idx), _ptr(num_sel), _ptr(dev_status),
+                                   _stream(stream)))
+    return block_idx, num_sel

@@ -286,6 +286,35 @@ ksa_status ksa_decode_select_blocks_ex(const ksa_shape *shape, const uint16_t *q
                        "ksa_decode_select_blocks launch");
 }
 
+ksa_status ksa_select_window(const ksa_shape *shape, const int32_t *seq_lens, int32_t k_blocks,
+                             int32_t *block_idx, int32_t *num_sel, uint32_t *dev_status,
+                             void *stream) {
+  ksa_status st = check_shape(shape, true);
+  if (st != KSA_OK) return st;
+  if (seq_lens == nullptr || block_idx == nullptr || num_sel == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "seq_lens, block_idx and num_sel must be non-NULL");
+  if (k_blocks < 1) return fail(KSA_ERR_INVALID_ARG, "k_blocks must be >= 1 (got %d)", k_blocks);
+  if (static_cast<long long>(shape->batch) * shape->num_kv_heads * k_blocks >= (1LL << 31))
+    return fail(KSA_ERR_UNSUPPORTED, "batch * num_kv_heads * k_blocks must be < 2^31");
+  ksa::SelectArgs a;
+  a.q = nullptr;
+  a.S = nullptr;
+  a.sbf16 = 0;
+  a.seq_lens = seq_lens;
+  a.block_idx = block_idx;
+  a.num_sel = num_sel;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hq = shape->num_q_heads;
+  a.Hkv = shape->num_kv_heads;
+  a.D = shape->head_dim;
+  a.T = shape->capacity;
+  a.bs = shape->block_size;
+  a.k = k_blocks;
+  return cuda_status(ksa::launch_select_window(a, static_cast<cudaStream_t>(stream)),
+                     "ksa_select_window launch");
+}
+
 ksa_status ksa_decode_select_blocks_paged(const ksa_shape *shape, const uint16_t *q,
                                           const uint16_t *K_pages, const ksa_pages *pages,
                                           void *summaries, int32_t summary_dtype,

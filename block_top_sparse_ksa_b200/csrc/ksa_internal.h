@@ -56,6 +56,8 @@ struct SelectArgs {
   int B, Hq, Hkv, D, T, bs, k;
   KvLayout kv;  // of the key cache given for the fused refresh
 };
+// Local-window block selection (reads only seq_lens; writes block_idx, num_sel).
+cudaError_t launch_select_window(const SelectArgs &a, cudaStream_t stream);
 // workspace: semaphores [B*Hkv] (zero between calls) + score keys [B*Hkv, ceil(T/bs)]
 size_t select_workspace_bytes(int B, int Hkv, int T, int bs);
 // K non-null: first refresh each row's last-block summary from K (fused maintenance).

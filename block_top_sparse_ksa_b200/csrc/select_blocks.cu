@@ -498,6 +498,23 @@ __global__ void __launch_bounds__(kRankThreads) rank_long_kernel(const ScoreDev 
   if (tid == 0) a.num_sel[row] = k;
 }
 
+// Local attention as a block selection: every (row, kv-head) keeps its last
+// min(k, NB_b) blocks, ascending, -1 padded.  One thread per output slot.
+__global__ void __launch_bounds__(256) window_blocks_kernel(const SelectArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= static_cast<long long>(a.B) * a.Hkv * a.k) return;
+  const int row = static_cast<int>(e / a.k), i = static_cast<int>(e % a.k);
+  const int b = row / a.Hkv;
+  const int L = clamp_len(a.seq_lens[b], a.T,
+                          (i == 0 && row == b * a.Hkv) ? a.status : nullptr);
+  const int nb = (L + a.bs - 1) / a.bs;
+  const int n = min(a.k, nb);
+  a.block_idx[e] = i < n ? nb - n + i : -1;
+  if (i == 0) a.num_sel[row] = n;
+}
+
 template <int D>
 cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) {
   ScoreDev p = p0;
@@ -538,6 +555,12 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
 
 // workspace: a leading region of one word per row plus two (reserved: zero)
 // + score keys [B*Hkv, nb_max]
+cudaError_t launch_select_window(const SelectArgs &a, cudaStream_t stream) {
+  const long long n = static_cast<long long>(a.B) * a.Hkv * a.k;
+  return launch_pdl(window_blocks_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256),
+                    0, stream, a);
+}
+
 size_t select_workspace_bytes(int B, int Hkv, int T, int bs) {
   const size_t rows = static_cast<size_t>(B) * Hkv;
   const size_t nb_max = static_cast<size_t>((T + bs - 1) / bs);

@@ -132,6 +132,17 @@ ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q,
                                     size_t ws_bytes, uint32_t *dev_status, void *stream);
 
 /*
+ * Local attention as a block selection [KIN s.5 compares block top-k with
+ * local attention, a fixed pattern over the nearest tokens]: every (b, g)
+ * keeps its last min(k_blocks, NB_b) blocks, NB_b - n .. NB_b - 1, ascending
+ * and -1 padded, in the layout of ksa_select_blocks, for the same attention
+ * call.  Reads only seq_lens; no workspace.
+ */
+ksa_status ksa_select_window(const ksa_shape *shape, const int32_t *seq_lens,
+                             int32_t k_blocks, int32_t *block_idx, int32_t *num_sel,
+                             uint32_t *dev_status, void *stream);
+
+/*
  * The same three calls with the summaries stored as bf16 or fp32
  * (summary_dtype: KSA_SUMMARIES_F32 or KSA_SUMMARIES_BF16).  With bf16 each
  * block mean is computed in fp32 as above and stored rounded to the nearest

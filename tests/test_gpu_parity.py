@@ -670,3 +670,60 @@ def test_paged_kv_bad_page_ids_are_flagged_not_read(ksa, oracle):
                                                tokens_per_idx=bs)
     # (another batch splits the work differently, so fp32 sums differ in the last bits)
     torch.testing.assert_close(out[:1], out0, atol=1e-5, rtol=1e-5)
+
+
+# ---------------------------------------------------------------------------
+# attention-recall diagnostic
+
+
+def test_attention_recall_matches_softmax_mass(ksa, oracle):
+    """recall = the dense softmax mass on the selected tokens (fp64 numpy softmax here);
+    the dense set recalls 1 and an empty selection 0."""
+    from block_top_sparse_ksa_b200.recall import attention_recall
+    rng = np.random.default_rng(1500)
+    B, Hq, Hkv, D, T, bs = 2, 8, 2, 64, 320, 16
+    G = Hq // Hkv
+    lens = np.array([T, 123], np.int32)
+    q, K, V = (rand_bits(rng, s) for s in [(B, Hq, D), (B, Hkv, T, D), (B, Hkv, T, D)])
+    nb = -(-lens // bs)
+    k = 6
+    idx = np.full((B, Hkv, k), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            pick = np.sort(rng.choice(int(nb[b]), size=k, replace=False))
+            idx[b, g] = pick
+            cnt[b, g] = k
+    qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
+    rec = attention_recall(qd, Kd, Vd, Ld, torch.from_numpy(idx).to(DEV),
+                           torch.from_numpy(cnt).to(DEV), tokens_per_idx=bs)
+    qv, Kv = bf16_value(q), bf16_value(K)
+    for b in range(B):
+        L = int(lens[b])
+        for h in range(Hq):
+            g = h // G
+            z = Kv[b, g, :L] @ qv[b, h] / math.sqrt(D)
+            w = np.exp(z - z.max())
+            w /= w.sum()
+            sel = np.zeros(L, bool)
+            for j in idx[b, g, :cnt[b, g]]:
+                sel[j * bs:min((j + 1) * bs, L)] = True
+            assert abs(rec[b, h] - w[sel].sum()) <= 3e-4 * max(1.0, w[sel].sum())
+    all_idx = torch.arange(int(nb.max()), dtype=torch.int32, device=DEV).repeat(B, Hkv, 1)
+    all_cnt = torch.from_numpy(np.repeat(nb[:, None], Hkv, 1).astype(np.int32)).to(DEV)
+    assert np.allclose(attention_recall(qd, Kd, Vd, Ld, all_idx, all_cnt, tokens_per_idx=bs),
+                       1.0, atol=1e-5)
+    none = torch.zeros((B, Hkv), dtype=torch.int32, device=DEV)
+    assert np.all(attention_recall(qd, Kd, Vd, Ld, all_idx, none, tokens_per_idx=bs) == 0.0)
+
+
+def test_select_window_matches_oracle(ksa, oracle):
+    """Local attention as a block selection: the oracle's last min(k, NB_b) blocks."""
+    lens = np.array([1000, 1, 33, 16 * 7], np.int32)
+    Ld = torch.from_numpy(lens).to(DEV)
+    for bs in (16, 64):
+        for k in (1, 5, 100):
+            idx, cnt = ksa.ksa_select_window(Ld, 3, bs, 1000, k)
+            ref_idx, ref_cnt = oracle.select_window(lens, 3, bs, k)
+            assert np.array_equal(idx.cpu().numpy(), ref_idx)
+            assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
