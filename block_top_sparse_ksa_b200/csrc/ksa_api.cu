@@ -491,6 +491,9 @@ ksa_status ksa_unified_select(const ksa_shape *shape, const uint16_t *q, const u
       ~static_cast<size_t>(255);
   a.keys = static_cast<uint32_t *>(ws);
   a.votes = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + keys_bytes);
+  const size_t votes_bytes =
+      (static_cast<size_t>(shape->batch) * shape->capacity * 4 + 255) & ~static_cast<size_t>(255);
+  a.bits = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + keys_bytes + votes_bytes);
   a.status = dev_status;
   a.B = shape->batch;
   a.Hq = shape->num_q_heads;

@@ -92,6 +92,7 @@ struct UnifiedArgs {
   int32_t *num_sel;
   uint32_t *keys;   // workspace [B, Hq, T] score keys
   int32_t *votes;   // workspace [B, T]
+  uint32_t *bits;   // workspace [B, Hq, ceil(T/32)]: each head's picks as a bit set
   uint32_t *status;
   int B, Hq, Hkv, D, T, P, budget, R;
 };
