@@ -510,7 +510,9 @@ def run_unified(args, dist, dev):
         "select_hbm": {"bytes_per_launch": sel_b, "gbs": sel_b / (t_sel * 1e-3) / 1e9},
         "step_hbm": {"bytes_per_step": sel_b + 3 * att_b,
                      "gbs": (sel_b + 3 * att_b) / per / 1e9},
-        "gpu_launches": (3 + len(inp.layers)) * args.steps, "clocks": clk,
+        # selection: scores, picks, (vote counting when the picks keep the row's keys in
+        # registers: capacity <= 24576), shared set; then one attention launch per layer
+        "gpu_launches": ((4 if T <= 24576 else 3) + len(inp.layers)) * args.steps, "clocks": clk,
         "config": {"workload": sh.name, "batch_per_gpu": B, "num_q_heads": Hq,
                    "num_kv_heads": Hkv, "head_dim": D, "context": sh.seq_len,
                    "per_head_topk": sh.per_head_topk, "token_budget": sh.token_budget,

@@ -397,6 +397,7 @@ __global__ void __launch_bounds__(256) unified_votes_kernel(const UnifiedArgs a)
   if (L <= a.budget || t >= L) return;  // warp-uniform up to the row's last word
   const uint32_t *bits = a.bits + static_cast<size_t>(b) * a.Hq * W32 + (t >> 5);
   int v = 0;
+#pragma unroll 16
   for (int h = 0; h < a.Hq; ++h) v += (__ldcg(bits + static_cast<size_t>(h) * W32) >> (t & 31)) & 1u;
   a.votes[static_cast<size_t>(b) * a.T + t] = v;
 }
