@@ -409,6 +409,45 @@ static int cmp_ranked(const void *a, const void *b) {
   return (x->t > y->t) - (x->t < y->t);
 }
 
+/*
+ * Kinetics section 5's ideal token-level sparse attention: every query head h
+ * keeps its own k highest-scoring tokens, s_t = sum_d q[b,h,d] * K[b,g,t,d]
+ * over t < L_b (g = h / G), ties to the lower t (the same full stable ranking
+ * as the LessIsMore per-head picks), listed ascending and -1 padded.  If
+ * k >= L_b every token is kept.
+ *   token_idx: [B, Hq, k];  num_sel: [B, Hq].
+ */
+void ksa_oracle_select_tokens_per_head(int B, int Hq, int Hkv, int D, int T,
+                                       const uint16_t *q, const uint16_t *K,
+                                       const int32_t *seq_lens, int k, int32_t *token_idx,
+                                       int32_t *num_sel) {
+  const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hq; ++h) {
+      const int L = seq_lens[b];
+      const int g = h / G;
+      int32_t *row = token_idx + ((size_t)b * Hq + h) * k;
+      for (int i = 0; i < k; ++i) row[i] = -1;
+      ranked_t *r = (ranked_t *)malloc(sizeof(ranked_t) * (size_t)(L > 0 ? L : 1));
+      const uint16_t *qrow = q + ((size_t)b * Hq + h) * D;
+      for (int t = 0; t < L; ++t) {
+        const uint16_t *krow = K + (((size_t)b * Hkv + g) * T + t) * D;
+        double sc = 0.0;
+        for (int d = 0; d < D; ++d) sc += bf16_to_f64(qrow[d]) * bf16_to_f64(krow[d]);
+        r[t].key = sc;
+        r[t].t = t;
+      }
+      qsort(r, (size_t)L, sizeof(ranked_t), cmp_ranked);
+      const int n = k < L ? k : L;
+      for (int i = 0; i < n; ++i) row[i] = r[i].t;
+      qsort(row, (size_t)n, sizeof(int32_t), cmp_int32);
+      num_sel[(size_t)b * Hq + h] = n;
+      free(r);
+    }
+  }
+}
+
 void ksa_oracle_unified_select(int B, int Hq, int Hkv, int D, int T,
                                const uint16_t *q, const uint16_t *K,
                                const int32_t *seq_lens, int P, int budget,

@@ -51,6 +51,8 @@ class Oracle:
                                                 _i32p, _i32p, nullable_f64])
         L.ksa_oracle_select_blocks_ex.argtypes = ([c_int] * 6 + [_u16p, _u16p, _i32p, c_int,
                                                    c_int, _i32p, _i32p, nullable_f64])
+        L.ksa_oracle_select_tokens_per_head.argtypes = ([c_int] * 5 + [_u16p, _u16p, _i32p,
+                                                        c_int, _i32p, _i32p])
         L.ksa_oracle_select_window.argtypes = [c_int] * 3 + [_i32p, c_int, _i32p, _i32p]
         L.ksa_oracle_gather_pages.argtypes = [c_int] * 6 + [_u16p, _i32p, _i32p, _u16p]
         L.ksa_oracle_round_bf16.argtypes = [c_double]
@@ -144,6 +146,20 @@ class Oracle:
             B, Hq, Hkv, D, T, bs, q, K, np.ascontiguousarray(seq_lens, np.int32), k,
             int(summary_bf16), idx, cnt, scores.ctypes.data if want_scores else None)
         return (idx, cnt, scores) if want_scores else (idx, cnt)
+
+    def select_tokens_per_head(self, q, K, seq_lens, k: int):
+        """Each query head's own top-k tokens (ties -> lower t), ascending, -1 padded:
+        (token_idx [B,Hq,k], num_sel [B,Hq])."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        K = np.ascontiguousarray(K, dtype=np.uint16)
+        B, Hq, D = q.shape
+        _, Hkv, T, _ = K.shape
+        idx = np.empty((B, Hq, k), np.int32)
+        cnt = np.empty((B, Hq), np.int32)
+        self.lib.ksa_oracle_select_tokens_per_head(B, Hq, Hkv, D, T, q, K,
+                                                   np.ascontiguousarray(seq_lens, np.int32),
+                                                   k, idx, cnt)
+        return idx, cnt
 
     def select_window(self, seq_lens, num_kv_heads: int, bs: int, k: int):
         """Local attention as a block selection: the last min(k, NB_b) blocks, ascending."""

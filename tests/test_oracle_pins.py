@@ -643,3 +643,46 @@ def test_select_window_is_topk_of_a_recency_score(oracle):
         want = oracle.select_blocks(bf16_bits(q), bf16_bits(K), lens, bs, k)
         got = oracle.select_window(lens, Hkv, bs, k)
         assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
+
+
+# ---------------------------------------------------------------------------
+# per-head token top-k (token-level sparse attention, one set per query head)
+
+
+def test_tokens_per_head_rank_counting(oracle):
+    """Brute force on small inputs: every kept token has fewer than k tokens ranked above it
+    (higher score, or equal score and lower index), and min(k, L) are kept."""
+    rng = np.random.default_rng(61)
+    B, Hq, Hkv, D, T = 2, 4, 2, 64, 90
+    G = Hq // Hkv
+    q = np.round(rng.standard_normal((B, Hq, D)) * 2) / 4      # coarse grid: exact ties
+    K = np.round(rng.standard_normal((B, Hkv, T, D)) * 2) / 4
+    lens = np.array([T, 37], np.int32)
+    for k in (1, 10, 40, 200):
+        idx, cnt = oracle.select_tokens_per_head(bf16_bits(q), bf16_bits(K), lens, k)
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(Hq):
+                s = K[b, h // G, :L] @ q[b, h]
+                n = int(cnt[b, h])
+                assert n == min(k, L)
+                got = idx[b, h, :n]
+                assert np.all(np.diff(got) > 0) and np.all(idx[b, h, n:] == -1)
+                for t in got:
+                    above = np.sum((s > s[t]) | ((s == s[t]) & (np.arange(L) < t)))
+                    assert above < k
+
+
+def test_tokens_per_head_equal_heads_match_unified_votes(oracle):
+    """With every query head identical, each head's top-k is the set every head votes for,
+    so it is the LessIsMore selection with budget k and no window."""
+    rng = np.random.default_rng(62)
+    B, Hq, Hkv, D, T, k = 2, 4, 1, 64, 300, 50
+    q1 = rng.standard_normal((B, 1, D)).astype(np.float32)
+    q = np.repeat(q1, Hq, axis=1)
+    K = rng.standard_normal((B, Hkv, T, D)).astype(np.float32)
+    lens = np.array([T, 120], np.int32)
+    idx, cnt = oracle.select_tokens_per_head(bf16_bits(q), bf16_bits(K), lens, k)
+    uni, ucnt = oracle.unified_select(bf16_bits(q), bf16_bits(K), lens, k, k, 0)
+    for h in range(Hq):
+        assert np.array_equal(idx[:, h], uni) and np.array_equal(cnt[:, h], ucnt)
