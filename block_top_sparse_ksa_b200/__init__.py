@@ -27,7 +27,8 @@ __all__ = [
     "ksa_unified_select_workspace", "ksa_status_string", "ksa_last_error", "ksa_version",
     "ksa_build_block_summaries_ex", "ksa_select_blocks_ex", "ksa_decode_select_blocks_ex",
     "ksa_build_block_summaries_paged", "ksa_decode_select_blocks_paged",
-    "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window",
+    "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window", "ksa_select_tokens_per_head",
+    "ksa_select_tokens_per_head_workspace", "IDX_PER_KV_HEAD", "IDX_SHARED", "IDX_PER_Q_HEAD",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -38,6 +39,7 @@ library_path = os.path.join(_HERE, "libksa.so")
 
 SUMMARY_ALL, SUMMARY_LAST_BLOCK = 0, 1
 SUMMARIES_F32, SUMMARIES_BF16 = 0, 1
+IDX_PER_KV_HEAD, IDX_SHARED, IDX_PER_Q_HEAD = 0, 1, 2
 OUT_F32, OUT_BF16 = 0, 1
 FLAG_SEQ_LEN_CLAMPED, FLAG_INDEX_SKIPPED, FLAG_NONFINITE_SCORE, FLAG_WAIT_TIMEOUT = 1, 2, 4, 8
 _STATUS = {0: "KSA_OK", 1: "KSA_ERR_INVALID_ARG", 2: "KSA_ERR_UNSUPPORTED",
@@ -82,6 +84,9 @@ _SIGS = {
                                             ctypes.POINTER(Pages), _vp, _vp, _vp, _i32, _i32,
                                             _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "ksa_select_window": (_i32, [ctypes.POINTER(Shape), _vp, _i32, _vp, _vp, _vp, _vp]),
+    "ksa_select_tokens_per_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
+    "ksa_select_tokens_per_head": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp,
+                                          _vp, _sz, _vp, _vp]),
     "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_blocks": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]),
@@ -280,7 +285,7 @@ ksa_decode_select_blocks_ex = ksa_decode_select_blocks
 def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                            seq_lens: torch.Tensor, idx: Optional[torch.Tensor] = None,
                            num_idx: Optional[torch.Tensor] = None, tokens_per_idx: int = 1,
-                           idx_shared: bool = False, scale: float = 0.0,
+                           idx_shared: int = IDX_PER_KV_HEAD, scale: float = 0.0,
                            out_dtype: int = OUT_F32, out: Optional[torch.Tensor] = None,
                            lse: Optional[torch.Tensor] = None,
                            workspace: Optional[torch.Tensor] = None,
@@ -308,7 +313,7 @@ def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         ctypes.byref(sh), int(cap), int(tokens_per_idx)), q.device)
     _check(lib().ksa_sparse_decode_attn(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx), _ptr(num_idx),
-        int(cap), int(tokens_per_idx), int(bool(idx_shared)), float(scale), int(out_dtype),
+        int(cap), int(tokens_per_idx), int(idx_shared), float(scale), int(out_dtype),
         _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status),
         _stream(stream)))
     return out, lse
@@ -317,7 +322,7 @@ def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
 def ksa_sparse_decode_attn_noalloc(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                                    seq_lens: torch.Tensor, idx: Optional[torch.Tensor] = None,
                                    num_idx: Optional[torch.Tensor] = None,
-                                   tokens_per_idx: int = 1, idx_shared: bool = False,
+                                   tokens_per_idx: int = 1, idx_shared: int = IDX_PER_KV_HEAD,
                                    scale: float = 0.0, out_dtype: int = OUT_F32,
                                    out: Optional[torch.Tensor] = None,
                                    lse: Optional[torch.Tensor] = None,
@@ -346,7 +351,7 @@ def ksa_sparse_decode_attn_noalloc(q: torch.Tensor, K: torch.Tensor, V: torch.Te
     sh = _shape(B, Hq, Hkv, D, T, max(1, tokens_per_idx))
     _check(lib().ksa_sparse_decode_attn_noalloc(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx), _ptr(num_idx),
-        int(cap), int(tokens_per_idx), int(bool(idx_shared)), float(scale), int(out_dtype),
+        int(cap), int(tokens_per_idx), int(idx_shared), float(scale), int(out_dtype),
         _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
     return out, lse
 
@@ -458,7 +463,7 @@ def ksa_sparse_decode_attn_paged(q: torch.Tensor, K_pages: torch.Tensor, V_pages
                                  block_table: torch.Tensor, seq_lens: torch.Tensor,
                                  idx: Optional[torch.Tensor] = None,
                                  num_idx: Optional[torch.Tensor] = None, tokens_per_idx: int = 1,
-                                 idx_shared: bool = False, scale: float = 0.0,
+                                 idx_shared: int = IDX_PER_KV_HEAD, scale: float = 0.0,
                                  out_dtype: int = OUT_F32, out: Optional[torch.Tensor] = None,
                                  lse: Optional[torch.Tensor] = None,
                                  workspace: Optional[torch.Tensor] = None,
@@ -489,7 +494,7 @@ def ksa_sparse_decode_attn_paged(q: torch.Tensor, K_pages: torch.Tensor, V_pages
     _check(lib().ksa_sparse_decode_attn_paged(
         ctypes.byref(sh), _ptr(q), _ptr(K_pages), _ptr(V_pages), ctypes.byref(pg),
         _ptr(seq_lens), _ptr(idx), _ptr(num_idx), int(cap), int(tokens_per_idx),
-        int(bool(idx_shared)), float(scale), int(out_dtype), _ptr(out), _ptr(lse), _ptr(ws),
+        int(idx_shared), float(scale), int(out_dtype), _ptr(out), _ptr(lse), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
     return out, lse
 
@@ -512,3 +517,36 @@ def ksa_select_window(seq_lens: torch.Tensor, num_kv_heads: int, block_size: int
                                    _ptr(block_idx), _ptr(num_sel), _ptr(dev_status),
                                    _stream(stream)))
     return block_idx, num_sel
+
+
+def ksa_select_tokens_per_head_workspace(B: int, Hq: int, Hkv: int, D: int, T: int,
+                                         k_tokens: int) -> int:
+    sh = _shape(B, Hq, Hkv, D, T)
+    return int(lib().ksa_select_tokens_per_head_workspace(ctypes.byref(sh), int(k_tokens)))
+
+
+def ksa_select_tokens_per_head(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor,
+                               k_tokens: int, token_idx: Optional[torch.Tensor] = None,
+                               num_sel: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None,
+                               dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Each query head's own top-k tokens: (token_idx [B,Hq,k] ascending -1 padded,
+    num_sel [B,Hq]); attend with idx_shared=IDX_PER_Q_HEAD, tokens_per_idx=1."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    need = ksa_select_tokens_per_head_workspace(B, Hq, Hkv, D, T, k_tokens)
+    if workspace is None:  # no initialisation needed
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    if token_idx is None:
+        token_idx = torch.empty((B, Hq, k_tokens), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+    sh = _shape(B, Hq, Hkv, D, T)
+    _check(lib().ksa_select_tokens_per_head(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(seq_lens), int(k_tokens), _ptr(token_idx),
+        _ptr(num_sel), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(dev_status), _stream(stream)))
+    return token_idx, num_sel

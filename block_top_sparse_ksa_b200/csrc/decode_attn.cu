@@ -69,6 +69,8 @@ struct Cfg {
 
 struct AttnDev {
   AttnArgs a;
+  int rpb;        // rows per batch row: Hkv, or Hq with per-query-head lists
+  int gw;         // query heads per row: G, or 1 with per-query-head lists
   int V;          // stages each row is padded to
   long long W;    // rows * V
   int N;          // CTAs in the grid
@@ -90,6 +92,25 @@ __device__ __forceinline__ void consumer_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
 }
 
+// Row r of the work: batch row b, kv-head g, and its query heads qh0 .. qh0 + gw - 1
+// (the G heads of kv-head g, or with per-query-head lists the one head h).
+struct RowGeom {
+  int b, g, qh0;
+};
+__device__ __forceinline__ RowGeom row_geom(const AttnDev &p, int r) {
+  RowGeom x;
+  x.b = r / p.rpb;
+  const int i = r - x.b * p.rpb;
+  if (p.gw == 1 && p.rpb == p.a.Hq) {  // per-query-head rows
+    x.g = i / (p.a.Hq / p.a.Hkv);
+    x.qh0 = i;
+  } else {
+    x.g = i;
+    x.qh0 = i * p.gw;
+  }
+  return x;
+}
+
 struct RowInfo {
   int L;
   const int32_t *list;
@@ -98,9 +119,8 @@ struct RowInfo {
 };
 
 template <int MODE>
-__device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int r, uint32_t *flag_sink) {
+__device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int r, int b, uint32_t *flag_sink) {
   RowInfo ri;
-  const int b = r / a.Hkv;
   ri.L = clamp_len(a.seq_lens[b], a.T, flag_sink);
   ri.list = nullptr;
   ri.n_idx = 0;
@@ -108,9 +128,9 @@ __device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int r, uint32_t *
     ri.n_st = (ri.L + kStageTok - 1) / kStageTok;
     return ri;
   }
-  ri.list = a.shared ? a.idx + static_cast<size_t>(b) * a.cap
-                     : a.idx + static_cast<size_t>(r) * a.cap;
-  int n = a.shared ? a.num_idx[b] : a.num_idx[r];
+  ri.list = a.shared == 1 ? a.idx + static_cast<size_t>(b) * a.cap
+                          : a.idx + static_cast<size_t>(r) * a.cap;
+  int n = a.shared == 1 ? a.num_idx[b] : a.num_idx[r];  // 0: per kv-head, 2: per query head rows
   if (n < 0 || n > a.cap) {
     flag_status(flag_sink, KSA_FLAG_INDEX_SKIPPED);
     n = n < 0 ? 0 : a.cap;
@@ -138,13 +158,13 @@ __device__ __forceinline__ void store_out(const AttnArgs &a, size_t oi, float v)
 template <int D>
 __device__ __forceinline__ void merge_partials(const AttnDev &p, int r, int tid) {
   const AttnArgs &a = p.a;
-  const int G = a.Hq / a.Hkv;
+  const int G = p.gw;  // query heads of the row
   const int SL = p.slot;
-  const int b = r / a.Hkv, g = r % a.Hkv;
+  const RowGeom rg = row_geom(p, r);
   const long long rv0 = static_cast<long long>(r) * p.V;
   const int c_first = cta_of(rv0, p.W, p.N);
   const int c_last = cta_of(rv0 + p.V - 1, p.W, p.N);
-  const size_t obase = (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G);
+  const size_t obase = static_cast<size_t>(rg.b) * a.Hq + rg.qh0;
   constexpr int NT = kConsumers * 32;
   for (int e0 = tid; e0 < G * D; e0 += 2 * NT) {
     float M[2] = {-INFINITY, -INFINITY}, o[2] = {0.f, 0.f}, l[2] = {0.f, 0.f};
@@ -218,7 +238,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
   float *merge = reinterpret_cast<float *>(smem + C::kMergeOffset);  // [4][2G + G*D]
 
   const AttnArgs &a = p.a;
-  const int G = a.Hq / a.Hkv;
+  const int G = p.gw;  // query heads per row
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x;
   const long long s0 = cta_start(c, p.W, p.N), s1 = cta_start(c + 1, p.W, p.N);
@@ -258,7 +278,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         const int spe = tpi >= kStageTok ? tpi / kStageTok : 1;  // stages per entry
         int r = r_first;
         long long rv0 = static_cast<long long>(r) * p.V;
-        RowInfo ri = row_info<MODE>(a, r, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
+        RowGeom rg = row_geom(p, r);
+        RowInfo ri = row_info<MODE>(a, r, rg.b, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
         int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
         int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
         int cnt = jb > ja ? jb - ja : 0;
@@ -268,7 +289,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
             row_base += cnt;
             if (++r > r_last) break;
             rv0 = static_cast<long long>(r) * p.V;
-            ri = row_info<MODE>(a, r, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
+            rg = row_geom(p, r);
+            ri = row_info<MODE>(a, r, rg.b, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
             ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
             jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
             cnt = jb > ja ? jb - ja : 0;
@@ -302,7 +324,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
             const long long left = ri.L - t0[u];
             nv[u] = (!ok || left <= 0) ? 0 : (left < seg ? static_cast<int>(left) : seg);
             if (nv[u] > 0) {  // the segment's first K/V row (its page, when paged)
-              yr[u] = kv_row(a.kv, r / a.Hkv, r % a.Hkv, a.Hkv, a.T, t0[u]);
+              yr[u] = kv_row(a.kv, rg.b, rg.g, a.Hkv, a.T, t0[u]);
               if (yr[u] < 0) {
                 nv[u] = 0;
                 skipped = KSA_FLAG_INDEX_SKIPPED;
@@ -345,7 +367,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
       for (int r = r_first; r <= r_last && !stop; ++r) {
         const long long rv0 = static_cast<long long>(r) * p.V;
         const bool reporter = lane == 0 && rv0 >= s0;
-        const RowInfo ri = row_info<MODE>(a, r, reporter ? a.status : nullptr);
+        const RowGeom rg = row_geom(p, r);
+        const RowInfo ri = row_info<MODE>(a, r, rg.b, reporter ? a.status : nullptr);
         const int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
         const int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
         const int eps = kStageTok / tpi;  // entries per stage
@@ -389,7 +412,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
                 (id < 0 || static_cast<long long>(id) * tpi >= ri.L))
               skipped = KSA_FLAG_INDEX_SKIPPED;
             if (valid) {
-              trow = kv_row(a.kv, r / a.Hkv, r % a.Hkv, a.Hkv, a.T, t);
+              trow = kv_row(a.kv, rg.b, rg.g, a.Hkv, a.T, t);
               if (trow < 0) {  // its page id names no page
                 valid = false;
                 skipped = KSA_FLAG_INDEX_SKIPPED;
@@ -433,9 +456,9 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
     float *wo = merge + 8 * G;  // [4][G][D]
     int i = 0;                  // ordinal of the next stage of this CTA
     for (int r = r_first; r <= r_last; ++r) {
-      const int b = r / a.Hkv, g = r % a.Hkv;
+      const RowGeom rg = row_geom(p, r);
       const long long rv0 = static_cast<long long>(r) * p.V;
-      const RowInfo ri = row_info<MODE>(a, r, nullptr);
+      const RowInfo ri = row_info<MODE>(a, r, rg.b, nullptr);
       const int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
       const int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
       const int cnt = jb > ja ? jb - ja : 0;
@@ -443,7 +466,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
       uint32_t qb[KT][2];
       {
         const uint16_t *qrow =
-            a.q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G + gid) * D;
+            a.q + (static_cast<size_t>(rg.b) * a.Hq + rg.qh0 + gid) * D;
 #pragma unroll
         for (int ks = 0; ks < KT; ++ks) {
           qb[ks][0] =
@@ -584,7 +607,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
         const int which = (r == static_cast<int>(s0 / p.V)) ? 0 : 1;
         myslot = p.part + (static_cast<size_t>(c) * 2 + which) * SL;
       }
-      const size_t obase = (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(g) * G);
+      const size_t obase = static_cast<size_t>(rg.b) * a.Hq + rg.qh0;
       for (int e = tid; e < G * D; e += kConsumers * 32) {
         const int hh = e / D, d = e % D;
         float M = -INFINITY;
@@ -646,7 +669,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
 template <int D, int MODE>
 cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, int num_sms,
                        cudaStream_t stream) {
-  const int G = p.a.Hq / p.a.Hkv;
+  const int G = p.gw;
   const size_t smem = Cfg<D>::kFixedSmem + static_cast<size_t>(kConsumers) * (2 * G + G * D) * 4;
   cudaError_t err = cudaFuncSetAttribute(sparse_decode_attn_kernel<D, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -673,7 +696,7 @@ size_t attn_workspace_bytes(int B, int Hq, int Hkv, int D, int num_sms) {
   const int G = Hq / Hkv;
   const size_t slot = static_cast<size_t>(2 * G + G * D) * sizeof(float);
   const size_t parts = static_cast<size_t>(num_sms) * kAttnMaxCtasPerSm * 2 * slot;
-  const size_t sems = static_cast<size_t>(B) * Hkv * sizeof(int32_t);
+  const size_t sems = static_cast<size_t>(B) * Hq * sizeof(int32_t);  // rows: B*Hkv, or B*Hq
   return ((sems + 255) & ~static_cast<size_t>(255)) + ((parts + 255) & ~static_cast<size_t>(255));
 }
 
@@ -700,15 +723,18 @@ cudaError_t launch_sparse_decode_attn(const AttnArgs &a, void *ws, int num_sms,
   else
     V = (static_cast<long long>(a.cap) * a.tpi + kStageTok - 1) / kStageTok;
   if (V < 1) V = 1;
-  const long long rows = static_cast<long long>(a.B) * a.Hkv;
-  const int G = a.Hq / a.Hkv;
   AttnDev p;
   p.a = a;
+  const bool per_q = a.shared == 2;  // one list per query head
+  p.rpb = per_q ? a.Hq : a.Hkv;
+  p.gw = per_q ? 1 : a.Hq / a.Hkv;
+  const long long rows = static_cast<long long>(a.B) * p.rpb;
   p.V = static_cast<int>(V);
   p.W = rows * V;
   p.N = 1;
-  p.slot = 2 * G + G * a.D;
-  const size_t sems = static_cast<size_t>(rows) * sizeof(int32_t);
+  p.slot = 2 * p.gw + p.gw * a.D;
+  // the semaphore region is sized for B*Hq rows in either case (attn_workspace_bytes)
+  const size_t sems = static_cast<size_t>(a.B) * a.Hq * sizeof(int32_t);
   p.sem = static_cast<int32_t *>(ws);
   p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
                                      ((sems + 255) & ~static_cast<size_t>(255)));

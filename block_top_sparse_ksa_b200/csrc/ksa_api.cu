@@ -63,8 +63,8 @@ ksa_status check_shape(const ksa_shape *s, bool need_block) {
   const long long rows = static_cast<long long>(s->batch) * s->num_kv_heads * s->capacity;
   if (rows >= (1LL << 31))
     return fail(KSA_ERR_UNSUPPORTED, "batch * num_kv_heads * capacity must be < 2^31");
-  if (static_cast<long long>(s->batch) * s->num_kv_heads * 8 >= (1LL << 31))
-    return fail(KSA_ERR_UNSUPPORTED, "batch * num_kv_heads too large");
+  if (static_cast<long long>(s->batch) * s->num_q_heads * 8 >= (1LL << 31))
+    return fail(KSA_ERR_UNSUPPORTED, "batch * num_q_heads too large");
   return KSA_OK;
 }
 
@@ -373,8 +373,9 @@ ksa_status attn_common(const ksa_shape *shape, const uint16_t *q, const uint16_t
         (tokens_per_idx & (tokens_per_idx - 1)) != 0)
       return fail(KSA_ERR_UNSUPPORTED, "tokens_per_idx %d is not a power of two in [1, 256]",
                   tokens_per_idx);
-    if (idx_shared != 0 && idx_shared != 1)
-      return fail(KSA_ERR_INVALID_ARG, "idx_shared must be 0 or 1");
+    if (idx_shared != KSA_IDX_PER_KV_HEAD && idx_shared != KSA_IDX_SHARED &&
+        idx_shared != KSA_IDX_PER_Q_HEAD)
+      return fail(KSA_ERR_INVALID_ARG, "idx_shared must be 0, 1 or 2");
     if (!aligned(idx, 4) || !aligned(num_idx, 4))
       return fail(KSA_ERR_INVALID_ARG, "idx and num_idx must be 4-byte aligned");
   }
@@ -506,6 +507,60 @@ ksa_status ksa_unified_select(const ksa_shape *shape, const uint16_t *q, const u
   return cuda_status(
       ksa::launch_unified_select(a, device_sm_count(), static_cast<cudaStream_t>(stream)),
       "ksa_unified_select launch");
+}
+
+size_t ksa_select_tokens_per_head_workspace(const ksa_shape *shape, int32_t k_tokens) {
+  (void)k_tokens;
+  if (shape == nullptr || shape->batch < 1 || shape->num_q_heads < 1 || shape->capacity < 1)
+    return 0;
+  return ksa::unified_workspace_bytes(shape->batch, shape->num_q_heads, shape->capacity);
+}
+
+ksa_status ksa_select_tokens_per_head(const ksa_shape *shape, const uint16_t *q,
+                                      const uint16_t *K, const int32_t *seq_lens,
+                                      int32_t k_tokens, int32_t *token_idx, int32_t *num_sel,
+                                      void *ws, size_t ws_bytes, uint32_t *dev_status,
+                                      void *stream) {
+  ksa_status st = check_shape(shape, false);
+  if (st != KSA_OK) return st;
+  if (q == nullptr || K == nullptr || seq_lens == nullptr || token_idx == nullptr ||
+      num_sel == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "q, K, seq_lens, token_idx and num_sel must be non-NULL");
+  const int G = shape->num_q_heads / shape->num_kv_heads;
+  if (G > 8) return fail(KSA_ERR_UNSUPPORTED, "query heads per kv-head = %d exceeds 8", G);
+  if (shape->capacity > 65536)
+    return fail(KSA_ERR_UNSUPPORTED, "capacity %d exceeds 65536", shape->capacity);
+  if (k_tokens < 1) return fail(KSA_ERR_INVALID_ARG, "k_tokens must be >= 1");
+  const size_t need =
+      ksa::unified_workspace_bytes(shape->batch, shape->num_q_heads, shape->capacity);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (!aligned(K, 16) || !aligned(q, 4))
+    return fail(KSA_ERR_INVALID_ARG, "K must be 16-byte aligned");
+  ksa::UnifiedArgs a;
+  a.q = q;
+  a.K = K;
+  a.seq_lens = seq_lens;
+  a.token_idx = token_idx;
+  a.num_sel = num_sel;
+  const size_t keys_bytes =
+      (static_cast<size_t>(shape->batch) * shape->num_q_heads * shape->capacity * 4 + 255) &
+      ~static_cast<size_t>(255);
+  a.keys = static_cast<uint32_t *>(ws);
+  a.votes = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + keys_bytes);
+  a.bits = nullptr;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hq = shape->num_q_heads;
+  a.Hkv = shape->num_kv_heads;
+  a.D = shape->head_dim;
+  a.T = shape->capacity;
+  a.P = k_tokens;
+  a.budget = k_tokens;  // rows with L <= k keep every token and need no scores
+  a.R = 0;
+  return cuda_status(ksa::launch_tokens_per_head(a, static_cast<cudaStream_t>(stream)),
+                     "ksa_select_tokens_per_head launch");
 }
 
 const char *ksa_status_string(ksa_status status) {

@@ -98,6 +98,8 @@ struct UnifiedArgs {
 };
 size_t unified_workspace_bytes(int B, int Hq, int T);
 cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream);
+// Per-head token top-k lists (P = k = budget; token_idx [B, Hq, k], num_sel [B, Hq]).
+cudaError_t launch_tokens_per_head(const UnifiedArgs &a, cudaStream_t stream);
 
 // Records a message for ksa_last_error() and returns `status`.
 ksa_status set_last_error(ksa_status status, const char *fmt, ...)

@@ -78,7 +78,8 @@ extern "C" ksa_status ksa_sparse_decode_attn_noalloc(
   if (st != KSA_OK) return st;
   // The scratch keeps whatever the previous call left; the per-row semaphores
   // at its start must be zero when the kernel starts.
-  const size_t rows = static_cast<size_t>(shape->batch) * shape->num_kv_heads;
+  // (the semaphore region covers B * Hq rows, the most any list mode uses)
+  const size_t rows = static_cast<size_t>(shape->batch) * shape->num_q_heads;
   const size_t sem_bytes = (rows * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
   const cudaError_t err =
       cudaMemsetAsync(scratch, 0, sem_bytes, static_cast<cudaStream_t>(stream));

@@ -402,6 +402,39 @@ __global__ void __launch_bounds__(256) unified_votes_kernel(const UnifiedArgs a)
   a.votes[static_cast<size_t>(b) * a.T + t] = v;
 }
 
+// Per-head token top-k lists: CTA per (row, query head), the k highest score
+// keys (ties to the lower token) listed ascending with -1 padding; rows with
+// L <= k keep every token.  Keys staged in shared memory when they fit.
+__global__ void __launch_bounds__(kPickThreads) unified_topk_list_kernel(const UnifiedArgs a,
+                                                                          int stage_in_smem) {
+  extern __shared__ uint32_t skeys[];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t info[4];
+  __shared__ uint32_t scratch[33];
+  const int b = blockIdx.x / a.Hq, h = blockIdx.x % a.Hq;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int L = clamp_len(a.seq_lens[b], a.T, (h == 0 && threadIdx.x == 0) ? a.status : nullptr);
+  const int k = a.P;
+  int32_t *out = a.token_idx + (static_cast<size_t>(b) * a.Hq + h) * k;
+  if (L <= k) {
+    for (int i = threadIdx.x; i < k; i += kPickThreads) out[i] = i < L ? i : -1;
+    if (threadIdx.x == 0) a.num_sel[static_cast<size_t>(b) * a.Hq + h] = L;
+    return;
+  }
+  const uint32_t *gkeys = a.keys + (static_cast<size_t>(b) * a.Hq + h) * a.T;
+  const uint32_t *keys = gkeys;
+  if (stage_in_smem) {
+    for (int t = threadIdx.x; t < L; t += kPickThreads) skeys[t] = gkeys[t];
+    __syncthreads();
+    keys = skeys;
+  }
+  uint32_t tau, n_gt, n_eq;
+  radix_select_desc<kPickThreads>(keys, L, k, 32, hist, info, tau, n_gt, n_eq);
+  select_ascending<kPickThreads>(keys, L, tau, n_gt, n_eq, k, out, scratch, [](int) {});
+  if (threadIdx.x == 0) a.num_sel[static_cast<size_t>(b) * a.Hq + h] = k;
+}
+
 // Shared set: CTA per row.
 __global__ void __launch_bounds__(kSetThreads) unified_set_kernel(const UnifiedArgs a) {
   __shared__ uint32_t hist[256];
@@ -455,6 +488,19 @@ size_t unified_workspace_bytes(int B, int Hq, int T) {
   const size_t bits =
       (static_cast<size_t>(B) * Hq * ((T + 31) / 32) * sizeof(uint32_t) + 255) & ~static_cast<size_t>(255);
   return keys + votes + bits;
+}
+
+cudaError_t launch_tokens_per_head(const UnifiedArgs &a, cudaStream_t stream) {
+  // the scoring launch skips rows with L <= budget: here the budget is k
+  cudaError_t err = a.D == 128 ? launch_scores<128>(a, stream) : launch_scores<64>(a, stream);
+  if (err != cudaSuccess) return err;
+  const int in_smem = a.T <= kSmemKeys ? 1 : 0;
+  const size_t smem = in_smem ? static_cast<size_t>(a.T) * sizeof(uint32_t) : 0;
+  err = cudaFuncSetAttribute(unified_topk_list_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(unified_topk_list_kernel, dim3(static_cast<unsigned>(a.B) * a.Hq),
+                    dim3(kPickThreads), smem, stream, a, in_smem);
 }
 
 cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream) {

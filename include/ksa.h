@@ -70,6 +70,8 @@ enum { KSA_SUMMARY_ALL = 0, KSA_SUMMARY_LAST_BLOCK = 1 };
 /* Storage type of the block summaries (the *_ex entry points). */
 enum { KSA_SUMMARIES_F32 = 0, KSA_SUMMARIES_BF16 = 1 };
 enum { KSA_OUT_F32 = 0, KSA_OUT_BF16 = 1 };
+/* Index-list layouts of ksa_sparse_decode_attn (idx_shared). */
+enum { KSA_IDX_PER_KV_HEAD = 0, KSA_IDX_SHARED = 1, KSA_IDX_PER_Q_HEAD = 2 };
 
 enum {
   KSA_FLAG_SEQ_LEN_CLAMPED = 1u << 0, /* some seq_len was outside [1, T] */
@@ -130,6 +132,27 @@ ksa_status ksa_decode_select_blocks(const ksa_shape *shape, const uint16_t *q,
                                     const int32_t *seq_lens, int32_t k_blocks,
                                     int32_t *block_idx, int32_t *num_sel, void *ws,
                                     size_t ws_bytes, uint32_t *dev_status, void *stream);
+
+/*
+ * Token-level sparse attention's selection [KIN s.5: the ideal, per-token
+ * top-K; costly, the reason for blocks]: every query head h of row b keeps its
+ * own k_tokens highest-scoring tokens, s_t = <q[b,h,:], K[b,g,t,:]> over
+ * t < L_b (exact fp32 products of bf16, ties to the lower t), listed
+ * ascending and -1 padded.  If L_b <= k_tokens every token is kept.  Use the
+ * lists with ksa_sparse_decode_attn, idx_shared = KSA_IDX_PER_Q_HEAD,
+ * tokens_per_idx = 1.
+ *   q: [B, Hq, D] bf16;  K: [B, Hkv, T, D] bf16
+ *   token_idx: [B, Hq, k_tokens] int32;  num_sel: [B, Hq] int32 (written)
+ *   ws: device scratch of ksa_select_tokens_per_head_workspace() bytes,
+ *       256-byte aligned, no initialisation needed.
+ * Limits: G <= 8; capacity <= 65536; k_tokens >= 1.
+ */
+size_t ksa_select_tokens_per_head_workspace(const ksa_shape *shape, int32_t k_tokens);
+ksa_status ksa_select_tokens_per_head(const ksa_shape *shape, const uint16_t *q,
+                                      const uint16_t *K, const int32_t *seq_lens,
+                                      int32_t k_tokens, int32_t *token_idx,
+                                      int32_t *num_sel, void *ws, size_t ws_bytes,
+                                      uint32_t *dev_status, void *stream);
 
 /*
  * Local attention as a block selection [KIN s.5 compares block top-k with
@@ -211,8 +234,12 @@ ksa_status ksa_decode_select_blocks_paged(const ksa_shape *shape, const uint16_t
  * of the list names tokens [idx*tpi, idx*tpi + tpi) with tpi =
  * tokens_per_idx (block_size for block lists, 1 for token lists); tokens
  * t >= L_b are dropped (partial tail block).  The list is [B, Hkv, cap]
- * with num_idx [B, Hkv] (idx_shared == 0), or [B, cap] with num_idx [B]
- * shared by every kv-head (idx_shared == 1, the LessIsMore layout).
+ * with num_idx [B, Hkv] (idx_shared == KSA_IDX_PER_KV_HEAD: one set per GQA
+ * group), [B, cap] with num_idx [B] shared by every kv-head (KSA_IDX_SHARED,
+ * the LessIsMore layout), or [B, Hq, cap] with num_idx [B, Hq], one set per
+ * query head (KSA_IDX_PER_Q_HEAD, e.g. the per-head token top-k of
+ * ksa_select_tokens_per_head; each head then reads its own K/V rows, so the
+ * group no longer shares one gather).
  * Entries are expected distinct; a negative entry or one naming no token
  * below L_b is skipped and flagged.  An empty set gives out = 0,
  * lse = -inf.  Accumulation is fp32; scale == 0 selects 1/sqrt(D).

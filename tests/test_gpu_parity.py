@@ -727,3 +727,38 @@ def test_select_window_matches_oracle(ksa, oracle):
             ref_idx, ref_cnt = oracle.select_window(lens, 3, bs, k)
             assert np.array_equal(idx.cpu().numpy(), ref_idx)
             assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+
+
+# ---------------------------------------------------------------------------
+# per-head token top-k and attention with one list per query head
+
+
+@pytest.mark.parametrize("L,k", [(300, 40), (1500, 400), (90, 200)])
+def test_tokens_per_head_and_per_query_head_attention(ksa, oracle, L, k):
+    """Dyadic q, K: exact scores, exact ties.  Every head's list equals the oracle's; the
+    attention over per-query-head lists equals the oracle run head by head."""
+    rng = np.random.default_rng(1600 + L)
+    B, Hq, Hkv, D = 2, 8, 2, 128
+    G = Hq // Hkv
+    T = L + 13
+    q = dyadic_bits(rng, (B, Hq, D))
+    K = dyadic_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([L, max(1, L // 3)], np.int32)
+    qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
+    st = status_tensor()
+    idx, cnt = ksa.ksa_select_tokens_per_head(qd, Kd, Ld, k, dev_status=st)
+    ref_idx, ref_cnt = oracle.select_tokens_per_head(q, K, lens, k)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=DEV)
+    out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, idx, cnt, tokens_per_idx=1,
+                                        idx_shared=ksa.IDX_PER_Q_HEAD, lse=lse, dev_status=st)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for h in range(Hq):
+        g = h // G
+        ref, ref_lse, _ = oracle.attention(q[:, h:h + 1], K[:, g:g + 1], V[:, g:g + 1], lens,
+                                           ref_idx[:, h:h + 1], ref_cnt[:, h:h + 1], 1)
+        assert_out_close(out[:, h], ref[:, 0])
+        np.testing.assert_allclose(lse[:, h], ref_lse[:, 0], rtol=0, atol=LSE_TOL)
+    assert st.item() == 0
