@@ -200,17 +200,6 @@ __device__ __forceinline__ void cp_async_16(void *dst, const void *src) {
                : "memory");
 }
 
-// Closes this thread's current group of cp.async copies.
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Waits until at most N of this thread's committed cp.async groups are pending.
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Arrive on `bar` once all cp.async issued so far by this thread have landed.
 // Counts as one of the barrier's expected arrivals.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
