@@ -509,7 +509,8 @@ def run_unified(args, dist, dev):
                      "bytes_per_launch": att_b},
         "select_hbm": {"bytes_per_launch": sel_b, "gbs": sel_b / (t_sel * 1e-3) / 1e9},
         "step_hbm": {"bytes_per_step": sel_b + 3 * att_b,
-                     "gbs": (sel_b + 3 * att_b) / per / 1e9},
+                     "gbs": (sel_b + 3 * att_b) / per / 1e9,
+                     "frac": (sel_b + 3 * att_b) / per / 1e9 / peak},
         # selection: scores, picks, (vote counting when the picks keep the row's keys in
         # registers: capacity <= 24576), shared set; then one attention launch per layer
         "gpu_launches": ((4 if T <= 24576 else 3) + len(inp.layers)) * args.steps, "clocks": clk,
