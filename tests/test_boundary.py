@@ -115,3 +115,43 @@ def test_missing_workspace_is_rejected(ksa):
                                  None) == 3
     assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, None, None, 0, 1,
                                       0, 0.0, 0, FAKE, None, None, 0, None, None) == 3
+
+
+def test_validation_of_the_newer_entry_points(ksa):
+    """Storage type, window, per-head top-k, paged caches and list layouts are checked on the
+    host before any device work."""
+    lib = ksa.lib()
+    sh = _shape(ksa)
+    BIG = 1 << 30
+    # summary storage type out of range
+    assert lib.ksa_build_block_summaries_ex(ctypes.byref(sh), FAKE, FAKE, 0, 7, FAKE, None,
+                                            None) == 1
+    assert lib.ksa_select_blocks_ex(ctypes.byref(sh), FAKE, FAKE, 2, FAKE, 4, FAKE, FAKE, FAKE,
+                                    BIG, None, None) == 1
+    # window: k < 1, NULL output, unsupported block size
+    assert lib.ksa_select_window(ctypes.byref(sh), FAKE, 0, FAKE, FAKE, None, None) == 1
+    assert lib.ksa_select_window(ctypes.byref(sh), FAKE, 4, None, FAKE, None, None) == 1
+    assert lib.ksa_select_window(ctypes.byref(_shape(ksa, bs=8)), FAKE, 4, FAKE, FAKE, None,
+                                 None) == 2
+    # per-head top-k: k < 1, G > 8, capacity above 65536
+    assert lib.ksa_select_tokens_per_head(ctypes.byref(sh), FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE,
+                                          BIG, None, None) == 1
+    assert lib.ksa_select_tokens_per_head(ctypes.byref(_shape(ksa, Hq=32, Hkv=2)), FAKE, FAKE,
+                                          FAKE, 4, FAKE, FAKE, FAKE, BIG, None, None) == 2
+    assert lib.ksa_select_tokens_per_head(ctypes.byref(_shape(ksa, T=70000)), FAKE, FAKE, FAKE, 4,
+                                          FAKE, FAKE, FAKE, BIG, None, None) == 2
+    # paged caches: no pages, capacity != max_blocks * block_size, empty pool
+    assert lib.ksa_build_block_summaries_paged(ctypes.byref(sh), FAKE, None, FAKE, 0, 0, FAKE,
+                                               None, None) == 1
+    bad_cap = ksa.Pages(FAKE, 3, 10)  # 3 * 16 != 64
+    assert lib.ksa_build_block_summaries_paged(ctypes.byref(sh), FAKE, ctypes.byref(bad_cap),
+                                               FAKE, 0, 0, FAKE, None, None) == 1
+    no_pages = ksa.Pages(FAKE, 4, 0)
+    assert lib.ksa_build_block_summaries_paged(ctypes.byref(sh), FAKE, ctypes.byref(no_pages),
+                                               FAKE, 0, 0, FAKE, None, None) == 1
+    assert lib.ksa_decode_select_blocks_paged(ctypes.byref(sh), FAKE, FAKE, ctypes.byref(bad_cap),
+                                              FAKE, 0, FAKE, 4, FAKE, FAKE, FAKE, BIG, None,
+                                              None) == 1
+    # attention list layout out of range
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1,
+                                      3, 0.0, 0, FAKE, None, None, 0, None, None) == 1
