@@ -4,6 +4,7 @@ Selected indices must match bit-exactly (inputs carry a planted score gap, or
 are dyadic so that every score is exact in fp32); attention outputs must meet
 max|d| <= 2e-3 and max|d| / max|ref| <= 1e-2, lse within 1e-4.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -422,6 +423,54 @@ def test_long_pipelines(ksa, oracle, mode):
         idx = np.sort(rng.choice(lens[0], size=8192, replace=False))[None].astype(np.int32)
         cnt = np.array([8192], np.int32)
         assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, 1, shared=True) == 0
+
+
+@pytest.mark.parametrize("mode", ["dense", "blocks", "tokens"])
+def test_long_rows_repeat_calls(ksa, oracle, mode):
+    """Rows of 1536-2048 stages, each split between many CTAs, over 24K+ stages in all.  Every
+    output matches the oracle; three calls on one workspace give the same bits (the split and
+    the merge order are fixed); the row semaphores are zero again after every call."""
+    rng = np.random.default_rng(810)
+    B, Hq, Hkv, D, T, bs = 4, 8, 4, 128, 32768, 16
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([T, T - 5, 25000, 30001], np.int32)
+    idx = cnt = None
+    tpi, shared = 1, False
+    if mode == "blocks":  # 1536 of each row's blocks: 1536 stages a row
+        tpi = bs
+        idx = np.zeros((B, Hkv, 1536), np.int32)
+        for b in range(B):
+            nb = -(-int(lens[b]) // bs)
+            for g in range(Hkv):
+                idx[b, g] = np.sort(rng.choice(nb, size=1536, replace=False))
+        cnt = np.full((B, Hkv), 1536, np.int32)
+    elif mode == "tokens":  # one shared set of 24576 tokens a row: 1536 stages a row
+        shared = True
+        idx = np.stack([np.sort(rng.choice(int(lens[b]), size=24576, replace=False))
+                        for b in range(B)]).astype(np.int32)
+        cnt = np.full((B,), 24576, np.int32)
+    qd, Kd, Vd = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V)
+    Ld = torch.from_numpy(lens).to(DEV)
+    idx_d = None if idx is None else torch.from_numpy(idx).to(DEV)
+    cnt_d = None if cnt is None else torch.from_numpy(cnt).to(DEV)
+    cap = T if mode == "dense" else idx.shape[-1]
+    ws = torch.zeros((ksa.lib().ksa_sparse_decode_attn_workspace(
+        ctypes.byref(ksa.Shape(B, Hq, Hkv, D, T, bs)), cap, tpi),), dtype=torch.uint8, device=DEV)
+    head = (B * Hq * 4 + 255) // 256 * 256  # the semaphores
+    outs = []
+    for _ in range(3):
+        st = status_tensor()
+        out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, idx_d, cnt_d, tokens_per_idx=tpi,
+                                            idx_shared=shared, workspace=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        assert int(ws[:head].count_nonzero()) == 0
+        outs.append(out.cpu().numpy())
+    assert all(np.array_equal(outs[0].view(np.uint32), o.view(np.uint32)) for o in outs[1:])
+    ref, _, _ = oracle.attention(q, K, V, lens, idx, cnt, tpi, shared)
+    assert_out_close(outs[0], ref)
 
 
 @pytest.mark.parametrize("D,bs,k,nblk", [(128, 16, 8, 40), (64, 32, 6, 40), (64, 16, 12, 1100)])

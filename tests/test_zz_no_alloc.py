@@ -61,6 +61,7 @@ def _raw_noalloc(ksa, q, K, V, lens, idx, cnt, bs, out, lse):
     (16, 16, 8, 128, 4096, 32, 16),   # many rows: most rows held by one CTA
     (1, 8, 2, 128, 32768, 16, 1024),  # two long rows split over many CTAs (partials + semaphores)
     (3, 8, 4, 64, 2048, 16, 40),      # D = 64
+    (8, 16, 8, 128, 16384, 16, 512),  # 32768 stages, ~74 per CTA: most rows split in two
 ])
 def test_noalloc_matches_workspace_entry_point_twice(ksa, B, Hq, Hkv, D, T, bs, k):
     q, K, V, lens, idx, cnt = _inputs(B, Hq, Hkv, D, T, bs, k, seed=B * 1000 + T)
@@ -82,7 +83,7 @@ def test_noalloc_binding_and_size_limit(ksa):
     out, _ = ksa.ksa_sparse_decode_attn_noalloc(q, K, V, lens, idx, cnt, tokens_per_idx=16)
     assert_out_close(out.cpu().numpy(), ref.cpu().numpy())
     # a shape whose workspace exceeds the fixed scratch is refused before any work
-    big = ksa.Shape(65536, 64, 64, 128, 16, 16)  # 4M (row, kv-head) semaphores alone = 16 MiB
+    big = ksa.Shape(65536, 64, 64, 128, 16, 16)  # 4M row semaphores alone fill the 16 MiB
     fake = ctypes.c_void_p(0x1000)
     st = ksa.lib().ksa_sparse_decode_attn_noalloc(
         ctypes.byref(big), fake, fake, fake, fake, None, None, 0, 1, 0, 0.0, 0, fake, None, None,
