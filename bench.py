@@ -248,13 +248,15 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
-def stored_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel source
-    is unchanged since the capture (else None)."""
+def stored_traffic(kernel: str, workload: str, batch: int):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken at this batch and
+    the kernel source is unchanged since (else None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
         ent = rec[kernel][workload]
+        if int(ent["batch"]) != batch:
+            return None
         src = open(os.path.join(ROOT, ent["source"]), "rb").read()
         if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha256_16"]:
             return None
@@ -355,7 +357,7 @@ def run_block(args, dist, dev, kind):
                        {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att}),
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                      "frac": attn_gbs / peak,
-                     "traffic": stored_traffic("sparse_decode_attn", args.workload),
+                     "traffic": stored_traffic("sparse_decode_attn", args.workload, shape.batch),
                      "kernel": "sparse_decode_attn", "peak_source": peak_kind,
                      "bytes_per_launch": attn_b},
         "step_hbm": {"bytes_per_step": total_b, "gbs": total_b / per_step_s / 1e9,
@@ -504,7 +506,7 @@ def run_unified(args, dist, dev):
         "kernels_ms": {"unified_select": t_sel, "sparse_decode_attn_per_layer": t_att},
         "roofline": {"bound": "hbm", "achieved": att_b / (t_att * 1e-3) / 1e9, "peak": peak,
                      "unit": "GB/s", "frac": att_b / (t_att * 1e-3) / 1e9 / peak,
-                     "traffic": stored_traffic("sparse_decode_attn", args.workload),
+                     "traffic": stored_traffic("sparse_decode_attn", args.workload, sh.batch),
                      "kernel": "sparse_decode_attn (token list)", "peak_source": peak_kind,
                      "bytes_per_launch": att_b},
         "select_hbm": {"bytes_per_launch": sel_b, "gbs": sel_b / (t_sel * 1e-3) / 1e9},
