@@ -1,7 +1,7 @@
 """Attention recall of a token selection, and the LessIsMore recency-ratio sweep.
 
 LessIsMore (evaluation of the unified selection and of the recency window)
-judges a selection by how much of each head's full attention it keeps.  For
+rates a selection by how much of each head's full attention it keeps.  For
 query head h of row b and a selected token set T_sel,
 
     recall[b, h] = sum_{t in T_sel} softmax(z)_t,   z_t = scale * <q_h, K_t>, t < L_b,
