@@ -47,6 +47,28 @@ MUTANTS = [
     ("recency window shifted by one", "for (int t = L - R; t < L; ++t) pick[n++] = t;",
      "for (int t = L - R - 1; t < L - 1; ++t) pick[n++] = t;", 0,
      [pins.test_unified_closed_forms]),
+    ("bf16 ties rounded away from zero",
+     "if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;",
+     "if (frac >= 0.5) r += 1.0;", 0,
+     [lambda o: pins.test_round_bf16_format_values(o, 1.0 + 2.0 ** -8, 0x3F80)]),
+    ("bf16 grid one bit too coarse", "int q = e - 8;", "int q = e - 7;", 0,
+     [pins.test_round_bf16_matches_torch_on_binary32]),
+    ("bf16 subnormal spacing of the normal range", "if (q < -133) q = -133;",
+     "if (q < -126) q = -126;", 0,
+     [lambda o: pins.test_round_bf16_format_values(o, 2.0 ** -133, 0x0001)]),
+    ("bf16 summary storage never applied", "if (summary_bf16) {", "if (0) {", 0,
+     [pins.test_select_blocks_bf16_storage_tie]),
+    ("page row ignores the kv-head",
+     "pages + (((size_t)page * Hkv + g) * bs + t % bs) * D;",
+     "pages + (((size_t)page * Hkv) * bs + t % bs) * D;", 0,
+     [pins.test_gather_pages_identity_table]),
+    ("token offset within a page off by one",
+     "pages + (((size_t)page * Hkv + g) * bs + t % bs) * D;",
+     "pages + (((size_t)page * Hkv + g) * bs + (t + 1) % bs) * D;", 0,
+     [pins.test_gather_pages_scatter_roundtrip_and_bad_pages]),
+    ("window one block early", "row[i] = i < n ? nb - n + i : -1;",
+     "row[i] = i < n ? nb - n + i - 1 : -1;", 0,
+     [pins.test_select_window_is_topk_of_a_recency_score]),
 ]
 
 
