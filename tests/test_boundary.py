@@ -155,3 +155,22 @@ def test_validation_of_the_newer_entry_points(ksa):
     # attention list layout out of range
     assert lib.ksa_sparse_decode_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1,
                                       3, 0.0, 0, FAKE, None, None, 0, None, None) == 1
+
+
+def test_sizes_past_32_bit_row_indices_are_refused(ksa):
+    """K/V row coordinates are 32-bit on the device: caches of 2^31 rows or more, and page
+    pools of that size, are refused on the host (KSA_ERR_UNSUPPORTED), never run."""
+    lib = ksa.lib()
+    big = _shape(ksa, B=1024, Hq=16, Hkv=8, T=1 << 18, bs=16)  # 1024 * 8 * 2^18 = 2^31 rows
+    assert lib.ksa_select_blocks(ctypes.byref(big), FAKE, FAKE, FAKE, 4, FAKE, FAKE, FAKE,
+                                 1 << 30, None, None) == 2
+    assert lib.ksa_sparse_decode_attn(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, None, None, 0,
+                                      1, 0, 0.0, 0, FAKE, None, None, 0, None, None) == 2
+    assert lib.ksa_select_blocks_workspace(ctypes.byref(big), 4) == 0
+    just_under = _shape(ksa, B=1023, Hq=16, Hkv=8, T=1 << 18, bs=16)
+    assert lib.ksa_select_blocks_workspace(ctypes.byref(just_under), 4) > 0
+    sh = _shape(ksa, B=1, Hq=4, Hkv=2, D=128, T=64, bs=16)
+    pool = ksa.Pages(FAKE, 4, 1 << 26)  # 2^26 pages * 2 kv-heads * 16 rows = 2^31
+    assert lib.ksa_sparse_decode_attn_paged(ctypes.byref(sh), FAKE, FAKE, FAKE,
+                                            ctypes.byref(pool), FAKE, FAKE, FAKE, 4, 16, 0, 0.0,
+                                            0, FAKE, None, FAKE, 1 << 30, None, None) == 2
