@@ -174,3 +174,52 @@ def test_sizes_past_32_bit_row_indices_are_refused(ksa):
     assert lib.ksa_sparse_decode_attn_paged(ctypes.byref(sh), FAKE, FAKE, FAKE,
                                             ctypes.byref(pool), FAKE, FAKE, FAKE, 4, 16, 0, 0.0,
                                             0, FAKE, None, FAKE, 1 << 30, None, None) == 2
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "ksa.h"
+
+int main(void) {
+  ksa_shape sh;
+  ksa_status st;
+  memset(&sh, 0, sizeof sh);
+  if (ksa_version() < 100) return 1;
+  if (strcmp(ksa_status_string(KSA_ERR_UNSUPPORTED), "KSA_ERR_UNSUPPORTED") != 0) return 2;
+  /* a NULL shape and an empty batch are refused on the host, with a message */
+  st = ksa_select_blocks(NULL, NULL, NULL, NULL, 4, NULL, NULL, NULL, 0, NULL, NULL);
+  if (st != KSA_ERR_INVALID_ARG || ksa_last_error()[0] == '\0') return 3;
+  sh.batch = 0; sh.num_q_heads = 4; sh.num_kv_heads = 2; sh.head_dim = 128;
+  sh.capacity = 64; sh.block_size = 16;
+  st = ksa_sparse_decode_attn(&sh, NULL, NULL, NULL, NULL, NULL, NULL, 0, 1, KSA_IDX_PER_KV_HEAD,
+                              0.0f, KSA_OUT_F32, NULL, NULL, NULL, 0, NULL, NULL);
+  if (st != KSA_ERR_INVALID_ARG) return 4;
+  sh.batch = 2;
+  if (ksa_select_blocks_workspace(&sh, 4) == 0) return 5;
+  printf("ok %d\n", (int)ksa_version());
+  return 0;
+}
+"""
+
+
+@pytest.mark.parametrize("lang", ["c99", "c++11"])
+def test_c_caller_builds_links_and_runs(ksa, tmp_path, lang):
+    """A plain C (and C++) program includes include/ksa.h, links libksa.so and makes the
+    host-only calls: version, status strings, validation errors, workspace sizes."""
+    import shutil
+    import subprocess
+    src = tmp_path / ("caller.c" if lang == "c99" else "caller.cpp")
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(ksa.library_path)
+    cc = "gcc" if lang == "c99" else "g++"
+    if shutil.which(cc) is None:
+        pytest.skip(f"{cc} not found")
+    cmd = [cc, f"-std={lang}", "-Wall", "-Wextra", "-Werror", "-pedantic",
+           "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+           "-L", libdir, "-l:" + os.path.basename(ksa.library_path), "-Wl,-rpath," + libdir]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.startswith("ok ")
