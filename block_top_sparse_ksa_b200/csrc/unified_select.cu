@@ -5,7 +5,8 @@
 // top tokens, the votes are pooled into one token set shared by all heads,
 // and the budget is split between voted tokens and the most recent tokens.
 //
-// Three launches on the caller's stream:
+// Launches on the caller's stream (four when every row has at most 24576 tokens:
+// the votes get a kernel of their own; three otherwise):
 //  1. scores: one CTA per (row, kv-head, 1024-token chunk).  A producer warp
 //     streams the chunk's keys with TMA (128B swizzle); four consumer warps
 //     form S^T = K_tile q^T for the kv-group's G heads with mma.sync
@@ -16,8 +17,8 @@
 //     lower token.  Rows of up to 24576 tokens keep their keys in registers,
 //     run an adaptive radix (each pass starts at the highest bit in which the
 //     remaining candidates differ) and write the picks as bit sets, from which
-//     a per-token kernel counts the votes; longer rows stage the keys in shared
-//     memory and add one atomic vote per pick.
+//     a per-token kernel then counts the votes (2b); longer rows stage the keys
+//     in shared memory and add one atomic vote per pick.
 //  3. shared set: one CTA per row.  Radix select on the vote counts of
 //     [0, L - R) for the (budget - R) most voted tokens (ties to the lower
 //     token), written ascending, followed by the window [L - R, L).
