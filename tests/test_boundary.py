@@ -223,3 +223,34 @@ def test_c_caller_builds_links_and_runs(ksa, tmp_path, lang):
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert out.stdout.startswith("ok ")
+
+
+def test_no_fallback_without_the_library_or_a_gpu(tmp_path):
+    """The product path has no CPU fallback: CPU tensors are refused before any call, and a
+    missing library is an error naming the build step (checked in a fresh interpreter)."""
+    import subprocess
+    import sys
+    code = (
+        "import sys, torch\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "import block_top_sparse_ksa_b200 as k\n"
+        "q = torch.zeros((1, 4, 128), dtype=torch.bfloat16)\n"
+        "K = torch.zeros((1, 2, 64, 128), dtype=torch.bfloat16)\n"
+        "L = torch.full((1,), 64, dtype=torch.int32)\n"
+        "try:\n"
+        "    k.ksa_sparse_decode_attn(q, K, K, L)\n"
+        "    sys.exit('CPU tensors were accepted')\n"
+        "except TypeError as e:\n"
+        "    assert 'CUDA tensor' in str(e), e\n"
+        f"k.library_path = {str(tmp_path / 'libksa_absent.so')!r}\n"
+        "k._LIB = None\n"
+        "try:\n"
+        "    k.lib()\n"
+        "    sys.exit('a missing library loaded')\n"
+        "except RuntimeError as e:\n"
+        "    assert 'missing' in str(e) and 'build' in str(e), e\n"
+        "print('ok')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip().endswith("ok")
