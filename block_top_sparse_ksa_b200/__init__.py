@@ -17,6 +17,7 @@ import ctypes
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 __all__ = [
@@ -28,7 +29,8 @@ __all__ = [
     "ksa_build_block_summaries_ex", "ksa_select_blocks_ex", "ksa_decode_select_blocks_ex",
     "ksa_build_block_summaries_paged", "ksa_decode_select_blocks_paged",
     "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window", "ksa_select_tokens_per_head",
-    "ksa_select_tokens_per_head_workspace", "IDX_PER_KV_HEAD", "IDX_SHARED", "IDX_PER_Q_HEAD",
+    "ksa_select_tokens_per_head_workspace", "ksa_select_tokens_one_head",
+    "ksa_select_tokens_one_head_workspace", "IDX_PER_KV_HEAD", "IDX_SHARED", "IDX_PER_Q_HEAD",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -85,6 +87,9 @@ _SIGS = {
                                             _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "ksa_select_window": (_i32, [ctypes.POINTER(Shape), _vp, _i32, _vp, _vp, _vp, _vp]),
     "ksa_select_tokens_per_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
+    "ksa_select_tokens_one_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
+    "ksa_select_tokens_one_head": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _i32, _vp,
+                                          _vp, _vp, _sz, _vp, _vp]),
     "ksa_select_tokens_per_head": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp,
                                           _vp, _sz, _vp, _vp]),
     "ksa_select_blocks_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
@@ -549,4 +554,50 @@ def ksa_select_tokens_per_head(q: torch.Tensor, K: torch.Tensor, seq_lens: torch
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(seq_lens), int(k_tokens), _ptr(token_idx),
         _ptr(num_sel), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(dev_status), _stream(stream)))
+    return token_idx, num_sel
+
+
+def ksa_select_tokens_one_head_workspace(B: int, Hq: int, Hkv: int, D: int, T: int,
+                                         k_tokens: int) -> int:
+    sh = _shape(B, Hq, Hkv, D, T)
+    return int(lib().ksa_select_tokens_one_head_workspace(ctypes.byref(sh), int(k_tokens)))
+
+
+def ksa_select_tokens_one_head(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor,
+                               head_of_row, k_tokens: int,
+                               token_idx: Optional[torch.Tensor] = None,
+                               num_sel: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None,
+                               dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Random-head aggregation: row b's set is query head head_of_row[b]'s own top-k tokens,
+    shared by every head: (token_idx [B,k] ascending -1 padded, num_sel [B]); attend with
+    idx_shared=IDX_SHARED, tokens_per_idx=1.  head_of_row: B heads in [0, Hq) on the host
+    (a list, a numpy array or a CPU tensor), drawn by the caller."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    heads = (head_of_row.detach().cpu().numpy() if isinstance(head_of_row, torch.Tensor)
+             else np.asarray(head_of_row))
+    heads = np.ascontiguousarray(heads, dtype=np.int32)
+    if heads.shape != (B,):
+        raise ValueError(f"head_of_row must hold {B} heads, got shape {heads.shape}")
+    need = ksa_select_tokens_one_head_workspace(B, Hq, Hkv, D, T, k_tokens)
+    if workspace is None:  # no initialisation needed
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    if token_idx is None:
+        token_idx = torch.empty((B, k_tokens), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B,), dtype=torch.int32, device=q.device)
+    _dev(token_idx, "token_idx", torch.int32)
+    _dev(num_sel, "num_sel", torch.int32)
+    if token_idx.numel() < B * k_tokens or num_sel.numel() < B:
+        raise ValueError("token_idx must hold [B, k_tokens] and num_sel [B] entries")
+    sh = _shape(B, Hq, Hkv, D, T)
+    _check(lib().ksa_select_tokens_one_head(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(seq_lens),
+        heads.ctypes.data_as(ctypes.c_void_p), int(k_tokens), _ptr(token_idx), _ptr(num_sel),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+        _stream(stream)))
     return token_idx, num_sel

@@ -563,6 +563,63 @@ ksa_status ksa_select_tokens_per_head(const ksa_shape *shape, const uint16_t *q,
                      "ksa_select_tokens_per_head launch");
 }
 
+// Random-head aggregation's workspace: the per-head workspace, then every head's lists
+// [B, Hq, k] and counts [B, Hq].
+size_t ksa_select_tokens_one_head_workspace(const ksa_shape *shape, int32_t k_tokens) {
+  if (shape == nullptr || shape->batch < 1 || shape->num_q_heads < 1 || shape->capacity < 1 ||
+      k_tokens < 1)
+    return 0;
+  const size_t heads = static_cast<size_t>(shape->batch) * shape->num_q_heads;
+  return ksa::unified_workspace_bytes(shape->batch, shape->num_q_heads, shape->capacity) +
+         ((heads * k_tokens * sizeof(int32_t) + 255) & ~static_cast<size_t>(255)) +
+         ((heads * sizeof(int32_t) + 255) & ~static_cast<size_t>(255));
+}
+
+ksa_status ksa_select_tokens_one_head(const ksa_shape *shape, const uint16_t *q,
+                                      const uint16_t *K, const int32_t *seq_lens,
+                                      const int32_t *head_of_row, int32_t k_tokens,
+                                      int32_t *token_idx, int32_t *num_sel, void *ws,
+                                      size_t ws_bytes, uint32_t *dev_status, void *stream) {
+  ksa_status st = check_shape(shape, false);
+  if (st != KSA_OK) return st;
+  if (head_of_row == nullptr || token_idx == nullptr || num_sel == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "head_of_row, token_idx and num_sel must be non-NULL");
+  if (k_tokens < 1) return fail(KSA_ERR_INVALID_ARG, "k_tokens must be >= 1");
+  const int B = shape->batch, Hq = shape->num_q_heads;
+  for (int b = 0; b < B; ++b) {  // the host array holds one head per row
+    if (head_of_row[b] < 0 || head_of_row[b] >= Hq)
+      return fail(KSA_ERR_INVALID_ARG, "head_of_row[%d] = %d is outside [0, %d)", b,
+                  head_of_row[b], Hq);
+  }
+  const size_t base = ksa::unified_workspace_bytes(B, Hq, shape->capacity);
+  const size_t heads = static_cast<size_t>(B) * Hq;
+  const size_t lists_bytes =
+      (heads * k_tokens * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  const size_t need = ksa_select_tokens_one_head_workspace(shape, k_tokens);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  int32_t *lists = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + base);
+  int32_t *counts = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + base + lists_bytes);
+  // every head's own set into the workspace (the per-head kernels) ...
+  st = ksa_select_tokens_per_head(shape, q, K, seq_lens, k_tokens, lists, counts, ws, base,
+                                  dev_status, stream);
+  if (st != KSA_OK) return st;
+  // ... then each row's chosen head's list and count, in stream order
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t k = static_cast<size_t>(k_tokens);
+  for (int b = 0; b < B; ++b) {
+    const size_t src = static_cast<size_t>(b) * Hq + head_of_row[b];
+    cudaError_t err = cudaMemcpyAsync(token_idx + b * k, lists + src * k, k * sizeof(int32_t),
+                                      cudaMemcpyDeviceToDevice, s);
+    if (err == cudaSuccess)
+      err = cudaMemcpyAsync(num_sel + b, counts + src, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                            s);
+    if (err != cudaSuccess) return cuda_status(err, "ksa_select_tokens_one_head copy");
+  }
+  return KSA_OK;
+}
+
 const char *ksa_status_string(ksa_status status) {
   switch (status) {
     case KSA_OK: return "KSA_OK";

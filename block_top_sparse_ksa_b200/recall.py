@@ -28,12 +28,13 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from . import ksa_sparse_decode_attn, ksa_unified_select
+from . import (IDX_PER_Q_HEAD, IDX_SHARED, ksa_select_tokens_one_head,
+               ksa_select_tokens_per_head, ksa_sparse_decode_attn, ksa_unified_select)
 
 
 def attention_recall(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor,
                      idx: torch.Tensor, num_idx: torch.Tensor, tokens_per_idx: int = 1,
-                     idx_shared: bool = False, scale: float = 0.0,
+                     idx_shared: int = 0, scale: float = 0.0,
                      workspace: Optional[torch.Tensor] = None, stream=None) -> np.ndarray:
     """recall [B, Hq] (fp64, host) of the selection (idx, num_idx) under the dense softmax."""
     B, Hq, D = q.shape
@@ -70,17 +71,49 @@ def recency_sweep(inp, ratios: Sequence[float]) -> list:
     return rows
 
 
+def aggregation_comparison(inp, budget: int, seed: int = 0) -> dict:
+    """The three ways LessIsMore's mechanism analysis turns the heads' choices into the set the
+    layers read, each with the same token budget and no recency window: the unified vote, a
+    set per query head, and one randomly drawn head's set (seeded draw, one head per row).
+    Returns the mean recall of each in the selection layer and in the sparse layers."""
+    B, Hq = inp.q_sel.shape[0], inp.q_sel.shape[1]
+    heads = np.random.default_rng(seed).integers(0, Hq, size=B).astype(np.int32)
+    sets = {
+        "unified": ksa_unified_select(inp.q_sel, inp.K_sel, inp.seq_lens, budget, budget, 0)
+        + (IDX_SHARED,),
+        "per_head": ksa_select_tokens_per_head(inp.q_sel, inp.K_sel, inp.seq_lens, budget)
+        + (IDX_PER_Q_HEAD,),
+        "random_head": ksa_select_tokens_one_head(inp.q_sel, inp.K_sel, inp.seq_lens, heads,
+                                                  budget) + (IDX_SHARED,),
+    }
+    res = {"budget": budget, "recent_tokens": 0, "heads": heads.tolist()}
+    for name, (tok, cnt, layout) in sets.items():
+        res[name] = {
+            "selection_layer": float(attention_recall(inp.q_sel, inp.K_sel, inp.K_sel,
+                                                      inp.seq_lens, tok, cnt,
+                                                      idx_shared=layout).mean()),
+            "sparse_layers": [float(attention_recall(q, K, V, inp.seq_lens, tok, cnt,
+                                                     idx_shared=layout).mean())
+                              for q, K, V in inp.layers]}
+    return res
+
+
 def main(argv=None) -> None:
     from . import synth
     p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     p.add_argument("--batch", type=int, default=4)
     p.add_argument("--ratios", default="0,0.1,0.25,0.5,0.75,1")
     p.add_argument("--seed", type=int, default=1004)
+    p.add_argument("--aggregation", action="store_true",
+                   help="also compare unified, per-head and random-head sets")
     args = p.parse_args(argv)
     shape = synth.dataclasses.replace(synth.LESSISMORE, batch=args.batch)
     inp = synth.lessismore_inputs(seed=args.seed, device="cuda", shape=shape)
     for row in recency_sweep(inp, [float(x) for x in args.ratios.split(",")]):
         print(json.dumps({"workload": shape.name, **row}))
+    if args.aggregation:
+        print(json.dumps({"workload": shape.name,
+                          **aggregation_comparison(inp, shape.token_budget, args.seed)}))
 
 
 if __name__ == "__main__":

@@ -155,6 +155,30 @@ ksa_status ksa_select_tokens_per_head(const ksa_shape *shape, const uint16_t *q,
                                       uint32_t *dev_status, void *stream);
 
 /*
+ * Random-head aggregation [LIM s.4, mechanism analysis: of three ways to turn
+ * the heads' choices into one set -- a randomly chosen head's selection used
+ * for all heads, a set per head, the unified vote -- the random head does
+ * worst]: row b takes query head head_of_row[b]'s own top-k_tokens set (the
+ * ranking of ksa_select_tokens_per_head) as the one set every head reads.
+ * The random draw is the caller's: head_of_row is a HOST array [B] of heads in
+ * [0, Hq), read before this call returns.  Use the lists with
+ * ksa_sparse_decode_attn, idx_shared = KSA_IDX_SHARED, tokens_per_idx = 1.
+ *   token_idx: [B, k_tokens] int32;  num_sel: [B] int32 (written)
+ *   ws: device scratch of ksa_select_tokens_one_head_workspace() bytes,
+ *       256-byte aligned, no initialisation needed.
+ * It runs the per-head kernels into the workspace, then copies each row's
+ * chosen list with one cudaMemcpyAsync per row (and one per count) on
+ * `stream`.  A head outside [0, Hq) is KSA_ERR_INVALID_ARG before any launch.
+ * Limits: as ksa_select_tokens_per_head.
+ */
+size_t ksa_select_tokens_one_head_workspace(const ksa_shape *shape, int32_t k_tokens);
+ksa_status ksa_select_tokens_one_head(const ksa_shape *shape, const uint16_t *q,
+                                      const uint16_t *K, const int32_t *seq_lens,
+                                      const int32_t *head_of_row, int32_t k_tokens,
+                                      int32_t *token_idx, int32_t *num_sel, void *ws,
+                                      size_t ws_bytes, uint32_t *dev_status, void *stream);
+
+/*
  * Local attention as a block selection [KIN s.5 compares block top-k with
  * local attention, a fixed pattern over the nearest tokens]: every (b, g)
  * keeps its last min(k_blocks, NB_b) blocks, NB_b - n .. NB_b - 1, ascending

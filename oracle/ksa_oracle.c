@@ -33,7 +33,9 @@
  *  (R9) per-head selection ranks raw q.k (softmax is monotone per head);
  *  (R10) bf16 block summaries are a storage format of the block mean: each
  *        mean is replaced by the nearest bf16 value (ties to even) and the
- *        scores read the stored values.
+ *        scores read the stored values;
+ *  (R11) random-head aggregation: the random head of each row is an input
+ *        drawn by the caller, and that head's own top-k set serves every head.
  *
  * Inputs: bf16 values arrive as their 16-bit patterns and are widened to fp64
  * exactly.  All arrays are dense row-major.  Threads: OpenMP over independent
@@ -446,6 +448,31 @@ void ksa_oracle_select_tokens_per_head(int B, int Hq, int Hkv, int D, int T,
       free(r);
     }
   }
+}
+
+/*
+ * LessIsMore section 4 (mechanism analysis) compares three ways of turning
+ * the heads' choices into the set the sparse layers read: one randomly chosen
+ * head's selection used for every head, a set kept per head (above), and the
+ * unified vote (below).  Random-head aggregation (R11): row b takes query head
+ * head_of_row[b]'s own top-k tokens, ranked as above, as the set shared by all
+ * heads.
+ *   head_of_row: [B], each in [0, Hq);  token_idx: [B, k];  num_sel: [B].
+ */
+void ksa_oracle_select_tokens_one_head(int B, int Hq, int Hkv, int D, int T,
+                                       const uint16_t *q, const uint16_t *K,
+                                       const int32_t *seq_lens, const int32_t *head_of_row,
+                                       int k, int32_t *token_idx, int32_t *num_sel) {
+  int32_t *all = (int32_t *)malloc(sizeof(int32_t) * (size_t)B * Hq * k);
+  int32_t *cnt = (int32_t *)malloc(sizeof(int32_t) * (size_t)B * Hq);
+  ksa_oracle_select_tokens_per_head(B, Hq, Hkv, D, T, q, K, seq_lens, k, all, cnt);
+  for (int b = 0; b < B; ++b) {
+    const int h = head_of_row[b];
+    memcpy(token_idx + (size_t)b * k, all + ((size_t)b * Hq + h) * k, sizeof(int32_t) * (size_t)k);
+    num_sel[b] = cnt[(size_t)b * Hq + h];
+  }
+  free(all);
+  free(cnt);
 }
 
 void ksa_oracle_unified_select(int B, int Hq, int Hkv, int D, int T,

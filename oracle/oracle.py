@@ -53,6 +53,8 @@ class Oracle:
                                                    c_int, _i32p, _i32p, nullable_f64])
         L.ksa_oracle_select_tokens_per_head.argtypes = ([c_int] * 5 + [_u16p, _u16p, _i32p,
                                                         c_int, _i32p, _i32p])
+        L.ksa_oracle_select_tokens_one_head.argtypes = ([c_int] * 5 + [_u16p, _u16p, _i32p,
+                                                        _i32p, c_int, _i32p, _i32p])
         L.ksa_oracle_select_window.argtypes = [c_int] * 3 + [_i32p, c_int, _i32p, _i32p]
         L.ksa_oracle_gather_pages.argtypes = [c_int] * 6 + [_u16p, _i32p, _i32p, _u16p]
         L.ksa_oracle_round_bf16.argtypes = [c_double]
@@ -159,6 +161,23 @@ class Oracle:
         self.lib.ksa_oracle_select_tokens_per_head(B, Hq, Hkv, D, T, q, K,
                                                    np.ascontiguousarray(seq_lens, np.int32),
                                                    k, idx, cnt)
+        return idx, cnt
+
+    def select_tokens_one_head(self, q, K, seq_lens, head_of_row, k: int):
+        """Random-head aggregation: row b's set is head head_of_row[b]'s own top-k tokens,
+        shared by every head: (token_idx [B,k], num_sel [B])."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        K = np.ascontiguousarray(K, dtype=np.uint16)
+        B, Hq, D = q.shape
+        _, Hkv, T, _ = K.shape
+        heads = np.ascontiguousarray(head_of_row, np.int32)
+        if heads.shape != (B,) or heads.min() < 0 or heads.max() >= Hq:
+            raise ValueError("head_of_row must hold one head in [0, Hq) per row")
+        idx = np.empty((B, k), np.int32)
+        cnt = np.empty((B,), np.int32)
+        self.lib.ksa_oracle_select_tokens_one_head(B, Hq, Hkv, D, T, q, K,
+                                                   np.ascontiguousarray(seq_lens, np.int32),
+                                                   heads, k, idx, cnt)
         return idx, cnt
 
     def select_window(self, seq_lens, num_kv_heads: int, bs: int, k: int):

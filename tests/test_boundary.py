@@ -254,3 +254,24 @@ def test_no_fallback_without_the_library_or_a_gpu(tmp_path):
                          timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip().endswith("ok")
+
+
+def test_validation_of_random_head_selection(ksa):
+    """The host array of heads is checked row by row before any launch."""
+    lib = ksa.lib()
+    sh = _shape(ksa, B=3, Hq=8, Hkv=2)
+    good = (ctypes.c_int32 * 3)(0, 7, 3)
+    bad = (ctypes.c_int32 * 3)(0, 8, 3)  # head 8 of 8
+    neg = (ctypes.c_int32 * 3)(-1, 0, 0)
+    BIG = 1 << 30
+    call = lambda heads, k, ws, n: lib.ksa_select_tokens_one_head(
+        ctypes.byref(sh), FAKE, FAKE, FAKE, heads, k, FAKE, FAKE, ws, n, None, None)
+    assert call(None, 4, FAKE, BIG) == 1
+    assert call(bad, 4, FAKE, BIG) == 1 and "head_of_row[1]" in ksa.ksa_last_error()
+    assert call(neg, 4, FAKE, BIG) == 1
+    assert call(good, 0, FAKE, BIG) == 1
+    assert call(good, 4, None, 0) == 3
+    per_head = lib.ksa_select_tokens_per_head_workspace(ctypes.byref(sh), 4)
+    one_head = lib.ksa_select_tokens_one_head_workspace(ctypes.byref(sh), 4)
+    assert one_head >= per_head + 3 * 8 * 4 * 4 + 3 * 8 * 4
+    assert call(good, 4, FAKE, one_head - 1) == 3

@@ -725,6 +725,41 @@ def test_paged_kv_bad_page_ids_are_flagged_not_read(ksa, oracle):
 # attention-recall diagnostic
 
 
+def test_aggregation_comparison_bounds(ksa, oracle):
+    """Unified, per-head and random-head sets of the same budget, scored by recall in the
+    selection layer: each head's own top-k carries the most softmax mass any k tokens can,
+    so the per-head recall bounds the other two head by head, and equals the random-head
+    recall for the drawn head.  With one kv-head and identical query heads all three sets
+    coincide."""
+    from block_top_sparse_ksa_b200 import recall
+    shape = synth.dataclasses.replace(synth.LESSISMORE, batch=2, num_q_heads=8, num_kv_heads=2,
+                                      capacity=600, seq_len=600, per_head_topk=120,
+                                      token_budget=120, recent_tokens=30)
+    inp = synth.lessismore_inputs(seed=5, device=DEV, shape=shape)
+    k, B = 120, 2
+    heads = np.array([6, 1], np.int32)
+    uni, ucnt = ksa.ksa_unified_select(inp.q_sel, inp.K_sel, inp.seq_lens, k, k, 0)
+    ph, phc = ksa.ksa_select_tokens_per_head(inp.q_sel, inp.K_sel, inp.seq_lens, k)
+    rh, rhc = ksa.ksa_select_tokens_one_head(inp.q_sel, inp.K_sel, inp.seq_lens, heads, k)
+    args = (inp.q_sel, inp.K_sel, inp.K_sel, inp.seq_lens)
+    r_uni = recall.attention_recall(*args, uni, ucnt, idx_shared=ksa.IDX_SHARED)
+    r_ph = recall.attention_recall(*args, ph, phc, idx_shared=ksa.IDX_PER_Q_HEAD)
+    r_rh = recall.attention_recall(*args, rh, rhc, idx_shared=ksa.IDX_SHARED)
+    tol = 1e-4
+    assert np.all(r_ph >= r_uni - tol) and np.all(r_ph >= r_rh - tol)
+    for b in range(B):
+        assert abs(r_rh[b, heads[b]] - r_ph[b, heads[b]]) <= tol
+    res = recall.aggregation_comparison(inp, k, seed=3)
+    assert res["per_head"]["selection_layer"] >= res["unified"]["selection_layer"] - tol
+    assert res["per_head"]["selection_layer"] >= res["random_head"]["selection_layer"] - tol
+    one = synth.dataclasses.replace(shape, num_kv_heads=1)
+    inp1 = synth.lessismore_inputs(seed=6, device=DEV, shape=one)
+    inp1.q_sel.copy_(inp1.q_sel[:, :1].clone().expand_as(inp1.q_sel))
+    res1 = recall.aggregation_comparison(inp1, k, seed=3)
+    vals = [res1[n]["selection_layer"] for n in ("unified", "per_head", "random_head")]
+    assert max(vals) - min(vals) <= tol, vals
+
+
 def test_attention_recall_matches_softmax_mass(ksa, oracle):
     """recall = the dense softmax mass on the selected tokens (fp64 numpy softmax here);
     the dense set recalls 1 and an empty selection 0."""
@@ -810,4 +845,32 @@ def test_tokens_per_head_and_per_query_head_attention(ksa, oracle, L, k):
                                            ref_idx[:, h:h + 1], ref_cnt[:, h:h + 1], 1)
         assert_out_close(out[:, h], ref[:, 0])
         np.testing.assert_allclose(lse[:, h], ref_lse[:, 0], rtol=0, atol=LSE_TOL)
+    assert st.item() == 0
+
+
+@pytest.mark.parametrize("L,k", [(300, 40), (1500, 400), (90, 200)])
+def test_random_head_selection_and_shared_attention(ksa, oracle, L, k):
+    """Random-head aggregation: dyadic q, K give exact scores and ties; each row's shared set
+    equals the oracle's for the drawn head, and attention over it (shared by all heads)
+    equals the oracle's."""
+    rng = np.random.default_rng(1700 + L)
+    B, Hq, Hkv, D = 3, 8, 2, 128
+    T = L + 13
+    q = dyadic_bits(rng, (B, Hq, D))
+    K = dyadic_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([L, max(1, L // 3), max(1, L - 7)], np.int32)
+    heads = rng.integers(0, Hq, size=B).astype(np.int32)  # the random draw: an input
+    qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
+    st = status_tensor()
+    idx, cnt = ksa.ksa_select_tokens_one_head(qd, Kd, Ld, heads, k, dev_status=st)
+    ref_idx, ref_cnt = oracle.select_tokens_one_head(q, K, lens, heads, k)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=DEV)
+    out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, idx, cnt, tokens_per_idx=1,
+                                        idx_shared=ksa.IDX_SHARED, lse=lse, dev_status=st)
+    ref, ref_lse, _ = oracle.attention(q, K, V, lens, ref_idx, ref_cnt, 1, True)
+    assert_out_close(out.cpu().numpy(), ref)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_TOL)
     assert st.item() == 0

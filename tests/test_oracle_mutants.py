@@ -66,6 +66,10 @@ MUTANTS = [
      "pages + (((size_t)page * Hkv + g) * bs + t % bs) * D;",
      "pages + (((size_t)page * Hkv + g) * bs + (t + 1) % bs) * D;", 0,
      [pins.test_gather_pages_scatter_roundtrip_and_bad_pages]),
+    ("random head: always head 0",
+     "memcpy(token_idx + (size_t)b * k, all + ((size_t)b * Hq + h) * k,",
+     "memcpy(token_idx + (size_t)b * k, all + ((size_t)b * Hq) * k,", 0,
+     [pins.test_one_head_set_is_that_heads_brute_force_topk]),
     ("window one block early", "row[i] = i < n ? nb - n + i : -1;",
      "row[i] = i < n ? nb - n + i - 1 : -1;", 0,
      [pins.test_select_window_is_topk_of_a_recency_score]),

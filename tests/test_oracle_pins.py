@@ -686,3 +686,51 @@ def test_tokens_per_head_equal_heads_match_unified_votes(oracle):
     uni, ucnt = oracle.unified_select(bf16_bits(q), bf16_bits(K), lens, k, k, 0)
     for h in range(Hq):
         assert np.array_equal(idx[:, h], uni) and np.array_equal(cnt[:, h], ucnt)
+
+
+# ---------------------------------------------------------------------------
+# random-head aggregation (one head's set shared by every head)
+
+
+def test_one_head_set_is_that_heads_brute_force_topk(oracle):
+    """Brute force on small inputs with distinct heads and exact ties: row b's set is the
+    min(k, L) tokens of the chosen head ranked first by (score desc, index asc), ascending."""
+    rng = np.random.default_rng(63)
+    B, Hq, Hkv, D, T = 3, 8, 2, 64, 80
+    G = Hq // Hkv
+    q = np.round(rng.standard_normal((B, Hq, D)) * 2) / 4      # coarse grid: exact ties
+    K = np.round(rng.standard_normal((B, Hkv, T, D)) * 2) / 4
+    lens = np.array([T, 45, 3], np.int32)
+    heads = np.array([5, 2, 7], np.int32)
+    for k in (1, 9, 30, 100):
+        idx, cnt = oracle.select_tokens_one_head(bf16_bits(q), bf16_bits(K), lens, heads, k)
+        assert idx.shape == (B, k) and cnt.shape == (B,)
+        for b in range(B):
+            L, h = int(lens[b]), int(heads[b])
+            s = (K[b, h // G, :L].astype(np.float64) @ q[b, h].astype(np.float64))
+            order = sorted(range(L), key=lambda t: (-s[t], t))
+            want = np.sort(np.array(order[:min(k, L)], np.int32))
+            assert cnt[b] == len(want)
+            assert np.array_equal(idx[b, :cnt[b]], want) and np.all(idx[b, cnt[b]:] == -1)
+
+
+def test_one_head_set_with_equal_heads_is_the_unified_set(oracle):
+    """With every query head identical, any chosen head's top-k is the set all heads vote
+    for: the LessIsMore selection with budget k and no window."""
+    rng = np.random.default_rng(64)
+    B, Hq, Hkv, D, T, k = 2, 4, 1, 64, 300, 40
+    q = np.repeat(rng.standard_normal((B, 1, D)).astype(np.float32), Hq, axis=1)
+    K = rng.standard_normal((B, Hkv, T, D)).astype(np.float32)
+    lens = np.array([T, 90], np.int32)
+    uni, ucnt = oracle.unified_select(bf16_bits(q), bf16_bits(K), lens, k, k, 0)
+    for heads in ([0, 3], [2, 1]):
+        idx, cnt = oracle.select_tokens_one_head(bf16_bits(q), bf16_bits(K), lens,
+                                                 np.array(heads, np.int32), k)
+        assert np.array_equal(idx, uni) and np.array_equal(cnt, ucnt)
+
+
+def test_one_head_rejects_heads_out_of_range(oracle):
+    q = np.zeros((1, 4, 64), np.uint16)
+    K = np.zeros((1, 2, 16, 64), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.select_tokens_one_head(q, K, np.array([16], np.int32), np.array([4], np.int32), 2)
