@@ -566,24 +566,53 @@ def oracle_step_units(o, shape, kind, q, K, V, S, lens, rows):
     o.attention(qv, Kv, Vv, Lv, idx, cnt, bs)
 
 
+def oracle_runner(shape, kind, n_rows, device):
+    """(oracle, step(i, rows), what a step computes) on a host sample of n_rows rows of the
+    workload.  A LessIsMore step is the unified selection followed by attention over the
+    shared set in each sparse layer, as on the GPU."""
+    if kind != "unified":
+        o, qb, K, V, S, lens = oracle_block_sample(shape, kind, n_rows, device)
+
+        def step(i, rows):
+            oracle_step_units(o, shape, kind, qb[i % len(qb)], K, V, S, lens, rows)
+        return o, step, ("oracle block scores + top-k + attention (summaries precomputed, as "
+                         "the GPU prefill)")
+    from block_top_sparse_ksa_b200 import synth
+    from oracle import oracle as O
+    inp = synth.lessismore_inputs(device=device, shape=synth.dataclasses.replace(shape,
+                                                                                 batch=n_rows))
+    o = O.get()
+    lens = inp.seq_lens.cpu().numpy()
+    q_sel, K_sel = synth.bits(inp.q_sel), synth.bits(inp.K_sel)
+    layers = [tuple(synth.bits(t) for t in layer) for layer in inp.layers]
+
+    def step(i, rows):
+        sel = np.asarray(rows)
+        tok, cnt = o.unified_select(q_sel[sel], K_sel[sel], lens[sel], shape.per_head_topk,
+                                    shape.token_budget, shape.recent_tokens)
+        for q, K, V in layers:
+            o.attention(q[sel], K[sel], V[sel], lens[sel], tok, cnt, 1, True)
+    return o, step, (f"oracle unified selection + attention over the shared set in "
+                     f"{len(layers)} sparse layers")
+
+
 def cpu_baseline(args, dev, kind, budget_s):
     _, shape = resolve_workload(args.workload, args.batch)
-    n_rows = min(8, shape.batch)
-    o, qb, K, V, S, lens = oracle_block_sample(shape, kind, n_rows, dev)
+    n_rows = 1 if kind == "unified" else min(8, shape.batch)
+    o, step, what = oracle_runner(shape, kind, n_rows, dev)
     o.set_threads(os.cpu_count() or 1)
     rows_done = 0
     t0 = time.perf_counter()
     i = 0
     while True:
-        oracle_step_units(o, shape, kind, qb[i % len(qb)], K, V, S, lens, list(range(n_rows)))
+        step(i, list(range(n_rows)))
         rows_done += n_rows
         i += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
     return {"value": rows_done / el, "unit": UNIT, "cores": o.max_threads(), "kind": "oracle",
-            "sample": f"{n_rows} rows of {shape.name}, {i} steps of oracle block scores + top-k "
-                      f"+ attention (summaries precomputed, as the GPU prefill), {el:.1f} s"}
+            "sample": f"{n_rows} rows of {shape.name}, {i} steps of {what}, {el:.1f} s"}
 
 
 def run_reference(args, dist):
@@ -592,28 +621,23 @@ def run_reference(args, dist):
         return
     kind, shape = resolve_workload(args.workload, args.batch)
     dev = torch.device("cuda", dist.local) if torch.cuda.is_available() else torch.device("cpu")
-    if kind == "unified":
-        print(json.dumps({"impl": "reference", "unavailable":
-                          "the oracle arm covers the block top-k workloads only"}))
-        return
     n_rows = min(8, shape.batch)
-    o, qb, K, V, S, lens = oracle_block_sample(shape, kind, n_rows, dev)
+    o, step, what = oracle_runner(shape, kind, n_rows, dev)
     o.set_threads(os.cpu_count() or 1)
     # size one step so that warmup + steps take about two minutes
     t0 = time.perf_counter()
-    oracle_step_units(o, shape, kind, qb[0], K, V, S, lens, [0])
+    step(0, [0])
     t_row = max(time.perf_counter() - t0, 1e-4)
     per_step = min(n_rows, max(1, int(120.0 / (args.steps + args.warmup) / t_row)))
     rows = list(range(per_step))
     for i in range(args.warmup):
-        oracle_step_units(o, shape, kind, qb[i % 4], K, V, S, lens, rows)
+        step(i, rows)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        oracle_step_units(o, shape, kind, qb[i % 4], K, V, S, lens, rows)
+        step(i, rows)
     el = time.perf_counter() - t0
     value = per_step * args.steps / el
-    sample = (f"{per_step} of {shape.batch} rows of {shape.name} per step (oracle block scores "
-              f"+ top-k + attention, fp64, summaries precomputed)")
+    sample = f"{per_step} of {shape.batch} rows of {shape.name} per step ({what}, fp64)"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
@@ -659,7 +683,7 @@ def main():
                 "gpu_launches": res["gpu_launches"], "clocks": res["clocks"]}
         if "e2e" in res:
             line["e2e"] = res["e2e"]
-        if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and kind != "unified":
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args, dev, kind, args.cpu_seconds)
         if dist.rank == 0:
             print(json.dumps(line), flush=True)

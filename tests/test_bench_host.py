@@ -75,3 +75,20 @@ def test_committed_traffic_record():
     assert len(ent["source_sha256_16"]) == 16 and ent["batch"] == 64
     # the capture agrees with the algorithmic bytes of one launch to within 1%
     assert abs(ent["dram_bytes_per_launch"] / 269_221_888 - 1) < 0.01
+
+
+@pytest.mark.parametrize("name", ["tiny", "lessismore"])
+def test_oracle_runner_steps_on_the_host(name):
+    """The oracle leg (cpu_baseline, --impl reference) runs a step of either workload kind on
+    a small host sample."""
+    from block_top_sparse_ksa_b200 import synth
+    import torch
+    kind, shape = bench.resolve_workload(name)
+    if kind == "unified":
+        shape = synth.dataclasses.replace(shape, num_q_heads=8, num_kv_heads=2, capacity=400,
+                                          seq_len=400, per_head_topk=80, token_budget=80,
+                                          recent_tokens=20)
+    o, step, what = bench.oracle_runner(shape, kind, 1, torch.device("cpu"))
+    step(0, [0])
+    step(1, [0])
+    assert "oracle" in what
