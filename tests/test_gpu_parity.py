@@ -107,12 +107,13 @@ def test_select_blocks_planted_gap(ksa, oracle, D, bs, k):
     _select_case(ksa, oracle, rng, B, Hq, Hkv, D, T, bs, k, lens)
 
 
-@pytest.mark.parametrize("nblk", [256, 700, 1100])
+@pytest.mark.parametrize("nblk", [256, 700, 1100, 3000, 7000, 16384])
 def test_select_blocks_exact_ties(ksa, oracle, nblk):
     """Dyadic inputs, full blocks: every score is exact in fp32, many tie
     exactly, and both sides must break ties toward the lower block.  Rows of
-    up to 1024 blocks are ranked inside the scoring launch, longer ones by the
-    separate ranking launch: 700 and 1100 blocks take one path each."""
+    up to 1024 blocks are ranked one warp per row (256 and 700 here); longer
+    rows one CTA per row with 8, 16, 32 or 64 keys per thread (1100, 3000,
+    7000, and 16384 blocks, the largest row the API accepts)."""
     rng = np.random.default_rng(210 + nblk)
     B, Hq, Hkv, D, bs = 2, 4, 2, 128, 16
     T = nblk * bs
