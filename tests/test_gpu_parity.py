@@ -276,6 +276,8 @@ def test_seq_len_out_of_range_is_clamped_and_flagged(ksa, oracle):
 @pytest.mark.parametrize("L,P,budget,R", [(300, 50, 64, 16), (1500, 400, 300, 75),
                                            (2500, 2600, 500, 125), (900, 120, 900, 225),
                                            (4100, 1000, 1000, 1000), (5000, 800, 1200, 0),
+                                           (11000, 2000, 3000, 750), (15500, 3000, 4000, 1000),
+                                           (24500, 4000, 4000, 1000),
                                            (30000, 3000, 4000, 1000)])
 def test_unified_select_exact(ksa, oracle, L, P, budget, R):
     rng = np.random.default_rng(700 + L)
