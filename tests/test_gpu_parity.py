@@ -877,3 +877,47 @@ def test_random_head_selection_and_shared_attention(ksa, oracle, L, k):
     assert_out_close(out.cpu().numpy(), ref)
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=LSE_TOL)
     assert st.item() == 0
+
+
+@pytest.mark.parametrize("tpi", [4, 16, 64])
+def test_per_query_head_lists_of_blocks(ksa, oracle, tpi):
+    """Lists per query head whose entries name runs of tpi tokens: runs of 16 or more go
+    through the TMA producer, shorter ones through cp.async.  Ragged counts, one empty
+    head, a partial last run; checked head by head against the oracle."""
+    rng = np.random.default_rng(1800 + tpi)
+    B, Hq, Hkv, D = 2, 8, 2, 128
+    G = Hq // Hkv
+    T = 64 * tpi
+    q, K, V = (rand_bits(rng, s) for s in [(B, Hq, D), (B, Hkv, T, D), (B, Hkv, T, D)])
+    lens = np.array([T - tpi // 2, 23 * tpi + 1], np.int32)
+    cap = 12
+    idx = np.full((B, Hq, cap), -1, np.int32)
+    cnt = np.zeros((B, Hq), np.int32)
+    for b in range(B):
+        n_runs = -(-int(lens[b]) // tpi)
+        for h in range(Hq):
+            n = 0 if (b, h) == (1, 3) else int(rng.integers(1, cap + 1))
+            pick = np.sort(rng.choice(n_runs, size=n, replace=False))
+            if n and b == 0 and h == 0:
+                pick[-1] = n_runs - 1  # the partial last run
+                pick = np.unique(pick)
+                n = len(pick)
+            idx[b, h, :n] = pick
+            cnt[b, h] = n
+    qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=DEV)
+    st = status_tensor()
+    out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, torch.from_numpy(idx).to(DEV),
+                                        torch.from_numpy(cnt).to(DEV), tokens_per_idx=tpi,
+                                        idx_shared=ksa.IDX_PER_Q_HEAD, lse=lse, dev_status=st)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for h in range(Hq):
+        g = h // G
+        ref, ref_lse, _ = oracle.attention(q[:, h:h + 1], K[:, g:g + 1], V[:, g:g + 1], lens,
+                                           idx[:, h:h + 1], cnt[:, h:h + 1], tpi)
+        assert_out_close(out[:, h], ref[:, 0], what=f"head {h}")
+        fin = np.isfinite(ref_lse[:, 0])
+        np.testing.assert_allclose(lse[fin, h], ref_lse[fin, 0], rtol=0, atol=LSE_TOL)
+        assert np.all(np.isneginf(lse[~fin, h]))
+    assert out[1, 3].max() == 0.0 and out[1, 3].min() == 0.0  # the empty head
+    assert st.item() == 0
