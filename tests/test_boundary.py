@@ -275,3 +275,27 @@ def test_validation_of_random_head_selection(ksa):
     one_head = lib.ksa_select_tokens_one_head_workspace(ctypes.byref(sh), 4)
     assert one_head >= per_head + 3 * 8 * 4 * 4 + 3 * 8 * 4
     assert call(good, 4, FAKE, one_head - 1) == 3
+
+
+def test_every_entry_point_refuses_a_null_shape(ksa):
+    """Driven by the binding's signature table: each call that takes a shape first returns
+    KSA_ERR_INVALID_ARG (status calls) or 0 bytes (workspace queries) for a NULL shape, with
+    every other pointer NULL and every number 0 -- validation first, nothing dereferenced."""
+    lib = ksa.lib()
+    checked = 0
+    for name, (res, args) in ksa._SIGS.items():
+        if not args or args[0] is not ctypes.POINTER(ksa.Shape):
+            continue
+        rest = []
+        for t in args[1:]:
+            if t in (ctypes.c_float, ctypes.c_double):
+                rest.append(0.0)
+            elif t in (ctypes.c_int32, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32):
+                rest.append(0)
+            else:
+                rest.append(None)
+        got = getattr(lib, name)(None, *rest)
+        want = 0 if res is ctypes.c_size_t else 1
+        assert got == want, (name, got)
+        checked += 1
+    assert checked >= 20
