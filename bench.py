@@ -379,8 +379,41 @@ def run_block(args, dist, dev, kind):
     }
     if not args.no_e2e:
         res["e2e"] = run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att)
+    if kind != "dense":
+        try:
+            res["prefill"] = time_prefill(ksa, inp, shape, S, stream, peak)
+        except Exception as e:  # a side figure: never lose the step's line for it
+            res["prefill"] = {"error": str(e)[:200]}
     res["_host"] = (inp, S, qs, shape, kind)
     return res
+
+
+def prefill_bytes(shape, seq_lens, summary_bytes: int = 4) -> int:
+    """The prefill's summary build (every block of every row): one read of the keys and one
+    write of the block means."""
+    bs, Hkv, D = shape.block_size, shape.num_kv_heads, shape.head_dim
+    return sum(Hkv * int(L) * D * 2 + Hkv * (-(-int(L) // bs)) * D * summary_bytes
+               for L in seq_lens)
+
+
+def time_prefill(ksa, inp, shape, S, stream, peak, reps: int = 5):
+    """ksa_build_block_summaries (mode ALL) over the whole cache, timed alone with CUDA events
+    (the cache is larger than L2, so the repetitions read from HBM)."""
+    S2 = torch.empty_like(S)
+    ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, shape.block_size, summaries=S2,
+                                  stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, shape.block_size, summaries=S2,
+                                      stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    b = prefill_bytes(shape, inp.seq_lens.cpu().tolist(), S.element_size())
+    return {"kernel": "block_summaries (mode ALL)", "ms": ms, "bytes": b,
+            "gbs": b / (ms * 1e-3) / 1e9, "frac": b / (ms * 1e-3) / 1e9 / peak}
 
 
 def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att):
@@ -683,6 +716,8 @@ def main():
                 "gpu_launches": res["gpu_launches"], "clocks": res["clocks"]}
         if "e2e" in res:
             line["e2e"] = res["e2e"]
+        if "prefill" in res:
+            line["prefill"] = res["prefill"]
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args, dev, kind, args.cpu_seconds)
         if dist.rank == 0:

@@ -92,3 +92,11 @@ def test_oracle_runner_steps_on_the_host(name):
     step(0, [0])
     step(1, [0])
     assert "oracle" in what
+
+
+def test_prefill_bytes():
+    _, sh = bench.resolve_workload("qwen3-0.6b")
+    # keys read: 64 rows x 8 kv-heads x 16384 tokens x 128 x 2 bytes; means written: 512 blocks
+    assert bench.prefill_bytes(sh, [16384] * 64) == 2_147_483_648 + 134_217_728
+    assert bench.prefill_bytes(sh, [16384] * 64, 2) == 2_147_483_648 + 67_108_864
+    assert bench.prefill_bytes(sh, [33]) == 8 * 33 * 128 * 2 + 8 * 2 * 128 * 4
