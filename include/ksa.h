@@ -7,11 +7,13 @@
  *   [KIN] Kinetics: Rethinking Test-Time Scaling Laws (press summary,
  *         news.43u.com.cn), section 5 "from theory to practice: block top-k".
  *   [LIM] LessIsMore (press summary, techwalker.com), section 2 "unified head
- *         selection" / "stable recency window", section 5 "implementation".
+ *         selection" / "stable recency window", section 4 "mechanism
+ *         analysis", section 5 "implementation".
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers, dense row-major, owned by the
- *     caller.  The library allocates nothing, keeps no state between calls,
+ *     caller; the one exception, head_of_row of ksa_select_tokens_one_head, is
+ *     a host array.  The library allocates nothing, keeps no state between calls,
  *     and never synchronises the host: work is enqueued on `stream`
  *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
  *   - bf16 tensors are passed as uint16_t* (the raw bf16 bit patterns).
