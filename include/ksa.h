@@ -121,11 +121,13 @@ ksa_status ksa_select_blocks(const ksa_shape *shape, const uint16_t *q,
                              uint32_t *dev_status, void *stream);
 
 /*
- * One decode step's selection in a single launch [KIN s.5]: for every row b
- * and kv-head g, first recompute the mean of the last block j = NB_b - 1 from
- * K and store it in `summaries` (what ksa_build_block_summaries does with
+ * One decode step's selection in one call [KIN s.5]: for every row b and
+ * kv-head g, first recompute the mean of the last block j = NB_b - 1 from K
+ * and store it in `summaries` (what ksa_build_block_summaries does with
  * KSA_SUMMARY_LAST_BLOCK, bit for bit), then score and select exactly as
- * ksa_select_blocks.  Use after appending the step's token to K.
+ * ksa_select_blocks.  The refresh runs inside the scoring launch, so the call
+ * is two launches (scoring, ranking), or one when no row can hold more than
+ * k_blocks blocks.  Use after appending the step's token to K.
  * Arguments as ksa_select_blocks, plus K [B, Hkv, T, D] bf16 (read);
  * `summaries` is read and its last-block entries are written.
  */
