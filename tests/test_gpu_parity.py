@@ -921,3 +921,52 @@ def test_per_query_head_lists_of_blocks(ksa, oracle, tpi):
         assert np.all(np.isneginf(lse[~fin, h]))
     assert out[1, 3].max() == 0.0 and out[1, 3].min() == 0.0  # the empty head
     assert st.item() == 0
+
+
+@pytest.mark.parametrize("layout", ["blocks", "shared_tokens", "dense"])
+def test_outputs_lie_in_the_hull_of_the_selected_values(ksa, oracle, layout):
+    """An invariant that needs no oracle: every output coordinate lies between the smallest
+    and largest value of that coordinate over the selected V rows (softmax weights are
+    non-negative and sum to 1), up to the fp32 accumulation tolerance."""
+    rng = np.random.default_rng(1900 + len(layout))
+    B, Hq, Hkv, D, T, bs = 3, 8, 2, 128, 1024, 16
+    G = Hq // Hkv
+    q, K, V = (rand_bits(rng, s, 2.0) for s in [(B, Hq, D), (B, Hkv, T, D), (B, Hkv, T, D)])
+    lens = np.array([T, 517, 40], np.int32)
+    qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
+    Vv = bf16_value(V)
+    sel = np.zeros((B, Hkv, T), bool)
+    if layout == "blocks":
+        k = 9
+        idx = np.full((B, Hkv, k), -1, np.int32)
+        cnt = np.zeros((B, Hkv), np.int32)
+        for b in range(B):
+            nb = -(-int(lens[b]) // bs)
+            for g in range(Hkv):
+                pick = np.sort(rng.choice(nb, size=min(k, nb), replace=False))
+                idx[b, g, :len(pick)] = pick
+                cnt[b, g] = len(pick)
+                for j in pick:
+                    sel[b, g, j * bs:min((j + 1) * bs, lens[b])] = True
+        out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, torch.from_numpy(idx).to(DEV),
+                                            torch.from_numpy(cnt).to(DEV), tokens_per_idx=bs)
+    elif layout == "shared_tokens":
+        k = 30
+        idx = np.stack([np.sort(rng.choice(int(lens[b]), size=k, replace=False))
+                        for b in range(B)]).astype(np.int32)
+        cnt = np.full((B,), k, np.int32)
+        for b in range(B):
+            sel[b, :, idx[b]] = True
+        out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld, torch.from_numpy(idx).to(DEV),
+                                            torch.from_numpy(cnt).to(DEV), tokens_per_idx=1,
+                                            idx_shared=ksa.IDX_SHARED)
+    else:
+        for b in range(B):
+            sel[b, :, :lens[b]] = True
+        out, _ = ksa.ksa_sparse_decode_attn(qd, Kd, Vd, Ld)
+    out = out.cpu().numpy()
+    for b in range(B):
+        for h in range(Hq):
+            rows = Vv[b, h // G][sel[b, h // G]]
+            assert np.all(out[b, h] >= rows.min(0) - 2e-3), (b, h)
+            assert np.all(out[b, h] <= rows.max(0) + 2e-3), (b, h)
