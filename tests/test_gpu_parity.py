@@ -970,3 +970,43 @@ def test_outputs_lie_in_the_hull_of_the_selected_values(ksa, oracle, layout):
             rows = Vv[b, h // G][sel[b, h // G]]
             assert np.all(out[b, h] >= rows.min(0) - 2e-3), (b, h)
             assert np.all(out[b, h] <= rows.max(0) + 2e-3), (b, h)
+
+
+@pytest.mark.parametrize("mode", ["dense", "blocks"])
+def test_nan_poisoned_partials_are_never_read_stale(ksa, oracle, mode):
+    """The workspace's split-row partial region starts as NaN (its semaphores zero, as the
+    API asks): rows split over a hundred or more CTAs still match the oracle, so every
+    partial the merge reads was written by this call."""
+    rng = np.random.default_rng(2000 + len(mode))
+    B, Hq, Hkv, D, T, bs = 2, 8, 2, 128, 32768, 16
+    q, K, V = (rand_bits(rng, s) for s in [(B, Hq, D), (B, Hkv, T, D), (B, Hkv, T, D)])
+    lens = np.array([T, T - 1000], np.int32)
+    idx = cnt = None
+    tpi = 1
+    cap = T
+    if mode == "blocks":
+        tpi, cap = bs, 1500
+        idx = np.full((B, Hkv, cap), -1, np.int32)
+        cnt = np.zeros((B, Hkv), np.int32)
+        for b in range(B):
+            nb = -(-int(lens[b]) // bs)
+            for g in range(Hkv):
+                idx[b, g] = np.sort(rng.choice(nb, size=cap, replace=False))
+                cnt[b, g] = cap
+    need = ksa.lib().ksa_sparse_decode_attn_workspace(
+        ctypes.byref(ksa.Shape(B, Hq, Hkv, D, T, bs)), cap, tpi)
+    head = (B * Hq * 4 + 255) // 256 * 256
+    ws = torch.zeros((need,), dtype=torch.uint8, device=DEV)
+    ws[head:].view(torch.float32).fill_(float("nan"))
+    qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
+    st = status_tensor()
+    out, _ = ksa.ksa_sparse_decode_attn(
+        qd, Kd, Vd, Ld, None if idx is None else torch.from_numpy(idx).to(DEV),
+        None if cnt is None else torch.from_numpy(cnt).to(DEV), tokens_per_idx=tpi,
+        workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    got = out.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    ref, _, _ = oracle.attention(q, K, V, lens, idx, cnt, tpi)
+    assert_out_close(got, ref)
