@@ -41,12 +41,17 @@ def log(*a):
 
 
 def parse_args():
-    p = argparse.ArgumentParser()
-    p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20000)
-    p.add_argument("--warmup", type=int, default=100)
-    p.add_argument("--impl", choices=["ksa", "reference"], default="ksa")
-    p.add_argument("--workload", default="qwen3-0.6b")
+    p = argparse.ArgumentParser(description="Decode-step throughput of libksa (or of the fp64 "
+                                "oracle with --impl reference); prints one JSON line.")
+    p.add_argument("--gpus", type=int, default=1,
+                   help="GPUs of the job (launch with torchrun for more than one)")
+    p.add_argument("--steps", type=int, default=20000, help="timed steps")
+    p.add_argument("--warmup", type=int, default=100, help="untimed steps before them")
+    p.add_argument("--impl", choices=["ksa", "reference"], default="ksa",
+                   help="ksa: the CUDA library; reference: the oracle on the host cores")
+    p.add_argument("--workload", default="qwen3-0.6b",
+                   help="qwen3-0.6b, qwen3-8b, lessismore, tiny, sweep-L<ctx>-B<budget>, "
+                        "dense-L<ctx>")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="wall-clock budget of the oracle CPU baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
