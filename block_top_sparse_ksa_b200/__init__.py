@@ -30,7 +30,8 @@ __all__ = [
     "ksa_build_block_summaries_paged", "ksa_decode_select_blocks_paged",
     "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window", "ksa_select_tokens_per_head",
     "ksa_select_tokens_per_head_workspace", "ksa_select_tokens_one_head",
-    "ksa_select_tokens_one_head_workspace", "IDX_PER_KV_HEAD", "IDX_SHARED", "IDX_PER_Q_HEAD",
+    "ksa_select_tokens_one_head_workspace", "ksa_get_device_status", "IDX_PER_KV_HEAD",
+    "IDX_SHARED", "IDX_PER_Q_HEAD",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -88,6 +89,7 @@ _SIGS = {
     "ksa_select_window": (_i32, [ctypes.POINTER(Shape), _vp, _i32, _vp, _vp, _vp, _vp]),
     "ksa_select_tokens_per_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_tokens_one_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
+    "ksa_get_device_status": (_i32, [_vp, _vp, _i32, ctypes.POINTER(ctypes.c_uint32)]),
     "ksa_select_tokens_one_head": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _i32, _vp,
                                           _vp, _vp, _sz, _vp, _vp]),
     "ksa_select_tokens_per_head": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _i32, _vp, _vp,
@@ -601,3 +603,16 @@ def ksa_select_tokens_one_head(q: torch.Tensor, K: torch.Tensor, seq_lens: torch
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
         _stream(stream)))
     return token_idx, num_sel
+
+
+def ksa_get_device_status(dev_status: torch.Tensor, clear: bool = False, stream=None) -> int:
+    """The KSA_FLAG_* bits collected in a device status word (waits for `stream`); with clear,
+    the word is zeroed afterwards on the stream."""
+    if not isinstance(dev_status, torch.Tensor) or not dev_status.is_cuda:
+        raise TypeError("dev_status must be a CUDA tensor")
+    if dev_status.element_size() * dev_status.numel() < 4:
+        raise ValueError("dev_status must hold one 32-bit word")
+    flags = ctypes.c_uint32(0)
+    _check(lib().ksa_get_device_status(_ptr(dev_status), _stream(stream), int(bool(clear)),
+                                       ctypes.byref(flags)))
+    return int(flags.value)

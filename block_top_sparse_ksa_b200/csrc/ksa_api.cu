@@ -620,6 +620,23 @@ ksa_status ksa_select_tokens_one_head(const ksa_shape *shape, const uint16_t *q,
   return KSA_OK;
 }
 
+ksa_status ksa_get_device_status(const uint32_t *dev_status, void *stream, int32_t clear,
+                                 uint32_t *flags) {
+  if (dev_status == nullptr || flags == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "dev_status and flags must be non-NULL");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0u;
+  cudaError_t err = cudaMemcpyAsync(&word, dev_status, sizeof word, cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+  if (err != cudaSuccess) return cuda_status(err, "reading the device status word");
+  *flags = word;
+  if (clear != 0) {
+    err = cudaMemsetAsync(const_cast<uint32_t *>(dev_status), 0, sizeof(uint32_t), s);
+    if (err != cudaSuccess) return cuda_status(err, "clearing the device status word");
+  }
+  return KSA_OK;
+}
+
 const char *ksa_status_string(ksa_status status) {
   switch (status) {
     case KSA_OK: return "KSA_OK";

@@ -359,6 +359,17 @@ ksa_status ksa_unified_select(const ksa_shape *shape, const uint16_t *q,
                               int32_t *num_sel, void *ws, size_t ws_bytes,
                               uint32_t *dev_status, void *stream);
 
+/*
+ * Reads back a device status word (the dev_status of earlier calls): copies it
+ * to *flags on `stream` and waits for the stream, so every call enqueued on
+ * it before has finished.  This is the one call that synchronises the host.
+ * clear != 0 then zeroes the word on `stream` for the next calls.  One word
+ * may collect the KSA_FLAG_* bits of a whole decode step.
+ *   dev_status: device uint32;  flags: host uint32 (written).
+ */
+ksa_status ksa_get_device_status(const uint32_t *dev_status, void *stream, int32_t clear,
+                                 uint32_t *flags);
+
 /* Human-readable name of a status code (static string). */
 const char *ksa_status_string(ksa_status status);
 /* Message describing the calling thread's last failed call ("" if none). */

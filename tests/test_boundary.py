@@ -299,3 +299,11 @@ def test_every_entry_point_refuses_a_null_shape(ksa):
         assert got == want, (name, got)
         checked += 1
     assert checked >= 20
+
+
+def test_device_status_read_back_validation(ksa):
+    lib = ksa.lib()
+    flags = ctypes.c_uint32(7)
+    assert lib.ksa_get_device_status(None, None, 0, ctypes.byref(flags)) == 1
+    assert lib.ksa_get_device_status(FAKE, None, 0, None) == 1
+    assert flags.value == 7  # untouched on a refused call

@@ -253,6 +253,26 @@ def test_attention_flags_bad_entries(ksa, oracle):
     assert st & 2  # KSA_FLAG_INDEX_SKIPPED
 
 
+def test_device_status_read_back_and_clear(ksa, oracle):
+    """ksa_get_device_status returns the bits a step's calls collected in one word, and
+    clears it on request."""
+    rng = np.random.default_rng(611)
+    B, Hq, Hkv, D, T, bs = 1, 4, 1, 128, 128, 16
+    q, K, V = (to_dev_bf16(rand_bits(rng, s)) for s in [(B, Hq, D), (B, Hkv, T, D),
+                                                         (B, Hkv, T, D)])
+    lens = torch.tensor([100], dtype=torch.int32, device=DEV)
+    idx = torch.tensor([[[1, -5, 3]]], dtype=torch.int32, device=DEV)  # -5 names no block
+    cnt = torch.tensor([[3]], dtype=torch.int32, device=DEV)
+    st = status_tensor()
+    ksa.ksa_sparse_decode_attn(q, K, V, lens, idx, cnt, tokens_per_idx=bs, dev_status=st)
+    assert ksa.ksa_get_device_status(st) == ksa.FLAG_INDEX_SKIPPED
+    assert ksa.ksa_get_device_status(st, clear=True) == ksa.FLAG_INDEX_SKIPPED
+    assert ksa.ksa_get_device_status(st) == 0
+    ksa.ksa_sparse_decode_attn(q, K, V, lens, idx[:, :, :1].contiguous(), cnt * 0 + 1,
+                               tokens_per_idx=bs, dev_status=st)
+    assert ksa.ksa_get_device_status(st) == 0  # a clean call adds nothing
+
+
 def test_seq_len_out_of_range_is_clamped_and_flagged(ksa, oracle):
     rng = np.random.default_rng(620)
     B, Hq, Hkv, D, T = 2, 4, 2, 64, 96
