@@ -15,6 +15,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libksa.so")
+# ptxas resource report of the last build (registers, spills, shared memory per kernel)
+REPORT = os.path.join(HERE, "_build", "ptxas.txt")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -43,13 +45,19 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+    if not force and up_to_date() and os.path.exists(REPORT):
         return LIB
-    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-           "-o", LIB + ".tmp", *sources()]
+    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xptxas=-v", "-Xcompiler", "-fPIC",
+           "-shared", "-o", LIB + ".tmp", *sources()]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise subprocess.CalledProcessError(res.returncode, cmd)
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+        sys.stderr.write(res.stderr)
+    os.makedirs(os.path.dirname(REPORT), exist_ok=True)
+    with open(REPORT, "w") as f:
+        f.write(res.stderr)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

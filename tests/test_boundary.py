@@ -307,3 +307,16 @@ def test_device_status_read_back_validation(ksa):
     assert lib.ksa_get_device_status(None, None, 0, ctypes.byref(flags)) == 1
     assert lib.ksa_get_device_status(FAKE, None, 0, None) == 1
     assert flags.value == 7  # untouched on a refused call
+
+
+def test_no_kernel_spills_registers(ksa):
+    """The last build's ptxas report: every kernel fits its registers (the selection and pick
+    kernels keep whole rows of keys in registers; a spill would send them to local memory)."""
+    from block_top_sparse_ksa_b200 import build
+    if not os.path.exists(build.REPORT):
+        build.build(force=True)
+    text = open(build.REPORT).read()
+    entries = re.findall(r"Compiling entry function '([^']+)'", text)
+    spills = re.findall(r"(\d+) bytes spill stores, (\d+) bytes spill loads", text)
+    assert len(entries) >= 30 and len(spills) >= len(entries)
+    assert all(a == "0" and b == "0" for a, b in spills), spills
