@@ -899,11 +899,12 @@ def test_random_head_selection_and_shared_attention(ksa, oracle, L, k):
     assert st.item() == 0
 
 
-@pytest.mark.parametrize("tpi", [4, 16, 64])
+@pytest.mark.parametrize("tpi", [4, 16, 64, 256])
 def test_per_query_head_lists_of_blocks(ksa, oracle, tpi):
     """Lists per query head whose entries name runs of tpi tokens: runs of 16 or more go
-    through the TMA producer, shorter ones through cp.async.  Ragged counts, one empty
-    head, a partial last run; checked head by head against the oracle."""
+    through the TMA producer (256, the largest run allowed, is 16 stages per entry), shorter
+    ones through cp.async.  Ragged counts, one empty head, a partial last run; checked head
+    by head against the oracle."""
     rng = np.random.default_rng(1800 + tpi)
     B, Hq, Hkv, D = 2, 8, 2, 128
     G = Hq // Hkv
