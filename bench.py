@@ -3,18 +3,28 @@
 
 One step = one decode step of one attention layer for a whole batch:
   block-summary maintenance (last block) + block scoring + top-k selection
-  (one fused kernel) -> gathered split-KV attention over the selected blocks,
-all in libksa's CUDA kernels.  Metric: queries/s, one query = one
-sequence's decode step for one layer (all query heads).
+  (the fused selection call: a scoring launch and a ranking launch) ->
+  gathered split-KV attention over the selected blocks, all in libksa's CUDA
+  kernels.  Metric: queries/s, one query = one sequence's decode step for one
+  layer (all query heads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ksa|reference]
-                  [--workload qwen3-0.6b|qwen3-8b|lessismore|sweep-L<ctx>-B<budget>|dense-L<ctx>]
+                  [--workload qwen3-8b|qwen3-0.6b|lessismore|tiny|sweep-L<ctx>-B<budget>|dense-L<ctx>]
 
-The default workload is the Qwen3-0.6B-shaped layer (batch 64, Hq 16, Hkv 8,
-D 128, context 16384, block 32, 32 blocks kept).  With N > 1 (torchrun, one
-rank per GPU) every rank runs the same per-GPU batch (weak scaling, no
-collective on the data path); the step time is the max over ranks.
-Rank 0 prints one JSON line on stdout; diagnostics go to stderr.
+The default workload is the Qwen3-8B-shaped layer at 16K-32K context (batch
+32, Hq 32, Hkv 8, D 128, lengths uniform in [16384, 32768], block 16, 128
+blocks kept).  The same line also carries the Qwen3-0.6B-shaped layer (batch
+64, context 16384) and the 32K-context sweep point with a 1024-token budget,
+timed the same way (--no-extra skips them).  With N > 1 (torchrun, one rank
+per GPU) every rank runs the same per-GPU batch (weak scaling, no collective
+on the data path); the step time is the max over ranks.  Rank 0 prints one
+JSON line on stdout; diagnostics go to stderr.
+
+Timing: W warm-up steps (and more, untimed, until at least --min-warmup-s of
+them have run, so the clocks have settled), then K steps back to back between
+two CUDA events on the launching stream, bracketed by barrier + synchronize.
+Nothing else is enqueued inside the timed region.  Per-kernel durations come
+from a second pass of the same steps with an event around each launch.
 """
 from __future__ import annotations
 
@@ -49,9 +59,13 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=100, help="untimed steps before them")
     p.add_argument("--impl", choices=["ksa", "reference"], default="ksa",
                    help="ksa: the CUDA library; reference: the oracle on the host cores")
-    p.add_argument("--workload", default="qwen3-0.6b",
-                   help="qwen3-0.6b, qwen3-8b, lessismore, tiny, sweep-L<ctx>-B<budget>, "
+    p.add_argument("--workload", default="qwen3-8b",
+                   help="qwen3-8b, qwen3-0.6b, lessismore, tiny, sweep-L<ctx>-B<budget>, "
                         "dense-L<ctx>")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the extra workloads carried in the default line")
+    p.add_argument("--min-warmup-s", type=float, default=0.25,
+                   help="keep running untimed warm-up steps until this much time has passed")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="wall-clock budget of the oracle CPU baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -190,13 +204,19 @@ def algorithmic_bytes(shape, seq_lens, kind: str, summary_bytes: int = 4):
 
 
 class ClockSampler:
-    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """nvidia-smi samples every 200 ms while it runs.  mark() notes the host time at the start
+    and end of the timed region; the summary keeps the samples from the warm-up before the
+    first mark (clocks under the same load) to the last mark, or all samples if that window
+    caught none."""
+    FIELDS = ("timestamp,index,uuid,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.proc = None
         self.path = None
+        self.marks = []
         try:
             self.uuid = str(torch.cuda.get_device_properties(device_index).uuid)
         except Exception:
@@ -209,12 +229,25 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.t_start = time.time()
         except Exception:
             self.proc = None
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    @staticmethod
+    def _when(stamp: str):
+        import datetime
+        try:
+            return datetime.datetime.strptime(stamp, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self):
         if self.proc is None:
             return None
+        time.sleep(0.25)  # one more sample after the last mark
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -223,22 +256,29 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 10:
+            if len(parts) < 11:
                 continue
-            if self.uuid and self.uuid not in parts[1] and parts[1] not in self.uuid:
+            if self.uuid and self.uuid not in parts[2] and parts[2] not in self.uuid:
                 continue
             rows.append(parts)
         os.unlink(self.path)
         if not rows:
             return None
-        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        window = "whole run"
+        if len(self.marks) >= 2:
+            lo, hi = self.marks[0] - 0.25, self.marks[-1] + 0.25
+            inside = [r for r in rows if (self._when(r[0]) or 0.0) >= lo
+                      and (self._when(r[0]) or 0.0) <= hi]
+            if inside:
+                rows, window = inside, "last warm-up samples + timed region"
+        sm = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        mx = [float(r[4]) for r in rows if r[4].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[6 + i]
-                          and "Not" not in r[6 + i]})
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[7 + i]
+                          and "Not" not in r[7 + i]})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "window": window}
 
 
 # ---------------------------------------------------------------------------
@@ -270,127 +310,204 @@ def stored_traffic(kernel: str, workload: str, batch: int):
         return None
 
 
-def run_block(args, dist, dev, kind):
-    import block_top_sparse_ksa_b200 as ksa
-    _, shape = resolve_workload(args.workload, args.batch)
-    torch.manual_seed(0)
-    inp = make_block_inputs(shape, dev)
-    B, Hq, Hkv, D, T, bs = (shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
-                            shape.capacity, shape.block_size)
-    k = shape.k_blocks
-    nq = 16
-    qs = query_sets(shape, nq, dev)
-    sdt = torch.bfloat16 if args.summaries == "bf16" else torch.float32
-    S = ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, bs, summary_dtype=sdt)  # prefill, untimed
-    ws_sel = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
-                         dtype=torch.uint8, device=dev)
-    ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
-                         dtype=torch.uint8, device=dev)
-    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
-    cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
-    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+def warm_up(step, warmup: int, min_s: float) -> int:
+    """W untimed steps, then more until min_s seconds have passed (SM clocks settle under
+    load); returns the number of warm-up steps run."""
+    n = 0
+    t0 = time.perf_counter()
+    while n < warmup or time.perf_counter() - t0 < min_s:
+        step(n)
+        n += 1
+        if n % 64 == 0:
+            torch.cuda.synchronize()  # keep the host from running far ahead of the device
+    return n
 
-    def step(i):
-        q = qs[i % nq]
-        if kind == "dense":
-            ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out, workspace=ws_att,
-                                       stream=stream)
-            return
-        ksa.ksa_decode_select_blocks(q, inp.K, S, inp.seq_lens, bs, k, block_idx=idx,
-                                     num_sel=cnt, workspace=ws_sel, stream=stream)
-        ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt, tokens_per_idx=bs,
-                                   out=out, workspace=ws_att, stream=stream)
 
-    # selection: a scoring launch (when some row can hold more than k blocks)
-    # and a ranking launch; then the attention launch
-    nb_max = -(-T // bs)
-    sel_launches = 2 if nb_max > k else 1
-    launches_per_step = 1 if kind == "dense" else sel_launches + 1
-    for i in range(args.warmup):
-        step(i)
-    # per-kernel events on a sample of the timed steps
-    every = max(1, args.steps // 400)
-    marks = []
+def timed_steps(step, steps: int, dist, stream):
+    """K steps back to back between two events on `stream`, bracketed by barrier +
+    synchronize.  Returns (device ms over all K steps, host enqueue us per step)."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev.index or 0)
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
     start.record(stream)
-    for i in range(args.steps):
-        if i % every == 0:
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            q = qs[i % nq]
-            ev[0].record(stream)
-            if kind == "dense":  # no selection: ev[1]..ev[2] is empty
-                ev[1].record(stream)
-                ev[2].record(stream)
-                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, out=out,
-                                           workspace=ws_att, stream=stream)
-            else:
-                ev[1].record(stream)
-                ksa.ksa_decode_select_blocks(q, inp.K, S, inp.seq_lens, bs, k, block_idx=idx,
-                                             num_sel=cnt, workspace=ws_sel, stream=stream)
-                ev[2].record(stream)
-                ksa.ksa_sparse_decode_attn(q, inp.K, inp.V, inp.seq_lens, idx, cnt,
-                                           tokens_per_idx=bs, out=out, workspace=ws_att,
-                                           stream=stream)
-            ev[3].record(stream)
-            marks.append(ev)
-        else:
-            step(i)
+    h0 = time.perf_counter()
+    for i in range(steps):
+        step(i)
+    h1 = time.perf_counter()
     end.record(stream)
     torch.cuda.synchronize()
-    clk = clocks.stop()
     dist.barrier()
-    value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), args.steps)
-    ms = ms_step * args.steps
-    t_sel = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
-    t_att = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
-    lens = inp.seq_lens.cpu().tolist()
-    total_b, attn_b, summ_b = algorithmic_bytes(shape, lens, kind, S.element_size())
-    per_step_s = ms / 1e3 / args.steps
-    peak, peak_kind = measured_peak()
+    return start.elapsed_time(end), (h1 - h0) * 1e6 / steps
+
+
+def kernel_pass(parts, steps: int, stream):
+    """Per-launch device time: the step's launches (`parts`, callables taking the step
+    index) with an event around each, over `steps` steps.  Returns mean ms per part."""
+    evs = []
+    for i in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+        ev[0].record(stream)
+        for j, part in enumerate(parts):
+            part(i)
+            ev[j + 1].record(stream)
+        evs.append(ev)
+    torch.cuda.synchronize()
+    return [statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in evs)
+            for j in range(len(parts))]
+
+
+class BlockWorkload:
+    """Device-resident inputs, prefilled summaries and workspaces of one block workload."""
+
+    def __init__(self, name: str, batch: int, dev, summaries: str):
+        import block_top_sparse_ksa_b200 as ksa
+        self.ksa = ksa
+        self.kind, self.shape = resolve_workload(name, batch)
+        sh = self.shape
+        torch.manual_seed(0)
+        self.inp = make_block_inputs(sh, dev)
+        self.nq = 16
+        self.qs = query_sets(sh, self.nq, dev)
+        sdt = torch.bfloat16 if summaries == "bf16" else torch.float32
+        B, Hq, Hkv, D, T, bs, k = (sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim,
+                                   sh.capacity, sh.block_size, sh.k_blocks)
+        self.S = ksa.ksa_build_block_summaries(self.inp.K, self.inp.seq_lens, bs,
+                                               summary_dtype=sdt)  # prefill, untimed
+        self.ws_sel = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
+                                  dtype=torch.uint8, device=dev)
+        self.ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
+                                  dtype=torch.uint8, device=dev)
+        self.idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        self.stream = torch.cuda.current_stream()
+        nb_max = -(-T // bs)
+        # selection: a scoring launch (when some row can hold more than k blocks) and a
+        # ranking launch; then the attention launch
+        self.launches_per_step = 1 if self.kind == "dense" else (2 if nb_max > k else 1) + 1
+
+    def select(self, i, q=None):
+        sh = self.shape
+        self.ksa.ksa_decode_select_blocks(self.qs[i % self.nq] if q is None else q, self.inp.K,
+                                          self.S, self.inp.seq_lens, sh.block_size, sh.k_blocks,
+                                          block_idx=self.idx, num_sel=self.cnt,
+                                          workspace=self.ws_sel, stream=self.stream)
+
+    def attend(self, i, q=None):
+        q = self.qs[i % self.nq] if q is None else q
+        if self.kind == "dense":
+            self.ksa.ksa_sparse_decode_attn(q, self.inp.K, self.inp.V, self.inp.seq_lens,
+                                            out=self.out, workspace=self.ws_att,
+                                            stream=self.stream)
+        else:
+            self.ksa.ksa_sparse_decode_attn(q, self.inp.K, self.inp.V, self.inp.seq_lens,
+                                            self.idx, self.cnt,
+                                            tokens_per_idx=self.shape.block_size, out=self.out,
+                                            workspace=self.ws_att, stream=self.stream)
+
+    def step(self, i):
+        if self.kind != "dense":
+            self.select(i)
+        self.attend(i)
+
+    def parts(self):
+        return [self.attend] if self.kind == "dense" else [self.select, self.attend]
+
+
+def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
+                  clocks: "ClockSampler | None" = None):
+    """Warm-up, the timed steps and the per-kernel pass of one block workload."""
+    sh, kind = wl.shape, wl.kind
+    n_warm = warm_up(wl.step, args.warmup, args.min_warmup_s)
+    if clocks is not None:
+        clocks.mark()
+    ms, host_us = timed_steps(wl.step, args.steps, dist, wl.stream)
+    if clocks is not None:
+        clocks.mark()
+    value, ms_step = weak_scaling(dist, sh.batch, ms, args.steps)
+    times = kernel_pass(wl.parts(), max(20, min(args.steps, 200)), wl.stream)
+    t_att = times[-1]
+    t_sel = times[0] if kind != "dense" else 0.0
+    lens = wl.inp.seq_lens.cpu().tolist()
+    total_b, attn_b, summ_b = algorithmic_bytes(sh, lens, kind, wl.S.element_size())
+    per_step_s = ms_step / 1e3
     attn_gbs = attn_b / (t_att * 1e-3) / 1e9
-    res = {
-        "ms_per_step": ms / args.steps,
-        "value": value,
+    return {
+        "value": value, "ms_per_step": ms_step, "warmup_steps_run": n_warm,
+        "host_enqueue_us_per_step": host_us,
         "kernels_ms": ({"sparse_decode_attn": t_att} if kind == "dense" else
                        {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att}),
+        "kernels_note": "mean of a second pass of the same steps with an event around each call "
+                        "(the selection call is its scoring and ranking launches)",
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                      "frac": attn_gbs / peak,
-                     "traffic": stored_traffic("sparse_decode_attn", args.workload, shape.batch),
+                     "traffic": stored_traffic("sparse_decode_attn", args.workload, sh.batch),
                      "kernel": "sparse_decode_attn", "peak_source": peak_kind,
                      "bytes_per_launch": attn_b},
         "step_hbm": {"bytes_per_step": total_b, "gbs": total_b / per_step_s / 1e9,
-                     "frac": total_b / per_step_s / 1e9 / peak},
+                     "frac": total_b / per_step_s / 1e9 / peak,
+                     "kernel_sum_ms": t_sel + t_att},
         "select_hbm": (None if kind == "dense" else
                        {"bytes_per_launch": summ_b,
                         "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None}),
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
-        "config": {"workload": shape.name, "batch_per_gpu": B, "num_q_heads": Hq,
-                   "num_kv_heads": Hkv, "head_dim": D, "capacity": T, "block_size": bs,
-                   "k_blocks": k if kind != "dense" else "all",
-                   "summaries": "bf16" if S.dtype == torch.bfloat16 else "f32",
+        "gpu_launches": wl.launches_per_step * args.steps,
+        "config": {"workload": sh.name, "batch_per_gpu": sh.batch, "num_q_heads": sh.num_q_heads,
+                   "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
+                   "capacity": sh.capacity, "block_size": sh.block_size,
+                   "seq_lens": ([sh.min_len, sh.max_len] if sh.min_len != sh.max_len
+                                else sh.max_len),
+                   "k_blocks": sh.k_blocks if kind != "dense" else "all",
+                   "summaries": "bf16" if wl.S.dtype == torch.bfloat16 else "f32",
                    "l2": "inputs larger than L2: K/V cache %.1f GB, %.0f MB read per step, %d "
-                         "rotating query sets" % (2 * inp.K.numel() * 2 / 1e9, total_b / 1e6, nq),
+                         "rotating query sets" % (2 * wl.inp.K.numel() * 2 / 1e9, total_b / 1e6,
+                                                  wl.nq),
                    "step": ("dense attention" if kind == "dense" else
                             "decode_select_blocks (last-block summary refresh + scoring + "
                             "top-k) + sparse_decode_attn")},
     }
+
+
+def run_block(args, dist, dev, kind):
+    wl = BlockWorkload(args.workload, args.batch, dev, args.summaries)
+    peak, peak_kind = measured_peak()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    res = measure_block(wl, args, dist, peak, peak_kind, clocks)
+    res["clocks"] = clocks.stop()
     if not args.no_e2e:
-        res["e2e"] = run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att)
+        res["e2e"] = run_block_e2e(args, dist, wl)
     if kind != "dense":
         try:
-            res["prefill"] = time_prefill(ksa, inp, shape, S, stream, peak)
+            res["prefill"] = time_prefill(wl.ksa, wl.inp, wl.shape, wl.S, wl.stream, peak)
         except Exception as e:  # a side figure: never lose the step's line for it
             res["prefill"] = {"error": str(e)[:200]}
-    res["_host"] = (inp, S, qs, shape, kind)
     return res
+
+
+EXTRA_WORKLOADS = ("qwen3-0.6b", "sweep-L32768-B1024")
+
+
+def run_extra(args, dist, dev):
+    """The other block workloads the line carries, each timed like the main one."""
+    peak, peak_kind = measured_peak()
+    out = {}
+    for name in EXTRA_WORKLOADS:
+        if name == args.workload:
+            continue
+        try:
+            wl = BlockWorkload(name, 0, dev, args.summaries)
+            r = measure_block(wl, args, dist, peak, peak_kind)
+            out[name] = {"workload": wl.shape.name, "value": r["value"], "unit": UNIT,
+                         "ms_per_step": r["ms_per_step"],
+                         "host_enqueue_us_per_step": r["host_enqueue_us_per_step"],
+                         "step_hbm": r["step_hbm"], "roofline_frac": r["roofline"]["frac"],
+                         "kernels_ms": r["kernels_ms"], "gpu_launches": r["gpu_launches"]}
+            del wl
+        except torch.cuda.OutOfMemoryError as e:  # never lose the main line for a side figure
+            out[name] = {"error": str(e)[:200]}
+        torch.cuda.empty_cache()
+    return out
 
 
 def prefill_bytes(shape, seq_lens, summary_bytes: int = 4) -> int:
@@ -421,62 +538,45 @@ def time_prefill(ksa, inp, shape, S, stream, peak, reps: int = 5):
             "gbs": b / (ms * 1e-3) / 1e9, "frac": b / (ms * 1e-3) / 1e9 / peak}
 
 
-def run_block_e2e(args, dist, dev, kind, inp, S, qs, shape, ws_sel, ws_att):
-    """Same step through the public API with host buffers: per step the new
-    query and the new token's K/V rows go host->device (pinned), the output
-    comes back device->host.  Copies are inside the timed region."""
+def run_block_e2e(args, dist, wl: BlockWorkload):
+    """The same step through the public API with host buffers.  Per step: the new query and
+    the new token's K/V rows go host->device from pinned memory, ksa_append_kv writes the
+    rows into their cache slot (token L_b - 1: the lengths stay fixed, so every step is the
+    same workload), then the selection and attention calls, and the output comes back
+    device->host.  The copies are inside the timed region."""
     import block_top_sparse_ksa_b200 as ksa
-    B, Hq, Hkv, D, T, bs = (shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
-                            shape.capacity, shape.block_size)
-    k = shape.k_blocks
-    nq = qs.shape[0]
-    h_q = qs.cpu().pin_memory()
+    sh = wl.shape
+    B, Hq, Hkv, D = sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim
+    dev = wl.qs.device
+    nq = wl.nq
+    h_q = wl.qs.cpu().pin_memory()
     h_kv = torch.randn((nq, 2, B, Hkv, D), dtype=torch.float32).to(torch.bfloat16).pin_memory()
     h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
     d_q = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
     d_kv = torch.empty((2, B, Hkv, D), dtype=torch.bfloat16, device=dev)
-    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
-    cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
-    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
-    lens = inp.seq_lens
-    pos = (lens.long() - 1)  # the newest token's slot per row
-    ar_b = torch.arange(B, device=dev)
+    stream = wl.stream
+    lens = wl.inp.seq_lens
 
     def step(i):
         d_q.copy_(h_q[i % nq], non_blocking=True)
         d_kv.copy_(h_kv[i % nq], non_blocking=True)
-        # append: write the new K/V rows into their cache slots
-        inp.K[ar_b, :, pos] = d_kv[0]
-        inp.V[ar_b, :, pos] = d_kv[1]
-        if kind == "dense":
-            ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, out=out, workspace=ws_att,
-                                       stream=stream)
-        else:
-            ksa.ksa_decode_select_blocks(d_q, inp.K, S, lens, bs, k, block_idx=idx,
-                                         num_sel=cnt, workspace=ws_sel, stream=stream)
-            ksa.ksa_sparse_decode_attn(d_q, inp.K, inp.V, lens, idx, cnt, tokens_per_idx=bs,
-                                       out=out, workspace=ws_att, stream=stream)
-        h_out.copy_(out, non_blocking=True)
+        ksa.ksa_append_kv(d_kv[0], d_kv[1], wl.inp.K, wl.inp.V, lens, stream=stream)
+        if wl.kind != "dense":
+            wl.select(i, d_q)
+        wl.attend(i, d_q)
+        h_out.copy_(wl.out, non_blocking=True)
 
-    steps = args.steps
-    for i in range(args.warmup):
-        step(i)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    dist.barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(steps):
-        step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), steps)
+    warm_up(step, args.warmup, 0.0)
+    ms, host_us = timed_steps(step, args.steps, dist, stream)
+    value, ms_step = weak_scaling(dist, B, ms, args.steps)
     h2d = (B * Hq * D + 2 * B * Hkv * D) * 2
     d2h = B * Hq * D * 4
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
-            "note": "cache append of the new token is a torch index copy"}
+            "host_enqueue_us_per_step": host_us,
+            "gpu_launches": (wl.launches_per_step + 1) * args.steps,
+            "note": "per step: q and the new token's K/V rows host->device (pinned), "
+                    "ksa_append_kv, selection, attention, out device->host"}
 
 
 def run_unified(args, dist, dev):
@@ -496,52 +596,40 @@ def run_unified(args, dist, dev):
                          dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(i, ev=None):
-        if ev:
-            ev[0].record(stream)
+    def select(i):
         ksa.ksa_unified_select(inp.q_sel, inp.K_sel, inp.seq_lens, sh.per_head_topk,
                                sh.token_budget, sh.recent_tokens, tok, cnt, ws, stream=stream)
-        if ev:
-            ev[1].record(stream)
+
+    def attend(i):
         for li, (q, K, V) in enumerate(inp.layers):
             ksa.ksa_sparse_decode_attn(q, K, V, inp.seq_lens, tok, cnt, tokens_per_idx=1,
                                        idx_shared=True, out=outs[li], workspace=ws_att,
                                        stream=stream)
-        if ev:
-            ev[2].record(stream)
 
-    for i in range(args.warmup):
-        step(i)
-    every = max(1, args.steps // 200)
-    marks = []
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    def step(i):
+        select(i)
+        attend(i)
+
     clocks = ClockSampler(dev.index or 0)
-    torch.cuda.synchronize()
-    dist.barrier()
     clocks.start()
-    time.sleep(0.3)
-    start.record(stream)
-    for i in range(args.steps):
-        if i % every == 0:
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-            step(i, ev)
-            marks.append(ev)
-        else:
-            step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
+    n_warm = warm_up(step, args.warmup, args.min_warmup_s)
+    clocks.mark()
+    ms, host_us = timed_steps(step, args.steps, dist, stream)
+    clocks.mark()
     clk = clocks.stop()
-    value, ms_step = weak_scaling(dist, B, start.elapsed_time(end), args.steps)
-    ms = ms_step * args.steps
-    t_sel = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
-    t_att = statistics.mean(m[1].elapsed_time(m[2]) for m in marks) / len(inp.layers)
-    per = ms / 1e3 / args.steps
+    value, ms_step = weak_scaling(dist, B, ms, args.steps)
+    t_sel, t_att3 = kernel_pass([select, attend], max(20, min(args.steps, 200)), stream)
+    t_att = t_att3 / len(inp.layers)
+    per = ms_step / 1e3
     sel_b = B * Hkv * sh.seq_len * D * 2 + B * Hq * D * 2
     att_b = B * Hkv * sh.token_budget * D * 2 * 2 + B * Hq * D * 6
     peak, peak_kind = measured_peak()
     return {
-        "ms_per_step": ms_step, "value": value,
+        "ms_per_step": ms_step, "value": value, "warmup_steps_run": n_warm,
+        "host_enqueue_us_per_step": host_us,
         "kernels_ms": {"unified_select": t_sel, "sparse_decode_attn_per_layer": t_att},
+        "kernels_note": "mean of a second pass of the same steps with an event around the "
+                        "selection call and around the three attention calls",
         "roofline": {"bound": "hbm", "achieved": att_b / (t_att * 1e-3) / 1e9, "peak": peak,
                      "unit": "GB/s", "frac": att_b / (t_att * 1e-3) / 1e9 / peak,
                      "traffic": stored_traffic("sparse_decode_attn", args.workload, sh.batch),
@@ -550,7 +638,8 @@ def run_unified(args, dist, dev):
         "select_hbm": {"bytes_per_launch": sel_b, "gbs": sel_b / (t_sel * 1e-3) / 1e9},
         "step_hbm": {"bytes_per_step": sel_b + 3 * att_b,
                      "gbs": (sel_b + 3 * att_b) / per / 1e9,
-                     "frac": (sel_b + 3 * att_b) / per / 1e9 / peak},
+                     "frac": (sel_b + 3 * att_b) / per / 1e9 / peak,
+                     "kernel_sum_ms": t_sel + t_att3},
         # selection: scores, picks, (vote counting when the picks keep the row's keys in
         # registers: capacity <= 24576), shared set; then one attention launch per layer
         "gpu_launches": ((4 if T <= 24576 else 3) + len(inp.layers)) * args.steps, "clocks": clk,
@@ -708,8 +797,6 @@ def main():
             res = run_unified(args, dist, dev)
         else:
             res = run_block(args, dist, dev, kind)
-        host = res.pop("_host", None)
-        del host
         line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": dist.world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -718,11 +805,16 @@ def main():
                                "replicas, no data-path collective)"),
                 "roofline": res["roofline"], "kernels_ms": res["kernels_ms"],
                 "step_hbm": res["step_hbm"], "select_hbm": res.get("select_hbm"),
-                "gpu_launches": res["gpu_launches"], "clocks": res["clocks"]}
+                "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+                "warmup_steps_run": res["warmup_steps_run"],
+                "host_enqueue_us_per_step": res["host_enqueue_us_per_step"],
+                "kernels_note": res["kernels_note"]}
         if "e2e" in res:
             line["e2e"] = res["e2e"]
         if "prefill" in res:
             line["prefill"] = res["prefill"]
+        if kind != "unified" and not args.no_extra and args.batch == 0:
+            line["extra_workloads"] = run_extra(args, dist, dev)
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args, dev, kind, args.cpu_seconds)
         if dist.rank == 0:

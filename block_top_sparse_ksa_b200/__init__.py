@@ -31,7 +31,7 @@ __all__ = [
     "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window", "ksa_select_tokens_per_head",
     "ksa_select_tokens_per_head_workspace", "ksa_select_tokens_one_head",
     "ksa_select_tokens_one_head_workspace", "ksa_get_device_status", "IDX_PER_KV_HEAD",
-    "IDX_SHARED", "IDX_PER_Q_HEAD",
+    "IDX_SHARED", "IDX_PER_Q_HEAD", "ksa_append_kv", "ksa_append_kv_paged",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -86,6 +86,9 @@ _SIGS = {
     "ksa_sparse_decode_attn_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp,
                                             ctypes.POINTER(Pages), _vp, _vp, _vp, _i32, _i32,
                                             _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "ksa_append_kv": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ksa_append_kv_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp,
+                                   ctypes.POINTER(Pages), _vp, _vp, _vp]),
     "ksa_select_window": (_i32, [ctypes.POINTER(Shape), _vp, _i32, _vp, _vp, _vp, _vp]),
     "ksa_select_tokens_per_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
     "ksa_select_tokens_one_head_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
@@ -214,12 +217,18 @@ def ksa_build_block_summaries(K: torch.Tensor, seq_lens: torch.Tensor, block_siz
 ksa_build_block_summaries_ex = ksa_build_block_summaries
 
 
-def _workspace(ws: Optional[torch.Tensor], need: int, device) -> torch.Tensor:
-    """The caller's workspace, or a fresh zero-filled one (see include/ksa.h)."""
-    if ws is None:
-        return torch.zeros((max(need, 1),), dtype=torch.uint8, device=device)
-    _dev(ws, "workspace", ws.dtype)
-    return ws
+def _workspace(ws: Optional[torch.Tensor], sh: Shape, args, kind: str, device) -> torch.Tensor:
+    """The caller's workspace as given (the library checks its size), or a fresh zero-filled
+    one of the size the matching *_workspace query returns (see include/ksa.h)."""
+    if ws is not None:
+        if not ws.is_cuda or not ws.is_contiguous():
+            raise TypeError("workspace must be a contiguous CUDA tensor")
+        return ws
+    if kind == "select":
+        need = lib().ksa_select_blocks_workspace(ctypes.byref(sh), args)
+    else:
+        need = lib().ksa_sparse_decode_attn_workspace(ctypes.byref(sh), *args)
+    return torch.zeros((max(int(need), 1),), dtype=torch.uint8, device=device)
 
 
 def ksa_select_blocks_workspace(B: int, Hq: int, Hkv: int, D: int, T: int, block_size: int,
@@ -246,8 +255,7 @@ def ksa_select_blocks(q: torch.Tensor, summaries: torch.Tensor, seq_lens: torch.
     if num_sel is None:
         num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     sh = _shape(B, Hq, Hkv, D, capacity, block_size)
-    ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
-                    q.device)
+    ws = _workspace(workspace, sh, int(k_blocks), "select", q.device)
     _check(lib().ksa_select_blocks_ex(ctypes.byref(sh), _ptr(q), _ptr(summaries),
                                       _summary_dtype(summaries), _ptr(seq_lens), int(k_blocks),
                                       _ptr(block_idx), _ptr(num_sel), _ptr(ws),
@@ -277,8 +285,7 @@ def ksa_decode_select_blocks(q: torch.Tensor, K: torch.Tensor, summaries: torch.
     if num_sel is None:
         num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     sh = _shape(B, Hq, Hkv, D, T, block_size)
-    ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
-                    q.device)
+    ws = _workspace(workspace, sh, int(k_blocks), "select", q.device)
     _check(lib().ksa_decode_select_blocks_ex(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(summaries), _summary_dtype(summaries),
         _ptr(seq_lens), int(k_blocks), _ptr(block_idx), _ptr(num_sel), _ptr(ws),
@@ -316,8 +323,7 @@ def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     if lse is not None:
         _dev(lse, "lse", torch.float32)
     sh = _shape(B, Hq, Hkv, D, T, max(1, tokens_per_idx))
-    ws = _workspace(workspace, lib().ksa_sparse_decode_attn_workspace(
-        ctypes.byref(sh), int(cap), int(tokens_per_idx)), q.device)
+    ws = _workspace(workspace, sh, (int(cap), int(tokens_per_idx)), "attn", q.device)
     _check(lib().ksa_sparse_decode_attn(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(seq_lens), _ptr(idx), _ptr(num_idx),
         int(cap), int(tokens_per_idx), int(idx_shared), float(scale), int(out_dtype),
@@ -389,8 +395,8 @@ def ksa_unified_select(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor,
     _dev(seq_lens, "seq_lens", torch.int32)
     B, Hq, D = q.shape
     _, Hkv, T, _ = K.shape
-    need = ksa_unified_select_workspace(B, Hq, Hkv, D, T, per_head_topk, token_budget)
     if workspace is None:  # the unified workspace needs no initialisation
+        need = ksa_unified_select_workspace(B, Hq, Hkv, D, T, per_head_topk, token_budget)
         workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     if token_idx is None:
         token_idx = torch.empty((B, token_budget), dtype=torch.int32, device=q.device)
@@ -457,8 +463,7 @@ def ksa_decode_select_blocks_paged(q: torch.Tensor, K_pages: torch.Tensor,
         num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     sh = _shape(B, Hq, Hkv, D, mb * bs, bs)
     pg = _pages(block_table, P)
-    ws = _workspace(workspace, lib().ksa_select_blocks_workspace(ctypes.byref(sh), int(k_blocks)),
-                    q.device)
+    ws = _workspace(workspace, sh, int(k_blocks), "select", q.device)
     _check(lib().ksa_decode_select_blocks_paged(
         ctypes.byref(sh), _ptr(q), _ptr(K_pages), ctypes.byref(pg), _ptr(summaries),
         _summary_dtype(summaries), _ptr(seq_lens), int(k_blocks), _ptr(block_idx), _ptr(num_sel),
@@ -496,14 +501,52 @@ def ksa_sparse_decode_attn_paged(q: torch.Tensor, K_pages: torch.Tensor, V_pages
         cap = idx.shape[-1]
     sh = _shape(B, Hq, Hkv, D, mb * bs, bs)
     pg = _pages(block_table, P)
-    ws = _workspace(workspace, lib().ksa_sparse_decode_attn_workspace(
-        ctypes.byref(sh), int(cap), int(tokens_per_idx)), q.device)
+    ws = _workspace(workspace, sh, (int(cap), int(tokens_per_idx)), "attn", q.device)
     _check(lib().ksa_sparse_decode_attn_paged(
         ctypes.byref(sh), _ptr(q), _ptr(K_pages), _ptr(V_pages), ctypes.byref(pg),
         _ptr(seq_lens), _ptr(idx), _ptr(num_idx), int(cap), int(tokens_per_idx),
         int(idx_shared), float(scale), int(out_dtype), _ptr(out), _ptr(lse), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
     return out, lse
+
+
+def ksa_append_kv(k_new: torch.Tensor, v_new: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                  seq_lens: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+                  stream=None) -> None:
+    """Write the new token's rows: K[b, g, L_b - 1] = k_new[b, g], V likewise (k_new, v_new
+    [B, Hkv, D] bf16; seq_lens already counts the new token)."""
+    _dev(k_new, "k_new", torch.bfloat16)
+    _dev(v_new, "v_new", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(V, "V", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hkv, T, D = K.shape
+    if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+        raise ValueError(f"k_new and v_new must be [{B}, {Hkv}, {D}]")
+    sh = _shape(B, Hkv, Hkv, D, T)
+    _check(lib().ksa_append_kv(ctypes.byref(sh), _ptr(k_new), _ptr(v_new), _ptr(K), _ptr(V),
+                               _ptr(seq_lens), _ptr(dev_status), _stream(stream)))
+
+
+def ksa_append_kv_paged(k_new: torch.Tensor, v_new: torch.Tensor, K_pages: torch.Tensor,
+                        V_pages: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ksa_append_kv on a paged K/V cache (pools [num_pages, Hkv, bs, D], block table
+    [B, max_blocks])."""
+    _dev(k_new, "k_new", torch.bfloat16)
+    _dev(v_new, "v_new", torch.bfloat16)
+    _dev(K_pages, "K_pages", torch.bfloat16)
+    _dev(V_pages, "V_pages", torch.bfloat16)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    P, Hkv, bs, D = K_pages.shape
+    B, mb = block_table.shape
+    if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+        raise ValueError(f"k_new and v_new must be [{B}, {Hkv}, {D}]")
+    sh = _shape(B, Hkv, Hkv, D, mb * bs, bs)
+    pg = _pages(block_table, P)
+    _check(lib().ksa_append_kv_paged(ctypes.byref(sh), _ptr(k_new), _ptr(v_new), _ptr(K_pages),
+                                     _ptr(V_pages), ctypes.byref(pg), _ptr(seq_lens),
+                                     _ptr(dev_status), _stream(stream)))
 
 
 def ksa_select_window(seq_lens: torch.Tensor, num_kv_heads: int, block_size: int, capacity: int,
@@ -544,8 +587,8 @@ def ksa_select_tokens_per_head(q: torch.Tensor, K: torch.Tensor, seq_lens: torch
     _dev(seq_lens, "seq_lens", torch.int32)
     B, Hq, D = q.shape
     _, Hkv, T, _ = K.shape
-    need = ksa_select_tokens_per_head_workspace(B, Hq, Hkv, D, T, k_tokens)
     if workspace is None:  # no initialisation needed
+        need = ksa_select_tokens_per_head_workspace(B, Hq, Hkv, D, T, k_tokens)
         workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     if token_idx is None:
         token_idx = torch.empty((B, Hq, k_tokens), dtype=torch.int32, device=q.device)
@@ -585,8 +628,8 @@ def ksa_select_tokens_one_head(q: torch.Tensor, K: torch.Tensor, seq_lens: torch
     heads = np.ascontiguousarray(heads, dtype=np.int32)
     if heads.shape != (B,):
         raise ValueError(f"head_of_row must hold {B} heads, got shape {heads.shape}")
-    need = ksa_select_tokens_one_head_workspace(B, Hq, Hkv, D, T, k_tokens)
     if workspace is None:  # no initialisation needed
+        need = ksa_select_tokens_one_head_workspace(B, Hq, Hkv, D, T, k_tokens)
         workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     if token_idx is None:
         token_idx = torch.empty((B, k_tokens), dtype=torch.int32, device=q.device)

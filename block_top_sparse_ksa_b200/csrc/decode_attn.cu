@@ -671,13 +671,9 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
                        cudaStream_t stream) {
   const int G = p.gw;
   const size_t smem = Cfg<D>::kFixedSmem + static_cast<size_t>(kConsumers) * (2 * G + G * D) * 4;
-  cudaError_t err = cudaFuncSetAttribute(sparse_decode_attn_kernel<D, MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
   int occ = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, sparse_decode_attn_kernel<D, MODE>,
-                                                      kAttnThreads, smem);
+  const cudaError_t err = kernel_occupancy(
+      reinterpret_cast<const void *>(sparse_decode_attn_kernel<D, MODE>), kAttnThreads, smem, &occ);
   if (err != cudaSuccess) return err;
   occ = occ < 1 ? 1 : (occ > kAttnMaxCtasPerSm ? kAttnMaxCtasPerSm : occ);
   long long n = static_cast<long long>(num_sms) * occ;

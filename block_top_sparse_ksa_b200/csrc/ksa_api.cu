@@ -8,8 +8,11 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+#include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 
 #include "../../include/ksa.h"
 #include "ksa_internal.h"
@@ -39,14 +42,7 @@ ksa_status cuda_status(cudaError_t err, const char *what) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int device_sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return 148;
-  return n;
-}
+using ksa::device_sm_count;
 
 ksa_status check_shape(const ksa_shape *s, bool need_block) {
   if (s == nullptr) return fail(KSA_ERR_INVALID_ARG, "shape is NULL");
@@ -90,6 +86,57 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 namespace ksa {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];  // 0: not yet queried
+std::mutex g_occ_mu;
+// (device, kernel) -> largest dynamic shared-memory size enabled so far
+std::map<std::tuple<int, const void *>, size_t> g_smem_enabled;
+// (device, kernel, threads, smem) -> resident CTAs per SM
+std::map<std::tuple<int, const void *, int, size_t>, int> g_occ;
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int n = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+cudaError_t kernel_occupancy(const void *func, int threads, size_t smem, int *occ) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(g_occ_mu);
+  const auto key = std::make_tuple(dev, func, threads, smem);
+  const auto hit = g_occ.find(key);
+  if (hit != g_occ.end()) {
+    *occ = hit->second;
+    return cudaSuccess;
+  }
+  // the limit only ever grows, so every size seen before stays launchable
+  size_t &enabled = g_smem_enabled[std::make_tuple(dev, func)];
+  if (smem > enabled) {
+    err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    enabled = smem;
+  }
+  int n = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem);
+  if (err != cudaSuccess) return err;
+  g_occ[key] = n;
+  *occ = n;
+  return cudaSuccess;
+}
 
 ksa_status set_last_error(ksa_status status, const char *fmt, ...) {
   char buf[512];
@@ -190,6 +237,51 @@ ksa_status ksa_build_block_summaries_paged(const ksa_shape *shape, const uint16_
   if (pages == nullptr) return fail(KSA_ERR_INVALID_ARG, "pages must be non-NULL");
   return summaries_common(shape, K_pages, pages, seq_lens, mode, summary_dtype, summaries,
                           dev_status, stream);
+}
+
+namespace {
+
+ksa_status append_common(const ksa_shape *shape, const uint16_t *k_new, const uint16_t *v_new,
+                         uint16_t *K, uint16_t *V, const ksa_pages *pages,
+                         const int32_t *seq_lens, uint32_t *dev_status, void *stream) {
+  ksa_status st = check_shape(shape, pages != nullptr);
+  if (st != KSA_OK) return st;
+  if (k_new == nullptr || v_new == nullptr || K == nullptr || V == nullptr || seq_lens == nullptr)
+    return fail(KSA_ERR_INVALID_ARG, "k_new, v_new, K, V and seq_lens must be non-NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(K, 16) || !aligned(V, 16) ||
+      !aligned(seq_lens, 4))
+    return fail(KSA_ERR_INVALID_ARG, "k_new, v_new, K and V must be 16-byte aligned");
+  ksa::AppendArgs a;
+  if (pages != nullptr && (st = check_pages(shape, pages, &a.kv)) != KSA_OK) return st;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.K = K;
+  a.V = V;
+  a.seq_lens = seq_lens;
+  a.status = dev_status;
+  a.B = shape->batch;
+  a.Hkv = shape->num_kv_heads;
+  a.T = shape->capacity;
+  a.D = shape->head_dim;
+  return cuda_status(ksa::launch_append_kv(a, static_cast<cudaStream_t>(stream)),
+                     "ksa_append_kv launch");
+}
+
+}  // namespace
+
+ksa_status ksa_append_kv(const ksa_shape *shape, const uint16_t *k_new, const uint16_t *v_new,
+                         uint16_t *K, uint16_t *V, const int32_t *seq_lens, uint32_t *dev_status,
+                         void *stream) {
+  return append_common(shape, k_new, v_new, K, V, nullptr, seq_lens, dev_status, stream);
+}
+
+ksa_status ksa_append_kv_paged(const ksa_shape *shape, const uint16_t *k_new,
+                               const uint16_t *v_new, uint16_t *K_pages, uint16_t *V_pages,
+                               const ksa_pages *pages, const int32_t *seq_lens,
+                               uint32_t *dev_status, void *stream) {
+  if (pages == nullptr) return fail(KSA_ERR_INVALID_ARG, "pages must be non-NULL");
+  return append_common(shape, k_new, v_new, K_pages, V_pages, pages, seq_lens, dev_status,
+                       stream);
 }
 
 ksa_status ksa_build_block_summaries(const ksa_shape *shape, const uint16_t *K,

@@ -45,6 +45,18 @@ struct SummaryArgs {
 };
 cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream);
 
+// The decode step's cache write: the new token's key and value rows of every
+// (b, g) go to token slot L_b - 1 (seq_lens counts the new token).
+struct AppendArgs {
+  const uint16_t *k_new, *v_new;  // [B, Hkv, D]
+  uint16_t *K, *V;                // caches (contiguous or paged, per kv)
+  const int32_t *seq_lens;
+  uint32_t *status;
+  int B, Hkv, T, D;
+  KvLayout kv;
+};
+cudaError_t launch_append_kv(const AppendArgs &a, cudaStream_t stream);
+
 struct SelectArgs {
   const uint16_t *q;
   void *S;    // fp32 or bf16; read; written only by the fused last-block refresh
@@ -100,6 +112,17 @@ size_t unified_workspace_bytes(int B, int Hq, int T);
 cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream);
 // Per-head token top-k lists (P = k = budget; token_idx [B, Hq, k], num_sel [B, Hq]).
 cudaError_t launch_tokens_per_head(const UnifiedArgs &a, cudaStream_t stream);
+
+// Resident CTAs per SM of `func` launched with `threads` threads and `smem`
+// bytes of dynamic shared memory, on the current device.  The first query per
+// (device, kernel, threads, smem) raises the kernel's dynamic shared-memory
+// limit as needed and asks the occupancy calculator; later ones read a memo,
+// so a launch pays no driver query.  Thread-safe.
+cudaError_t kernel_occupancy(const void *func, int threads, size_t smem, int *occ);
+
+// Streaming multiprocessors of the current device (memo per device; 148 if
+// the query fails).
+int device_sm_count();
 
 // Records a message for ksa_last_error() and returns `status`.
 ksa_status set_last_error(ksa_status status, const char *fmt, ...)

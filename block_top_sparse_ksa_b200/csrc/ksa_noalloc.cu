@@ -1,18 +1,17 @@
 // ksa_noalloc.cu -- sparse decode attention without any allocation.
 //
 // ksa_sparse_decode_attn needs a caller-allocated workspace.  Some callers
-// must not allocate device memory: a serving loop that forbids new device
-// memory after start-up (cudaMalloc synchronizes the device and can fragment
-// a pre-sized pool), code being recorded into a CUDA graph while stream
-// capture is active (cudaMalloc is not permitted then), or an integration
-// layer that is handed only its input and output buffers.  For them this file
-// keeps one fixed scratch area inside the library and runs the same attention
-// kernel on it.
+// cannot allocate device memory: a serving loop that allows no new device
+// memory after start-up (cudaMalloc synchronizes the device and can fragment a
+// pre-sized pool), or an integration layer that is handed only its input and
+// output buffers and owns no allocator.  For them this file keeps one fixed
+// scratch area inside the library and runs the same attention kernel on it.
 //
 // The scratch is a file-scope __device__ array, so every GPU that loads the
 // library holds kNoAllocScratchBytes of it until the process exits.  In host
 // code the array's name only stands in for it: its device address is looked
-// up once per device with cudaGetSymbolAddress, on that device's first call.
+// up with cudaGetSymbolAddress on a device's first call, and again whenever
+// the device's current context has changed since (a device reset).
 #include <mutex>
 
 #include "../../include/ksa.h"
@@ -29,10 +28,34 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices];  // device address of the scratch, per device ordinal
+// Device address of the scratch per device ordinal, with the context it was
+// looked up in: after a device reset the primary context is a new one, the old
+// address is stale, and the next call looks it up again.
+struct ScratchAddr {
+  CUcontext ctx;
+  void *addr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of the scratch on the current device (looked up once per device).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+
+// The driver's cuCtxGetCurrent, fetched through the runtime (no link to libcuda).
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch on the current device (looked up once per
+// device and context).
 ksa_status scratch_on_current_device(void **out) {
   int dev = -1;
   cudaError_t err = cudaGetDevice(&dev);
@@ -41,16 +64,25 @@ ksa_status scratch_on_current_device(void **out) {
   if (dev < 0 || dev >= kMaxDevices)
     return ksa::set_last_error(KSA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev,
                                kMaxDevices - 1);
+  const CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr)
+    return ksa::set_last_error(KSA_ERR_CUDA, "cuCtxGetCurrent is not available");
+  CUcontext ctx = nullptr;  // null before the runtime has made the device's context
+  if (get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
+  ScratchAddr &e = g_scratch_addr[dev];
+  if (e.addr == nullptr || ctx == nullptr || e.ctx != ctx) {
+    void *p = nullptr;  // (the lookup makes the context if there was none)
     err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (err != cudaSuccess || p == nullptr)
       return ksa::set_last_error(KSA_ERR_CUDA, "cudaGetSymbolAddress of the scratch: %s",
                                  cudaGetErrorString(err));
-    g_scratch_addr[dev] = p;
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+      return ksa::set_last_error(KSA_ERR_CUDA, "no current CUDA context on device %d", dev);
+    e.ctx = ctx;
+    e.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return KSA_OK;
 }
 

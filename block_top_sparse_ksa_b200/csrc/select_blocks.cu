@@ -525,7 +525,7 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
   if (nb_max > a.k) {  // otherwise no row has a block to score
     const auto kern = a.sbf16 ? score_blocks_kernel<D, true> : score_blocks_kernel<D, false>;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kScThreads, 0);
+    err = kernel_occupancy(reinterpret_cast<const void *>(kern), kScThreads, 0, &per_sm);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     constexpr int kWarps = kScThreads / 32;

@@ -10,6 +10,10 @@
 // independent (in flight together).  Partial sums meet through warp shuffles;
 // then one IEEE division by n_j, in fp32, and the mean is stored as fp32 or
 // as bf16 rounded to nearest even.
+//
+// Also here: the decode step's cache append (the new token's key and value
+// rows written into their slot), the write that the last-block refresh of the
+// summaries follows.
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
 
@@ -60,7 +64,44 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
   }
 }
 
+// One thread per 16-byte chunk of the new K rows, then of the new V rows.  A
+// row whose seq_len is outside [1, T], or whose slot's page id names no page,
+// is not written (a clamped slot would overwrite a valid token) and is flagged.
+__global__ void __launch_bounds__(256) append_kv_kernel(const AppendArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int ch = a.D / 8;  // 16-byte chunks per row
+  const long long n = static_cast<long long>(a.B) * a.Hkv * ch;
+  long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= 2 * n) return;
+  const bool is_v = e >= n;
+  if (is_v) e -= n;
+  const int c = static_cast<int>(e % ch);
+  const long long bg = e / ch;
+  const int b = static_cast<int>(bg / a.Hkv), g = static_cast<int>(bg - static_cast<long long>(b) * a.Hkv);
+  const bool reporter = c == 0 && !is_v;
+  const int len = a.seq_lens[b];
+  if (len < 1 || len > a.T) {
+    if (reporter && g == 0) flag_status(a.status, KSA_FLAG_SEQ_LEN_CLAMPED);
+    return;
+  }
+  const long long row = kv_row(a.kv, b, g, a.Hkv, a.T, len - 1);
+  if (row < 0) {
+    if (reporter) flag_status(a.status, KSA_FLAG_INDEX_SKIPPED);
+    return;
+  }
+  const uint16_t *src = (is_v ? a.v_new : a.k_new) + bg * a.D + c * 8;
+  uint16_t *dst = (is_v ? a.V : a.K) + row * a.D + c * 8;
+  *reinterpret_cast<uint4 *>(dst) = __ldg(reinterpret_cast<const uint4 *>(src));
+}
+
 }  // namespace
+
+cudaError_t launch_append_kv(const AppendArgs &a, cudaStream_t stream) {
+  const long long n = 2LL * a.B * a.Hkv * (a.D / 8);
+  return launch_pdl(append_kv_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0,
+                    stream, a);
+}
 
 cudaError_t launch_block_summaries(const SummaryArgs &a, cudaStream_t stream) {
   const int nb_max = (a.T + a.bs - 1) / a.bs;

@@ -472,9 +472,9 @@ cudaError_t launch_scores(const UnifiedArgs &a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   const int n_chunks = (a.T + kChunk - 1) / kChunk;
   const size_t smem = SCfg<D>::kSmemBytes;
-  cudaError_t err = cudaFuncSetAttribute(unified_scores_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  int occ = 0;  // (the memo raises the kernel's shared-memory limit once per device)
+  const cudaError_t err = kernel_occupancy(reinterpret_cast<const void *>(unified_scores_kernel<D>),
+                                           kScoreThreads, smem, &occ);
   if (err != cudaSuccess) return err;
   const unsigned grid = static_cast<unsigned>(a.B) * a.Hkv * n_chunks;
   return launch_pdl(unified_scores_kernel<D>, dim3(grid), dim3(kScoreThreads), smem, stream, km,
@@ -497,8 +497,9 @@ cudaError_t launch_tokens_per_head(const UnifiedArgs &a, cudaStream_t stream) {
   if (err != cudaSuccess) return err;
   const int in_smem = a.T <= kSmemKeys ? 1 : 0;
   const size_t smem = in_smem ? static_cast<size_t>(a.T) * sizeof(uint32_t) : 0;
-  err = cudaFuncSetAttribute(unified_topk_list_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+  int occ = 0;
+  err = kernel_occupancy(reinterpret_cast<const void *>(unified_topk_list_kernel), kPickThreads,
+                         smem, &occ);
   if (err != cudaSuccess) return err;
   return launch_pdl(unified_topk_list_kernel, dim3(static_cast<unsigned>(a.B) * a.Hq),
                     dim3(kPickThreads), smem, stream, a, in_smem);
@@ -525,8 +526,9 @@ cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_
   } else {  // longer rows: keys staged in shared memory (or read from L2)
     const int in_smem = a.T <= kSmemKeys ? 1 : 0;
     const size_t pick_smem = in_smem ? static_cast<size_t>(a.T) * sizeof(uint32_t) : 0;
-    err = cudaFuncSetAttribute(unified_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(pick_smem));
+    int occ = 0;
+    err = kernel_occupancy(reinterpret_cast<const void *>(unified_pick_kernel), kPickThreads,
+                           pick_smem, &occ);
     if (err != cudaSuccess) return err;
     err = launch_pdl(unified_pick_kernel, pgrid, dim3(kPickThreads), pick_smem, stream, a,
                      in_smem);

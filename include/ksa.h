@@ -253,6 +253,32 @@ ksa_status ksa_decode_select_blocks_paged(const ksa_shape *shape, const uint16_t
                                           size_t ws_bytes, uint32_t *dev_status, void *stream);
 
 /*
+ * Cache append: the decode step's write of the new token [KIN s.5: the
+ * history the blocks are cut from is the cached keys and values of every
+ * token so far; each step adds one].  For every (b, kv-head g):
+ *   K[b,g,L_b-1,:] = k_new[b,g,:],   V[b,g,L_b-1,:] = v_new[b,g,:]
+ * where L_b = seq_lens[b] already counts the new token.  Run it before the
+ * step's selection and attention (ksa_decode_select_blocks then refreshes the
+ * summary of the block the token landed in).
+ *   k_new, v_new: [B, Hkv, D] bf16 (read)
+ *   K, V:         [B, Hkv, T, D] bf16 (one row of each (b, g) written)
+ * A row whose seq_len is outside [1, T] is not written and sets
+ * KSA_FLAG_SEQ_LEN_CLAMPED (a clamped slot would overwrite a valid token).
+ * shape->num_q_heads and block_size are not used (any valid values).
+ * Pointers 16-byte aligned, else KSA_ERR_INVALID_ARG.
+ */
+ksa_status ksa_append_kv(const ksa_shape *shape, const uint16_t *k_new,
+                         const uint16_t *v_new, uint16_t *K, uint16_t *V,
+                         const int32_t *seq_lens, uint32_t *dev_status, void *stream);
+/* ksa_append_kv on a paged cache: the token goes to slot (L_b-1) % bs of page
+ * block_table[b, (L_b-1) / bs]; a page id outside the pool is not written and
+ * sets KSA_FLAG_INDEX_SKIPPED. */
+ksa_status ksa_append_kv_paged(const ksa_shape *shape, const uint16_t *k_new,
+                               const uint16_t *v_new, uint16_t *K_pages, uint16_t *V_pages,
+                               const ksa_pages *pages, const int32_t *seq_lens,
+                               uint32_t *dev_status, void *stream);
+
+/*
  * Sparse decode attention over a selected token set [KIN s.5; LIM s.5
  * "sparse attention layer", GQA kernel sharing one KV set per group].
  * For query head h of row b (kv-head g = h / G) and selected tokens T_sel:
@@ -307,10 +333,9 @@ ksa_status ksa_sparse_decode_attn_paged(const ksa_shape *shape, const uint16_t *
 
 /*
  * ksa_sparse_decode_attn without a workspace argument: the same computation,
- * arguments and results, for callers that must not allocate device memory
- * (a serving loop that allows no new device memory after start-up, code
- * recorded into a CUDA graph while capture is active, or a layer handed only
- * its input and output buffers).  The sources describe no such entry point;
+ * arguments and results, for callers that cannot allocate device memory (a
+ * serving loop that allows no new device memory after start-up, or a layer
+ * handed only its input and output buffers, with no allocator of its own).  The sources describe no such entry point;
  * it is an integration convenience with no counterpart in the method.
  * The library keeps one fixed 8 MiB scratch area per GPU (held from the first
  * call on that GPU, or from library load when CUDA loads modules eagerly,
@@ -319,7 +344,9 @@ ksa_status ksa_sparse_decode_attn_paged(const ksa_shape *shape, const uint16_t *
  * with a message.  It allocates nothing: it clears the scratch's semaphores
  * with cudaMemsetAsync on `stream` and launches the attention kernel.
  * The first call on a device looks up the scratch's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * (cudaGetSymbolAddress), and so does the first call after the device's
+ * context has changed (cudaDeviceReset); make that first call before any
+ * stream capture.
  * Every call shares the one scratch area, so calls that may overlap on the
  * GPU (different streams, or different host threads) race: issue them one
  * after another on one stream.

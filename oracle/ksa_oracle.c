@@ -35,7 +35,9 @@
  *        mean is replaced by the nearest bf16 value (ties to even) and the
  *        scores read the stored values;
  *  (R11) random-head aggregation: the random head of each row is an input
- *        drawn by the caller, and that head's own top-k set serves every head.
+ *        drawn by the caller, and that head's own top-k set serves every head;
+ *  (R12) attention recall of a selection is the share of the dense softmax
+ *        weight (over every cached token) that falls on the selected tokens.
  *
  * Inputs: bf16 values arrive as their 16-bit patterns and are widened to fp64
  * exactly.  All arrays are dense row-major.  Threads: OpenMP over independent
@@ -403,6 +405,79 @@ typedef struct {
   double key; /* sort descending on key */
   int32_t t;  /* then ascending on t */
 } ranked_t;
+
+/* ---- (f4) attention recall ----------------------------------------------
+ * LessIsMore, section 3 (accuracy and efficiency) and section 4 (mechanism
+ * analysis) rate a token selection by attention recall: how much of a query
+ * head's full softmax attention falls on the selected tokens.  Written as the
+ * definition: the dense weights w_t = exp(z_t - max z) / sum_u exp(z_u - max z)
+ * over every t < L_b, z_t = scale * <q_h, K_t>, then the sum of w_t over the
+ * distinct selected tokens t < L_b.  Layouts of the selection as for
+ * attention; shared = 2 means one list per query head [B, Hq, cap].
+ * recall: [B, Hq]. */
+void ksa_oracle_attention_recall(int B, int Hq, int Hkv, int D, int T,
+                                 const uint16_t *q, const uint16_t *K,
+                                 const int32_t *seq_lens, const int32_t *idx,
+                                 const int32_t *num_idx, int cap, int tpi,
+                                 int shared, double scale, double *recall) {
+  const int G = Hq / Hkv;
+  if (scale == 0.0) scale = 1.0 / sqrt((double)D); /* R7 */
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hq; ++h) {
+      const int g = h / G;
+      const int L = seq_lens[b];
+      double *r = recall + (size_t)b * Hq + h;
+      if (L <= 0) {
+        *r = 0.0;
+        continue;
+      }
+      /* the dense softmax over every cached token */
+      double *w = (double *)malloc(sizeof(double) * (size_t)L);
+      const uint16_t *qrow = q + ((size_t)b * Hq + h) * D;
+      double zmax = -INFINITY;
+      for (int t = 0; t < L; ++t) {
+        const uint16_t *krow = K + (((size_t)b * Hkv + g) * T + t) * D;
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += bf16_to_f64(qrow[d]) * bf16_to_f64(krow[d]);
+        w[t] = scale * acc;
+        if (w[t] > zmax) zmax = w[t];
+      }
+      double denom = 0.0;
+      for (int t = 0; t < L; ++t) {
+        w[t] = exp(w[t] - zmax);
+        denom += w[t];
+      }
+      /* the selected tokens, each counted once */
+      char *sel = (char *)calloc((size_t)L, 1);
+      const int32_t *list;
+      int cnt;
+      if (shared == 1) {
+        list = idx + (size_t)b * cap;
+        cnt = num_idx[b];
+      } else if (shared == 2) {
+        list = idx + ((size_t)b * Hq + h) * cap;
+        cnt = num_idx[b * Hq + h];
+      } else {
+        list = idx + ((size_t)b * Hkv + g) * cap;
+        cnt = num_idx[b * Hkv + g];
+      }
+      for (int e = 0; e < cnt; ++e) {
+        if (list[e] < 0) continue;
+        for (int u = 0; u < tpi; ++u) {
+          const long t = (long)list[e] * tpi + u;
+          if (t < L) sel[t] = 1;
+        }
+      }
+      double mass = 0.0;
+      for (int t = 0; t < L; ++t)
+        if (sel[t]) mass += w[t] / denom;
+      *r = mass;
+      free(sel);
+      free(w);
+    }
+  }
+}
 
 static int cmp_ranked(const void *a, const void *b) {
   const ranked_t *x = (const ranked_t *)a, *y = (const ranked_t *)b;

@@ -64,6 +64,8 @@ class Oracle:
                                            ctypes.c_void_p, ctypes.c_void_p, c_int, c_int,
                                            c_int, c_double, _f64p, nullable_f64,
                                            nullable_f64])
+        L.ksa_oracle_attention_recall.argtypes = ([c_int] * 5 + [_u16p, _u16p, _i32p, _i32p,
+                                                  _i32p, c_int, c_int, c_int, c_double, _f64p])
         L.ksa_oracle_unified_select.argtypes = ([c_int] * 5 + [_u16p, _u16p, _i32p, c_int,
                                                 c_int, c_int, _i32p, _i32p,
                                                 ctypes.c_void_p])
@@ -217,6 +219,24 @@ class Oracle:
                                       lse.ctypes.data, wsum.ctypes.data)
         del keep
         return out, lse, wsum
+
+    def attention_recall(self, q, K, seq_lens, idx, num_idx, tokens_per_idx: int = 1,
+                         shared: int = 0, scale: float = 0.0) -> np.ndarray:
+        """Share of each query head's dense softmax weight on the selected tokens -> fp64
+        [B,Hq].  shared: 0 lists per kv-head [B,Hkv,cap], 1 one list per row [B,cap],
+        2 one list per query head [B,Hq,cap]."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        K = np.ascontiguousarray(K, dtype=np.uint16)
+        B, Hq, D = q.shape
+        _, Hkv, T, _ = K.shape
+        idx = np.ascontiguousarray(idx, np.int32)
+        num_idx = np.ascontiguousarray(num_idx, np.int32)
+        rec = np.empty((B, Hq), np.float64)
+        self.lib.ksa_oracle_attention_recall(B, Hq, Hkv, D, T, q, K,
+                                             np.ascontiguousarray(seq_lens, np.int32), idx,
+                                             num_idx, idx.shape[-1], tokens_per_idx, int(shared),
+                                             float(scale), rec)
+        return rec
 
     # -- A6 -----------------------------------------------------------------
     def unified_select(self, q, K, seq_lens, per_head_topk: int, token_budget: int,

@@ -113,7 +113,8 @@ def test_select_blocks_exact_ties(ksa, oracle, nblk):
     exactly, and both sides must break ties toward the lower block.  Rows of
     up to 1024 blocks are ranked one warp per row (256 and 700 here); longer
     rows one CTA per row with 8, 16, 32 or 64 keys per thread (1100, 3000,
-    7000, and 16384 blocks, the largest row the API accepts)."""
+    7000, and 16384 blocks, the largest row the API accepts).  k runs up to
+    512, the largest budget of the sweep (8192 tokens in blocks of 16)."""
     rng = np.random.default_rng(210 + nblk)
     B, Hq, Hkv, D, bs = 2, 4, 2, 128, 16
     T = nblk * bs
@@ -122,7 +123,7 @@ def test_select_blocks_exact_ties(ksa, oracle, nblk):
     K = bf16_bits(np.clip(np.round(rng.standard_normal((B, Hkv, T, D)) * 0.5), -2, 2) * 0.25)
     qd, Kd, Ld = to_dev_bf16(q), to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
     S = ksa.ksa_build_block_summaries(Kd, Ld, bs)
-    for k in (1, 7, 50, 99, 100, 255):
+    for k in (1, 7, 50, 99, 100, 255, 256, 512):
         idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k)
         ref_idx, ref_cnt, scores = oracle.select_blocks(q, K, lens, bs, k, want_scores=True)
         assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
@@ -385,6 +386,112 @@ def test_decode_step_qwen3_8b_full_size(ksa, oracle):
     _plant(oracle, inp, rows, inp.shape.k_blocks)
     res = _decode_step(ksa, inp, inp.shape.k_blocks)
     _check_rows(oracle, inp, rows, *res, inp.shape.k_blocks)
+
+
+def _fused_step(ksa, inp, k, stale_last_block=True):
+    """What bench.py times: the fused selection call (last-block refresh + scoring + top-k)
+    then the attention call.  The summaries are prefilled from the cache as it was before
+    the newest token (seq_lens - 1; blocks never built hold NaN), so the call must refresh
+    the block the newest token landed in before it scores."""
+    sh = inp.shape
+    B, Hq, Hkv, D, T, bs = (sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, sh.capacity,
+                            sh.block_size)
+    S = torch.full((B, Hkv, -(-T // bs), D), float("nan"), dtype=torch.float32, device=DEV)
+    before = (inp.seq_lens - 1).clamp_min(1) if stale_last_block else inp.seq_lens
+    ksa.ksa_build_block_summaries(inp.K, before, bs, summaries=S)
+    st = status_tensor()
+    ws_sel = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
+                         dtype=torch.uint8, device=DEV)
+    ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
+                         dtype=torch.uint8, device=DEV)
+    idx, cnt = ksa.ksa_decode_select_blocks(inp.q, inp.K, S, inp.seq_lens, bs, k,
+                                            workspace=ws_sel, dev_status=st)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=DEV)
+    out, _ = ksa.ksa_sparse_decode_attn(inp.q, inp.K, inp.V, inp.seq_lens, idx, cnt,
+                                        tokens_per_idx=bs, lse=lse, workspace=ws_att,
+                                        dev_status=st)
+    assert st.item() == 0
+    return idx, cnt, out, lse
+
+
+@pytest.mark.parametrize("which", ["qwen3-0.6b", "qwen3-8b"])
+def test_fused_decode_step_full_size(ksa, oracle, which):
+    """The bench's own call sequence at the full Qwen3-0.6B (batch 64, 512 blocks, k 32) and
+    Qwen3-8B (batch 32, 1024-2048 blocks, k 128) shapes, planted score gap on the sampled
+    rows: indices bit-exact, outputs within 2e-3 of the oracle."""
+    if which == "qwen3-0.6b":
+        inp = synth.qwen3_0_6b_inputs(device=DEV)
+    else:
+        inp = synth.qwen3_8b_inputs(device=DEV, poison_tail=64.0)
+    rows = sample_rows(inp.shape.batch, 11, extra=3)
+    _plant(oracle, inp, rows, inp.shape.k_blocks)
+    res = _fused_step(ksa, inp, inp.shape.k_blocks)
+    _check_rows(oracle, inp, rows, *res, inp.shape.k_blocks)
+
+
+@pytest.mark.parametrize("context,budget", [(131072, 8192), (32768, 256), (4096, 8192)])
+def test_sweep_points_fused_step(ksa, oracle, context, budget):
+    """Sparse points of the throughput sweep (Hq 32, Hkv 8, D 128, bs 16) at their own
+    context and budget, two rows each, through the fused selection call and attention:
+    128K / 8192 tokens (k = 512 of 8192 blocks), 32K / 256 (k = 16), and 4K / 8192, where
+    k = 512 covers all 256 blocks so the step must equal dense attention."""
+    sh = synth.dataclasses.replace(synth.sweep_shape(context, budget), batch=2)
+    inp = synth.sweep_inputs(sh, seed=1005 + context + budget, device=DEV)
+    k = sh.k_blocks
+    rows = [0, 1]
+    _plant(oracle, inp, rows, k)
+    idx, cnt, out, lse = _fused_step(ksa, inp, k)
+    _check_rows(oracle, inp, rows, idx, cnt, out, lse, k)
+    nb = -(-context // sh.block_size)
+    if k >= nb:
+        assert torch.all(cnt == nb)
+        dense = torch.empty_like(out)
+        dense_lse = torch.empty_like(lse)
+        ksa.ksa_sparse_decode_attn(inp.q, inp.K, inp.V, inp.seq_lens, out=dense, lse=dense_lse)
+        assert_out_close(out.cpu().numpy(), dense.cpu().numpy(), what="k covers every block")
+        np.testing.assert_allclose(lse.cpu().numpy(), dense_lse.cpu().numpy(), rtol=0,
+                                   atol=LSE_TOL)
+
+
+def test_append_kv_writes_the_newest_slot(ksa, oracle):
+    """ksa_append_kv: K[b, g, L_b - 1] and V[b, g, L_b - 1] take the new rows bit for bit and
+    nothing else changes; a row whose seq_len is outside [1, T] is left alone and flagged.
+    The paged form writes the same rows into the pages the block table names."""
+    rng = np.random.default_rng(1600)
+    B, Hkv, T, D, bs = 4, 3, 96, 128, 16
+    K, V = rand_bits(rng, (B, Hkv, T, D)), rand_bits(rng, (B, Hkv, T, D))
+    kn, vn = rand_bits(rng, (B, Hkv, D)), rand_bits(rng, (B, Hkv, D))
+    lens = np.array([1, 50, 96, 97], np.int32)  # the last is out of range
+    Kd, Vd = to_dev_bf16(K), to_dev_bf16(V)
+    st = status_tensor()
+    ksa.ksa_append_kv(to_dev_bf16(kn), to_dev_bf16(vn), Kd, Vd, torch.from_numpy(lens).to(DEV),
+                      dev_status=st)
+    wantK, wantV = K.copy(), V.copy()
+    for b in range(3):
+        wantK[b, :, lens[b] - 1] = kn[b]
+        wantV[b, :, lens[b] - 1] = vn[b]
+    assert np.array_equal(host_bits(Kd), wantK) and np.array_equal(host_bits(Vd), wantV)
+    assert st.item() == ksa.FLAG_SEQ_LEN_CLAMPED
+    # paged: a shuffled pool with a spare page; row 3's slot names a page outside the pool
+    mb = T // bs
+    P = B * mb + 1
+    perm = rng.permutation(P)[:B * mb].astype(np.int32).reshape(B, mb)
+    perm[3, (30 - 1) // bs] = P + 5
+    plens = np.array([1, 50, 96, 30], np.int32)
+    pages_k = rand_bits(rng, (P, Hkv, bs, D))
+    pages_v = rand_bits(rng, (P, Hkv, bs, D))
+    Kp, Vp = to_dev_bf16(pages_k), to_dev_bf16(pages_v)
+    st.zero_()
+    ksa.ksa_append_kv_paged(to_dev_bf16(kn), to_dev_bf16(vn), Kp, Vp,
+                            torch.from_numpy(perm).to(DEV), torch.from_numpy(plens).to(DEV),
+                            dev_status=st)
+    wk, wv = pages_k.copy(), pages_v.copy()
+    for b in range(3):
+        t = plens[b] - 1
+        wk[perm[b, t // bs], :, t % bs] = kn[b]
+        wv[perm[b, t // bs], :, t % bs] = vn[b]
+    assert np.array_equal(host_bits(Kp), wk) and np.array_equal(host_bits(Vp), wv)
+    assert st.item() == ksa.FLAG_INDEX_SKIPPED
 
 
 def test_lessismore_full_size(ksa, oracle):
@@ -783,45 +890,80 @@ def test_aggregation_comparison_bounds(ksa, oracle):
     assert max(vals) - min(vals) <= tol, vals
 
 
-def test_attention_recall_matches_softmax_mass(ksa, oracle):
-    """recall = the dense softmax mass on the selected tokens (fp64 numpy softmax here);
-    the dense set recalls 1 and an empty selection 0."""
+# recall = exp(lse_sel - lse_all) from two attention launches; each lse is within 1e-4 of the
+# oracle's, so the recall is within (e^{2e-4} - 1) * recall <= 2.1e-4 of the oracle's recall
+RECALL_TOL = 2.5e-4
+
+
+@pytest.mark.parametrize("layout", ["blocks", "shared_tokens", "per_q_head"])
+def test_attention_recall_matches_oracle(ksa, oracle, layout):
+    """The GPU recall of a selection against the oracle's: the share of each head's dense
+    softmax weight on the selected tokens, element by element; the dense set recalls 1 and
+    an empty selection 0."""
     from block_top_sparse_ksa_b200.recall import attention_recall
     rng = np.random.default_rng(1500)
     B, Hq, Hkv, D, T, bs = 2, 8, 2, 64, 320, 16
-    G = Hq // Hkv
     lens = np.array([T, 123], np.int32)
     q, K, V = (rand_bits(rng, s) for s in [(B, Hq, D), (B, Hkv, T, D), (B, Hkv, T, D)])
     nb = -(-lens // bs)
-    k = 6
-    idx = np.full((B, Hkv, k), -1, np.int32)
-    cnt = np.zeros((B, Hkv), np.int32)
-    for b in range(B):
-        for g in range(Hkv):
-            pick = np.sort(rng.choice(int(nb[b]), size=k, replace=False))
-            idx[b, g] = pick
-            cnt[b, g] = k
+    if layout == "blocks":
+        tpi, shared, k = bs, ksa.IDX_PER_KV_HEAD, 6
+        idx = np.stack([np.stack([np.sort(rng.choice(int(nb[b]), size=k, replace=False))
+                                  for _ in range(Hkv)]) for b in range(B)]).astype(np.int32)
+        cnt = np.full((B, Hkv), k, np.int32)
+    elif layout == "shared_tokens":
+        tpi, shared, k = 1, ksa.IDX_SHARED, 40
+        idx = np.stack([np.sort(rng.choice(int(lens[b]), size=k, replace=False))
+                        for b in range(B)]).astype(np.int32)
+        cnt = np.array([k, k - 7], np.int32)
+    else:
+        tpi, shared, k = 1, ksa.IDX_PER_Q_HEAD, 25
+        idx = np.stack([np.stack([np.sort(rng.choice(int(lens[b]), size=k, replace=False))
+                                  for _ in range(Hq)]) for b in range(B)]).astype(np.int32)
+        cnt = np.full((B, Hq), k, np.int32)
     qd, Kd, Vd, Ld = to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(lens).to(DEV)
     rec = attention_recall(qd, Kd, Vd, Ld, torch.from_numpy(idx).to(DEV),
-                           torch.from_numpy(cnt).to(DEV), tokens_per_idx=bs)
-    qv, Kv = bf16_value(q), bf16_value(K)
-    for b in range(B):
-        L = int(lens[b])
-        for h in range(Hq):
-            g = h // G
-            z = Kv[b, g, :L] @ qv[b, h] / math.sqrt(D)
-            w = np.exp(z - z.max())
-            w /= w.sum()
-            sel = np.zeros(L, bool)
-            for j in idx[b, g, :cnt[b, g]]:
-                sel[j * bs:min((j + 1) * bs, L)] = True
-            assert abs(rec[b, h] - w[sel].sum()) <= 3e-4 * max(1.0, w[sel].sum())
+                           torch.from_numpy(cnt).to(DEV), tokens_per_idx=tpi, idx_shared=shared)
+    ref = oracle.attention_recall(q, K, lens, idx, cnt, tpi, shared)
+    assert np.all(ref > 0.0) and np.all(ref < 1.0)
+    np.testing.assert_allclose(rec, ref, rtol=0, atol=RECALL_TOL)
     all_idx = torch.arange(int(nb.max()), dtype=torch.int32, device=DEV).repeat(B, Hkv, 1)
     all_cnt = torch.from_numpy(np.repeat(nb[:, None], Hkv, 1).astype(np.int32)).to(DEV)
     assert np.allclose(attention_recall(qd, Kd, Vd, Ld, all_idx, all_cnt, tokens_per_idx=bs),
-                       1.0, atol=1e-5)
+                       1.0, atol=RECALL_TOL)
     none = torch.zeros((B, Hkv), dtype=torch.int32, device=DEV)
     assert np.all(attention_recall(qd, Kd, Vd, Ld, all_idx, none, tokens_per_idx=bs) == 0.0)
+
+
+def test_recency_sweep_matches_oracle(ksa, oracle):
+    """The LessIsMore recency-share sweep (0 to 100% of the budget given to the recent
+    window) on a small seeded shape: for every share the GPU's unified set equals the
+    oracle's, and the mean recall of that set in the selection layer and in each sparse
+    layer equals the oracle's recall of the oracle's set."""
+    from block_top_sparse_ksa_b200 import recall
+    shape = synth.dataclasses.replace(synth.LESSISMORE, batch=2, num_q_heads=8, num_kv_heads=2,
+                                      capacity=1500, seq_len=1500, per_head_topk=300,
+                                      token_budget=300, recent_tokens=75)
+    inp = synth.lessismore_inputs(seed=21, device=DEV, shape=shape)
+    ratios = [0.0, 0.25, 0.5, 0.75, 1.0]
+    rows = recall.recency_sweep(inp, ratios)
+    q_sel, K_sel = host_bits(inp.q_sel), host_bits(inp.K_sel)
+    lens = inp.seq_lens.cpu().numpy()
+    layers = [tuple(host_bits(t) for t in layer) for layer in inp.layers]
+    for ratio, row in zip(ratios, rows):
+        R = int(round(ratio * shape.token_budget))
+        assert row["recent_tokens"] == R
+        tok, cnt = oracle.unified_select(q_sel, K_sel, lens, shape.per_head_topk,
+                                         shape.token_budget, R)
+        g_tok, g_cnt = ksa.ksa_unified_select(inp.q_sel, inp.K_sel, inp.seq_lens,
+                                              shape.per_head_topk, shape.token_budget, R)
+        assert np.array_equal(g_tok.cpu().numpy(), tok) and np.array_equal(g_cnt.cpu().numpy(),
+                                                                           cnt)
+        want = oracle.attention_recall(q_sel, K_sel, lens, tok, cnt, 1, 1).mean()
+        assert abs(row["selection_layer"] - want) <= RECALL_TOL, (ratio, row, want)
+        for got, (q, K, _) in zip(row["sparse_layers"], layers):
+            want = oracle.attention_recall(q, K, lens, tok, cnt, 1, 1).mean()
+            assert abs(got - want) <= RECALL_TOL, (ratio, got, want)
 
 
 def test_select_window_matches_oracle(ksa, oracle):

@@ -40,10 +40,16 @@ MUTANTS = [
      "const int n_cand = L;", 0, [pins.test_unified_window_excluded_from_voted_part]),
     ("unified ties go to the higher token", "return (x->t > y->t) - (x->t < y->t);",
      "return (x->t < y->t) - (x->t > y->t);", 0, [pins.test_unified_bruteforce_small]),
+    ("wrong kv-head for a query head in recall", "const int g = h / G;",
+     "const int g = h % Hkv;", 1, [pins.test_recall_is_the_lse_difference]),
+    ("recall without the max subtraction", "w[t] = exp(w[t] - zmax);", "w[t] = exp(w[t]);", 0,
+     [pins.test_recall_with_huge_logits]),
+    ("recall weights not divided by the dense sum", "if (sel[t]) mass += w[t] / denom;",
+     "if (sel[t]) mass += w[t];\n      denom = mass;", 0, [pins.test_golden_recall]),
     ("wrong kv-head for a query head in per-head top-k", "const int g = h / G;",
-     "const int g = h % Hkv;", 1, [pins.test_tokens_per_head_rank_counting]),
+     "const int g = h % Hkv;", 2, [pins.test_tokens_per_head_rank_counting]),
     ("wrong kv-head for a query head in voting", "const int g = h / G;",
-     "const int g = h % Hkv;", 2, [pins.test_unified_bruteforce_small]),
+     "const int g = h % Hkv;", 3, [pins.test_unified_bruteforce_small]),
     ("recency window shifted by one", "for (int t = L - R; t < L; ++t) pick[n++] = t;",
      "for (int t = L - R - 1; t < L - 1; ++t) pick[n++] = t;", 0,
      [pins.test_unified_closed_forms]),

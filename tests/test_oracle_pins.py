@@ -734,3 +734,87 @@ def test_one_head_rejects_heads_out_of_range(oracle):
     K = np.zeros((1, 2, 16, 64), np.uint16)
     with pytest.raises(ValueError):
         oracle.select_tokens_one_head(q, K, np.array([16], np.int32), np.array([4], np.int32), 2)
+
+
+# --------------------------------------------------------------------------
+# attention recall (LessIsMore press summary, sections 3 and 4)
+
+
+def test_golden_recall(oracle):
+    rows, cases = _read_golden("recall_hand.txt")
+    sh = _shape(rows)
+    B, Hq, Hkv, D, T = sh["B"], sh["Hq"], sh["Hkv"], sh["D"], sh["T"]
+    L = _nums(rows["seq_lens"], int).astype(np.int32)
+    q = bf16_bits(_nums(rows["q"]).reshape(B, Hq, D))
+    K = bf16_bits(_nums(rows["K"]).reshape(B, Hkv, T, D))
+    for case in cases:
+        sel, _, want = case.partition(":")
+        idx = _nums(sel, int).astype(np.int32).reshape(1, -1)
+        cnt = np.array([idx.shape[-1]], np.int32)
+        r = oracle.attention_recall(q, K, L, idx, cnt, 1, 1, float(rows["scale"]))
+        np.testing.assert_allclose(r.reshape(-1), _nums(want), rtol=0, atol=1e-15)
+
+
+def test_recall_of_every_token_is_one_and_of_none_is_zero(oracle):
+    rng = np.random.default_rng(71)
+    B, Hq, Hkv, D, T, bs = 2, 6, 3, 32, 90, 16
+    q, K = rnd_bits(rng, (B, Hq, D), 2.0), rnd_bits(rng, (B, Hkv, T, D))
+    L = np.array([90, 37], np.int32)
+    nb = -(-T // bs)
+    idx = np.tile(np.arange(nb, dtype=np.int32), (B, Hkv, 1))
+    cnt = np.tile(-(-L // bs)[:, None], (1, Hkv)).astype(np.int32)
+    np.testing.assert_allclose(oracle.attention_recall(q, K, L, idx, cnt, bs), 1.0, atol=1e-13)
+    none = np.zeros((B, Hkv), np.int32)
+    assert np.all(oracle.attention_recall(q, K, L, idx, none, bs) == 0.0)
+    # slots past L_b (block 2 holds tokens 32..47 of the 37-token row) count once, if at all
+    np.testing.assert_allclose(oracle.attention_recall(q, K, L, idx, cnt * 0 + nb, bs), 1.0,
+                               atol=1e-13)
+
+
+def test_recall_is_the_lse_difference(oracle):
+    """Mass on a set = exp(lse(set) - lse(all)): the log-sum-exps come from the attention
+    routine (itself pinned against torch SDPA), a separate computation."""
+    rng = np.random.default_rng(72)
+    B, Hq, Hkv, D, T = 2, 8, 2, 64, 200
+    q, K, V = (rnd_bits(rng, s) for s in [(B, Hq, D), (B, Hkv, T, D), (B, Hkv, T, D)])
+    L = np.array([200, 131], np.int32)
+    k = 17
+    idx = np.full((B, Hkv, k), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            m = 9 + 4 * g + b
+            idx[b, g, :m] = np.sort(rng.choice(int(L[b]), size=m, replace=False))
+            cnt[b, g] = m
+    r = oracle.attention_recall(q, K, L, idx, cnt, 1, 0)
+    _, lse_all, _ = oracle.attention(q, K, V, L)
+    _, lse_sel, _ = oracle.attention(q, K, V, L, idx, cnt, 1)
+    np.testing.assert_allclose(r, np.exp(lse_sel - lse_all), rtol=1e-12, atol=0)
+    # the same selections as one list per query head (each head of a group repeats its
+    # kv-head's list), and as one shared list when every kv-head has the same list
+    G = Hq // Hkv
+    per_q = np.repeat(idx, G, axis=1)
+    per_q_cnt = np.repeat(cnt, G, axis=1)
+    np.testing.assert_allclose(oracle.attention_recall(q, K, L, per_q, per_q_cnt, 1, 2), r,
+                               rtol=0, atol=0)
+    shared = oracle.attention_recall(q, K, L, idx[:, 0], cnt[:, 0], 1, 1)
+    same = oracle.attention_recall(q, K, L, np.repeat(idx[:, :1], Hkv, 1),
+                                   np.repeat(cnt[:, :1], Hkv, 1), 1, 0)
+    np.testing.assert_allclose(shared, same, rtol=0, atol=0)
+
+
+def test_recall_with_huge_logits(oracle):
+    """Logits near 1000: the dense weights must still be formed stably (e^1024 overflows
+    fp64).  Weights are proportional to (1, e^-64, e^-128)."""
+    q = bf16_bits(np.array([[[64.0, 0.0]]]))
+    K = bf16_bits(np.array([[[[16.0, 0.0], [15.0, 0.0], [14.0, 0.0]]]]))
+    L = np.array([3], np.int32)
+    one = np.array([[[0]]], np.int32), np.array([[1]], np.int32)
+    mid = np.array([[[1]]], np.int32), np.array([[1]], np.int32)
+    r0 = oracle.attention_recall(q, K, L, *one, 1, 0, 1.0)
+    r1 = oracle.attention_recall(q, K, L, *mid, 1, 0, 1.0)
+    assert np.isfinite(r0).all() and np.isfinite(r1).all()
+    assert r0[0, 0] == pytest.approx(1.0, abs=1e-15)
+    assert r1[0, 0] == pytest.approx(math.exp(-64) / (1 + math.exp(-64) + math.exp(-128)),
+                                     rel=1e-12)
+
