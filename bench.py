@@ -378,14 +378,21 @@ class BlockWorkload:
                                   dtype=torch.uint8, device=dev)
         self.ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
                                   dtype=torch.uint8, device=dev)
+        self.ws_step = torch.zeros((ksa.ksa_decode_step_workspace(B, Hq, Hkv, D, T, bs, k),),
+                                   dtype=torch.uint8, device=dev)
         self.idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
         self.cnt = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
         self.out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
         self.stream = torch.cuda.current_stream()
         nb_max = -(-T // bs)
-        # selection: a scoring launch (when some row can hold more than k blocks) and a
-        # ranking launch; then the attention launch
-        self.launches_per_step = 1 if self.kind == "dense" else (2 if nb_max > k else 1) + 1
+        # the two calls: a scoring launch (when some row can hold more than k blocks), a
+        # ranking launch, the attention launch; ksa_decode_step is one launch for rows of up
+        # to 2048 blocks and those three beyond
+        self.two_call_launches = (2 if nb_max > k else 1) + 1
+        if self.kind == "dense":
+            self.launches_per_step = 1
+        else:
+            self.launches_per_step = 1 if nb_max <= 2048 else self.two_call_launches
 
     def select(self, i, q=None):
         sh = self.shape
@@ -406,18 +413,29 @@ class BlockWorkload:
                                             tokens_per_idx=self.shape.block_size, out=self.out,
                                             workspace=self.ws_att, stream=self.stream)
 
-    def step(self, i):
-        if self.kind != "dense":
-            self.select(i)
-        self.attend(i)
+    def decode_step(self, i, q=None):
+        sh = self.shape
+        self.ksa.ksa_decode_step(self.qs[i % self.nq] if q is None else q, self.inp.K,
+                                 self.inp.V, self.S, self.inp.seq_lens, sh.block_size,
+                                 sh.k_blocks, block_idx=self.idx, num_sel=self.cnt, out=self.out,
+                                 workspace=self.ws_step, stream=self.stream)
 
-    def parts(self):
-        return [self.attend] if self.kind == "dense" else [self.select, self.attend]
+    def step(self, i):
+        """The timed step: ksa_decode_step (dense attention for the k = all workloads)."""
+        if self.kind == "dense":
+            self.attend(i)
+        else:
+            self.decode_step(i)
+
+    def step_two_calls(self, i):
+        self.select(i)
+        self.attend(i)
 
 
 def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
                   clocks: "ClockSampler | None" = None):
-    """Warm-up, the timed steps and the per-kernel pass of one block workload."""
+    """Warm-up, the timed steps and the per-kernel pass of one block workload; then the
+    same steps through the two calls (selection, attention) for comparison."""
     sh, kind = wl.shape, wl.kind
     n_warm = warm_up(wl.step, args.warmup, args.min_warmup_s)
     if clocks is not None:
@@ -426,31 +444,26 @@ def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
     if clocks is not None:
         clocks.mark()
     value, ms_step = weak_scaling(dist, sh.batch, ms, args.steps)
-    times = kernel_pass(wl.parts(), max(20, min(args.steps, 200)), wl.stream)
-    t_att = times[-1]
-    t_sel = times[0] if kind != "dense" else 0.0
+    n_pass = max(20, min(args.steps, 200))
+    (t_step,) = kernel_pass([wl.step], n_pass, wl.stream)
     lens = wl.inp.seq_lens.cpu().tolist()
     total_b, attn_b, summ_b = algorithmic_bytes(sh, lens, kind, wl.S.element_size())
     per_step_s = ms_step / 1e3
-    attn_gbs = attn_b / (t_att * 1e-3) / 1e9
-    return {
+    name = "sparse_decode_attn" if kind == "dense" else "decode_step"
+    # the dominant (here: only) kernel of the step, its algorithmic bytes per launch
+    roof_b = attn_b if kind == "dense" else total_b
+    roof_gbs = roof_b / (t_step * 1e-3) / 1e9
+    res = {
         "value": value, "ms_per_step": ms_step, "warmup_steps_run": n_warm,
         "host_enqueue_us_per_step": host_us,
-        "kernels_ms": ({"sparse_decode_attn": t_att} if kind == "dense" else
-                       {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att}),
-        "kernels_note": "mean of a second pass of the same steps with an event around each call "
-                        "(the selection call is its scoring and ranking launches)",
-        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": attn_gbs / peak,
-                     "traffic": stored_traffic("sparse_decode_attn", args.workload, sh.batch),
-                     "kernel": "sparse_decode_attn", "peak_source": peak_kind,
-                     "bytes_per_launch": attn_b},
+        "kernels_ms": {name: t_step},
+        "kernels_note": "mean of a second pass of the same steps with an event around each call",
+        "roofline": {"bound": "hbm", "achieved": roof_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": roof_gbs / peak,
+                     "traffic": stored_traffic(name, args.workload, sh.batch),
+                     "kernel": name, "peak_source": peak_kind, "bytes_per_launch": roof_b},
         "step_hbm": {"bytes_per_step": total_b, "gbs": total_b / per_step_s / 1e9,
-                     "frac": total_b / per_step_s / 1e9 / peak,
-                     "kernel_sum_ms": t_sel + t_att},
-        "select_hbm": (None if kind == "dense" else
-                       {"bytes_per_launch": summ_b,
-                        "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None}),
+                     "frac": total_b / per_step_s / 1e9 / peak, "kernel_sum_ms": t_step},
         "gpu_launches": wl.launches_per_step * args.steps,
         "config": {"workload": sh.name, "batch_per_gpu": sh.batch, "num_q_heads": sh.num_q_heads,
                    "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
@@ -463,9 +476,26 @@ def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
                          "rotating query sets" % (2 * wl.inp.K.numel() * 2 / 1e9, total_b / 1e6,
                                                   wl.nq),
                    "step": ("dense attention" if kind == "dense" else
-                            "decode_select_blocks (last-block summary refresh + scoring + "
-                            "top-k) + sparse_decode_attn")},
+                            "ksa_decode_step: last-block summary refresh + scoring + top-k + "
+                            "sparse attention (%d launch%s)" % (
+                                wl.launches_per_step,
+                                "" if wl.launches_per_step == 1 else "es"))},
     }
+    if kind != "dense":
+        ms2, _ = timed_steps(wl.step_two_calls, args.steps, dist, wl.stream)
+        _, ms2_step = weak_scaling(dist, sh.batch, ms2, args.steps)
+        t_sel, t_att = kernel_pass([wl.select, wl.attend], n_pass, wl.stream)
+        attn_gbs = attn_b / (t_att * 1e-3) / 1e9
+        res["two_calls"] = {
+            "what": "ksa_decode_select_blocks + ksa_sparse_decode_attn (%d launches)"
+                    % wl.two_call_launches,
+            "ms_per_step": ms2_step, "value": sh.batch / (ms2_step * 1e-3),
+            "kernels_ms": {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att},
+            "attention_roofline": {"bytes_per_launch": attn_b, "achieved": attn_gbs,
+                                   "frac": attn_gbs / peak},
+            "select_hbm": {"bytes_per_launch": summ_b,
+                           "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None}}
+    return res
 
 
 def run_block(args, dist, dev, kind):
@@ -502,7 +532,8 @@ def run_extra(args, dist, dev):
                          "ms_per_step": r["ms_per_step"],
                          "host_enqueue_us_per_step": r["host_enqueue_us_per_step"],
                          "step_hbm": r["step_hbm"], "roofline_frac": r["roofline"]["frac"],
-                         "kernels_ms": r["kernels_ms"], "gpu_launches": r["gpu_launches"]}
+                         "kernels_ms": r["kernels_ms"], "gpu_launches": r["gpu_launches"],
+                         "two_calls": r.get("two_calls")}
             del wl
         except torch.cuda.OutOfMemoryError as e:  # never lose the main line for a side figure
             out[name] = {"error": str(e)[:200]}
@@ -561,9 +592,10 @@ def run_block_e2e(args, dist, wl: BlockWorkload):
         d_q.copy_(h_q[i % nq], non_blocking=True)
         d_kv.copy_(h_kv[i % nq], non_blocking=True)
         ksa.ksa_append_kv(d_kv[0], d_kv[1], wl.inp.K, wl.inp.V, lens, stream=stream)
-        if wl.kind != "dense":
-            wl.select(i, d_q)
-        wl.attend(i, d_q)
+        if wl.kind == "dense":
+            wl.attend(i, d_q)
+        else:
+            wl.decode_step(i, d_q)
         h_out.copy_(wl.out, non_blocking=True)
 
     warm_up(step, args.warmup, 0.0)
@@ -576,7 +608,7 @@ def run_block_e2e(args, dist, wl: BlockWorkload):
             "host_enqueue_us_per_step": host_us,
             "gpu_launches": (wl.launches_per_step + 1) * args.steps,
             "note": "per step: q and the new token's K/V rows host->device (pinned), "
-                    "ksa_append_kv, selection, attention, out device->host"}
+                    "ksa_append_kv, ksa_decode_step, out device->host"}
 
 
 def run_unified(args, dist, dev):
@@ -804,11 +836,15 @@ def main():
                 "config": dict(res["config"], parallelism=f"dp{dist.world} (batch-sharded "
                                "replicas, no data-path collective)"),
                 "roofline": res["roofline"], "kernels_ms": res["kernels_ms"],
-                "step_hbm": res["step_hbm"], "select_hbm": res.get("select_hbm"),
+                "step_hbm": res["step_hbm"],
                 "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
                 "warmup_steps_run": res["warmup_steps_run"],
                 "host_enqueue_us_per_step": res["host_enqueue_us_per_step"],
                 "kernels_note": res["kernels_note"]}
+        if "two_calls" in res:
+            line["two_calls"] = res["two_calls"]
+        if "select_hbm" in res:
+            line["select_hbm"] = res["select_hbm"]
         if "e2e" in res:
             line["e2e"] = res["e2e"]
         if "prefill" in res:

@@ -31,7 +31,8 @@ __all__ = [
     "ksa_sparse_decode_attn_paged", "Pages", "ksa_select_window", "ksa_select_tokens_per_head",
     "ksa_select_tokens_per_head_workspace", "ksa_select_tokens_one_head",
     "ksa_select_tokens_one_head_workspace", "ksa_get_device_status", "IDX_PER_KV_HEAD",
-    "IDX_SHARED", "IDX_PER_Q_HEAD", "ksa_append_kv", "ksa_append_kv_paged",
+    "IDX_SHARED", "IDX_PER_Q_HEAD", "ksa_append_kv", "ksa_append_kv_paged", "ksa_decode_step",
+    "ksa_decode_step_workspace",
     "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
@@ -86,6 +87,9 @@ _SIGS = {
     "ksa_sparse_decode_attn_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp,
                                             ctypes.POINTER(Pages), _vp, _vp, _vp, _i32, _i32,
                                             _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "ksa_decode_step_workspace": (_sz, [ctypes.POINTER(Shape), _i32]),
+    "ksa_decode_step": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp,
+                               _vp, _f32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "ksa_append_kv": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ksa_append_kv_paged": (_i32, [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp,
                                    ctypes.POINTER(Pages), _vp, _vp, _vp]),
@@ -294,6 +298,53 @@ def ksa_decode_select_blocks(q: torch.Tensor, K: torch.Tensor, summaries: torch.
 
 
 ksa_decode_select_blocks_ex = ksa_decode_select_blocks
+
+
+def ksa_decode_step_workspace(B: int, Hq: int, Hkv: int, D: int, T: int, block_size: int,
+                              k_blocks: int) -> int:
+    sh = _shape(B, Hq, Hkv, D, T, block_size)
+    return int(lib().ksa_decode_step_workspace(ctypes.byref(sh), int(k_blocks)))
+
+
+def ksa_decode_step(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, summaries: torch.Tensor,
+                    seq_lens: torch.Tensor, block_size: int, k_blocks: int,
+                    block_idx: Optional[torch.Tensor] = None,
+                    num_sel: Optional[torch.Tensor] = None, scale: float = 0.0,
+                    out_dtype: int = OUT_F32, out: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None,
+                    dev_status: Optional[torch.Tensor] = None, stream=None):
+    """One decode step in one call: last-block refresh, scoring, top-k and attention over the
+    kept blocks -> (block_idx [B,Hkv,k], num_sel [B,Hkv], out [B,Hq,D], lse or None)."""
+    _dev(q, "q", torch.bfloat16)
+    _dev(K, "K", torch.bfloat16)
+    _dev(V, "V", torch.bfloat16)
+    _dev(summaries, "summaries", summaries.dtype)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    B, Hq, D = q.shape
+    _, Hkv, T, _ = K.shape
+    if block_idx is None:
+        block_idx = torch.empty((B, Hkv, k_blocks), dtype=torch.int32, device=q.device)
+    if num_sel is None:
+        num_sel = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    odt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=odt, device=q.device)
+    _dev(out, "out", odt)
+    if lse is not None:
+        _dev(lse, "lse", torch.float32)
+    sh = _shape(B, Hq, Hkv, D, T, block_size)
+    if workspace is None:  # zero-filled once (see include/ksa.h)
+        need = lib().ksa_decode_step_workspace(ctypes.byref(sh), int(k_blocks))
+        workspace = torch.zeros((max(int(need), 1),), dtype=torch.uint8, device=q.device)
+    elif not workspace.is_cuda or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    _check(lib().ksa_decode_step(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(V), _ptr(summaries), _summary_dtype(summaries),
+        _ptr(seq_lens), int(k_blocks), _ptr(block_idx), _ptr(num_sel), float(scale),
+        int(out_dtype), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+    return block_idx, num_sel, out, lse
 
 
 def ksa_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,

@@ -300,12 +300,11 @@ size_t ksa_select_blocks_workspace(const ksa_shape *shape, int32_t k_blocks) {
 
 namespace {
 
-// Shared by the selection entry points; K non-NULL fuses the last-block refresh.
-ksa_status select_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
-                         const ksa_pages *pages, void *summaries, int32_t summary_dtype,
-                         const int32_t *seq_lens,
-                         int32_t k_blocks, int32_t *block_idx, int32_t *num_sel, void *ws,
-                         size_t ws_bytes, uint32_t *dev_status, void *stream, const char *what) {
+// Validates a selection call's arguments (not its workspace) and fills *a.
+ksa_status select_args(const ksa_shape *shape, const uint16_t *q, const ksa_pages *pages,
+                       void *summaries, int32_t summary_dtype, const int32_t *seq_lens,
+                       int32_t k_blocks, int32_t *block_idx, int32_t *num_sel,
+                       uint32_t *dev_status, ksa::SelectArgs *a) {
   ksa_status st = check_shape(shape, true);
   if (st != KSA_OK) return st;
   if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
@@ -319,27 +318,39 @@ ksa_status select_common(const ksa_shape *shape, const uint16_t *q, const uint16
     return fail(KSA_ERR_UNSUPPORTED, "ceil(capacity/block_size) = %d exceeds 16384", nb_max);
   if (!aligned(summaries, 16) || !aligned(q, 4))
     return fail(KSA_ERR_INVALID_ARG, "summaries must be 16-byte aligned");
+  if (pages != nullptr && (st = check_pages(shape, pages, &a->kv)) != KSA_OK) return st;
+  a->q = q;
+  a->S = summaries;  // written only when K is given (the fused refresh)
+  a->sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
+  a->seq_lens = seq_lens;
+  a->block_idx = block_idx;
+  a->num_sel = num_sel;
+  a->status = dev_status;
+  a->B = shape->batch;
+  a->Hq = shape->num_q_heads;
+  a->Hkv = shape->num_kv_heads;
+  a->D = shape->head_dim;
+  a->T = shape->capacity;
+  a->bs = shape->block_size;
+  a->k = k_blocks;
+  return KSA_OK;
+}
+
+// Shared by the selection entry points; K non-NULL fuses the last-block refresh.
+ksa_status select_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                         const ksa_pages *pages, void *summaries, int32_t summary_dtype,
+                         const int32_t *seq_lens,
+                         int32_t k_blocks, int32_t *block_idx, int32_t *num_sel, void *ws,
+                         size_t ws_bytes, uint32_t *dev_status, void *stream, const char *what) {
+  ksa::SelectArgs a;
+  ksa_status st = select_args(shape, q, pages, summaries, summary_dtype, seq_lens, k_blocks,
+                              block_idx, num_sel, dev_status, &a);
+  if (st != KSA_OK) return st;
   const size_t need = ksa::select_workspace_bytes(shape->batch, shape->num_kv_heads,
                                                   shape->capacity, shape->block_size);
   if (ws == nullptr || ws_bytes < need)
     return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  ksa::SelectArgs a;
-  if (pages != nullptr && (st = check_pages(shape, pages, &a.kv)) != KSA_OK) return st;
-  a.q = q;
-  a.S = summaries;  // written only when K is given (the fused refresh)
-  a.sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
-  a.seq_lens = seq_lens;
-  a.block_idx = block_idx;
-  a.num_sel = num_sel;
-  a.status = dev_status;
-  a.B = shape->batch;
-  a.Hq = shape->num_q_heads;
-  a.Hkv = shape->num_kv_heads;
-  a.D = shape->head_dim;
-  a.T = shape->capacity;
-  a.bs = shape->block_size;
-  a.k = k_blocks;
   return cuda_status(
       ksa::launch_select_blocks(a, K, ws, device_sm_count(), static_cast<cudaStream_t>(stream)),
       what);
@@ -441,12 +452,12 @@ size_t ksa_sparse_decode_attn_workspace(const ksa_shape *shape, int32_t idx_capa
 
 namespace {
 
-ksa_status attn_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
-                       const uint16_t *V, const ksa_pages *pages, const int32_t *seq_lens,
-                       const int32_t *idx, const int32_t *num_idx, int32_t idx_capacity,
-                       int32_t tokens_per_idx, int32_t idx_shared, float scale, int32_t out_dtype,
-                       void *out, float *lse, void *ws, size_t ws_bytes, uint32_t *dev_status,
-                       void *stream) {
+// Validates an attention call's arguments (not its workspace) and fills *a.
+ksa_status attn_args(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                     const uint16_t *V, const ksa_pages *pages, const int32_t *seq_lens,
+                     const int32_t *idx, const int32_t *num_idx, int32_t idx_capacity,
+                     int32_t tokens_per_idx, int32_t idx_shared, float scale, int32_t out_dtype,
+                     void *out, float *lse, uint32_t *dev_status, ksa::AttnArgs *a) {
   ksa_status st = check_shape(shape, pages != nullptr);
   if (st != KSA_OK) return st;
   if (q == nullptr || K == nullptr || V == nullptr || seq_lens == nullptr || out == nullptr)
@@ -474,34 +485,47 @@ ksa_status attn_common(const ksa_shape *shape, const uint16_t *q, const uint16_t
   if (!aligned(K, 16) || !aligned(V, 16) || !aligned(q, 4) ||
       !aligned(out, out_dtype == KSA_OUT_F32 ? 4 : 2) || (lse && !aligned(lse, 4)))
     return fail(KSA_ERR_INVALID_ARG, "K and V must be 16-byte aligned, q and out element-aligned");
+  if (pages != nullptr && (st = check_pages(shape, pages, &a->kv)) != KSA_OK) return st;
+  a->q = q;
+  a->K = K;
+  a->V = V;
+  a->seq_lens = seq_lens;
+  a->idx = idx;
+  a->num_idx = num_idx;
+  a->out_f32 = out_dtype == KSA_OUT_F32 ? static_cast<float *>(out) : nullptr;
+  a->out_bf16 = out_dtype == KSA_OUT_BF16 ? static_cast<uint16_t *>(out) : nullptr;
+  a->lse = lse;
+  a->status = dev_status;
+  a->B = shape->batch;
+  a->Hq = shape->num_q_heads;
+  a->Hkv = shape->num_kv_heads;
+  a->D = shape->head_dim;
+  a->T = shape->capacity;
+  a->cap = idx ? idx_capacity : 0;
+  a->tpi = idx ? tokens_per_idx : 1;
+  a->shared = idx ? idx_shared : 0;
+  a->scale = scale == 0.f ? static_cast<float>(1.0 / sqrt(static_cast<double>(shape->head_dim)))
+                          : scale;
+  return KSA_OK;
+}
+
+ksa_status attn_common(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                       const uint16_t *V, const ksa_pages *pages, const int32_t *seq_lens,
+                       const int32_t *idx, const int32_t *num_idx, int32_t idx_capacity,
+                       int32_t tokens_per_idx, int32_t idx_shared, float scale, int32_t out_dtype,
+                       void *out, float *lse, void *ws, size_t ws_bytes, uint32_t *dev_status,
+                       void *stream) {
+  ksa::AttnArgs a;
+  const ksa_status st = attn_args(shape, q, K, V, pages, seq_lens, idx, num_idx, idx_capacity,
+                                  tokens_per_idx, idx_shared, scale, out_dtype, out, lse,
+                                  dev_status, &a);
+  if (st != KSA_OK) return st;
   const int sms = device_sm_count();
   const size_t need = ksa::attn_workspace_bytes(shape->batch, shape->num_q_heads,
                                                 shape->num_kv_heads, shape->head_dim, sms);
   if (ws == nullptr || ws_bytes < need)
     return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  ksa::AttnArgs a;
-  if (pages != nullptr && (st = check_pages(shape, pages, &a.kv)) != KSA_OK) return st;
-  a.q = q;
-  a.K = K;
-  a.V = V;
-  a.seq_lens = seq_lens;
-  a.idx = idx;
-  a.num_idx = num_idx;
-  a.out_f32 = out_dtype == KSA_OUT_F32 ? static_cast<float *>(out) : nullptr;
-  a.out_bf16 = out_dtype == KSA_OUT_BF16 ? static_cast<uint16_t *>(out) : nullptr;
-  a.lse = lse;
-  a.status = dev_status;
-  a.B = shape->batch;
-  a.Hq = shape->num_q_heads;
-  a.Hkv = shape->num_kv_heads;
-  a.D = shape->head_dim;
-  a.T = shape->capacity;
-  a.cap = idx ? idx_capacity : 0;
-  a.tpi = idx ? tokens_per_idx : 1;
-  a.shared = idx ? idx_shared : 0;
-  a.scale = scale == 0.f ? static_cast<float>(1.0 / sqrt(static_cast<double>(shape->head_dim)))
-                         : scale;
   return cuda_status(
       ksa::launch_sparse_decode_attn(a, ws, sms, static_cast<cudaStream_t>(stream)),
       "ksa_sparse_decode_attn launch");
@@ -532,6 +556,42 @@ ksa_status ksa_sparse_decode_attn_paged(const ksa_shape *shape, const uint16_t *
   return attn_common(shape, q, K_pages, V_pages, pages, seq_lens, idx, num_idx, idx_capacity,
                      tokens_per_idx, idx_shared, scale, out_dtype, out, lse, ws, ws_bytes,
                      dev_status, stream);
+}
+
+size_t ksa_decode_step_workspace(const ksa_shape *shape, int32_t k_blocks) {
+  (void)k_blocks;
+  if (check_shape(shape, true) != KSA_OK) return 0;
+  return ksa::decode_step_workspace_bytes(shape->batch, shape->num_q_heads, shape->num_kv_heads,
+                                          shape->head_dim, shape->capacity, shape->block_size,
+                                          device_sm_count());
+}
+
+ksa_status ksa_decode_step(const ksa_shape *shape, const uint16_t *q, const uint16_t *K,
+                           const uint16_t *V, void *summaries, int32_t summary_dtype,
+                           const int32_t *seq_lens, int32_t k_blocks, int32_t *block_idx,
+                           int32_t *num_sel, float scale, int32_t out_dtype, void *out,
+                           float *lse, void *ws, size_t ws_bytes, uint32_t *dev_status,
+                           void *stream) {
+  if (K == nullptr) return fail(KSA_ERR_INVALID_ARG, "K must be non-NULL");
+  ksa::SelectArgs sa;
+  ksa_status st = select_args(shape, q, nullptr, summaries, summary_dtype, seq_lens, k_blocks,
+                              block_idx, num_sel, dev_status, &sa);
+  if (st != KSA_OK) return st;
+  ksa::AttnArgs aa;
+  st = attn_args(shape, q, K, V, nullptr, seq_lens, block_idx, num_sel, k_blocks,
+                 shape->block_size, KSA_IDX_PER_KV_HEAD, scale, out_dtype, out, lse, dev_status,
+                 &aa);
+  if (st != KSA_OK) return st;
+  const int sms = device_sm_count();
+  const size_t need = ksa::decode_step_workspace_bytes(
+      shape->batch, shape->num_q_heads, shape->num_kv_heads, shape->head_dim, shape->capacity,
+      shape->block_size, sms);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(KSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  return cuda_status(
+      ksa::launch_decode_step(sa, K, aa, ws, sms, static_cast<cudaStream_t>(stream)),
+      "ksa_decode_step launch");
 }
 
 size_t ksa_unified_select_workspace(const ksa_shape *shape, int32_t per_head_topk,

@@ -97,6 +97,15 @@ size_t attn_workspace_bytes(int B, int Hq, int Hkv, int D, int num_sms);
 cudaError_t launch_sparse_decode_attn(const AttnArgs &a, void *ws, int num_sms,
                                       cudaStream_t stream);
 
+// The decode step in one launch: last-block refresh, scoring, top-k (into
+// a.block_idx / a.num_sel) and attention over the kept blocks (aa's lists are
+// those outputs).  Workspace: the selection workspace followed by the attention
+// workspace; falls back to the two-launch form where the one-launch kernel does
+// not apply.
+size_t decode_step_workspace_bytes(int B, int Hq, int Hkv, int D, int T, int bs, int num_sms);
+cudaError_t launch_decode_step(const SelectArgs &sa, const uint16_t *K, const AttnArgs &aa,
+                               void *ws, int num_sms, cudaStream_t stream);
+
 struct UnifiedArgs {
   const uint16_t *q, *K;
   const int32_t *seq_lens;

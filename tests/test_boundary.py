@@ -320,3 +320,28 @@ def test_no_kernel_spills_registers(ksa):
     spills = re.findall(r"(\d+) bytes spill stores, (\d+) bytes spill loads", text)
     assert len(entries) >= 30 and len(spills) >= len(entries)
     assert all(a == "0" and b == "0" for a, b in spills), spills
+
+
+def test_validation_of_the_decode_step_and_append(ksa):
+    """ksa_decode_step checks the arguments of both calls it stands for, then its own
+    workspace; ksa_append_kv checks pointers and alignment.  Nothing reaches the device."""
+    lib = ksa.lib()
+    sh = _shape(ksa, B=2, Hq=8, Hkv=2, D=128, T=256, bs=16)
+    args = lambda **kw: [kw.get("q", FAKE), kw.get("K", FAKE), FAKE, FAKE, 0, FAKE,
+                         kw.get("k", 8), FAKE, FAKE, kw.get("scale", 0.0), 0, FAKE, None,
+                         kw.get("ws", None), kw.get("ws_bytes", 0), None, None]
+    assert lib.ksa_decode_step(None, *args()) == 1
+    assert lib.ksa_decode_step(ctypes.byref(sh), *args(K=None)) == 1
+    assert lib.ksa_decode_step(ctypes.byref(sh), *args(k=0)) == 1
+    assert lib.ksa_decode_step(ctypes.byref(sh), *args(scale=-1.0)) == 1
+    assert lib.ksa_decode_step(ctypes.byref(sh), *args()) == 3  # no workspace
+    need = lib.ksa_decode_step_workspace(ctypes.byref(sh), 8)
+    assert need >= (lib.ksa_select_blocks_workspace(ctypes.byref(sh), 8) +
+                    lib.ksa_sparse_decode_attn_workspace(ctypes.byref(sh), 8, 16))
+    assert lib.ksa_decode_step(ctypes.byref(sh), *args(ws=FAKE, ws_bytes=need - 1)) == 3
+    bad = _shape(ksa, B=2, Hq=8, Hkv=2, D=128, T=256, bs=8)
+    assert lib.ksa_decode_step(ctypes.byref(bad), *args()) == 2
+    assert lib.ksa_append_kv(ctypes.byref(sh), FAKE, None, FAKE, FAKE, FAKE, None, None) == 1
+    odd = ctypes.c_void_p(0x1008)  # 8-byte aligned only
+    assert lib.ksa_append_kv(ctypes.byref(sh), odd, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert "aligned" in ksa.ksa_last_error()

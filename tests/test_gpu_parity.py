@@ -388,11 +388,12 @@ def test_decode_step_qwen3_8b_full_size(ksa, oracle):
     _check_rows(oracle, inp, rows, *res, inp.shape.k_blocks)
 
 
-def _fused_step(ksa, inp, k, stale_last_block=True):
-    """What bench.py times: the fused selection call (last-block refresh + scoring + top-k)
-    then the attention call.  The summaries are prefilled from the cache as it was before
-    the newest token (seq_lens - 1; blocks never built hold NaN), so the call must refresh
-    the block the newest token landed in before it scores."""
+def _fused_step(ksa, inp, k, one_call=False, stale_last_block=True):
+    """The decode step as bench.py times it: ksa_decode_step (one_call), or the fused
+    selection call (last-block refresh + scoring + top-k) then the attention call.  The
+    summaries are prefilled from the cache as it was before the newest token (seq_lens - 1;
+    blocks never built hold NaN), so the step must refresh the block the newest token
+    landed in before it scores."""
     sh = inp.shape
     B, Hq, Hkv, D, T, bs = (sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, sh.capacity,
                             sh.block_size)
@@ -400,6 +401,12 @@ def _fused_step(ksa, inp, k, stale_last_block=True):
     before = (inp.seq_lens - 1).clamp_min(1) if stale_last_block else inp.seq_lens
     ksa.ksa_build_block_summaries(inp.K, before, bs, summaries=S)
     st = status_tensor()
+    if one_call:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=DEV)
+        idx, cnt, out, _ = ksa.ksa_decode_step(inp.q, inp.K, inp.V, S, inp.seq_lens, bs, k,
+                                               lse=lse, dev_status=st)
+        assert st.item() == 0
+        return idx, cnt, out, lse
     ws_sel = torch.zeros((ksa.ksa_select_blocks_workspace(B, Hq, Hkv, D, T, bs, k),),
                          dtype=torch.uint8, device=DEV)
     ws_att = torch.zeros((ksa.ksa_sparse_decode_attn_workspace(B, Hq, Hkv, D, T, k, bs),),
@@ -414,25 +421,28 @@ def _fused_step(ksa, inp, k, stale_last_block=True):
     return idx, cnt, out, lse
 
 
+@pytest.mark.parametrize("one_call", [True, False], ids=["decode_step", "two_calls"])
 @pytest.mark.parametrize("which", ["qwen3-0.6b", "qwen3-8b"])
-def test_fused_decode_step_full_size(ksa, oracle, which):
-    """The bench's own call sequence at the full Qwen3-0.6B (batch 64, 512 blocks, k 32) and
-    Qwen3-8B (batch 32, 1024-2048 blocks, k 128) shapes, planted score gap on the sampled
-    rows: indices bit-exact, outputs within 2e-3 of the oracle."""
+def test_fused_decode_step_full_size(ksa, oracle, which, one_call):
+    """The decode step at the full Qwen3-0.6B (batch 64, 512 blocks, k 32) and Qwen3-8B
+    (batch 32, 1024-2048 blocks, k 128) shapes, through ksa_decode_step (what bench.py times)
+    and through the two calls, planted score gap on the sampled rows: indices bit-exact,
+    outputs within 2e-3 of the oracle."""
     if which == "qwen3-0.6b":
         inp = synth.qwen3_0_6b_inputs(device=DEV)
     else:
         inp = synth.qwen3_8b_inputs(device=DEV, poison_tail=64.0)
     rows = sample_rows(inp.shape.batch, 11, extra=3)
     _plant(oracle, inp, rows, inp.shape.k_blocks)
-    res = _fused_step(ksa, inp, inp.shape.k_blocks)
+    res = _fused_step(ksa, inp, inp.shape.k_blocks, one_call)
     _check_rows(oracle, inp, rows, *res, inp.shape.k_blocks)
 
 
 @pytest.mark.parametrize("context,budget", [(131072, 8192), (32768, 256), (4096, 8192)])
 def test_sweep_points_fused_step(ksa, oracle, context, budget):
     """Sparse points of the throughput sweep (Hq 32, Hkv 8, D 128, bs 16) at their own
-    context and budget, two rows each, through the fused selection call and attention:
+    context and budget, two rows each, through ksa_decode_step (one launch up to 2048
+    blocks per row, the two calls' launches beyond):
     128K / 8192 tokens (k = 512 of 8192 blocks), 32K / 256 (k = 16), and 4K / 8192, where
     k = 512 covers all 256 blocks so the step must equal dense attention."""
     sh = synth.dataclasses.replace(synth.sweep_shape(context, budget), batch=2)
@@ -440,7 +450,7 @@ def test_sweep_points_fused_step(ksa, oracle, context, budget):
     k = sh.k_blocks
     rows = [0, 1]
     _plant(oracle, inp, rows, k)
-    idx, cnt, out, lse = _fused_step(ksa, inp, k)
+    idx, cnt, out, lse = _fused_step(ksa, inp, k, one_call=True)
     _check_rows(oracle, inp, rows, idx, cnt, out, lse, k)
     nb = -(-context // sh.block_size)
     if k >= nb:
