@@ -13,15 +13,17 @@
 //     flat sequence of 8 KB summary pieces -- the same pieces, the same fused
 //     last-block refresh and the same arithmetic as the scoring kernel;
 //  2. a grid-wide barrier: every score key is written;
-//  3. ranking: row r goes to warp r / N of CTA r % N (N CTAs), which selects
-//     its k best blocks with the ranking kernel's warp radix select (keys in
-//     registers), writes the ascending list and the count, and publishes the
+//  3. ranking: rows of up to 1024 blocks go one per warp (row r to warp r / N
+//     of CTA r % N, N CTAs) and use the ranking kernel's warp radix select;
+//     longer rows go one per CTA (row r to CTA r % N) and use the block-wide
+//     radix select of the long-row ranking kernel; keys stay in registers.
+//     The ranker writes the ascending list and the count and publishes the
 //     row (release) tagged with this launch's epoch;
 //  4. attention: the attention kernel's own stream-K partition and pipeline;
 //     each CTA first waits (acquire) until every row it reads is published.
 // The attention grid is the attention kernel's (same CTA shape, shared memory
 // and occupancy), so the results equal the two calls' bit for bit.  Rows of
-// more than 2048 blocks (more keys than one warp holds in registers) take the
+// more than 2048 blocks (more keys than the CTA ranks from registers) take the
 // two-launch path.
 #include <string.h>
 
@@ -39,7 +41,7 @@ using sel::ScoreDev;
 
 constexpr int kStepThreads = att::kAttnThreads;  // 4 consumer warps + 1 producer warp
 constexpr int kStepWarps = kStepThreads / 32;
-constexpr int kMaxFusedBlocks = 2048;  // 64 keys per lane in warp_topk
+constexpr int kMaxFusedBlocks = 2048;  // longest row the one-launch ranking holds in registers
 
 // Flags and barrier words of the step, in the leading (reserved) region of the
 // selection part of the workspace.
@@ -82,29 +84,54 @@ __global__ void __launch_bounds__(kStepThreads, 3)
   uint32_t epoch = 0u;
   if (!grid_barrier(st.bar, a.status, &epoch)) return;  // flagged; rows stay unpublished
 
-  // ---- 3. ranking: one warp per row, its 256-bin histogram in the stage buffers
+  // ---- 3. ranking.  Shared memory for it lies in the stage buffers (unused until phase 4).
   {
-    uint32_t *hist = reinterpret_cast<uint32_t *>(
-                         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023)) +
-                     warp * 256;
+    uint32_t *sm = reinterpret_cast<uint32_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int rows = a.B * a.Hkv;
     const int nb_max = (a.T + a.bs - 1) / a.bs;
-    for (int row = blockIdx.x + static_cast<int>(gridDim.x) * warp; row < rows;
-         row += static_cast<int>(gridDim.x) * kStepWarps) {
-      const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, lane == 0 ? a.status : nullptr);
-      const int nb = (L + a.bs - 1) / a.bs;
-      if (nb <= a.k) {
-        sel::keep_all_blocks<D>(sp, row, L, nb);
-      } else {
-        sel::warp_topk<KPL>(sp.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
-                            a.block_idx + static_cast<size_t>(row) * a.k, hist);
-        if (lane == 0) a.num_sel[row] = a.k;
+    if constexpr (KPL <= 32) {
+      // rows of up to 1024 blocks: one warp per row, a 256-bin histogram per warp
+      uint32_t *hist = sm + warp * 256;
+      for (int row = blockIdx.x + static_cast<int>(gridDim.x) * warp; row < rows;
+           row += static_cast<int>(gridDim.x) * kStepWarps) {
+        const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, lane == 0 ? a.status : nullptr);
+        const int nb = (L + a.bs - 1) / a.bs;
+        if (nb <= a.k) {
+          sel::keep_all_blocks<D>(sp, row, L, nb);
+        } else {
+          sel::warp_topk<KPL>(sp.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
+                              a.block_idx + static_cast<size_t>(row) * a.k, hist);
+          if (lane == 0) a.num_sel[row] = a.k;
+        }
+        __threadfence();  // this lane's list entries before the publication
+        __syncwarp();
+        if (lane == 0) st_release_gpu(st.ready + row, epoch);
       }
-      __threadfence();  // this lane's list entries before the publication
-      __syncwarp();
-      if (lane == 0) st_release_gpu(st.ready + row, epoch);
+    } else {
+      // longer rows (up to 2048 blocks): the CTA's five warps rank one row together
+      constexpr int kCtaKeys = (kMaxFusedBlocks + kStepThreads - 1) / kStepThreads;
+      static_assert(sel::block_topk_words<kStepThreads>() * 4 <= 8 * 8192,
+                    "the ranking's shared arrays fit in the stage buffers");
+      for (int row = blockIdx.x; row < rows; row += static_cast<int>(gridDim.x)) {
+        const int L =
+            clamp_len(a.seq_lens[row / a.Hkv], a.T, threadIdx.x == 0 ? a.status : nullptr);
+        const int nb = (L + a.bs - 1) / a.bs;
+        if (nb <= a.k) {
+          if (warp == 0) sel::keep_all_blocks<D>(sp, row, L, nb);
+        } else {
+          sel::block_topk<kStepThreads, kCtaKeys>(sp.keys + static_cast<size_t>(row) * nb_max,
+                                                  nb, a.k,
+                                                  a.block_idx + static_cast<size_t>(row) * a.k,
+                                                  sm);
+          if (threadIdx.x == 0) a.num_sel[row] = a.k;
+        }
+        __threadfence();  // this thread's list entries before the publication
+        __syncthreads();  // (also: the shared arrays are free for the next row)
+        if (threadIdx.x == 0) st_release_gpu(st.ready + row, epoch);
+      }
     }
-    fence_proxy_async_smem();  // the histograms' stores before the TMA writes that follow
+    fence_proxy_async_smem();  // the ranking's shared stores before the TMA writes that follow
   }
   __syncthreads();
 

@@ -94,21 +94,15 @@ __global__ void __launch_bounds__(kRankWarpThreads) rank_rows_kernel(const Score
   if (lane == 0) a.num_sel[row] = a.k;
 }
 
-// Ranking for rows of more than 1024 blocks (up to 256 KPL): one CTA of
-// kRankThreads per (row, kv-head), keys in registers (thread t holds blocks
-// t, t + NT, ... so that (slot, thread) order is block order).  The same exact
-// radix select as warp_topk, block-wide: per pass, per-warp 256-bin shared
-// histograms (fewer same-address atomics), summed by warp 0, which finds the
-// digit.  Output: per slot, ballots and one exchange of per-warp counts give
-// every winner its place, ascending.
+// Ranking for rows of more than 1024 blocks (up to 64 keys per thread): one
+// CTA of kRankThreads per (row, kv-head), block_topk over its keys.
+// (With 32 or more keys per thread one CTA per SM: the register file holds them
+// all, with no spill.)
 template <int D, int KPL>
-__global__ void __launch_bounds__(kRankThreads) rank_long_kernel(const ScoreDev p) {
-  constexpr int NT = kRankThreads, NW = NT / 32;
-  __shared__ __align__(16) uint32_t hist[NW][256];
-  __shared__ uint32_t red[2][NW];
-  __shared__ uint32_t xinfo[2];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
+__global__ void __launch_bounds__(kRankThreads, KPL >= 32 ? 1 : 0)
+    rank_long_kernel(const ScoreDev p) {
+  __shared__ __align__(16) uint32_t sm[block_topk_words<kRankThreads>()];
+  const int tid = threadIdx.x, warp = tid >> 5;
   pdl_wait();
   pdl_launch_dependents();
   const SelectArgs &a = p.a;
@@ -116,125 +110,13 @@ __global__ void __launch_bounds__(kRankThreads) rank_long_kernel(const ScoreDev 
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, tid == 0 ? a.status : nullptr);
   const int nb = (L + a.bs - 1) / a.bs;
-  const int k = a.k;
-  if (nb <= k) {
+  if (nb <= a.k) {
     if (warp == 0) keep_all_blocks<D>(p, row, L, nb);
     return;
   }
-  int32_t *out = a.block_idx + static_cast<size_t>(row) * k;
-  const uint32_t *krow = p.keys + static_cast<size_t>(row) * nb_max;
-  uint32_t key[KPL];
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const int j = tid + NT * e;
-    key[e] = j < nb ? __ldcg(krow + j) : 0u;
-    if (j < nb) {
-      kmin = min(kmin, key[e]);
-      kmax = max(kmax, key[e]);
-    }
-  }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if (lane == 0) {
-    red[0][warp] = kmin;
-    red[1][warp] = kmax;
-  }
-  __syncthreads();
-  kmin = red[0][0];
-  kmax = red[1][0];
-#pragma unroll
-  for (int w = 1; w < NW; ++w) {
-    kmin = min(kmin, red[0][w]);
-    kmax = max(kmax, red[1][w]);
-  }
-  uint32_t tau = kmin;
-  uint32_t remaining = static_cast<uint32_t>(k);  // keys still to take at or below tau
-  if (kmin != kmax) {
-    const int hb = 31 - __clz(kmin ^ kmax);
-    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
-    uint32_t prefix = kmin & pmask;
-    for (int shift = hb - 7;; shift -= 8) {
-      const int sh = shift > 0 ? shift : 0;
-      for (int i = tid; i < NW * 256; i += NT) (&hist[0][0])[i] = 0u;
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < KPL; ++e) {
-        if (tid + NT * e < nb && (key[e] & pmask) == prefix)
-          atomicAdd(&hist[warp][(key[e] >> sh) & 255u], 1u);
-      }
-      __syncthreads();
-      if (warp == 0) {  // lane l owns bins [8l, 8l + 8); counts from the top bin down
-        uint32_t c[8];
-        uint32_t tot = 0u;
-#pragma unroll
-        for (int jb = 0; jb < 8; ++jb) {
-          uint32_t v = 0u;
-#pragma unroll
-          for (int w = 0; w < NW; ++w) v += hist[w][lane * 8 + jb];
-          c[jb] = v;
-          tot += v;
-        }
-        uint32_t incl = tot;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
-          if (lane + off < 32) incl += y;
-        }
-        uint32_t run = incl - tot;
-#pragma unroll
-        for (int jb = 7; jb >= 0; --jb) {
-          const uint32_t before = run;
-          run += c[jb];
-          if (before < remaining && run >= remaining) {
-            xinfo[0] = static_cast<uint32_t>(lane * 8 + jb);
-            xinfo[1] = before;
-          }
-        }
-      }
-      __syncthreads();
-      const uint32_t digit = xinfo[0];
-      remaining -= xinfo[1];
-      prefix = (prefix & ~(255u << sh)) | (digit << sh);
-      pmask |= 255u << sh;
-      __syncthreads();  // xinfo and the bins are read before the next pass
-      if (sh == 0) break;
-    }
-    tau = prefix;
-  }
-  const uint32_t take_eq = remaining;
-  uint32_t base = 0u, eq_seen = 0u;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const int j = tid + NT * e;
-    const bool ok = j < nb;
-    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) red[0][warp] = __popc(eb);
-    __syncthreads();
-    uint32_t eq_below = 0u, eq_tot = 0u;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const uint32_t v = red[0][w];
-      eq_below += w < warp ? v : 0u;
-      eq_tot += v;
-    }
-    const bool sel = gt || (eq && eq_seen + eq_below + __popc(eb & lt) < take_eq);
-    eq_seen += eq_tot;
-    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) red[1][warp] = __popc(sb);
-    __syncthreads();
-    uint32_t sel_below = 0u, sel_tot = 0u;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const uint32_t v = red[1][w];
-      sel_below += w < warp ? v : 0u;
-      sel_tot += v;
-    }
-    if (sel) out[base + sel_below + __popc(sb & lt)] = j;
-    base += sel_tot;
-  }
-  if (tid == 0) a.num_sel[row] = k;
+  block_topk<kRankThreads, KPL>(p.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
+                                a.block_idx + static_cast<size_t>(row) * a.k, sm);
+  if (tid == 0) a.num_sel[row] = a.k;
 }
 
 // Local attention as a block selection: every (row, kv-head) keeps its last

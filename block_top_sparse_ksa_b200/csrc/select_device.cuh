@@ -86,6 +86,7 @@ __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const ui
 template <int KPL>
 __device__ __forceinline__ void warp_topk(const uint32_t *krow, int nb, int k, int32_t *out,
                                           uint32_t *hist) {
+  static_assert(KPL >= 1 && KPL <= 32, "the live-slot mask is one 32-bit word");
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
   uint32_t key[KPL];
@@ -166,6 +167,142 @@ __device__ __forceinline__ void warp_topk(const uint32_t *krow, int nb, int k, i
     const uint32_t sb = __ballot_sync(0xffffffffu, sel);
     if (sel) out[base + __popc(sb & lt)] = lane + 32 * e;
     base += __popc(sb);
+  }
+}
+
+// Exact top-k of one row's nb (k < nb <= NT KPL) score keys by a whole CTA
+// of NT threads, keys in registers (thread t holds blocks t, t + NT, ... so
+// that (slot, thread) order is block order).  The same radix select as
+// warp_topk, block-wide: per pass, per-warp 256-bin shared histograms (fewer
+// same-address atomics), summed by warp 0, which finds the digit.  Output: per
+// slot, ballots and one exchange of per-warp counts give every winner its
+// place, ascending.  Shared memory `sm`, 16-byte aligned: block_topk_words<NT>
+// words (per-warp histograms, then two words per warp and two more).  All NT
+// threads call it.
+template <int NT>
+__host__ __device__ constexpr int block_topk_words() {
+  return (NT / 32) * 256 + 2 * (NT / 32) + 2;
+}
+
+template <int NT, int KPL>
+__device__ __forceinline__ void block_topk(const uint32_t *krow, int nb, int k, int32_t *out,
+                                           uint32_t *sm) {
+  constexpr int NW = NT / 32;
+  uint32_t(*hist)[256] = reinterpret_cast<uint32_t(*)[256]>(sm);
+  uint32_t(*red)[NW] = reinterpret_cast<uint32_t(*)[NW]>(sm + NW * 256);
+  uint32_t *xinfo = sm + NW * 256 + 2 * NW;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t key[KPL];
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = tid + NT * e;
+    key[e] = j < nb ? __ldcg(krow + j) : 0u;
+    if (j < nb) {
+      kmin = min(kmin, key[e]);
+      kmax = max(kmax, key[e]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    red[0][warp] = kmin;
+    red[1][warp] = kmax;
+  }
+  __syncthreads();
+  kmin = red[0][0];
+  kmax = red[1][0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    kmin = min(kmin, red[0][w]);
+    kmax = max(kmax, red[1][w]);
+  }
+  uint32_t tau = kmin;
+  uint32_t remaining = static_cast<uint32_t>(k);  // keys still to take at or below tau
+  if (kmin != kmax) {
+    const int hb = 31 - __clz(kmin ^ kmax);
+    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
+    uint32_t prefix = kmin & pmask;
+    for (int shift = hb - 7;; shift -= 8) {
+      const int sh = shift > 0 ? shift : 0;
+      for (int i = tid; i < NW * 256; i += NT) (&hist[0][0])[i] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) {
+        if (tid + NT * e < nb && (key[e] & pmask) == prefix)
+          atomicAdd(&hist[warp][(key[e] >> sh) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {  // lane l owns bins [8l, 8l + 8); counts from the top bin down
+        uint32_t c[8];
+        uint32_t tot = 0u;
+#pragma unroll
+        for (int jb = 0; jb < 8; ++jb) {
+          uint32_t v = 0u;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) v += hist[w][lane * 8 + jb];
+          c[jb] = v;
+          tot += v;
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+          if (lane + off < 32) incl += y;
+        }
+        uint32_t run = incl - tot;
+#pragma unroll
+        for (int jb = 7; jb >= 0; --jb) {
+          const uint32_t before = run;
+          run += c[jb];
+          if (before < remaining && run >= remaining) {
+            xinfo[0] = static_cast<uint32_t>(lane * 8 + jb);
+            xinfo[1] = before;
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t digit = xinfo[0];
+      remaining -= xinfo[1];
+      prefix = (prefix & ~(255u << sh)) | (digit << sh);
+      pmask |= 255u << sh;
+      __syncthreads();  // xinfo and the bins are read before the next pass
+      if (sh == 0) break;
+    }
+    tau = prefix;
+  }
+  const uint32_t take_eq = remaining;
+  uint32_t base = 0u, eq_seen = 0u;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = tid + NT * e;
+    const bool ok = j < nb;
+    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) red[0][warp] = __popc(eb);
+    __syncthreads();
+    uint32_t eq_below = 0u, eq_tot = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t v = red[0][w];
+      eq_below += w < warp ? v : 0u;
+      eq_tot += v;
+    }
+    const bool sel = gt || (eq && eq_seen + eq_below + __popc(eb & lt) < take_eq);
+    eq_seen += eq_tot;
+    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) red[1][warp] = __popc(sb);
+    __syncthreads();
+    uint32_t sel_below = 0u, sel_tot = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t v = red[1][w];
+      sel_below += w < warp ? v : 0u;
+      sel_tot += v;
+    }
+    if (sel) out[base + sel_below + __popc(sb & lt)] = j;
+    base += sel_tot;
   }
 }
 
