@@ -13,12 +13,10 @@
 //     flat sequence of 8 KB summary pieces -- the same pieces, the same fused
 //     last-block refresh and the same arithmetic as the scoring kernel;
 //  2. a grid-wide barrier: every score key is written;
-//  3. ranking: rows of up to 1024 blocks go one per warp (row r to warp r / N
-//     of CTA r % N, N CTAs) and use the ranking kernel's warp radix select;
-//     longer rows go one per CTA (row r to CTA r % N) and use the block-wide
-//     radix select of the long-row ranking kernel; keys stay in registers.
-//     The ranker writes the ascending list and the count and publishes the
-//     row (release) tagged with this launch's epoch;
+//  3. ranking: row r goes to CTA r % N (N CTAs), whose threads hold its keys
+//     in registers and run the ranking kernel's fast_topk; the CTA writes the
+//     ascending list and the count and publishes the row (release) tagged
+//     with this launch's epoch;
 //  4. attention: the attention kernel's own stream-K partition and pipeline;
 //     each CTA first waits (acquire) until every row it reads is published.
 // The attention grid is the attention kernel's (same CTA shape, shared memory
@@ -50,7 +48,7 @@ struct StepDev {
   uint32_t *bar;    // [2]: grid barrier (arrivals, generation)
 };
 
-template <int D, bool SBF, int KPL>
+template <int D, bool SBF, int RK>
 __global__ void __launch_bounds__(kStepThreads, 3)
     decode_step_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const ScoreDev sp,
@@ -66,9 +64,12 @@ __global__ void __launch_bounds__(kStepThreads, 3)
     float4 qv[D / 32];
     const long long NW = static_cast<long long>(gridDim.x) * kStepWarps;
     const long long gw = static_cast<long long>(blockIdx.x) * kStepWarps + warp;
-    const long long u0 = gw * sp.units / NW, u1 = (gw + 1) * sp.units / NW;
+    int pcs[sel::kWalkPerLane];
+    sel::PieceWalk walk = sel::walk_begin(sp, pcs);
+    const long long u0 = gw * walk.total / NW, u1 = (gw + 1) * walk.total / NW;
+    if (walk.compact && u0 < u1) sel::walk_seek(sp, walk, pcs, u0);
     for (long long u = u0; u < u1; ++u) {
-      const sel::Piece x = sel::piece_of(sp, u);
+      const sel::Piece x = sel::walk_next(sp, walk, u);
       if (x.n == 0) continue;
       if (x.row != qrow) {
         qrow = x.row;
@@ -84,52 +85,29 @@ __global__ void __launch_bounds__(kStepThreads, 3)
   uint32_t epoch = 0u;
   if (!grid_barrier(st.bar, a.status, &epoch)) return;  // flagged; rows stay unpublished
 
-  // ---- 3. ranking.  Shared memory for it lies in the stage buffers (unused until phase 4).
+  // ---- 3. ranking: one CTA per row; its shared memory lies in the stage buffers, which
+  // are unused until phase 4
   {
+    static_assert(sel::fast_topk_words<kStepThreads, RK>() * 4 <= 8 * 4096,
+                  "the ranking's shared arrays fit in the stage buffers");
     uint32_t *sm = reinterpret_cast<uint32_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int rows = a.B * a.Hkv;
     const int nb_max = (a.T + a.bs - 1) / a.bs;
-    if constexpr (KPL <= 32) {
-      // rows of up to 1024 blocks: one warp per row, a 256-bin histogram per warp
-      uint32_t *hist = sm + warp * 256;
-      for (int row = blockIdx.x + static_cast<int>(gridDim.x) * warp; row < rows;
-           row += static_cast<int>(gridDim.x) * kStepWarps) {
-        const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, lane == 0 ? a.status : nullptr);
-        const int nb = (L + a.bs - 1) / a.bs;
-        if (nb <= a.k) {
-          sel::keep_all_blocks<D>(sp, row, L, nb);
-        } else {
-          sel::warp_topk<KPL>(sp.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
-                              a.block_idx + static_cast<size_t>(row) * a.k, hist);
-          if (lane == 0) a.num_sel[row] = a.k;
-        }
-        __threadfence();  // this lane's list entries before the publication
-        __syncwarp();
-        if (lane == 0) st_release_gpu(st.ready + row, epoch);
+    for (int row = blockIdx.x; row < rows; row += static_cast<int>(gridDim.x)) {
+      const int L =
+          clamp_len(a.seq_lens[row / a.Hkv], a.T, threadIdx.x == 0 ? a.status : nullptr);
+      const int nb = (L + a.bs - 1) / a.bs;
+      if (nb <= a.k) {
+        if (warp == 0) sel::keep_all_blocks<D>(sp, row, L, nb);
+      } else {
+        sel::fast_topk<kStepThreads, RK>(sp.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
+                                         a.block_idx + static_cast<size_t>(row) * a.k, sm);
+        if (threadIdx.x == 0) a.num_sel[row] = a.k;
       }
-    } else {
-      // longer rows (up to 2048 blocks): the CTA's five warps rank one row together
-      constexpr int kCtaKeys = (kMaxFusedBlocks + kStepThreads - 1) / kStepThreads;
-      static_assert(sel::block_topk_words<kStepThreads>() * 4 <= 8 * 8192,
-                    "the ranking's shared arrays fit in the stage buffers");
-      for (int row = blockIdx.x; row < rows; row += static_cast<int>(gridDim.x)) {
-        const int L =
-            clamp_len(a.seq_lens[row / a.Hkv], a.T, threadIdx.x == 0 ? a.status : nullptr);
-        const int nb = (L + a.bs - 1) / a.bs;
-        if (nb <= a.k) {
-          if (warp == 0) sel::keep_all_blocks<D>(sp, row, L, nb);
-        } else {
-          sel::block_topk<kStepThreads, kCtaKeys>(sp.keys + static_cast<size_t>(row) * nb_max,
-                                                  nb, a.k,
-                                                  a.block_idx + static_cast<size_t>(row) * a.k,
-                                                  sm);
-          if (threadIdx.x == 0) a.num_sel[row] = a.k;
-        }
-        __threadfence();  // this thread's list entries before the publication
-        __syncthreads();  // (also: the shared arrays are free for the next row)
-        if (threadIdx.x == 0) st_release_gpu(st.ready + row, epoch);
-      }
+      __threadfence();  // this thread's list entries before the publication
+      __syncthreads();  // (also: the shared arrays are free for the next row)
+      if (threadIdx.x == 0) st_release_gpu(st.ready + row, epoch);
     }
     fence_proxy_async_smem();  // the ranking's shared stores before the TMA writes that follow
   }
@@ -145,11 +123,9 @@ cudaError_t launch_fused(const CUtensorMap &km, const CUtensorMap &vm, const Sco
                          cudaStream_t stream, bool *launched) {
   const void *fn;
   void (*k4)(CUtensorMap, CUtensorMap, ScoreDev, AttnDev, StepDev) = nullptr;
-  if (nb_max <= 128) k4 = decode_step_kernel<D, SBF, 4>;
-  else if (nb_max <= 256) k4 = decode_step_kernel<D, SBF, 8>;
-  else if (nb_max <= 512) k4 = decode_step_kernel<D, SBF, 16>;
-  else if (nb_max <= 1024) k4 = decode_step_kernel<D, SBF, 32>;
-  else k4 = decode_step_kernel<D, SBF, 64>;
+  if (nb_max <= 4 * kStepThreads) k4 = decode_step_kernel<D, SBF, 4>;
+  else if (nb_max <= 8 * kStepThreads) k4 = decode_step_kernel<D, SBF, 8>;
+  else k4 = decode_step_kernel<D, SBF, (kMaxFusedBlocks + kStepThreads - 1) / kStepThreads>;
   fn = reinterpret_cast<const void *>(k4);
   const size_t smem = att::attn_smem_bytes(D, ap.gw);
   int occ = 0;

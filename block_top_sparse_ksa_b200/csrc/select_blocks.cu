@@ -8,20 +8,19 @@
 // Two launches:
 //  1. scoring, persistent.  The summaries of every (row b, kv-head g) are cut
 //     into pieces of 8 KB (2048 / D consecutive blocks of D fp32, or 4096 / D
-//     of D bf16, contiguous); each row is padded to the same number of pieces
-//     and the grid's warps take equal contiguous slices of the flat piece sequence, so
-//     a warp streams one region front to back and forms each row's group
-//     query sum once.  A warp pulls a whole piece into registers with 16-byte
+//     of D bf16, contiguous); the grid's warps take equal contiguous slices of
+//     the sequence of the rows' real pieces (PieceWalk), so a warp streams one
+//     region front to back, forms each row's group query sum once, and every
+//     warp has the same bytes to read whatever the mix of lengths.  A warp pulls a whole piece into registers with 16-byte
 //     loads (all in flight at once), then scores it -- 8 lanes per summary
 //     row, warp shuffles -- and stores order-preserving uint32 keys in the
 //     workspace.  No shared memory, no barriers.  Pieces of rows with at most
 //     k blocks are skipped: nothing is read.
-//  2. ranking.  Rows of up to 1024 blocks: one warp per (row, kv-head) holds
-//     the row's keys (just written, in L2) in registers and runs an exact
-//     radix select for the k-th largest key (ties at the threshold go to the
-//     lower block); ballots place the winners in ascending block order.
-//     Longer rows: one CTA per row, keys in registers, the same selection
-//     block-wide.  Rows with at most k blocks keep every block.
+//  2. ranking: one CTA per (row, kv-head) holds the row's keys (just written,
+//     in L2) in registers and runs fast_topk: histogram passes over shrinking
+//     key ranges (usually two) find the k best, ties at the threshold going
+//     to the lower block, and a bitmap of the winners gives their places in
+//     ascending block order.  Rows with at most k blocks keep every block.
 //
 // With a key cache given (the fused decode-step entry point), the last block
 // of every row is first re-averaged from the keys -- the per-step maintenance
@@ -55,9 +54,12 @@ __global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev
   float4 qv[D / 32];
   const long long NW = static_cast<long long>(p.N) * kWarps;
   const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
-  const long long s0 = gw * p.units / NW, s1 = (gw + 1) * p.units / NW;
+  int pcs[kWalkPerLane];
+  PieceWalk walk = walk_begin(p, pcs);
+  const long long s0 = gw * walk.total / NW, s1 = (gw + 1) * walk.total / NW;
+  if (walk.compact && s0 < s1) walk_seek(p, walk, pcs, s0);
   for (long long u = s0; u < s1; ++u) {  // warp-uniform control flow throughout
-    const Piece x = piece_of(p, u);
+    const Piece x = walk_next(p, walk, u);
     if (x.n == 0) continue;
     if (x.row != qrow) {
       qrow = x.row;
@@ -69,54 +71,26 @@ __global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev
   if (bad != 0u && lane == 0) flag_status(p.a.status, bad);
 }
 
-// Ranking, one warp per (row, kv-head), for rows of at most 32 KPL blocks:
-// the row's keys (just written, in L2) go into registers and warp_topk picks
-// the k best.  Rows with at most k blocks keep every block.
-template <int D, int KPL>
-__global__ void __launch_bounds__(kRankWarpThreads) rank_rows_kernel(const ScoreDev p) {
-  constexpr int kWarps = kRankWarpThreads / 32;
-  __shared__ __align__(16) uint32_t s_hist[kWarps][256];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  pdl_wait();
-  pdl_launch_dependents();
-  const SelectArgs &a = p.a;
-  const int row = blockIdx.x * kWarps + warp;
-  if (row >= a.B * a.Hkv) return;
-  const int nb_max = (a.T + a.bs - 1) / a.bs;
-  const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, lane == 0 ? a.status : nullptr);
-  const int nb = (L + a.bs - 1) / a.bs;
-  if (nb <= a.k) {
-    keep_all_blocks<D>(p, row, L, nb);
-    return;
-  }
-  warp_topk<KPL>(p.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
-                 a.block_idx + static_cast<size_t>(row) * a.k, s_hist[warp]);
-  if (lane == 0) a.num_sel[row] = a.k;
-}
-
-// Ranking for rows of more than 1024 blocks (up to 64 keys per thread): one
-// CTA of kRankThreads per (row, kv-head), block_topk over its keys.
-// (With 32 or more keys per thread one CTA per SM: the register file holds them
-// all, with no spill.)
-template <int D, int KPL>
-__global__ void __launch_bounds__(kRankThreads, KPL >= 32 ? 1 : 0)
-    rank_long_kernel(const ScoreDev p) {
-  __shared__ __align__(16) uint32_t sm[block_topk_words<kRankThreads>()];
-  const int tid = threadIdx.x, warp = tid >> 5;
+// Ranking, one CTA of NT threads per (row, kv-head): the row's keys (just
+// written, in L2) go into registers and fast_topk keeps the k best.  Rows with
+// at most k blocks keep every block.
+template <int D, int NT, int KPL>
+__global__ void __launch_bounds__(NT) rank_rows_kernel(const ScoreDev p) {
+  __shared__ __align__(16) uint32_t sm[fast_topk_words<NT, KPL>()];
   pdl_wait();
   pdl_launch_dependents();
   const SelectArgs &a = p.a;
   const int row = blockIdx.x;
   const int nb_max = (a.T + a.bs - 1) / a.bs;
-  const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, tid == 0 ? a.status : nullptr);
+  const int L = clamp_len(a.seq_lens[row / a.Hkv], a.T, threadIdx.x == 0 ? a.status : nullptr);
   const int nb = (L + a.bs - 1) / a.bs;
   if (nb <= a.k) {
-    if (warp == 0) keep_all_blocks<D>(p, row, L, nb);
+    if (threadIdx.x < 32) keep_all_blocks<D>(p, row, L, nb);
     return;
   }
-  block_topk<kRankThreads, KPL>(p.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
-                                a.block_idx + static_cast<size_t>(row) * a.k, sm);
-  if (tid == 0) a.num_sel[row] = a.k;
+  fast_topk<NT, KPL>(p.keys + static_cast<size_t>(row) * nb_max, nb, a.k,
+                     a.block_idx + static_cast<size_t>(row) * a.k, sm);
+  if (threadIdx.x == 0) a.num_sel[row] = a.k;
 }
 
 // Local attention as a block selection: every (row, kv-head) keeps its last
@@ -157,19 +131,15 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
     err = launch_pdl(kern, dim3(static_cast<unsigned>(p.N)), dim3(kScThreads), 0, stream, p);
     if (err != cudaSuccess) return err;
   }
-  // rows of up to 1024 blocks: one warp per row; longer rows: one CTA per row
-  constexpr int kRw = kRankWarpThreads / 32;
-  const dim3 wgrid(static_cast<unsigned>((rows + kRw - 1) / kRw)), wblock(kRankWarpThreads);
-  if (nb_max <= 128) return launch_pdl(rank_rows_kernel<D, 4>, wgrid, wblock, 0, stream, p);
-  if (nb_max <= 256) return launch_pdl(rank_rows_kernel<D, 8>, wgrid, wblock, 0, stream, p);
-  if (nb_max <= 512) return launch_pdl(rank_rows_kernel<D, 16>, wgrid, wblock, 0, stream, p);
-  if (nb_max <= 1024) return launch_pdl(rank_rows_kernel<D, 32>, wgrid, wblock, 0, stream, p);
-  // longer rows (nb_max <= 16384 is checked by the API): one CTA per row
-  const dim3 rgrid(static_cast<unsigned>(rows)), rblock(kRankThreads);
-  if (nb_max <= 8 * kRankThreads) return launch_pdl(rank_long_kernel<D, 8>, rgrid, rblock, 0, stream, p);
-  if (nb_max <= 16 * kRankThreads) return launch_pdl(rank_long_kernel<D, 16>, rgrid, rblock, 0, stream, p);
-  if (nb_max <= 32 * kRankThreads) return launch_pdl(rank_long_kernel<D, 32>, rgrid, rblock, 0, stream, p);
-  return launch_pdl(rank_long_kernel<D, 64>, rgrid, rblock, 0, stream, p);
+  // one CTA per row; its threads hold the row's keys in registers
+  const dim3 grid(static_cast<unsigned>(rows));
+  if (nb_max <= 512) return launch_pdl(rank_rows_kernel<D, 128, 4>, grid, dim3(128), 0, stream, p);
+  if (nb_max <= 1024) return launch_pdl(rank_rows_kernel<D, 128, 8>, grid, dim3(128), 0, stream, p);
+  if (nb_max <= 2048) return launch_pdl(rank_rows_kernel<D, 256, 8>, grid, dim3(256), 0, stream, p);
+  if (nb_max <= 4096) return launch_pdl(rank_rows_kernel<D, 256, 16>, grid, dim3(256), 0, stream, p);
+  if (nb_max <= 8192) return launch_pdl(rank_rows_kernel<D, 256, 32>, grid, dim3(256), 0, stream, p);
+  // (nb_max <= 16384 is checked by the API)
+  return launch_pdl(rank_rows_kernel<D, 512, 32>, grid, dim3(512), 0, stream, p);
 }
 
 }  // namespace

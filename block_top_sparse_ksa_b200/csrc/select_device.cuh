@@ -16,8 +16,6 @@ namespace sel {
 
 constexpr int kPieceBytes = 8192;  // one piece: 2048 / D fp32 or 4096 / D bf16 summary rows
 constexpr int kScThreads = 256;
-constexpr int kRankWarpThreads = 128;
-constexpr int kRankThreads = 256;
 
 struct ScoreDev {
   SelectArgs a;
@@ -33,7 +31,6 @@ struct Piece {
   int row, b, g, L, nb, j0, n;  // blocks [j0, j0 + n) of the row; n == 0: nothing to score
 };
 
-// `report`: flag an out-of-range sequence length in the status word (once per row).
 static __device__ __forceinline__ Piece piece_of(const ScoreDev &p, long long u, bool report = false) {
   Piece x;
   x.row = static_cast<int>(u / p.pieces);
@@ -46,6 +43,116 @@ static __device__ __forceinline__ Piece piece_of(const ScoreDev &p, long long u,
   x.n = (x.nb > p.a.k && x.j0 < x.nb) ? min(p.prow, x.nb - x.j0) : 0;
   return x;
 }
+
+// Work partition of the scoring.  Only rows with more than k blocks are scored,
+// in pieces of prow blocks, so row (b, g) has P_b = ceil(NB_b / prow) pieces (0
+// if NB_b <= k), the same for every kv-head g of batch row b.  The scoring
+// warps take equal slices of the sequence of these pieces, rows in order, so
+// every warp streams the same number of bytes whatever the mix of lengths.
+// A warp locates its slice from the batch rows' lengths held in its lanes'
+// registers (lane l: rows l, l + 32, ...), which bounds B by kWalkMaxRows; for
+// larger batches each row is padded to the longest row's pieces instead.
+constexpr int kWalkMaxRows = 512;
+constexpr int kWalkPerLane = kWalkMaxRows / 32;
+
+static __device__ __forceinline__ int pieces_of_row(const ScoreDev &p, int L) {
+  const int nb = (L + p.a.bs - 1) / p.a.bs;
+  return nb > p.a.k ? (nb + p.prow - 1) / p.prow : 0;
+}
+
+struct PieceWalk {
+  long long total;  // pieces in the sequence
+  int b, g, piece;  // the cursor
+  int pb, L;        // pieces and length of batch row b
+  bool compact;     // false: the padded layout (rows * p.pieces units)
+};
+
+// Total pieces of the sequence (warp-uniform; every lane calls it).
+static __device__ __forceinline__ PieceWalk walk_begin(const ScoreDev &p, int (&pcs)[kWalkPerLane]) {
+  PieceWalk w;
+  const int lane = threadIdx.x & 31;
+  const SelectArgs &a = p.a;
+  w.compact = a.B <= kWalkMaxRows;
+  if (!w.compact) {
+    w.total = p.units;
+    return w;
+  }
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kWalkPerLane; ++i) {
+    const int b = lane + 32 * i;
+    pcs[i] = b < a.B ? pieces_of_row(p, clamp_len(a.seq_lens[b], a.T, nullptr)) : 0;
+    sum += pcs[i];
+  }
+  w.total = static_cast<long long>(__reduce_add_sync(0xffffffffu, sum)) * a.Hkv;
+  return w;
+}
+
+// Moves the cursor to unit u0 < w.total of the compact sequence.
+static __device__ __forceinline__ void walk_seek(const ScoreDev &p, PieceWalk &w,
+                                                 const int (&pcs)[kWalkPerLane], long long u0) {
+  const int lane = threadIdx.x & 31;
+  const SelectArgs &a = p.a;
+  long long before = 0;  // pieces of the batch rows below the current chunk of 32
+  int fb = 0, fpb = 1, foff = 0;
+  bool found = false;
+#pragma unroll
+  for (int i = 0; i < kWalkPerLane; ++i) {
+    const int mine = pcs[i] * a.Hkv;
+    int incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int chunk = __shfl_sync(0xffffffffu, incl, 31);
+    const unsigned hit = __ballot_sync(0xffffffffu, before + incl > u0);
+    const int src = hit != 0u ? __ffs(hit) - 1 : 0;
+    const int at_incl = __shfl_sync(0xffffffffu, incl, src);
+    const int at_mine = __shfl_sync(0xffffffffu, mine, src);
+    const int at_pcs = __shfl_sync(0xffffffffu, pcs[i], src);
+    if (!found && hit != 0u) {
+      found = true;
+      fb = 32 * i + src;
+      fpb = at_pcs;
+      foff = static_cast<int>(u0 - before) - (at_incl - at_mine);
+    }
+    before += chunk;
+  }
+  w.b = fb;
+  w.pb = fpb;
+  w.g = foff / fpb;
+  w.piece = foff - w.g * fpb;
+  w.L = clamp_len(a.seq_lens[fb], a.T, nullptr);
+}
+
+// The piece under the cursor (then advances it).  Padded layout: unit u.
+static __device__ __forceinline__ Piece walk_next(const ScoreDev &p, PieceWalk &w, long long u) {
+  if (!w.compact) return piece_of(p, u);
+  const SelectArgs &a = p.a;
+  Piece x;
+  x.b = w.b;
+  x.g = w.g;
+  x.row = w.b * a.Hkv + w.g;
+  x.L = w.L;
+  x.nb = (w.L + a.bs - 1) / a.bs;
+  x.j0 = w.piece * p.prow;
+  x.n = min(p.prow, x.nb - x.j0);
+  if (++w.piece == w.pb) {
+    w.piece = 0;
+    if (++w.g == a.Hkv) {
+      w.g = 0;
+      do {  // the next batch row that has pieces (the slice ends before running out)
+        if (++w.b >= a.B) break;
+        w.L = clamp_len(a.seq_lens[w.b], a.T, nullptr);
+        w.pb = pieces_of_row(p, w.L);
+      } while (w.pb == 0);
+    }
+  }
+  return x;
+}
+
+// `report`: flag an out-of-range sequence length in the status word (once per row).
 
 // Re-averages block nb-1 of `row` from K and stores it in the summaries.
 // Lanes l < D/8 get dims [8 (l % (D/8)), +8) in mean[] and return true.
@@ -73,236 +180,196 @@ __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const ui
   return mine;
 }
 
-// Exact top-k of one row's nb (k < nb <= 32 KPL) score keys by one warp, the
-// keys held in registers: lane l holds blocks l, l + 32, l + 64, ... so that
-// (slot, lane) order is block order.  Radix select for the k-th largest key
-// tau, 8 bits a pass from the highest bit in which the row's keys differ (the
-// bits above are common to all): a 256-bin shared-memory histogram of the
-// keys that match the digits fixed so far, then the bin where the count from
-// the top reaches the number still to take.  Every key above tau is kept, and
-// of the keys equal to tau the lowest-index ones, k in all; ballots give each
-// winner its place, so out[0..k) comes out in ascending block order.
-// `hist`: 256 words of this warp's shared memory, 16-byte aligned.
-template <int KPL>
-__device__ __forceinline__ void warp_topk(const uint32_t *krow, int nb, int k, int32_t *out,
-                                          uint32_t *hist) {
-  static_assert(KPL >= 1 && KPL <= 32, "the live-slot mask is one 32-bit word");
-  const int lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
+// Shared-memory words of fast_topk<NT, KPL>: a 1024-bin histogram, the
+// selected and the tied-candidate bitmaps (one bit per block), and 64 words
+// for reductions and broadcasts.
+template <int NT, int KPL>
+__host__ __device__ constexpr int fast_topk_words() {
+  return 1024 + 2 * ((NT * KPL + 31) / 32) + 64;
+}
+
+// Exact top-k of one row's n (k < n <= NT KPL) uint32 score keys by a CTA of
+// NT threads (all of them call it), the keys in registers: thread t holds
+// blocks t, t + NT, t + 2 NT, ...  Selection by shrinking key ranges: the live
+// keys span [lo, hi]; a pass drops them into 1024 buckets of width 2^s
+// ((hi - lo) >> s < 1024), the bucket holding the k-th largest live key is
+// found from a histogram, keys in higher buckets are selected, in lower ones
+// dropped, and the bucket's keys stay live with a range 1024 times narrower.
+// Done when the live keys are exactly the ones still needed (usually after two
+// passes on continuous scores), or all equal: then the lowest-index ones are
+// taken (ties go to the lower block).  At most four passes.  The winners are
+// written to out[0..k) in ascending block order through a bitmap of the
+// selection and one prefix count over its words.  `sm`: fast_topk_words words
+// of shared memory, 16-byte aligned.
+template <int NT, int KPL>
+__device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, int32_t *out,
+                                          uint32_t *sm) {
+  static_assert(NT % 32 == 0 && NT >= 64 && NT <= 1024, "whole warps");
+  static_assert(KPL >= 1 && KPL <= 64, "a 64-bit slot mask per thread");
+  constexpr int NW = NT / 32;
+  constexpr int W = (NT * KPL + 31) / 32;  // bitmap words; block j is bit j % 32 of word j / 32
+  uint32_t *hist = sm;
+  uint32_t *selw = sm + 1024;
+  uint32_t *livew = selw + W;
+  uint32_t *misc = livew + W;  // [0..3) the pass's bucket, count above, count in it; [8..) reductions
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t key[KPL];
-  uint32_t live = 0u;  // bit e: block lane + 32 e exists
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  uint64_t live = 0ull, sel = 0ull;
+  uint32_t lo = 0xffffffffu, hi = 0u;
 #pragma unroll
   for (int e = 0; e < KPL; ++e) {
-    const bool ok = lane + 32 * e < nb;
-    key[e] = ok ? __ldcg(krow + lane + 32 * e) : 0u;
-    live |= ok ? (1u << e) : 0u;
-    if (ok) {
-      kmin = min(kmin, key[e]);
-      kmax = max(kmax, key[e]);
+    const int j = tid + NT * e;
+    key[e] = j < n ? __ldcg(krow + j) : 0u;
+    if (j < n) {
+      live |= 1ull << e;
+      lo = min(lo, key[e]);
+      hi = max(hi, key[e]);
     }
   }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  uint32_t tau = kmin;                            // every key equal: tau is that key
-  uint32_t remaining = static_cast<uint32_t>(k);  // keys still to take at or below tau
-  if (kmin != kmax) {
-    const int hb = 31 - __clz(kmin ^ kmax);  // highest bit in which keys differ
-    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);  // bits fixed so far
-    uint32_t prefix = kmin & pmask;
-    for (int shift = hb - 7;; shift -= 8) {
-      const int sh = shift > 0 ? shift : 0;
-      reinterpret_cast<uint4 *>(hist)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
-      reinterpret_cast<uint4 *>(hist)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
-      __syncwarp();
+  uint32_t remaining = static_cast<uint32_t>(k);  // winners still to find among the live keys
+  for (int pass = 0;; ++pass) {
+    // range of the live keys, block-wide
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+      misc[8 + warp] = lo;
+      misc[8 + NW + warp] = hi;
+    }
+    __syncthreads();
+    lo = misc[8];
+    hi = misc[8 + NW];
 #pragma unroll
-      for (int e = 0; e < KPL; ++e) {
-        if (((live >> e) & 1u) && (key[e] & pmask) == prefix)
-          atomicAdd(&hist[(key[e] >> sh) & 255u], 1u);
+    for (int w = 1; w < NW; ++w) {
+      lo = min(lo, misc[8 + w]);
+      hi = max(hi, misc[8 + NW + w]);
+    }
+    if (lo == hi || pass == 4) break;  // all live keys equal: the index rule decides
+    const int bits = 32 - __clz(hi - lo);
+    const int sh = bits > 10 ? bits - 10 : 0;
+    for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < KPL; ++e)
+      if ((live >> e) & 1ull) atomicAdd(&hist[(key[e] - lo) >> sh], 1u);
+    __syncthreads();
+    if (warp == 0) {  // lane l owns buckets [32 l, 32 l + 32); count from the top down
+      uint32_t c[32];
+      uint32_t tot = 0u;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 v = reinterpret_cast<const uint4 *>(hist + 32 * lane)[q];
+        c[4 * q] = v.x;
+        c[4 * q + 1] = v.y;
+        c[4 * q + 2] = v.z;
+        c[4 * q + 3] = v.w;
+        tot += v.x + v.y + v.z + v.w;
       }
-      __syncwarp();
-      // lane l owns bins [8l, 8l + 8); counts from the top bin down
-      const uint4 h0 = reinterpret_cast<const uint4 *>(hist)[2 * lane];
-      const uint4 h1 = reinterpret_cast<const uint4 *>(hist)[2 * lane + 1];
-      const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-      const uint32_t tot = c[0] + c[1] + c[2] + c[3] + c[4] + c[5] + c[6] + c[7];
-      uint32_t incl = tot;  // keys in the bins of lanes >= this lane
+      uint32_t incl = tot;  // keys in the buckets of lanes >= this one
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
         if (lane + off < 32) incl += y;
       }
-      uint32_t run = incl - tot, digit = 0u, above = 0u;
-      bool found = false;
+      uint32_t run = incl - tot;
 #pragma unroll
-      for (int j = 7; j >= 0; --j) {
+      for (int b = 31; b >= 0; --b) {
         const uint32_t before = run;
-        run += c[j];
+        run += c[b];
         if (before < remaining && run >= remaining) {
-          found = true;
-          digit = static_cast<uint32_t>(lane * 8 + j);
-          above = before;
+          misc[0] = static_cast<uint32_t>(32 * lane + b);
+          misc[1] = before;
+          misc[2] = c[b];
         }
       }
-      const int src = __ffs(__ballot_sync(0xffffffffu, found)) - 1;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      remaining -= above;
-      prefix = (prefix & ~(255u << sh)) | (digit << sh);
-      pmask |= 255u << sh;
-      __syncwarp();  // the bins are read before the next pass clears them
-      if (sh == 0) break;
     }
-    tau = prefix;
-  }
-  const uint32_t take_eq = remaining;  // k minus the keys above tau
-  uint32_t base = 0u, eq_seen = 0u;
+    __syncthreads();
+    const uint32_t bstar = misc[0], above = misc[1], inb = misc[2];
+    remaining -= above;
+    const bool exact = inb == remaining;  // every live key of the bucket is needed
+    const uint32_t base = lo;
+    lo = 0xffffffffu;
+    hi = 0u;
 #pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const bool ok = (live >> e) & 1u;
-    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    const bool sel = gt || (eq && eq_seen + __popc(eb & lt) < take_eq);
-    eq_seen += __popc(eb);
-    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[base + __popc(sb & lt)] = lane + 32 * e;
-    base += __popc(sb);
-  }
-}
-
-// Exact top-k of one row's nb (k < nb <= NT KPL) score keys by a whole CTA
-// of NT threads, keys in registers (thread t holds blocks t, t + NT, ... so
-// that (slot, thread) order is block order).  The same radix select as
-// warp_topk, block-wide: per pass, per-warp 256-bin shared histograms (fewer
-// same-address atomics), summed by warp 0, which finds the digit.  Output: per
-// slot, ballots and one exchange of per-warp counts give every winner its
-// place, ascending.  Shared memory `sm`, 16-byte aligned: block_topk_words<NT>
-// words (per-warp histograms, then two words per warp and two more).  All NT
-// threads call it.
-template <int NT>
-__host__ __device__ constexpr int block_topk_words() {
-  return (NT / 32) * 256 + 2 * (NT / 32) + 2;
-}
-
-template <int NT, int KPL>
-__device__ __forceinline__ void block_topk(const uint32_t *krow, int nb, int k, int32_t *out,
-                                           uint32_t *sm) {
-  constexpr int NW = NT / 32;
-  uint32_t(*hist)[256] = reinterpret_cast<uint32_t(*)[256]>(sm);
-  uint32_t(*red)[NW] = reinterpret_cast<uint32_t(*)[NW]>(sm + NW * 256);
-  uint32_t *xinfo = sm + NW * 256 + 2 * NW;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
-  uint32_t key[KPL];
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const int j = tid + NT * e;
-    key[e] = j < nb ? __ldcg(krow + j) : 0u;
-    if (j < nb) {
-      kmin = min(kmin, key[e]);
-      kmax = max(kmax, key[e]);
+    for (int e = 0; e < KPL; ++e) {
+      if (!((live >> e) & 1ull)) continue;
+      const uint32_t bk = (key[e] - base) >> sh;
+      if (bk > bstar || (bk == bstar && exact)) {
+        sel |= 1ull << e;
+        live &= ~(1ull << e);
+      } else if (bk < bstar) {
+        live &= ~(1ull << e);
+      } else {
+        lo = min(lo, key[e]);
+        hi = max(hi, key[e]);
+      }
+    }
+    __syncthreads();  // misc and the histogram are rewritten by the next pass
+    if (exact) {
+      remaining = 0u;
+      break;
     }
   }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if (lane == 0) {
-    red[0][warp] = kmin;
-    red[1][warp] = kmax;
+  // bitmaps of the selected and of the still-live (all equal) keys, in block order
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const uint32_t sb = __ballot_sync(0xffffffffu, (sel >> e) & 1ull);
+    const uint32_t lb = __ballot_sync(0xffffffffu, (live >> e) & 1ull);
+    if (lane == 0) {
+      selw[warp + NW * e] = sb;
+      livew[warp + NW * e] = lb;
+    }
   }
   __syncthreads();
-  kmin = red[0][0];
-  kmax = red[1][0];
+  if (warp == 0) {
+    // lane l owns words [WPL l, WPL l + WPL): the lowest-index `remaining` live keys join the
+    // selection, then every winner gets its place from a prefix count of the words
+    constexpr int WPL = (W + 31) / 32;
+    uint32_t wl[WPL], ws[WPL];
+    uint32_t nl = 0u;
 #pragma unroll
-  for (int w = 1; w < NW; ++w) {
-    kmin = min(kmin, red[0][w]);
-    kmax = max(kmax, red[1][w]);
-  }
-  uint32_t tau = kmin;
-  uint32_t remaining = static_cast<uint32_t>(k);  // keys still to take at or below tau
-  if (kmin != kmax) {
-    const int hb = 31 - __clz(kmin ^ kmax);
-    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
-    uint32_t prefix = kmin & pmask;
-    for (int shift = hb - 7;; shift -= 8) {
-      const int sh = shift > 0 ? shift : 0;
-      for (int i = tid; i < NW * 256; i += NT) (&hist[0][0])[i] = 0u;
-      __syncthreads();
+    for (int q = 0; q < WPL; ++q) {
+      const int w = lane * WPL + q;
+      wl[q] = w < W ? livew[w] : 0u;
+      ws[q] = w < W ? selw[w] : 0u;
+      nl += __popc(wl[q]);
+    }
+    uint32_t pl = nl;  // inclusive prefix of live bits over the lanes
 #pragma unroll
-      for (int e = 0; e < KPL; ++e) {
-        if (tid + NT * e < nb && (key[e] & pmask) == prefix)
-          atomicAdd(&hist[warp][(key[e] >> sh) & 255u], 1u);
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, pl, off);
+      if (lane >= off) pl += y;
+    }
+    pl -= nl;
+    uint32_t ns = 0u;
+#pragma unroll
+    for (int q = 0; q < WPL; ++q) {
+      uint32_t take = 0u, x = wl[q];
+      while (x != 0u && pl < remaining) {  // lowest set bits first: ascending blocks
+        const uint32_t b = x & (0u - x);
+        take |= b;
+        x ^= b;
+        ++pl;
       }
-      __syncthreads();
-      if (warp == 0) {  // lane l owns bins [8l, 8l + 8); counts from the top bin down
-        uint32_t c[8];
-        uint32_t tot = 0u;
+      pl += __popc(x);
+      ws[q] |= take;
+      ns += __popc(ws[q]);
+    }
+    uint32_t ps = ns;
 #pragma unroll
-        for (int jb = 0; jb < 8; ++jb) {
-          uint32_t v = 0u;
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, ps, off);
+      if (lane >= off) ps += y;
+    }
+    ps -= ns;
 #pragma unroll
-          for (int w = 0; w < NW; ++w) v += hist[w][lane * 8 + jb];
-          c[jb] = v;
-          tot += v;
-        }
-        uint32_t incl = tot;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
-          if (lane + off < 32) incl += y;
-        }
-        uint32_t run = incl - tot;
-#pragma unroll
-        for (int jb = 7; jb >= 0; --jb) {
-          const uint32_t before = run;
-          run += c[jb];
-          if (before < remaining && run >= remaining) {
-            xinfo[0] = static_cast<uint32_t>(lane * 8 + jb);
-            xinfo[1] = before;
-          }
-        }
+    for (int q = 0; q < WPL; ++q) {
+      uint32_t x = ws[q];
+      while (x != 0u) {
+        const int b = __ffs(x) - 1;
+        x &= x - 1u;
+        out[ps++] = 32 * (lane * WPL + q) + b;
       }
-      __syncthreads();
-      const uint32_t digit = xinfo[0];
-      remaining -= xinfo[1];
-      prefix = (prefix & ~(255u << sh)) | (digit << sh);
-      pmask |= 255u << sh;
-      __syncthreads();  // xinfo and the bins are read before the next pass
-      if (sh == 0) break;
     }
-    tau = prefix;
-  }
-  const uint32_t take_eq = remaining;
-  uint32_t base = 0u, eq_seen = 0u;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const int j = tid + NT * e;
-    const bool ok = j < nb;
-    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) red[0][warp] = __popc(eb);
-    __syncthreads();
-    uint32_t eq_below = 0u, eq_tot = 0u;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const uint32_t v = red[0][w];
-      eq_below += w < warp ? v : 0u;
-      eq_tot += v;
-    }
-    const bool sel = gt || (eq && eq_seen + eq_below + __popc(eb & lt) < take_eq);
-    eq_seen += eq_tot;
-    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) red[1][warp] = __popc(sb);
-    __syncthreads();
-    uint32_t sel_below = 0u, sel_tot = 0u;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const uint32_t v = red[1][w];
-      sel_below += w < warp ? v : 0u;
-      sel_tot += v;
-    }
-    if (sel) out[base + sel_below + __popc(sb & lt)] = j;
-    base += sel_tot;
   }
 }
 
