@@ -1,12 +1,12 @@
 #!/usr/bin/env python
 """Throughput of block top-k sparse decode attention on B200.
 
-One step = one decode step of one attention layer for a whole batch:
-  block-summary maintenance (last block) + block scoring + top-k selection
-  (the fused selection call: a scoring launch and a ranking launch) ->
-  gathered split-KV attention over the selected blocks, all in libksa's CUDA
-  kernels.  Metric: queries/s, one query = one sequence's decode step for one
-  layer (all query heads).
+One step = one decode step of one attention layer for a whole batch, one
+ksa_decode_step call: block-summary maintenance (last block) + block scoring
+(one launch), top-k selection (one launch), gathered split-KV attention over
+the selected blocks (one launch), all in libksa's CUDA kernels.  Metric:
+queries/s, one query = one sequence's decode step for one layer (all query
+heads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ksa|reference]
                   [--workload qwen3-8b|qwen3-0.6b|lessismore|tiny|sweep-L<ctx>-B<budget>|dense-L<ctx>]
@@ -24,7 +24,8 @@ Timing: W warm-up steps (and more, untimed, until at least --min-warmup-s of
 them have run, so the clocks have settled), then K steps back to back between
 two CUDA events on the launching stream, bracketed by barrier + synchronize.
 Nothing else is enqueued inside the timed region.  Per-kernel durations come
-from a second pass of the same steps with an event around each launch.
+from a second pass of the same steps with an event around the selection call
+and the attention call.
 """
 from __future__ import annotations
 
@@ -385,14 +386,9 @@ class BlockWorkload:
         self.out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
         self.stream = torch.cuda.current_stream()
         nb_max = -(-T // bs)
-        # the two calls: a scoring launch (when some row can hold more than k blocks), a
-        # ranking launch, the attention launch; ksa_decode_step is one launch for rows of up
-        # to 2048 blocks and those three beyond
-        self.two_call_launches = (2 if nb_max > k else 1) + 1
-        if self.kind == "dense":
-            self.launches_per_step = 1
-        else:
-            self.launches_per_step = 1 if nb_max <= 2048 else self.two_call_launches
+        # ksa_decode_step: a scoring launch (when some row can hold more than k blocks), a
+        # ranking launch, the attention launch
+        self.launches_per_step = 1 if self.kind == "dense" else (2 if nb_max > k else 1) + 1
 
     def select(self, i, q=None):
         sh = self.shape
@@ -427,15 +423,14 @@ class BlockWorkload:
         else:
             self.decode_step(i)
 
-    def step_two_calls(self, i):
-        self.select(i)
-        self.attend(i)
+    def parts(self):
+        """The step's calls, one by one (for per-kernel times)."""
+        return [self.attend] if self.kind == "dense" else [self.select, self.attend]
 
 
 def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
                   clocks: "ClockSampler | None" = None):
-    """Warm-up, the timed steps and the per-kernel pass of one block workload; then the
-    same steps through the two calls (selection, attention) for comparison."""
+    """Warm-up, the timed steps and the per-kernel pass of one block workload."""
     sh, kind = wl.shape, wl.kind
     n_warm = warm_up(wl.step, args.warmup, args.min_warmup_s)
     if clocks is not None:
@@ -444,26 +439,31 @@ def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
     if clocks is not None:
         clocks.mark()
     value, ms_step = weak_scaling(dist, sh.batch, ms, args.steps)
-    n_pass = max(20, min(args.steps, 200))
-    (t_step,) = kernel_pass([wl.step], n_pass, wl.stream)
+    times = kernel_pass(wl.parts(), max(20, min(args.steps, 200)), wl.stream)
+    t_att = times[-1]
+    t_sel = times[0] if kind != "dense" else 0.0
     lens = wl.inp.seq_lens.cpu().tolist()
     total_b, attn_b, summ_b = algorithmic_bytes(sh, lens, kind, wl.S.element_size())
     per_step_s = ms_step / 1e3
-    name = "sparse_decode_attn" if kind == "dense" else "decode_step"
-    # the dominant (here: only) kernel of the step, its algorithmic bytes per launch
-    roof_b = attn_b if kind == "dense" else total_b
-    roof_gbs = roof_b / (t_step * 1e-3) / 1e9
-    res = {
+    attn_gbs = attn_b / (t_att * 1e-3) / 1e9
+    return {
         "value": value, "ms_per_step": ms_step, "warmup_steps_run": n_warm,
         "host_enqueue_us_per_step": host_us,
-        "kernels_ms": {name: t_step},
-        "kernels_note": "mean of a second pass of the same steps with an event around each call",
-        "roofline": {"bound": "hbm", "achieved": roof_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": roof_gbs / peak,
-                     "traffic": stored_traffic(name, args.workload, sh.batch),
-                     "kernel": name, "peak_source": peak_kind, "bytes_per_launch": roof_b},
+        "kernels_ms": ({"sparse_decode_attn": t_att} if kind == "dense" else
+                       {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att}),
+        "kernels_note": "mean of a second pass of the same steps with an event around each call "
+                        "(the selection call is its scoring and ranking launches)",
+        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": attn_gbs / peak,
+                     "traffic": stored_traffic("sparse_decode_attn", args.workload, sh.batch),
+                     "kernel": "sparse_decode_attn", "peak_source": peak_kind,
+                     "bytes_per_launch": attn_b},
         "step_hbm": {"bytes_per_step": total_b, "gbs": total_b / per_step_s / 1e9,
-                     "frac": total_b / per_step_s / 1e9 / peak, "kernel_sum_ms": t_step},
+                     "frac": total_b / per_step_s / 1e9 / peak,
+                     "kernel_sum_ms": t_sel + t_att},
+        "select_hbm": (None if kind == "dense" else
+                       {"bytes_per_launch": summ_b,
+                        "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None}),
         "gpu_launches": wl.launches_per_step * args.steps,
         "config": {"workload": sh.name, "batch_per_gpu": sh.batch, "num_q_heads": sh.num_q_heads,
                    "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim,
@@ -476,26 +476,9 @@ def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
                          "rotating query sets" % (2 * wl.inp.K.numel() * 2 / 1e9, total_b / 1e6,
                                                   wl.nq),
                    "step": ("dense attention" if kind == "dense" else
-                            "ksa_decode_step: last-block summary refresh + scoring + top-k + "
-                            "sparse attention (%d launch%s)" % (
-                                wl.launches_per_step,
-                                "" if wl.launches_per_step == 1 else "es"))},
+                            "ksa_decode_step: last-block summary refresh + scoring + top-k "
+                            "(2 launches) + sparse attention (1 launch)")},
     }
-    if kind != "dense":
-        ms2, _ = timed_steps(wl.step_two_calls, args.steps, dist, wl.stream)
-        _, ms2_step = weak_scaling(dist, sh.batch, ms2, args.steps)
-        t_sel, t_att = kernel_pass([wl.select, wl.attend], n_pass, wl.stream)
-        attn_gbs = attn_b / (t_att * 1e-3) / 1e9
-        res["two_calls"] = {
-            "what": "ksa_decode_select_blocks + ksa_sparse_decode_attn (%d launches)"
-                    % wl.two_call_launches,
-            "ms_per_step": ms2_step, "value": sh.batch / (ms2_step * 1e-3),
-            "kernels_ms": {"decode_select_blocks": t_sel, "sparse_decode_attn": t_att},
-            "attention_roofline": {"bytes_per_launch": attn_b, "achieved": attn_gbs,
-                                   "frac": attn_gbs / peak},
-            "select_hbm": {"bytes_per_launch": summ_b,
-                           "gbs": summ_b / (t_sel * 1e-3) / 1e9 if t_sel > 0 else None}}
-    return res
 
 
 def run_block(args, dist, dev, kind):
@@ -532,8 +515,7 @@ def run_extra(args, dist, dev):
                          "ms_per_step": r["ms_per_step"],
                          "host_enqueue_us_per_step": r["host_enqueue_us_per_step"],
                          "step_hbm": r["step_hbm"], "roofline_frac": r["roofline"]["frac"],
-                         "kernels_ms": r["kernels_ms"], "gpu_launches": r["gpu_launches"],
-                         "two_calls": r.get("two_calls")}
+                         "kernels_ms": r["kernels_ms"], "gpu_launches": r["gpu_launches"]}
             del wl
         except torch.cuda.OutOfMemoryError as e:  # never lose the main line for a side figure
             out[name] = {"error": str(e)[:200]}
@@ -606,7 +588,7 @@ def run_block_e2e(args, dist, wl: BlockWorkload):
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
             "host_enqueue_us_per_step": host_us,
-            "gpu_launches": (wl.launches_per_step + 1) * args.steps,
+            "gpu_launches": (wl.launches_per_step + 1) * args.steps,  # + the append
             "note": "per step: q and the new token's K/V rows host->device (pinned), "
                     "ksa_append_kv, ksa_decode_step, out device->host"}
 
@@ -841,9 +823,7 @@ def main():
                 "warmup_steps_run": res["warmup_steps_run"],
                 "host_enqueue_us_per_step": res["host_enqueue_us_per_step"],
                 "kernels_note": res["kernels_note"]}
-        if "two_calls" in res:
-            line["two_calls"] = res["two_calls"]
-        if "select_hbm" in res:
+        if res.get("select_hbm") is not None:
             line["select_hbm"] = res["select_hbm"]
         if "e2e" in res:
             line["e2e"] = res["e2e"]

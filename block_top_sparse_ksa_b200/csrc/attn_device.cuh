@@ -1,6 +1,6 @@
-// attn_device.cuh -- device pieces of the gathered split-KV flash-decode,
-// shared by the attention kernel (decode_attn.cu) and the one-launch decode
-// step (decode_step.cu).  The design is described at the top of decode_attn.cu.
+// attn_device.cuh -- device pieces of the gathered split-KV flash-decode (the
+// attention kernel's body and its helpers) and the host-side preparation of an
+// attention launch.  The design is described at the top of decode_attn.cu.
 #pragma once
 
 #include "ksa_device.cuh"
@@ -91,14 +91,7 @@ struct RowInfo {
   int n_st;  // real stages of the row
 };
 
-// A list entry: through the read-only path when the lists come from an earlier
-// launch, through L2 when they were written earlier in this launch.
-template <bool FUSED>
-__device__ __forceinline__ int ld_list(const int32_t *p) {
-  return FUSED ? __ldcg(p) : __ldg(p);
-}
-
-template <int MODE, bool FUSED = false>
+template <int MODE>
 __device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int r, int b, uint32_t *flag_sink) {
   RowInfo ri;
   ri.L = clamp_len(a.seq_lens[b], a.T, flag_sink);
@@ -110,8 +103,7 @@ __device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int r, int b, uin
   }
   ri.list = a.shared == 1 ? a.idx + static_cast<size_t>(b) * a.cap
                           : a.idx + static_cast<size_t>(r) * a.cap;
-  // 0: per kv-head, 2: per query head rows
-  int n = ld_list<FUSED>(a.shared == 1 ? a.num_idx + b : a.num_idx + r);
+  int n = a.shared == 1 ? a.num_idx[b] : a.num_idx[r];  // 0: per kv-head, 2: per query head rows
   if (n < 0 || n > a.cap) {
     flag_status(flag_sink, KSA_FLAG_INDEX_SKIPPED);
     n = n < 0 ? 0 : a.cap;
@@ -200,17 +192,10 @@ __device__ __forceinline__ void merge_partials(const AttnDev &p, int r, int tid)
   }
 }
 
-// One CTA's share of the attention: the body of the attention kernel, and the
-// last phase of the one-launch decode step.  FUSED: the index lists and counts
-// were written earlier in the same launch; before any read of a row's list
-// the CTA waits (bounded) until row_ready[r] == epoch, and lists are read
-// through L2 (no read-only path).  Otherwise the lists come from a finished
-// launch and the CTA waits for it through programmatic dependent launch.
-template <int D, int MODE, bool FUSED>
+// One CTA's share of the attention (the body of the attention kernel).
+template <int D, int MODE>
 __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensorMap &vmap,
-                                         const AttnDev &p, uint8_t *smem_raw,
-                                         const uint32_t *row_ready = nullptr,
-                                         uint32_t epoch = 0u) {
+                                         const AttnDev &p, uint8_t *smem_raw) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
   constexpr int KT = C::kKT;
@@ -245,22 +230,9 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
   }
-  if (FUSED) {
-    if (tid == 0) {  // every row this CTA touches has its list
-      for (int r = r_first; r <= r_last; ++r) {
-        if (!wait_flag_eq(row_ready + r, epoch)) {
-          *abort_flag = 1u;
-          flag_status(a.status, KSA_FLAG_WAIT_TIMEOUT);
-          break;
-        }
-      }
-    }
-  } else {
-    pdl_wait();
-    pdl_launch_dependents();
-  }
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
-  if (FUSED && *abort_flag != 0u) return;  // nothing was issued yet
 
   int issued = 0;  // stages the producer filled (TMA modes: uses of the lane's own buffer)
 
@@ -279,7 +251,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
         int r = r_first;
         long long rv0 = static_cast<long long>(r) * p.V;
         RowGeom rg = row_geom(p, r);
-        RowInfo ri = row_info<MODE, FUSED>(a, r, rg.b, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
+        RowInfo ri = row_info<MODE>(a, r, rg.b, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
         int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
         int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
         int cnt = jb > ja ? jb - ja : 0;
@@ -290,7 +262,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
             if (++r > r_last) break;
             rv0 = static_cast<long long>(r) * p.V;
             rg = row_geom(p, r);
-            ri = row_info<MODE, FUSED>(a, r, rg.b, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
+            ri = row_info<MODE>(a, r, rg.b, (lane == 0 && rv0 >= s0) ? a.status : nullptr);
             ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
             jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
             cnt = jb > ja ? jb - ja : 0;
@@ -314,7 +286,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
               const int part = (tpi >= kStageTok) ? j % spe : 0;
               // read the entry without waiting for the count (any e < cap is in
               // bounds): one dependent round trip fewer per row
-              const int id_any = e < a.cap ? ld_list<FUSED>(ri.list + e) : -1;
+              const int id_any = e < a.cap ? __ldg(ri.list + e) : -1;
               const int id = e < ri.n_idx ? id_any : -1;
               ok = e < ri.n_idx && id >= 0;
               t0[u] = static_cast<long long>(id) * tpi + static_cast<long long>(part) * kStageTok;
@@ -368,7 +340,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
         const long long rv0 = static_cast<long long>(r) * p.V;
         const bool reporter = lane == 0 && rv0 >= s0;
         const RowGeom rg = row_geom(p, r);
-        const RowInfo ri = row_info<MODE, FUSED>(a, r, rg.b, reporter ? a.status : nullptr);
+        const RowInfo ri = row_info<MODE>(a, r, rg.b, reporter ? a.status : nullptr);
         const int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
         const int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
         const int eps = kStageTok / tpi;  // entries per stage
@@ -376,9 +348,9 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
         if (ja < jb) {
           wbase = (ja * eps) & ~31;
           // entries are read before the count is known (any index < cap is in bounds)
-          const int c0 = (wbase + lane < a.cap) ? ld_list<FUSED>(ri.list + wbase + lane) : -1;
+          const int c0 = (wbase + lane < a.cap) ? ri.list[wbase + lane] : -1;
           const int c1 =
-              (wbase + 32 + lane < a.cap) ? ld_list<FUSED>(ri.list + wbase + 32 + lane) : -1;
+              (wbase + 32 + lane < a.cap) ? ri.list[wbase + 32 + lane] : -1;
           cur = (wbase + lane < ri.n_idx) ? c0 : -1;
           nxt = (wbase + 32 + lane < ri.n_idx) ? c1 : -1;
         }
@@ -400,7 +372,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
           if (j * eps >= wbase + 32) {  // stages advance by at most one window
             wbase += 32;
             cur = nxt;
-            nxt = (wbase + 32 + lane < ri.n_idx) ? ld_list<FUSED>(ri.list + wbase + 32 + lane) : -1;
+            nxt = (wbase + 32 + lane < ri.n_idx) ? ri.list[wbase + 32 + lane] : -1;
           }
           const int e = j * eps + lane / tpi;
           const int id = __shfl_sync(0xffffffffu, cur, (e - wbase) & 31);
@@ -459,7 +431,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
     for (int r = r_first; r <= r_last; ++r) {
       const RowGeom rg = row_geom(p, r);
       const long long rv0 = static_cast<long long>(r) * p.V;
-      const RowInfo ri = row_info<MODE, FUSED>(a, r, rg.b, nullptr);
+      const RowInfo ri = row_info<MODE>(a, r, rg.b, nullptr);
       const int ja = static_cast<int>((s0 > rv0 ? s0 : rv0) - rv0);
       const int jb = min(static_cast<int>((s1 < rv0 + p.V ? s1 : rv0 + p.V) - rv0), ri.n_st);
       const int cnt = jb > ja ? jb - ja : 0;

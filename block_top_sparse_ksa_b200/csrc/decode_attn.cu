@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
     sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap,
                               const __grid_constant__ CUtensorMap vmap, const AttnDev p) {
   extern __shared__ uint8_t smem_raw[];
-  attn_cta<D, MODE, false>(kmap, vmap, p, smem_raw);
+  attn_cta<D, MODE>(kmap, vmap, p, smem_raw);
 }
 
 template <int D, int MODE>

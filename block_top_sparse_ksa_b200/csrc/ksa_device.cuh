@@ -82,62 +82,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // ---------------------------------------------------------------------------
-// flags between CTAs of one launch (GPU scope)
-
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Waits until *flag == want (acquire); false once kWaitTimeoutNs have passed.
-__device__ __forceinline__ bool wait_flag_eq(const uint32_t *flag, uint32_t want) {
-  if (ld_acquire_gpu(flag) == want) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (ld_acquire_gpu(flag) != want) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
-    __nanosleep(64);
-  }
-  return true;
-}
-
-// Barrier over every CTA of a cooperative launch (all of them resident, so
-// every CTA reaches it).  words[0] counts arrivals and words[1] is the
-// generation; both sit in the caller's workspace, zero-filled once, and the
-// last arrival resets the count, so they serve the next launch as they are.
-// Every thread returns true with *epoch = the new generation (never 0; the
-// same in every CTA), which tags this launch's flags apart from earlier
-// launches'.  False (with KSA_FLAG_WAIT_TIMEOUT) if the bounded wait gave up.
-__device__ __forceinline__ bool grid_barrier(uint32_t *words, uint32_t *status, uint32_t *epoch) {
-  __shared__ uint32_t s_epoch;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t gen = ld_acquire_gpu(words + 1);  // read before arriving
-    const uint32_t next = gen + 1u == 0u ? 1u : gen + 1u;
-    const uint32_t nblocks = gridDim.x * gridDim.y * gridDim.z;
-    __threadfence();  // this CTA's writes (ordered before by the barrier above) first
-    uint32_t out = next;
-    if (atomicAdd(words, 1u) == nblocks - 1u) {
-      atomicExch(words, 0u);
-      __threadfence();
-      st_release_gpu(words + 1, next);
-    } else if (!wait_flag_eq(words + 1, next)) {
-      flag_status(status, KSA_FLAG_WAIT_TIMEOUT);
-      out = 0u;
-    }
-    __threadfence();
-    s_epoch = out;
-  }
-  __syncthreads();
-  *epoch = s_epoch;
-  return s_epoch != 0u;
-}
-
-// ---------------------------------------------------------------------------
 // programmatic dependent launch
 //
 // A kernel reads no input before pdl_wait(), which returns once the previous

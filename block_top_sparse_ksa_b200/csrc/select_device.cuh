@@ -1,6 +1,4 @@
-// select_device.cuh -- device pieces of block scoring and top-k selection,
-// shared by the two-launch selection (select_blocks.cu) and the one-launch
-// decode step (decode_step.cu).
+// select_device.cuh -- device pieces of block scoring and top-k selection.
 //
 // Kinetics (block top-k section): every block's mean key is scored against
 // the query and the K' most relevant blocks are kept.  Reading of the
@@ -44,116 +42,6 @@ static __device__ __forceinline__ Piece piece_of(const ScoreDev &p, long long u,
   return x;
 }
 
-// Work partition of the scoring.  Only rows with more than k blocks are scored,
-// in pieces of prow blocks, so row (b, g) has P_b = ceil(NB_b / prow) pieces (0
-// if NB_b <= k), the same for every kv-head g of batch row b.  The scoring
-// warps take equal slices of the sequence of these pieces, rows in order, so
-// every warp streams the same number of bytes whatever the mix of lengths.
-// A warp locates its slice from the batch rows' lengths held in its lanes'
-// registers (lane l: rows l, l + 32, ...), which bounds B by kWalkMaxRows; for
-// larger batches each row is padded to the longest row's pieces instead.
-constexpr int kWalkMaxRows = 512;
-constexpr int kWalkPerLane = kWalkMaxRows / 32;
-
-static __device__ __forceinline__ int pieces_of_row(const ScoreDev &p, int L) {
-  const int nb = (L + p.a.bs - 1) / p.a.bs;
-  return nb > p.a.k ? (nb + p.prow - 1) / p.prow : 0;
-}
-
-struct PieceWalk {
-  long long total;  // pieces in the sequence
-  int b, g, piece;  // the cursor
-  int pb, L;        // pieces and length of batch row b
-  bool compact;     // false: the padded layout (rows * p.pieces units)
-};
-
-// Total pieces of the sequence (warp-uniform; every lane calls it).
-static __device__ __forceinline__ PieceWalk walk_begin(const ScoreDev &p, int (&pcs)[kWalkPerLane]) {
-  PieceWalk w;
-  const int lane = threadIdx.x & 31;
-  const SelectArgs &a = p.a;
-  w.compact = a.B <= kWalkMaxRows;
-  if (!w.compact) {
-    w.total = p.units;
-    return w;
-  }
-  int sum = 0;
-#pragma unroll
-  for (int i = 0; i < kWalkPerLane; ++i) {
-    const int b = lane + 32 * i;
-    pcs[i] = b < a.B ? pieces_of_row(p, clamp_len(a.seq_lens[b], a.T, nullptr)) : 0;
-    sum += pcs[i];
-  }
-  w.total = static_cast<long long>(__reduce_add_sync(0xffffffffu, sum)) * a.Hkv;
-  return w;
-}
-
-// Moves the cursor to unit u0 < w.total of the compact sequence.
-static __device__ __forceinline__ void walk_seek(const ScoreDev &p, PieceWalk &w,
-                                                 const int (&pcs)[kWalkPerLane], long long u0) {
-  const int lane = threadIdx.x & 31;
-  const SelectArgs &a = p.a;
-  long long before = 0;  // pieces of the batch rows below the current chunk of 32
-  int fb = 0, fpb = 1, foff = 0;
-  bool found = false;
-#pragma unroll
-  for (int i = 0; i < kWalkPerLane; ++i) {
-    const int mine = pcs[i] * a.Hkv;
-    int incl = mine;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const int chunk = __shfl_sync(0xffffffffu, incl, 31);
-    const unsigned hit = __ballot_sync(0xffffffffu, before + incl > u0);
-    const int src = hit != 0u ? __ffs(hit) - 1 : 0;
-    const int at_incl = __shfl_sync(0xffffffffu, incl, src);
-    const int at_mine = __shfl_sync(0xffffffffu, mine, src);
-    const int at_pcs = __shfl_sync(0xffffffffu, pcs[i], src);
-    if (!found && hit != 0u) {
-      found = true;
-      fb = 32 * i + src;
-      fpb = at_pcs;
-      foff = static_cast<int>(u0 - before) - (at_incl - at_mine);
-    }
-    before += chunk;
-  }
-  w.b = fb;
-  w.pb = fpb;
-  w.g = foff / fpb;
-  w.piece = foff - w.g * fpb;
-  w.L = clamp_len(a.seq_lens[fb], a.T, nullptr);
-}
-
-// The piece under the cursor (then advances it).  Padded layout: unit u.
-static __device__ __forceinline__ Piece walk_next(const ScoreDev &p, PieceWalk &w, long long u) {
-  if (!w.compact) return piece_of(p, u);
-  const SelectArgs &a = p.a;
-  Piece x;
-  x.b = w.b;
-  x.g = w.g;
-  x.row = w.b * a.Hkv + w.g;
-  x.L = w.L;
-  x.nb = (w.L + a.bs - 1) / a.bs;
-  x.j0 = w.piece * p.prow;
-  x.n = min(p.prow, x.nb - x.j0);
-  if (++w.piece == w.pb) {
-    w.piece = 0;
-    if (++w.g == a.Hkv) {
-      w.g = 0;
-      do {  // the next batch row that has pieces (the slice ends before running out)
-        if (++w.b >= a.B) break;
-        w.L = clamp_len(a.seq_lens[w.b], a.T, nullptr);
-        w.pb = pieces_of_row(p, w.L);
-      } while (w.pb == 0);
-    }
-  }
-  return x;
-}
-
-// `report`: flag an out-of-range sequence length in the status word (once per row).
-
 // Re-averages block nb-1 of `row` from K and stores it in the summaries.
 // Lanes l < D/8 get dims [8 (l % (D/8)), +8) in mean[] and return true.
 // One whole warp.
@@ -185,27 +73,38 @@ __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const ui
 // for reductions and broadcasts.
 template <int NT, int KPL>
 __host__ __device__ constexpr int fast_topk_words() {
-  return 1024 + 2 * ((NT * KPL + 31) / 32) + 64;
+  return 1024 + 2 * ((NT * KPL + 31) / 32) + 64;  // misc: 8 + 3 * (NT / 32) <= 64 words
+}
+
+// The score an order-preserving key stands for (score_key's inverse); the key
+// of a NaN score (0) gives -inf.
+__device__ __forceinline__ float key_score(uint32_t key) {
+  if (key == 0u) return -INFINITY;
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // Exact top-k of one row's n (k < n <= NT KPL) uint32 score keys by a CTA of
 // NT threads (all of them call it), the keys in registers: thread t holds
-// blocks t, t + NT, t + 2 NT, ...  Selection by shrinking key ranges: the live
-// keys span [lo, hi]; a pass drops them into 1024 buckets of width 2^s
-// ((hi - lo) >> s < 1024), the bucket holding the k-th largest live key is
-// found from a histogram, keys in higher buckets are selected, in lower ones
-// dropped, and the bucket's keys stay live with a range 1024 times narrower.
-// Done when the live keys are exactly the ones still needed (usually after two
-// passes on continuous scores), or all equal: then the lowest-index ones are
-// taken (ties go to the lower block).  At most four passes.  The winners are
-// written to out[0..k) in ascending block order through a bitmap of the
-// selection and one prefix count over its words.  `sm`: fast_topk_words words
-// of shared memory, 16-byte aligned.
+// blocks t, t + NT, t + 2 NT, ...  Selection by shrinking ranges: a pass drops
+// the live keys into 1024 buckets, the bucket holding the k-th largest live
+// key is found from a histogram, keys in higher buckets are selected, in lower
+// ones dropped, and the bucket's keys stay live.  The first pass buckets by
+// score value over [min, max] (linear in the score, so continuous scores
+// spread over many buckets and the boundary one holds a few); later passes
+// bucket the live keys' range [lo, hi] by key bits, 2^s wide ((hi - lo) >> s <
+// 1024), each 1024 times narrower.  Every bucket map is monotone in the key,
+// so a higher bucket means a higher score.  Done when the live keys are
+// exactly the ones still needed (usually after two passes), or all equal: then
+// the lowest-index ones are taken (ties go to the lower block).  At most five
+// passes.  The winners are written to out[0..k) in ascending block order
+// through a bitmap of the selection and one prefix count over its words.
+// `sm`: fast_topk_words words of shared memory, 16-byte aligned.
 template <int NT, int KPL>
 __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, int32_t *out,
                                           uint32_t *sm) {
   static_assert(NT % 32 == 0 && NT >= 64 && NT <= 1024, "whole warps");
   static_assert(KPL >= 1 && KPL <= 64, "a 64-bit slot mask per thread");
+  static_assert(8 + 3 * (NT / 32) <= 64, "the reduction words fit in misc");
   constexpr int NW = NT / 32;
   constexpr int W = (NT * KPL + 31) / 32;  // bitmap words; block j is bit j % 32 of word j / 32
   uint32_t *hist = sm;
@@ -215,7 +114,7 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t key[KPL];
   uint64_t live = 0ull, sel = 0ull;
-  uint32_t lo = 0xffffffffu, hi = 0u;
+  uint32_t lo = 0xffffffffu, hi = 0u, lo_real = 0xffffffffu;  // lo_real: over keys of real scores
 #pragma unroll
   for (int e = 0; e < KPL; ++e) {
     const int j = tid + NT * e;
@@ -224,6 +123,7 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
       live |= 1ull << e;
       lo = min(lo, key[e]);
       hi = max(hi, key[e]);
+      if (key[e] != 0u) lo_real = min(lo_real, key[e]);
     }
   }
   uint32_t remaining = static_cast<uint32_t>(k);  // winners still to find among the live keys
@@ -231,26 +131,43 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     // range of the live keys, block-wide
     lo = __reduce_min_sync(0xffffffffu, lo);
     hi = __reduce_max_sync(0xffffffffu, hi);
+    if (pass == 0) lo_real = __reduce_min_sync(0xffffffffu, lo_real);
     if (lane == 0) {
       misc[8 + warp] = lo;
       misc[8 + NW + warp] = hi;
+      misc[8 + 2 * NW + warp] = lo_real;
     }
     __syncthreads();
     lo = misc[8];
     hi = misc[8 + NW];
+    if (pass == 0) lo_real = misc[8 + 2 * NW];
 #pragma unroll
     for (int w = 1; w < NW; ++w) {
       lo = min(lo, misc[8 + w]);
       hi = max(hi, misc[8 + NW + w]);
+      if (pass == 0) lo_real = min(lo_real, misc[8 + 2 * NW + w]);
     }
-    if (lo == hi || pass == 4) break;  // all live keys equal: the index rule decides
+    if (lo == hi || pass == 5) break;  // all live keys equal: the index rule decides
+    // pass 0 by score value when the real scores span a finite, non-empty range
+    const float v0 = key_score(lo_real), v1 = key_score(hi);
+    const float vscale = 1024.f / (v1 - v0);
+    const bool by_value = pass == 0 && lo_real < hi && isfinite(vscale) && vscale > 0.f;
     const int bits = 32 - __clz(hi - lo);
     const int sh = bits > 10 ? bits - 10 : 0;
     for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
     __syncthreads();
 #pragma unroll
-    for (int e = 0; e < KPL; ++e)
-      if ((live >> e) & 1ull) atomicAdd(&hist[(key[e] - lo) >> sh], 1u);
+    for (int e = 0; e < KPL; ++e) {
+      if (!((live >> e) & 1ull)) continue;
+      uint32_t bk;
+      if (by_value) {  // NaN keys (0) and the lowest scores share bucket 0
+        const float f = (key_score(key[e]) - v0) * vscale;
+        bk = key[e] == 0u ? 0u : static_cast<uint32_t>(fminf(fmaxf(f, 0.f), 1023.f));
+      } else {
+        bk = (key[e] - lo) >> sh;
+      }
+      atomicAdd(&hist[bk], 1u);
+    }
     __syncthreads();
     if (warp == 0) {  // lane l owns buckets [32 l, 32 l + 32); count from the top down
       uint32_t c[32];
@@ -292,7 +209,13 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
 #pragma unroll
     for (int e = 0; e < KPL; ++e) {
       if (!((live >> e) & 1ull)) continue;
-      const uint32_t bk = (key[e] - base) >> sh;
+      uint32_t bk;
+      if (by_value) {
+        const float f = (key_score(key[e]) - v0) * vscale;
+        bk = key[e] == 0u ? 0u : static_cast<uint32_t>(fminf(fmaxf(f, 0.f), 1023.f));
+      } else {
+        bk = (key[e] - base) >> sh;
+      }
       if (bk > bstar || (bk == bstar && exact)) {
         sel |= 1ull << e;
         live &= ~(1ull << e);

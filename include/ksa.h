@@ -255,22 +255,19 @@ ksa_status ksa_decode_select_blocks_paged(const ksa_shape *shape, const uint16_t
 /*
  * The decode step in one call [KIN s.5: keep the block representation
  * current, score every block against the query, keep the K' best, attend
- * over their tokens]: the results of ksa_decode_select_blocks_ex followed by
+ * over their tokens]: ksa_decode_select_blocks_ex followed by
  * ksa_sparse_decode_attn over its block lists (tokens_per_idx = block_size,
- * KSA_IDX_PER_KV_HEAD), bit for bit.  When ceil(T/bs) <= 2048 the step runs
- * as one cooperative launch: its CTAs are all resident and wait for one
- * another inside the launch (every wait bounded; on expiry
- * KSA_FLAG_WAIT_TIMEOUT is set and the results are invalid).  Longer rows,
- * or a device with no room for that grid, run as the two calls' launches.
+ * KSA_IDX_PER_KV_HEAD), issued from one call on one workspace -- the same
+ * launches, so the same results bit for bit.
  *   q, K, V, summaries, summary_dtype, seq_lens, k_blocks: as
  *              ksa_decode_select_blocks_ex (the summary of each row's last
  *              block is refreshed from K and written back)
  *   block_idx: [B, Hkv, k_blocks] int32 and num_sel [B, Hkv] (written)
  *   scale, out_dtype, out, lse: as ksa_sparse_decode_attn
- *   ws:        ksa_decode_step_workspace() bytes, 256-byte aligned.  Zero-fill
- *              it once after allocating it; each call leaves it ready for the
- *              next (the per-row flags it keeps carry a per-call tag).  Calls
- *              that may run concurrently need separate workspaces.
+ *   ws:        ksa_decode_step_workspace() bytes, 256-byte aligned: the
+ *              selection workspace followed by the attention workspace, with
+ *              their rules (zero-fill once; calls that may run concurrently
+ *              need separate workspaces).
  * Limits and errors: those of both calls.
  */
 size_t ksa_decode_step_workspace(const ksa_shape *shape, int32_t k_blocks);

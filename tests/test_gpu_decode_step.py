@@ -1,11 +1,9 @@
 """ksa_decode_step: one decode step in one call -- the last-block summary refresh, block
 scoring, top-k and attention over the kept blocks (Kinetics press summary, section 5:
-block top-k).  For rows of up to 2048 blocks it is one cooperative launch whose CTAs wait
-for one another; beyond that it runs the two calls' launches.  Either way its results must
-equal those of ksa_decode_select_blocks followed by ksa_sparse_decode_attn bit for bit:
-the same pieces are scored with the same arithmetic, the top-k is exact with the same tie
-rule, and the attention runs the same partition and pipeline on the same grid.  (Parity
-with the oracle is in test_gpu_parity.py.)"""
+block top-k), issued as the launches of ksa_decode_select_blocks followed by
+ksa_sparse_decode_attn on one workspace.  Its results must equal the two calls' bit for
+bit, on repeated calls over one workspace too.  (Parity with the oracle is in
+test_gpu_parity.py.)"""
 import numpy as np
 import pytest
 import torch
@@ -72,10 +70,10 @@ CASES = [
     (3, 8, 2, 128, 40 * 16 + 7, 16, 8, torch.float32, 0),     # ragged capacity
     (4, 16, 8, 128, 4096, 32, 16, torch.float32, 0),          # the Qwen3-0.6B layout, short
     (3, 8, 4, 64, 2048, 16, 40, torch.float32, 1),            # D 64, bf16 output
-    (5, 32, 8, 128, 32768, 16, 128, torch.float32, 0),        # 2048 blocks: 64 keys per lane
+    (5, 32, 8, 128, 32768, 16, 128, torch.float32, 0),        # 2048 blocks
     (3, 16, 8, 128, 8192, 32, 32, torch.bfloat16, 0),         # bf16 summaries
-    (3, 8, 2, 128, 1100 * 16, 16, 50, torch.float32, 0),      # 1100 blocks, one warp per row
-    (2, 8, 2, 128, 3000 * 16, 16, 64, torch.float32, 0),      # 3000 blocks: two launches
+    (3, 8, 2, 128, 1100 * 16, 16, 50, torch.float32, 0),      # 1100 blocks
+    (2, 8, 2, 128, 3000 * 16, 16, 64, torch.float32, 0),      # 3000 blocks
     (4, 8, 2, 128, 512, 16, 64, torch.float32, 0),            # k covers every block
     (64, 16, 8, 128, 16384, 32, 32, torch.float32, 0),        # Qwen3-0.6B step shape
 ]
@@ -103,8 +101,8 @@ def test_decode_step_equals_the_two_calls(ksa, B, Hq, Hkv, D, T, bs, k, sdt, odt
 
 def test_decode_step_repeated_calls_on_one_workspace(ksa):
     """Calls back to back on one workspace, alternating two query sets and two caches: each
-    result equals the first result for its inputs (the flags a call leaves carry its own
-    tag, so a stale flag never releases a later call's attention early)."""
+    result equals the first result for its inputs (every call leaves the workspace's
+    semaphores as it found them)."""
     B, Hq, Hkv, D, T, bs, k = 16, 32, 8, 128, 16384, 16, 64
     qa, Ka, Va, la = _inputs(B, Hq, Hkv, D, T, bs, seed=1)
     qb, Kb, Vb, lb = _inputs(B, Hq, Hkv, D, T, bs, seed=2)
