@@ -99,9 +99,14 @@ __device__ __forceinline__ float key_score(uint32_t key) {
 // passes.  The winners are written to out[0..k) in ascending block order
 // through a bitmap of the selection and one prefix count over its words.
 // `sm`: fast_topk_words words of shared memory, 16-byte aligned.
-template <int NT, int KPL>
+//
+// kValuePass = false: the keys are plain unsigned ranks (vote counts), not
+// score keys, and every pass buckets by key bits.  bits_out non-null: instead
+// of the list, the selection is written as a bit set, bit j % 32 of word j / 32
+// for j < n (the words of [0, n) only).
+template <int NT, int KPL, bool kValuePass = true>
 __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, int32_t *out,
-                                          uint32_t *sm) {
+                                          uint32_t *sm, uint32_t *bits_out = nullptr) {
   static_assert(NT % 32 == 0 && NT >= 64 && NT <= 1024, "whole warps");
   static_assert(KPL >= 1 && KPL <= 64, "a 64-bit slot mask per thread");
   static_assert(8 + 3 * (NT / 32) <= 64, "the reduction words fit in misc");
@@ -151,7 +156,8 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     // pass 0 by score value when the real scores span a finite, non-empty range
     const float v0 = key_score(lo_real), v1 = key_score(hi);
     const float vscale = 1024.f / (v1 - v0);
-    const bool by_value = pass == 0 && lo_real < hi && isfinite(vscale) && vscale > 0.f;
+    const bool by_value =
+        kValuePass && pass == 0 && lo_real < hi && isfinite(vscale) && vscale > 0.f;
     const int bits = 32 - __clz(hi - lo);
     const int sh = bits > 10 ? bits - 10 : 0;
     for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
@@ -170,15 +176,10 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     }
     __syncthreads();
     if (warp == 0) {  // lane l owns buckets [32 l, 32 l + 32); count from the top down
-      uint32_t c[32];
       uint32_t tot = 0u;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const uint4 v = reinterpret_cast<const uint4 *>(hist + 32 * lane)[q];
-        c[4 * q] = v.x;
-        c[4 * q + 1] = v.y;
-        c[4 * q + 2] = v.z;
-        c[4 * q + 3] = v.w;
         tot += v.x + v.y + v.z + v.w;
       }
       uint32_t incl = tot;  // keys in the buckets of lanes >= this one
@@ -188,14 +189,16 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
         if (lane + off < 32) incl += y;
       }
       uint32_t run = incl - tot;
-#pragma unroll
-      for (int b = 31; b >= 0; --b) {
-        const uint32_t before = run;
-        run += c[b];
-        if (before < remaining && run >= remaining) {
-          misc[0] = static_cast<uint32_t>(32 * lane + b);
-          misc[1] = before;
-          misc[2] = c[b];
+      if (run < remaining && incl >= remaining) {  // the one lane holding the k-th key
+        for (int b = 31; b >= 0; --b) {
+          const uint32_t before = run, c = hist[32 * lane + b];
+          run += c;
+          if (run >= remaining) {
+            misc[0] = static_cast<uint32_t>(32 * lane + b);
+            misc[1] = before;
+            misc[2] = c;
+            break;
+          }
         }
       }
     }
@@ -245,17 +248,12 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
   __syncthreads();
   if (warp == 0) {
     // lane l owns words [WPL l, WPL l + WPL): the lowest-index `remaining` live keys join the
-    // selection, then every winner gets its place from a prefix count of the words
+    // selection (written back into selw), then every winner gets its place from a prefix
+    // count of the words
     constexpr int WPL = (W + 31) / 32;
-    uint32_t wl[WPL], ws[WPL];
+    const int w0 = lane * WPL, w1 = min(w0 + WPL, W);
     uint32_t nl = 0u;
-#pragma unroll
-    for (int q = 0; q < WPL; ++q) {
-      const int w = lane * WPL + q;
-      wl[q] = w < W ? livew[w] : 0u;
-      ws[q] = w < W ? selw[w] : 0u;
-      nl += __popc(wl[q]);
-    }
+    for (int w = w0; w < w1; ++w) nl += __popc(livew[w]);
     uint32_t pl = nl;  // inclusive prefix of live bits over the lanes
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -264,9 +262,8 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     }
     pl -= nl;
     uint32_t ns = 0u;
-#pragma unroll
-    for (int q = 0; q < WPL; ++q) {
-      uint32_t take = 0u, x = wl[q];
+    for (int w = w0; w < w1; ++w) {
+      uint32_t take = 0u, x = livew[w];
       while (x != 0u && pl < remaining) {  // lowest set bits first: ascending blocks
         const uint32_t b = x & (0u - x);
         take |= b;
@@ -274,8 +271,14 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
         ++pl;
       }
       pl += __popc(x);
-      ws[q] |= take;
-      ns += __popc(ws[q]);
+      const uint32_t sw = selw[w] | take;
+      selw[w] = sw;
+      ns += __popc(sw);
+    }
+    if (bits_out != nullptr) {
+      const int nwords = (n + 31) / 32;
+      for (int w = w0; w < w1 && w < nwords; ++w) bits_out[w] = selw[w];
+      return;
     }
     uint32_t ps = ns;
 #pragma unroll
@@ -284,13 +287,12 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
       if (lane >= off) ps += y;
     }
     ps -= ns;
-#pragma unroll
-    for (int q = 0; q < WPL; ++q) {
-      uint32_t x = ws[q];
+    for (int w = w0; w < w1; ++w) {
+      uint32_t x = selw[w];
       while (x != 0u) {
         const int b = __ffs(x) - 1;
         x &= x - 1u;
-        out[ps++] = 32 * (lane * WPL + q) + b;
+        out[ps++] = 32 * w + b;
       }
     }
   }
