@@ -73,7 +73,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--batch", type=int, default=0,
                    help="override the per-GPU batch (small profiling cases only)")
-    p.add_argument("--summaries", choices=["f32", "bf16"], default="f32",
+    p.add_argument("--summaries", choices=["f32", "bf16", "fp8"], default="f32",
                    help="storage type of the block summaries (block workloads)")
     return p.parse_args()
 
@@ -181,10 +181,12 @@ def query_sets(shape, count, device):
     return synth.make_queries(shape, 5000, count, device, group_noise=noise)
 
 
-def algorithmic_bytes(shape, seq_lens, kind: str, summary_bytes: int = 4):
+def algorithmic_bytes(shape, seq_lens, kind: str, summary_bytes: int = 4,
+                      summary_extra: int = 0):
     """Per step: summaries read (when k < NB_b) + selected K/V + q + out (fp32).
     Also returns the attention kernel's share (selected K/V + q + out).
-    summary_bytes: 4 for fp32-stored summaries, 2 for bf16."""
+    summary_bytes: bytes per summary value (4 fp32, 2 bf16, 1 fp8); summary_extra: bytes
+    per block besides the values (4: the fp8 scale)."""
     bs, Hkv, Hq, D = shape.block_size, shape.num_kv_heads, shape.num_q_heads, shape.head_dim
     k = shape.k_blocks
     summ = kv = 0
@@ -194,7 +196,7 @@ def algorithmic_bytes(shape, seq_lens, kind: str, summary_bytes: int = 4):
             kv += Hkv * int(L) * D * 2 * 2
             continue
         if k < nb:
-            summ += Hkv * nb * D * summary_bytes
+            summ += Hkv * nb * (D * summary_bytes + summary_extra)
         kv += Hkv * min(k * bs, int(L)) * D * 2 * 2
     qo = len(seq_lens) * Hq * D * (2 + 4)
     return summ + kv + qo, kv + qo, summ
@@ -370,7 +372,7 @@ class BlockWorkload:
         self.inp = make_block_inputs(sh, dev)
         self.nq = 16
         self.qs = query_sets(sh, self.nq, dev)
-        sdt = torch.bfloat16 if summaries == "bf16" else torch.float32
+        sdt = {"bf16": torch.bfloat16, "fp8": "fp8"}.get(summaries, torch.float32)
         B, Hq, Hkv, D, T, bs, k = (sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim,
                                    sh.capacity, sh.block_size, sh.k_blocks)
         self.S = ksa.ksa_build_block_summaries(self.inp.K, self.inp.seq_lens, bs,
@@ -443,7 +445,8 @@ def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
     t_att = times[-1]
     t_sel = times[0] if kind != "dense" else 0.0
     lens = wl.inp.seq_lens.cpu().tolist()
-    total_b, attn_b, summ_b = algorithmic_bytes(sh, lens, kind, wl.S.element_size())
+    total_b, attn_b, summ_b = algorithmic_bytes(sh, lens, kind, wl.S.element_size(),
+                                                4 if wl.S.dtype == torch.uint8 else 0)
     per_step_s = ms_step / 1e3
     attn_gbs = attn_b / (t_att * 1e-3) / 1e9
     return {
@@ -471,7 +474,8 @@ def measure_block(wl: BlockWorkload, args, dist, peak: float, peak_kind: str,
                    "seq_lens": ([sh.min_len, sh.max_len] if sh.min_len != sh.max_len
                                 else sh.max_len),
                    "k_blocks": sh.k_blocks if kind != "dense" else "all",
-                   "summaries": "bf16" if wl.S.dtype == torch.bfloat16 else "f32",
+                   "summaries": {torch.bfloat16: "bf16", torch.uint8: "fp8 e4m3 + fp32 "
+                                 "scale per block"}.get(wl.S.dtype, "f32"),
                    "l2": "inputs larger than L2: K/V cache %.1f GB, %.0f MB read per step, %d "
                          "rotating query sets" % (2 * wl.inp.K.numel() * 2 / 1e9, total_b / 1e6,
                                                   wl.nq),
@@ -523,18 +527,20 @@ def run_extra(args, dist, dev):
     return out
 
 
-def prefill_bytes(shape, seq_lens, summary_bytes: int = 4) -> int:
+def prefill_bytes(shape, seq_lens, summary_bytes: int = 4, summary_extra: int = 0) -> int:
     """The prefill's summary build (every block of every row): one read of the keys and one
-    write of the block means."""
+    write of the block means (summary_extra: bytes per block besides the values)."""
     bs, Hkv, D = shape.block_size, shape.num_kv_heads, shape.head_dim
-    return sum(Hkv * int(L) * D * 2 + Hkv * (-(-int(L) // bs)) * D * summary_bytes
+    return sum(Hkv * int(L) * D * 2 +
+               Hkv * (-(-int(L) // bs)) * (D * summary_bytes + summary_extra)
                for L in seq_lens)
 
 
 def time_prefill(ksa, inp, shape, S, stream, peak, reps: int = 5):
     """ksa_build_block_summaries (mode ALL) over the whole cache, timed alone with CUDA events
     (the cache is larger than L2, so the repetitions read from HBM)."""
-    S2 = torch.empty_like(S)
+    fp8 = S.dtype == torch.uint8
+    S2 = ksa.alloc_summaries(*S.shape, "fp8" if fp8 else S.dtype, S.device)
     ksa.ksa_build_block_summaries(inp.K, inp.seq_lens, shape.block_size, summaries=S2,
                                   stream=stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -546,7 +552,7 @@ def time_prefill(ksa, inp, shape, S, stream, peak, reps: int = 5):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
-    b = prefill_bytes(shape, inp.seq_lens.cpu().tolist(), S.element_size())
+    b = prefill_bytes(shape, inp.seq_lens.cpu().tolist(), S.element_size(), 4 if fp8 else 0)
     return {"kernel": "block_summaries (mode ALL)", "ms": ms, "bytes": b,
             "gbs": b / (ms * 1e-3) / 1e9, "frac": b / (ms * 1e-3) / 1e9 / peak}
 

@@ -9,7 +9,10 @@ an error that says how to build it.
 
 Layouts (row-major, contiguous):
   q [B, Hq, D] bf16;  K, V [B, Hkv, T, D] bf16;  seq_lens [B] int32;
-  summaries [B, Hkv, ceil(T/bs), D] fp32;  block_idx [B, Hkv, k] int32.
+  summaries [B, Hkv, ceil(T/bs), D] fp32 or bf16, or fp8: a uint8 tensor of
+  that shape (the e4m3 values) whose storage holds the per-block fp32 scales
+  right after it (alloc_summaries, fp8_summary_scales);  block_idx [B, Hkv, k]
+  int32.
 """
 from __future__ import annotations
 
@@ -33,7 +36,8 @@ __all__ = [
     "ksa_select_tokens_one_head_workspace", "ksa_get_device_status", "IDX_PER_KV_HEAD",
     "IDX_SHARED", "IDX_PER_Q_HEAD", "ksa_append_kv", "ksa_append_kv_paged", "ksa_decode_step",
     "ksa_decode_step_workspace",
-    "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "OUT_F32", "OUT_BF16",
+    "SUMMARY_ALL", "SUMMARY_LAST_BLOCK", "SUMMARIES_F32", "SUMMARIES_BF16", "SUMMARIES_FP8",
+    "OUT_F32", "OUT_BF16", "alloc_summaries", "fp8_summary_scales",
     "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_INDEX_SKIPPED", "FLAG_NONFINITE_SCORE", "FLAG_WAIT_TIMEOUT",
 ]
@@ -42,7 +46,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libksa.so")
 
 SUMMARY_ALL, SUMMARY_LAST_BLOCK = 0, 1
-SUMMARIES_F32, SUMMARIES_BF16 = 0, 1
+SUMMARIES_F32, SUMMARIES_BF16, SUMMARIES_FP8 = 0, 1, 2
 IDX_PER_KV_HEAD, IDX_SHARED, IDX_PER_Q_HEAD = 0, 1, 2
 OUT_F32, OUT_BF16 = 0, 1
 FLAG_SEQ_LEN_CLAMPED, FLAG_INDEX_SKIPPED, FLAG_NONFINITE_SCORE, FLAG_WAIT_TIMEOUT = 1, 2, 4, 8
@@ -190,26 +194,62 @@ def _shape(B, Hq, Hkv, D, T, bs=16) -> Shape:
 
 
 def _summary_dtype(summaries: torch.Tensor) -> int:
-    """KSA_SUMMARIES_* code of a summaries tensor (fp32 or bf16)."""
+    """KSA_SUMMARIES_* code of a summaries tensor (fp32, bf16, or uint8 for fp8)."""
     if summaries.dtype == torch.float32:
         return SUMMARIES_F32
     if summaries.dtype == torch.bfloat16:
         return SUMMARIES_BF16
-    raise TypeError(f"summaries must be float32 or bfloat16, not {summaries.dtype}")
+    if summaries.dtype == torch.uint8:
+        room = summaries.untyped_storage().nbytes() - summaries.storage_offset()
+        if summaries.dim() != 4 or room < summaries.numel() * (summaries.shape[-1] + 4) // (
+                summaries.shape[-1]):
+            raise ValueError("fp8 summaries: a [B, Hkv, nb, D] uint8 tensor whose storage holds "
+                             "B*Hkv*nb fp32 scales after it (see alloc_summaries)")
+        return SUMMARIES_FP8
+    raise TypeError(f"summaries must be float32, bfloat16 or uint8 (fp8), not {summaries.dtype}")
+
+
+def alloc_summaries(B: int, Hkv: int, nb: int, D: int, dtype="fp32", device="cuda",
+                    fill: Optional[float] = None) -> torch.Tensor:
+    """Block-summary storage [B, Hkv, nb, D]: dtype torch.float32 / "fp32", torch.bfloat16 /
+    "bf16", or "fp8" (uint8 e4m3 values, the nb fp32 scales per (row, kv-head) stored right
+    after them in the same allocation).  `fill`: an initial value for fp32/bf16 storage."""
+    if dtype in (torch.float32, "fp32", "f32"):
+        S = torch.empty((B, Hkv, nb, D), dtype=torch.float32, device=device)
+    elif dtype in (torch.bfloat16, "bf16"):
+        S = torch.empty((B, Hkv, nb, D), dtype=torch.bfloat16, device=device)
+    elif dtype == "fp8":
+        n = B * Hkv * nb
+        return torch.zeros((n * (D + 4),), dtype=torch.uint8, device=device)[:n * D].view(
+            B, Hkv, nb, D)
+    else:
+        raise ValueError(f"unknown summary dtype {dtype!r}")
+    if fill is not None:
+        S.fill_(fill)
+    return S
+
+
+def fp8_summary_scales(S: torch.Tensor) -> torch.Tensor:
+    """The per-block fp32 scales [B, Hkv, nb] stored after fp8 summaries S."""
+    B, Hkv, nb, D = S.shape
+    n = B * Hkv * nb
+    raw = torch.as_strided(S, (n * 4,), (1,), S.storage_offset() + S.numel())
+    return raw.view(torch.float32).view(B, Hkv, nb)
 
 
 def ksa_build_block_summaries(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
                               mode: int = SUMMARY_ALL, summaries: Optional[torch.Tensor] = None,
                               dev_status: Optional[torch.Tensor] = None, stream=None,
-                              summary_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+                              summary_dtype=torch.float32) -> torch.Tensor:
     """Block mean keys S [B, Hkv, ceil(T/bs), D] (all blocks, or the last one), stored as
-    fp32 or bf16: the given tensor's dtype, else `summary_dtype`."""
+    fp32, bf16 or fp8: the given tensor's type, else `summary_dtype` (torch.float32,
+    torch.bfloat16 or "fp8"; see alloc_summaries)."""
     _dev(K, "K", torch.bfloat16)
     _dev(seq_lens, "seq_lens", torch.int32)
     B, Hkv, T, D = K.shape
     nb = -(-T // block_size)
     if summaries is None:
-        summaries = torch.empty((B, Hkv, nb, D), dtype=summary_dtype, device=K.device)
+        summaries = alloc_summaries(B, Hkv, nb, D, summary_dtype, K.device)
     _dev(summaries, "summaries", summaries.dtype)
     sh = _shape(B, Hkv, Hkv, D, T, block_size)
     _check(lib().ksa_build_block_summaries_ex(
@@ -476,14 +516,14 @@ def ksa_build_block_summaries_paged(K_pages: torch.Tensor, block_table: torch.Te
                                     seq_lens: torch.Tensor, mode: int = SUMMARY_ALL,
                                     summaries: Optional[torch.Tensor] = None,
                                     dev_status: Optional[torch.Tensor] = None, stream=None,
-                                    summary_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+                                    summary_dtype=torch.float32) -> torch.Tensor:
     """ksa_build_block_summaries on a paged key cache; the page size is the block size."""
     _dev(K_pages, "K_pages", torch.bfloat16)
     _dev(seq_lens, "seq_lens", torch.int32)
     P, Hkv, bs, D = K_pages.shape
     B, mb = block_table.shape
     if summaries is None:
-        summaries = torch.empty((B, Hkv, mb, D), dtype=summary_dtype, device=K_pages.device)
+        summaries = alloc_summaries(B, Hkv, mb, D, summary_dtype, K_pages.device)
     _dev(summaries, "summaries", summaries.dtype)
     sh = _shape(B, Hkv, Hkv, D, mb * bs, bs)
     pg = _pages(block_table, P)

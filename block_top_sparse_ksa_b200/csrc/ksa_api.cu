@@ -199,8 +199,12 @@ ksa_status summaries_common(const ksa_shape *shape, const uint16_t *K, const ksa
     return fail(KSA_ERR_INVALID_ARG, "K, seq_lens and summaries must be non-NULL");
   if (mode != KSA_SUMMARY_ALL && mode != KSA_SUMMARY_LAST_BLOCK)
     return fail(KSA_ERR_INVALID_ARG, "mode %d is neither ALL nor LAST_BLOCK", mode);
-  if (summary_dtype != KSA_SUMMARIES_F32 && summary_dtype != KSA_SUMMARIES_BF16)
-    return fail(KSA_ERR_INVALID_ARG, "summary_dtype %d is neither F32 nor BF16", summary_dtype);
+  if (summary_dtype != KSA_SUMMARIES_F32 && summary_dtype != KSA_SUMMARIES_BF16 &&
+      summary_dtype != KSA_SUMMARIES_FP8)
+    return fail(KSA_ERR_INVALID_ARG, "summary_dtype %d is not F32, BF16 or FP8", summary_dtype);
+  if (summary_dtype == KSA_SUMMARIES_FP8 && shape->head_dim != 128)
+    return fail(KSA_ERR_UNSUPPORTED, "fp8 summaries need head_dim 128 (got %d)",
+                shape->head_dim);
   if (!aligned(K, 16) || !aligned(summaries, 16) || !aligned(seq_lens, 4))
     return fail(KSA_ERR_INVALID_ARG, "K and summaries must be 16-byte aligned");
   ksa::SummaryArgs a;
@@ -208,7 +212,7 @@ ksa_status summaries_common(const ksa_shape *shape, const uint16_t *K, const ksa
   a.K = K;
   a.seq_lens = seq_lens;
   a.S = summaries;
-  a.sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
+  a.sfmt = summary_dtype;
   a.status = dev_status;
   a.B = shape->batch;
   a.Hkv = shape->num_kv_heads;
@@ -310,8 +314,12 @@ ksa_status select_args(const ksa_shape *shape, const uint16_t *q, const ksa_page
   if (q == nullptr || summaries == nullptr || seq_lens == nullptr || block_idx == nullptr ||
       num_sel == nullptr)
     return fail(KSA_ERR_INVALID_ARG, "q, summaries, seq_lens, block_idx, num_sel must be non-NULL");
-  if (summary_dtype != KSA_SUMMARIES_F32 && summary_dtype != KSA_SUMMARIES_BF16)
-    return fail(KSA_ERR_INVALID_ARG, "summary_dtype %d is neither F32 nor BF16", summary_dtype);
+  if (summary_dtype != KSA_SUMMARIES_F32 && summary_dtype != KSA_SUMMARIES_BF16 &&
+      summary_dtype != KSA_SUMMARIES_FP8)
+    return fail(KSA_ERR_INVALID_ARG, "summary_dtype %d is not F32, BF16 or FP8", summary_dtype);
+  if (summary_dtype == KSA_SUMMARIES_FP8 && shape->head_dim != 128)
+    return fail(KSA_ERR_UNSUPPORTED, "fp8 summaries need head_dim 128 (got %d)",
+                shape->head_dim);
   if (k_blocks < 1) return fail(KSA_ERR_INVALID_ARG, "k_blocks must be >= 1 (got %d)", k_blocks);
   const int nb_max = (shape->capacity + shape->block_size - 1) / shape->block_size;
   if (nb_max > 16384)
@@ -321,7 +329,7 @@ ksa_status select_args(const ksa_shape *shape, const uint16_t *q, const ksa_page
   if (pages != nullptr && (st = check_pages(shape, pages, &a->kv)) != KSA_OK) return st;
   a->q = q;
   a->S = summaries;  // written only when K is given (the fused refresh)
-  a->sbf16 = summary_dtype == KSA_SUMMARIES_BF16 ? 1 : 0;
+  a->sfmt = summary_dtype;
   a->seq_lens = seq_lens;
   a->block_idx = block_idx;
   a->num_sel = num_sel;
@@ -402,7 +410,7 @@ ksa_status ksa_select_window(const ksa_shape *shape, const int32_t *seq_lens, in
   ksa::SelectArgs a;
   a.q = nullptr;
   a.S = nullptr;
-  a.sbf16 = 0;
+  a.sfmt = KSA_SUMMARIES_F32;
   a.seq_lens = seq_lens;
   a.block_idx = block_idx;
   a.num_sel = num_sel;

@@ -42,6 +42,34 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
   return static_cast<uint16_t>(pack_bf16x2(x, 0.f) & 0xffffu);
 }
 
+// Packs two fp32 values as fp8 e4m3 (round to nearest even, held at +-448):
+// `lo` in bits 0..7.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The two fp8 e4m3 values of `v` (bits 0..7 -> .x), exactly, as fp32.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  float lo, hi;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(static_cast<uint16_t>(h & 0xffffu)));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(static_cast<uint16_t>(h >> 16)));
+  return make_float2(lo, hi);
+}
+
+// Scale exponent of an fp8 block: the smallest e with amax <= 448 * 2^e (448 =
+// 0.875 * 2^9, so with amax = f 2^E, 0.5 <= f < 1: e = E - 9 if f <= 0.875,
+// else E - 8); 0 for an all-zero block.
+__device__ __forceinline__ int e4m3_scale_exp(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int E;
+  const float f = frexpf(amax, &E);
+  return f <= 0.875f ? E - 9 : E - 8;
+}
+
 // 2^x with the hardware approximation (relative error ~2^-22); -inf -> +0.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -292,12 +320,12 @@ __device__ __forceinline__ bool warp_block_mean(const uint16_t *rows, int n, flo
   return rp == 0;
 }
 
-// Stores dims [c8, c8 + 8) of a block mean at element offset `row` of the
-// summaries: fp32, or (sbf16) bf16 rounded to nearest even.  Every writer of
-// summaries goes through here, so all of them store the same bits.
-__device__ __forceinline__ void store_mean8(void *S, int sbf16, size_t row, int c8,
+// Stores dims [c8, c8 + 8) of a block mean at element offset `row` of fp32
+// summaries, or of bf16 ones (sfmt KSA_SUMMARIES_BF16: rounded to nearest
+// even).
+__device__ __forceinline__ void store_mean8(void *S, int sfmt, size_t row, int c8,
                                             const float (&m)[8]) {
-  if (sbf16) {
+  if (sfmt == KSA_SUMMARIES_BF16) {
     *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(S) + row + c8) =
         make_uint4(pack_bf16x2(m[0], m[1]), pack_bf16x2(m[2], m[3]), pack_bf16x2(m[4], m[5]),
                    pack_bf16x2(m[6], m[7]));
@@ -306,6 +334,53 @@ __device__ __forceinline__ void store_mean8(void *S, int sbf16, size_t row, int 
     dst[0] = make_float4(m[0], m[1], m[2], m[3]);
     dst[1] = make_float4(m[4], m[5], m[6], m[7]);
   }
+}
+
+// Stores the mean of block `blk` (flat index over the n_blocks blocks [B, Hkv,
+// ceil(T/bs)] of the summaries), held by the lanes l < D/8 (`mine`: dims
+// [8 (l % (D/8)), +8) in m[]).  Every writer of summaries goes through here,
+// so all of them store the same bits.  fp32 and bf16: per lane.  fp8: the
+// block's scale exponent e comes from the warp's largest |mean|, each lane
+// stores round_e4m3(m 2^-e) as 8 bytes and lane 0 the scale 2^e (the scales
+// follow the n_blocks * D value bytes).  All 32 lanes call it.
+template <int D, int FMT>
+__device__ __forceinline__ void store_block_mean(void *S, size_t n_blocks, size_t blk, bool mine,
+                                                 const float (&m)[8]) {
+  const int lane = threadIdx.x & 31;
+  const int c8 = (lane % (D / 8)) * 8;
+  if (FMT != KSA_SUMMARIES_FP8) {
+    if (mine) store_mean8(S, FMT, blk * D, c8, m);
+    return;
+  }
+  float amax = 0.f;
+  if (mine) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(m[i]));
+  }
+  // non-negative floats order like their bit patterns
+  amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+  const int e = e4m3_scale_exp(amax);
+  if (mine) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = pack_e4m3x2(ldexpf(m[2 * i], -e), ldexpf(m[2 * i + 1], -e));
+    *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(S) + blk * D + c8) =
+        make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+  }
+  if (lane == 0)
+    reinterpret_cast<float *>(static_cast<uint8_t *>(S) + n_blocks * D)[blk] = ldexpf(1.f, e);
+}
+
+// store_block_mean with the format chosen at run time.
+template <int D>
+__device__ __forceinline__ void store_block_mean_any(void *S, int sfmt, size_t n_blocks,
+                                                     size_t blk, bool mine, const float (&m)[8]) {
+  if (sfmt == KSA_SUMMARIES_FP8)
+    store_block_mean<D, KSA_SUMMARIES_FP8>(S, n_blocks, blk, mine, m);
+  else if (sfmt == KSA_SUMMARIES_BF16)
+    store_block_mean<D, KSA_SUMMARIES_BF16>(S, n_blocks, blk, mine, m);
+  else
+    store_block_mean<D, KSA_SUMMARIES_F32>(S, n_blocks, blk, mine, m);
 }
 
 // ---------------------------------------------------------------------------

@@ -37,8 +37,8 @@ __device__ __forceinline__ long long kv_row(const KvLayout &kv, int b, int g, in
 struct SummaryArgs {
   const uint16_t *K;
   const int32_t *seq_lens;
-  void *S;    // fp32 or bf16 [B, Hkv, ceil(T/bs), D]
-  int sbf16;  // summaries stored as bf16
+  void *S;   // [B, Hkv, ceil(T/bs), D] fp32 / bf16 / fp8 values (+ fp8 scales)
+  int sfmt;  // storage: KSA_SUMMARIES_F32, _BF16 or _FP8
   uint32_t *status;
   int B, Hkv, T, D, bs, mode;
   KvLayout kv;
@@ -59,8 +59,8 @@ cudaError_t launch_append_kv(const AppendArgs &a, cudaStream_t stream);
 
 struct SelectArgs {
   const uint16_t *q;
-  void *S;    // fp32 or bf16; read; written only by the fused last-block refresh
-  int sbf16;  // summaries stored as bf16
+  void *S;   // fp32 / bf16 / fp8; read; written only by the fused last-block refresh
+  int sfmt;  // storage: KSA_SUMMARIES_F32, _BF16 or _FP8
   const int32_t *seq_lens;
   int32_t *block_idx;
   int32_t *num_sel;

@@ -41,11 +41,16 @@ using namespace sel;
 
 namespace {
 
+// The scoring kernel's format for fp8 summaries: fp8 at D = 128; other head
+// sizes never reach it (the API refuses fp8 there), so they map to fp32.
+template <int D>
+constexpr int kFp8For = D == 128 ? KSA_SUMMARIES_FP8 : KSA_SUMMARIES_F32;
+
 // Scoring.  The grid's warps take equal contiguous slices of the flat piece
 // sequence: a warp streams one region of the summaries front to back (the
 // pattern the DRAM serves best, measured against round-robin and
 // counter-driven orders) and forms each row's group query sum once.
-template <int D, bool SBF>
+template <int D, int FMT>
 __global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev p) {
   constexpr int kWarps = kScThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane & 7;
@@ -62,9 +67,9 @@ __global__ void __launch_bounds__(kScThreads) score_blocks_kernel(const ScoreDev
     if (x.n == 0) continue;
     if (x.row != qrow) {
       qrow = x.row;
-      load_qsum<D, SBF>(p.a, x.b, x.g, sub, qv);
+      load_qsum<D, FMT>(p.a, x.b, x.g, sub, qv);
     }
-    score_piece<D, SBF>(p, x, qv, bad);
+    score_piece<D, FMT>(p, x, qv, bad);
   }
   bad = __reduce_or_sync(0xffffffffu, bad);
   if (bad != 0u && lane == 0) flag_status(p.a.status, bad);
@@ -117,7 +122,9 @@ cudaError_t launch_select(const ScoreDev &p0, int num_sms, cudaStream_t stream) 
   const int rows = a.B * a.Hkv;
   cudaError_t err;
   if (nb_max > a.k) {  // otherwise no row has a block to score
-    const auto kern = a.sbf16 ? score_blocks_kernel<D, true> : score_blocks_kernel<D, false>;
+    const auto kern = a.sfmt == KSA_SUMMARIES_BF16 ? score_blocks_kernel<D, KSA_SUMMARIES_BF16>
+                      : a.sfmt == KSA_SUMMARIES_FP8 ? score_blocks_kernel<D, kFp8For<D>>
+                                                    : score_blocks_kernel<D, KSA_SUMMARIES_F32>;
     int per_sm = 0;
     err = kernel_occupancy(reinterpret_cast<const void *>(kern), kScThreads, 0, &per_sm);
     if (err != cudaSuccess) return err;
@@ -169,7 +176,9 @@ cudaError_t launch_select_blocks(const SelectArgs &a, const uint16_t *K, void *w
   p.a = a;
   p.K = K;
   p.keys = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + sems);
-  p.prow = kPieceBytes / (a.D * (a.sbf16 ? 2 : 4));
+  p.prow = kPieceBytes / (a.D * (a.sfmt == KSA_SUMMARIES_F32    ? 4
+                                  : a.sfmt == KSA_SUMMARIES_BF16 ? 2
+                                                                 : 1));
   p.pieces = (nb_max + p.prow - 1) / p.prow;
   p.units = static_cast<long long>(rows) * p.pieces;
   p.N = 1;

@@ -45,7 +45,8 @@ static __device__ __forceinline__ Piece piece_of(const ScoreDev &p, long long u,
 // Re-averages block nb-1 of `row` from K and stores it in the summaries.
 // Lanes l < D/8 get dims [8 (l % (D/8)), +8) in mean[] and return true.
 // One whole warp.
-template <int D>
+// FMT: the summaries' storage format (a.sfmt), or -1 to read it at run time.
+template <int D, int FMT = -1>
 __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const uint16_t *K,
                                                    int row, int L, int nb, float (&mean)[8]) {
   const int nb_max = (a.T + a.bs - 1) / a.bs;
@@ -62,9 +63,12 @@ __device__ __forceinline__ bool refresh_last_block(const SelectArgs &a, const ui
   } else {
     mine = warp_block_mean<D>(K + static_cast<size_t>(row0) * D, L - jl * a.bs, mean);
   }
-  if (mine)
-    store_mean8(a.S, a.sbf16, (static_cast<size_t>(row) * nb_max + jl) * D,
-                ((threadIdx.x & 31) % (D / 8)) * 8, mean);
+  const size_t n_blocks = static_cast<size_t>(a.B) * a.Hkv * nb_max;
+  const size_t blk = static_cast<size_t>(row) * nb_max + jl;
+  if (FMT < 0)
+    store_block_mean_any<D>(a.S, a.sfmt, n_blocks, blk, mine, mean);
+  else
+    store_block_mean<D, (FMT < 0 ? 0 : FMT)>(a.S, n_blocks, blk, mine, mean);
   return mine;
 }
 
@@ -99,14 +103,9 @@ __device__ __forceinline__ float key_score(uint32_t key) {
 // passes.  The winners are written to out[0..k) in ascending block order
 // through a bitmap of the selection and one prefix count over its words.
 // `sm`: fast_topk_words words of shared memory, 16-byte aligned.
-//
-// kValuePass = false: the keys are plain unsigned ranks (vote counts), not
-// score keys, and every pass buckets by key bits.  bits_out non-null: instead
-// of the list, the selection is written as a bit set, bit j % 32 of word j / 32
-// for j < n (the words of [0, n) only).
-template <int NT, int KPL, bool kValuePass = true>
+template <int NT, int KPL>
 __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, int32_t *out,
-                                          uint32_t *sm, uint32_t *bits_out = nullptr) {
+                                          uint32_t *sm) {
   static_assert(NT % 32 == 0 && NT >= 64 && NT <= 1024, "whole warps");
   static_assert(KPL >= 1 && KPL <= 64, "a 64-bit slot mask per thread");
   static_assert(8 + 3 * (NT / 32) <= 64, "the reduction words fit in misc");
@@ -156,8 +155,7 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     // pass 0 by score value when the real scores span a finite, non-empty range
     const float v0 = key_score(lo_real), v1 = key_score(hi);
     const float vscale = 1024.f / (v1 - v0);
-    const bool by_value =
-        kValuePass && pass == 0 && lo_real < hi && isfinite(vscale) && vscale > 0.f;
+    const bool by_value = pass == 0 && lo_real < hi && isfinite(vscale) && vscale > 0.f;
     const int bits = 32 - __clz(hi - lo);
     const int sh = bits > 10 ? bits - 10 : 0;
     for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
@@ -264,6 +262,11 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     uint32_t ns = 0u;
     for (int w = w0; w < w1; ++w) {
       uint32_t take = 0u, x = livew[w];
+      if (pl + __popc(x) <= remaining) {  // the whole word
+        take = x;
+        pl += __popc(x);
+        x = 0u;
+      }
       while (x != 0u && pl < remaining) {  // lowest set bits first: ascending blocks
         const uint32_t b = x & (0u - x);
         take |= b;
@@ -274,11 +277,6 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
       const uint32_t sw = selw[w] | take;
       selw[w] = sw;
       ns += __popc(sw);
-    }
-    if (bits_out != nullptr) {
-      const int nwords = (n + 31) / 32;
-      for (int w = w0; w < w1 && w < nwords; ++w) bits_out[w] = selw[w];
-      return;
     }
     uint32_t ps = ns;
 #pragma unroll
@@ -314,9 +312,10 @@ __device__ __forceinline__ void keep_all_blocks(const ScoreDev &p, int row, int 
 
 // Group query sum of kv-head g of batch row b over this lane's columns,
 // summed over the heads in order.  The lane reads 16-byte chunks sub + 8 j of
-// a summary row: 4 fp32 dims each (qv[j]), or with bf16 summaries 8 dims each
-// (qv[2j], qv[2j+1]).  Either way qv covers D/8 dims in D/32 float4.
-template <int D, bool SBF>
+// a summary row: 4 fp32 dims each (qv[j]), with bf16 summaries 8 dims each
+// (qv[2j], qv[2j+1]), with fp8 ones (D = 128: one chunk) 16 dims (qv[0..3]).
+// Either way qv covers D/8 dims in D/32 float4.
+template <int D, int FMT>
 __device__ __forceinline__ void load_qsum(const SelectArgs &a, int b, int g, int sub,
                                           float4 (&qv)[D / 32]) {
   constexpr int NQ = D / 32;
@@ -329,7 +328,9 @@ __device__ __forceinline__ void load_qsum(const SelectArgs &a, int b, int g, int
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
       // dims 4 c .. 4 c + 3 with c the 4-dim group of qv[j]
-      const int c4 = SBF ? 2 * (sub + 8 * (j >> 1)) + (j & 1) : sub + 8 * j;
+      const int c4 = FMT == KSA_SUMMARIES_FP8    ? 4 * sub + j
+                     : FMT == KSA_SUMMARIES_BF16 ? 2 * (sub + 8 * (j >> 1)) + (j & 1)
+                                                 : sub + 8 * j;
       const uint32_t *q2 =
           reinterpret_cast<const uint32_t *>(qg + static_cast<size_t>(h) * D + 4 * c4);
       const uint32_t w0 = __ldg(q2), w1 = __ldg(q2 + 1);
@@ -346,10 +347,11 @@ __device__ __forceinline__ void load_qsum(const SelectArgs &a, int b, int g, int
 // of rows 4 it + r), each summary row is reduced over its 8 lanes, and the
 // keys are stored.  With a key cache given, the piece holding the row's last
 // block first re-averages that block, so the fresh value is the one scored.
-template <int D, bool SBF>
+template <int D, int FMT>
 __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
                                             const float4 (&qv)[D / 32], uint32_t &bad) {
-  constexpr int RB = D * (SBF ? 2 : 4);  // bytes per summary row
+  static_assert(FMT != KSA_SUMMARIES_FP8 || D == 128, "fp8 rows are one 16-byte chunk per lane");
+  constexpr int RB = D * (FMT == KSA_SUMMARIES_F32 ? 4 : FMT == KSA_SUMMARIES_BF16 ? 2 : 1);
   constexpr int R = kPieceBytes / RB;     // rows per piece
   constexpr int PER = RB / 16 / 8;        // 16-byte chunks per lane and row
   constexpr int IT = R / 4;
@@ -358,7 +360,7 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
   const int nb_max = (a.T + a.bs - 1) / a.bs;
   if (p.K != nullptr && x.j0 + x.n == x.nb) {
     float mean[8];
-    refresh_last_block<D>(a, p.K, x.row, x.L, x.nb, mean);
+    refresh_last_block<D, FMT>(a, p.K, x.row, x.L, x.nb, mean);
     __syncwarp();  // the fresh summary is visible to the whole warp's loads below
   }
   const uint4 *src = reinterpret_cast<const uint4 *>(
@@ -371,6 +373,15 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
     for (int j = 0; j < PER; ++j)
       v[it][j] = jr < x.n ? __ldcg(src + jr * (RB / 16) + sub + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
   }
+  // fp8: the piece's block scales, row jr's in lane jr % 32 of sa (jr < 32) or sb
+  float sa = 1.f, sb = 1.f;
+  if (FMT == KSA_SUMMARIES_FP8) {
+    const float *scales = reinterpret_cast<const float *>(
+        static_cast<const uint8_t *>(a.S) + static_cast<size_t>(a.B) * a.Hkv * nb_max * D);
+    const size_t s0 = static_cast<size_t>(x.row) * nb_max + x.j0;
+    if (lane < x.n) sa = __ldcg(scales + s0 + lane);
+    if (32 + lane < x.n) sb = __ldcg(scales + s0 + 32 + lane);
+  }
   uint32_t *krow = p.keys + static_cast<size_t>(x.row) * nb_max + x.j0;
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
@@ -379,7 +390,18 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
       const uint4 w = v[it][j];
-      if (SBF) {
+      if (FMT == KSA_SUMMARIES_FP8) {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // dims 16 sub + 4 c .. + 3
+          const float2 lo = e4m3x2_to_float2(static_cast<uint16_t>(ww[c] & 0xffffu));
+          const float2 hi = e4m3x2_to_float2(static_cast<uint16_t>(ww[c] >> 16));
+          sc = fmaf(qv[c].x, lo.x, sc);
+          sc = fmaf(qv[c].y, lo.y, sc);
+          sc = fmaf(qv[c].z, hi.x, sc);
+          sc = fmaf(qv[c].w, hi.y, sc);
+        }
+      } else if (FMT == KSA_SUMMARIES_BF16) {
         const float4 qa = qv[2 * j], qb = qv[2 * j + 1];
         sc = fmaf(qa.x, bf16_lo(w.x), sc);
         sc = fmaf(qa.y, bf16_hi(w.x), sc);
@@ -399,6 +421,11 @@ __device__ __forceinline__ void score_piece(const ScoreDev &p, const Piece &x,
     sc += __shfl_xor_sync(0xffffffffu, sc, 1);
     sc += __shfl_xor_sync(0xffffffffu, sc, 2);
     sc += __shfl_xor_sync(0xffffffffu, sc, 4);
+    if (FMT == KSA_SUMMARIES_FP8) {  // the stored values times the block's scale (exact)
+      const float ga = __shfl_sync(0xffffffffu, sa, jr & 31);
+      const float gb = __shfl_sync(0xffffffffu, sb, jr & 31);
+      sc *= jr < 32 ? ga : gb;
+    }
     if (jr < x.n && sub == 0) {
       bool nan;
       krow[jr] = score_key(sc, nan);

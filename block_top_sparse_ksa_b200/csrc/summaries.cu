@@ -8,8 +8,8 @@
 // rows l / (D/8), l / (D/8) + 32/(D/8), ... so every warp-wide load covers
 // 2 (D = 128) or 4 (D = 64) whole key rows and all of a block's loads are
 // independent (in flight together).  Partial sums meet through warp shuffles;
-// then one IEEE division by n_j, in fp32, and the mean is stored as fp32 or
-// as bf16 rounded to nearest even.
+// then one IEEE division by n_j, in fp32, and the mean is stored as fp32, as
+// bf16 rounded to nearest even, or as fp8 e4m3 with a per-block scale.
 //
 // Also here: the decode step's cache append (the new token's key and value
 // rows written into their slot), the write that the last-block refresh of the
@@ -58,9 +58,8 @@ __global__ void __launch_bounds__(256) block_summaries_kernel(SummaryArgs a) {
     } else {
       mine = warp_block_mean<D>(a.K + static_cast<size_t>(row0) * D, n, mean);
     }
-    if (mine)
-      store_mean8(a.S, a.sbf16, (static_cast<size_t>(bg) * nb_max + j) * D, (lane % (D / 8)) * 8,
-                  mean);
+    store_block_mean_any<D>(a.S, a.sfmt, static_cast<size_t>(a.B) * a.Hkv * nb_max,
+                            static_cast<size_t>(bg) * nb_max + j, mine, mean);
   }
 }
 

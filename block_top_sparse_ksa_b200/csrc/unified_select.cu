@@ -12,22 +12,20 @@
 //     form S^T = K_tile q^T for the kv-group's G heads with mma.sync
 //     (fp32 accumulate) and store order-preserving uint32 score keys
 //     [B, Hq, T].  The g == 0 CTAs also clear the vote table.
-//  2. per-head picks: one CTA per (row, query head) selects the P highest
-//     keys of the row's L, ties at the threshold to the lower token.  Rows of
-//     up to 24576 tokens keep their keys in registers and run sel::fast_topk
-//     (histogram passes over shrinking ranges, the first by score value),
-//     writing the picks as bit sets, from which a per-token kernel then counts
-//     the votes (2b); longer rows stage the keys in shared memory, run a radix
-//     select and add one atomic vote per pick.
-//  3. shared set: one CTA per row selects the (budget - R) most voted tokens
-//     of [0, L - R) (ties to the lower token; fast_topk on the vote counts for
-//     rows of up to 24576 tokens, a radix select beyond), written ascending,
-//     followed by the window [L - R, L).
+//  2. per-head picks: one CTA per (row, query head).  Exact radix select of the
+//     P-th largest key over the row's L keys, ties at the threshold to the
+//     lower token.  Rows of up to 24576 tokens keep their keys in registers,
+//     run an adaptive radix (each pass starts at the highest bit in which the
+//     remaining candidates differ) and write the picks as bit sets, from which
+//     a per-token kernel then counts the votes (2b); longer rows stage the keys
+//     in shared memory and add one atomic vote per pick.
+//  3. shared set: one CTA per row.  Radix select on the vote counts of
+//     [0, L - R) for the (budget - R) most voted tokens (ties to the lower
+//     token), written ascending, followed by the window [L - R, L).
 #include <string.h>
 
 #include "ksa_device.cuh"
 #include "ksa_internal.h"
-#include "select_device.cuh"
 
 namespace ksa {
 
@@ -37,9 +35,8 @@ constexpr int kTok = 32;            // tokens per pipeline stage
 constexpr int kChunk = 1024;        // tokens per scoring CTA
 constexpr int kScoreThreads = 160;  // 4 consumer warps + 1 producer warp
 constexpr int kPickThreads = 512;
-// picks and shared set with the row's keys in registers: 256 threads for rows of up to
-// 16384 tokens, 384 up to 24576 (64 keys per thread at most, with no spill)
-constexpr int kFastMaxTokens = 24576;
+constexpr int kPickRegThreads = 256;  // picks with the row's keys in registers
+constexpr int kPickRegMaxKeys = 96;   // keys per thread of that kernel (rows <= 24576 tokens)
 constexpr int kSetThreads = 1024;
 constexpr int kSmemKeys = 40960;    // keys of one head staged in shared memory
 
@@ -205,29 +202,185 @@ __global__ void __launch_bounds__(kPickThreads) unified_pick_kernel(const Unifie
                                  [&](int t) { atomicAdd(&votes[t], 1); });
 }
 
-// Per-head picks for rows that fit in registers (L <= NT * KPL): CTA
-// per (row, query head); sel::fast_topk finds the P highest score keys (ties to
-// the lower token) by histogram passes over shrinking ranges -- the first by
-// score value, so scores on a coarse grid spread over many buckets -- and
-// writes them as the head's bit set, from which unified_votes_kernel counts
-// the votes.
-template <int NT, int KPL>
-__global__ void __launch_bounds__(NT) unified_pick_fast_kernel(const UnifiedArgs a) {
-  __shared__ __align__(16) uint32_t sm[sel::fast_topk_words<NT, KPL>()];
+// Per-head picks for rows that fit in registers (L <= kPickRegThreads * KPL):
+// CTA per (row, query head), thread t holds tokens t, t + NT, ...  The P-th
+// largest key is found by a radix select that, before every 8-bit pass,
+// recomputes the min and max of the keys still in play and starts the pass at
+// their highest differing bit: bits all candidates share cost nothing, and a
+// pass never piles equal digits of tied keys into one bin (scores on a coarse
+// grid tie a lot).  Once the candidates are all equal the threshold is found.
+// Keys above it vote; of the keys equal to it the lowest-index ones vote
+// (ballots and per-warp counts, in token order).
+template <int KPL>
+__global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const UnifiedArgs a) {
+  constexpr int NT = kPickRegThreads, NW = NT / 32;
+  __shared__ __align__(16) uint32_t hist[NW][256];
+  __shared__ uint32_t red[3][NW];
+  __shared__ uint32_t xinfo[3];
   const int b = blockIdx.x / a.Hq, h = blockIdx.x % a.Hq;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
   pdl_wait();
   pdl_launch_dependents();
   const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
   if (L <= a.budget) return;
-  const int W32 = (a.T + 31) / 32;
-  uint32_t *bits = a.bits + (static_cast<size_t>(b) * a.Hq + h) * W32;
   if (a.P >= L) {  // the head picks every token
-    for (int w = threadIdx.x; w < (L + 31) / 32; w += NT)
+    const int W32 = (a.T + 31) / 32;
+    uint32_t *bits = a.bits + (static_cast<size_t>(b) * a.Hq + h) * W32;
+    for (int w = tid; w < (L + 31) / 32; w += NT)
       bits[w] = (w + 1) * 32 <= L ? 0xffffffffu : ((1u << (L - w * 32)) - 1u);
     return;
   }
-  sel::fast_topk<NT, KPL>(a.keys + (static_cast<size_t>(b) * a.Hq + h) * a.T, L, a.P,
-                                    nullptr, sm, bits);
+  const uint32_t *gkeys = a.keys + (static_cast<size_t>(b) * a.Hq + h) * a.T;
+  uint32_t key[KPL];
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = tid + NT * e;
+    key[e] = j < L ? __ldcg(gkeys + j) : 0u;
+  }
+  uint32_t prefix = 0u, pmask = 0u;
+  uint32_t remaining = static_cast<uint32_t>(a.P);  // still to take among the candidates
+  uint32_t tau = 0u, n_eq = 0u;
+  for (int pass = 0; pass < 5; ++pass) {  // at most 4 passes of 8 bits, then all equal
+    // min / max / count of the candidates (keys matching the digits fixed so far)
+    uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      if (tid + NT * e < L && (key[e] & pmask) == prefix) {
+        kmin = min(kmin, key[e]);
+        kmax = max(kmax, key[e]);
+        ++cnt;
+      }
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) {
+      red[0][warp] = kmin;
+      red[1][warp] = kmax;
+      red[2][warp] = cnt;
+    }
+    __syncthreads();
+    kmin = red[0][0];
+    kmax = red[1][0];
+    cnt = red[2][0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) {
+      kmin = min(kmin, red[0][w]);
+      kmax = max(kmax, red[1][w]);
+      cnt += red[2][w];
+    }
+    if (kmin == kmax) {  // every candidate equal: the threshold
+      tau = kmin;
+      n_eq = cnt;
+      break;
+    }
+    const int hb = 31 - __clz(kmin ^ kmax);  // candidates share every bit above hb
+    const uint32_t above = hb == 31 ? 0u : ~((2u << hb) - 1u);
+    prefix = kmin & above;
+    pmask = above;
+    const int sh = hb >= 7 ? hb - 7 : 0;
+    for (int i = tid; i < NW * 256; i += NT) (&hist[0][0])[i] = 0u;
+    __syncthreads();  // also: red was read by everyone
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      if (tid + NT * e < L && (key[e] & pmask) == prefix)
+        atomicAdd(&hist[warp][(key[e] >> sh) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {  // lane l owns bins [8l, 8l + 8); counts from the top bin down
+      uint32_t c[8];
+      uint32_t tot = 0u;
+#pragma unroll
+      for (int jb = 0; jb < 8; ++jb) {
+        uint32_t v = 0u;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) v += hist[w][lane * 8 + jb];
+        c[jb] = v;
+        tot += v;
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl += y;
+      }
+      uint32_t run = incl - tot;
+#pragma unroll
+      for (int jb = 7; jb >= 0; --jb) {
+        const uint32_t before = run;
+        run += c[jb];
+        if (before < remaining && run >= remaining) {
+          xinfo[0] = static_cast<uint32_t>(lane * 8 + jb);
+          xinfo[1] = before;
+          xinfo[2] = c[jb];
+        }
+      }
+    }
+    __syncthreads();
+    remaining -= xinfo[1];
+    prefix = (prefix & ~(255u << sh)) | (xinfo[0] << sh);
+    pmask |= 255u << sh;
+    n_eq = xinfo[2];
+    tau = prefix;
+    __syncthreads();  // xinfo, hist and red are rewritten by the next pass
+    if (sh == 0) break;  // every bit fixed
+  }
+  __syncthreads();  // red is read above before it is rewritten below
+  const uint32_t take_eq = remaining;  // keys equal to tau to take, lowest token first
+  const bool all_eq = take_eq == n_eq;  // block-uniform
+  uint32_t *pre = &hist[0][0];          // [KPL][NW] exclusive counts of tied keys, token order
+  if (!all_eq) {
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      const bool eq = tid + NT * e < L && key[e] == tau;
+      const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+      if (lane == 0) pre[e * NW + warp] = __popc(eb);
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the KPL * NW counts, slot-major = token order
+      constexpr int N = KPL * NW, PERL = (N + 31) / 32;
+      uint32_t v[PERL];
+      uint32_t s = 0u;
+#pragma unroll
+      for (int i = 0; i < PERL; ++i) {
+        const int x = lane * PERL + i;
+        v[i] = x < N ? pre[x] : 0u;
+        s += v[i];
+      }
+      uint32_t incl = s;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      uint32_t run = incl - s;
+#pragma unroll
+      for (int i = 0; i < PERL; ++i) {
+        const int x = lane * PERL + i;
+        if (x < N) pre[x] = run;
+        run += v[i];
+      }
+    }
+    __syncthreads();
+  }
+  const int W32 = (a.T + 31) / 32;
+  const int nwords = (L + 31) / 32;
+  uint32_t *bits = a.bits + (static_cast<size_t>(b) * a.Hq + h) * W32;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = tid + NT * e;
+    const bool ok = j < L;
+    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
+    bool sel = gt || eq;
+    if (!all_eq) {
+      const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+      sel = gt || (eq && pre[e * NW + warp] + __popc(eb & lt) < take_eq);
+    }
+    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+    const int word = NW * e + warp;  // tokens NT e + 32 warp + [0, 32)
+    if (lane == 0 && word < nwords) bits[word] = sb;
+  }
 }
 
 // Votes from the pick bit sets (rows whose picks were written as bits): one
@@ -283,34 +436,7 @@ __global__ void __launch_bounds__(kPickThreads) unified_topk_list_kernel(const U
   if (threadIdx.x == 0) a.num_sel[static_cast<size_t>(b) * a.Hq + h] = k;
 }
 
-// Shared set for rows whose candidates fit in registers (L - R <= NT * KPL):
-// CTA per row; the (budget - R) most voted tokens of [0, L - R) by
-// sel::fast_topk on the vote counts (plain ranks: no score-value pass; equal
-// counts go to the lower token), written ascending, then the window.
-template <int NT, int KPL>
-__global__ void __launch_bounds__(NT) unified_set_fast_kernel(const UnifiedArgs a) {
-  __shared__ __align__(16) uint32_t sm[sel::fast_topk_words<NT, KPL>()];
-  const int b = blockIdx.x;
-  pdl_wait();
-  pdl_launch_dependents();
-  const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
-  int32_t *out = a.token_idx + static_cast<size_t>(b) * a.budget;
-  if (L <= a.budget) {
-    for (int i = threadIdx.x; i < a.budget; i += NT) out[i] = i < L ? i : -1;
-    if (threadIdx.x == 0) a.num_sel[b] = L;
-    return;
-  }
-  const int n = L - a.R;  // candidates [0, L - R); n > k since L > budget
-  const int k = a.budget - a.R;
-  if (k > 0)
-    sel::fast_topk<NT, KPL, false>(
-        reinterpret_cast<const uint32_t *>(a.votes + static_cast<size_t>(b) * a.T), n, k, out,
-        sm);
-  for (int i = threadIdx.x; i < a.R; i += NT) out[k + i] = n + i;
-  if (threadIdx.x == 0) a.num_sel[b] = a.budget;
-}
-
-// Shared set for longer rows: CTA per row.
+// Shared set: CTA per row.
 __global__ void __launch_bounds__(kSetThreads) unified_set_kernel(const UnifiedArgs a) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t info[4];
@@ -384,13 +510,15 @@ cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_
   cudaError_t err = a.D == 128 ? launch_scores<128>(a, stream) : launch_scores<64>(a, stream);
   if (err != cudaSuccess) return err;
   const dim3 pgrid(static_cast<unsigned>(a.B) * a.Hq);
-  const bool fast = a.T <= kFastMaxTokens;
-  if (fast) {
-    if (a.T <= 2048) err = launch_pdl(unified_pick_fast_kernel<256, 8>, pgrid, dim3(256), 0, stream, a);
-    else if (a.T <= 4096) err = launch_pdl(unified_pick_fast_kernel<256, 16>, pgrid, dim3(256), 0, stream, a);
-    else if (a.T <= 8192) err = launch_pdl(unified_pick_fast_kernel<256, 32>, pgrid, dim3(256), 0, stream, a);
-    else if (a.T <= 16384) err = launch_pdl(unified_pick_fast_kernel<256, 64>, pgrid, dim3(256), 0, stream, a);
-    else err = launch_pdl(unified_pick_fast_kernel<384, 64>, pgrid, dim3(384), 0, stream, a);
+  const int per = (a.T + kPickRegThreads - 1) / kPickRegThreads;  // keys per thread
+  if (per <= kPickRegMaxKeys) {
+    const dim3 pblock(kPickRegThreads);
+    if (per <= 16) err = launch_pdl(unified_pick_reg_kernel<16>, pgrid, pblock, 0, stream, a);
+    else if (per <= 32) err = launch_pdl(unified_pick_reg_kernel<32>, pgrid, pblock, 0, stream, a);
+    else if (per <= 48) err = launch_pdl(unified_pick_reg_kernel<48>, pgrid, pblock, 0, stream, a);
+    else if (per <= 64) err = launch_pdl(unified_pick_reg_kernel<64>, pgrid, pblock, 0, stream, a);
+    else if (per <= 80) err = launch_pdl(unified_pick_reg_kernel<80>, pgrid, pblock, 0, stream, a);
+    else err = launch_pdl(unified_pick_reg_kernel<96>, pgrid, pblock, 0, stream, a);
     if (err != cudaSuccess) return err;
     const long long nt = static_cast<long long>(a.B) * ((a.T + 31) / 32) * 32;
     err = launch_pdl(unified_votes_kernel, dim3(static_cast<unsigned>((nt + 255) / 256)),
@@ -406,14 +534,6 @@ cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_
                      in_smem);
   }
   if (err != cudaSuccess) return err;
-  if (fast) {  // the candidates [0, L - R) number at most T
-    const dim3 sgrid(static_cast<unsigned>(a.B));
-    if (a.T <= 2048) return launch_pdl(unified_set_fast_kernel<256, 8>, sgrid, dim3(256), 0, stream, a);
-    if (a.T <= 4096) return launch_pdl(unified_set_fast_kernel<256, 16>, sgrid, dim3(256), 0, stream, a);
-    if (a.T <= 8192) return launch_pdl(unified_set_fast_kernel<256, 32>, sgrid, dim3(256), 0, stream, a);
-    if (a.T <= 16384) return launch_pdl(unified_set_fast_kernel<256, 64>, sgrid, dim3(256), 0, stream, a);
-    return launch_pdl(unified_set_fast_kernel<384, 64>, sgrid, dim3(384), 0, stream, a);
-  }
   return launch_pdl(unified_set_kernel, dim3(static_cast<unsigned>(a.B)), dim3(kSetThreads), 0,
                     stream, a);
 }

@@ -70,7 +70,7 @@ typedef struct {
 
 enum { KSA_SUMMARY_ALL = 0, KSA_SUMMARY_LAST_BLOCK = 1 };
 /* Storage type of the block summaries (the *_ex entry points). */
-enum { KSA_SUMMARIES_F32 = 0, KSA_SUMMARIES_BF16 = 1 };
+enum { KSA_SUMMARIES_F32 = 0, KSA_SUMMARIES_BF16 = 1, KSA_SUMMARIES_FP8 = 2 };
 enum { KSA_OUT_F32 = 0, KSA_OUT_BF16 = 1 };
 /* Index-list layouts of ksa_sparse_decode_attn (idx_shared). */
 enum { KSA_IDX_PER_KV_HEAD = 0, KSA_IDX_SHARED = 1, KSA_IDX_PER_Q_HEAD = 2 };
@@ -194,16 +194,24 @@ ksa_status ksa_select_window(const ksa_shape *shape, const int32_t *seq_lens,
                              uint32_t *dev_status, void *stream);
 
 /*
- * The same three calls with the summaries stored as bf16 or fp32
- * (summary_dtype: KSA_SUMMARIES_F32 or KSA_SUMMARIES_BF16).  With bf16 each
- * block mean is computed in fp32 as above and stored rounded to the nearest
- * bf16 (ties to even): half the bytes for the maintenance writes and, above
- * all, for the scoring reads, which dominate at long context and small budget
- * [KIN s.5 names the block mean; the storage precision is this library's
- * option, not the source's].  Scores are accumulated in fp32 from the stored
- * values, so blocks whose scores differ by less than the rounding of their
- * means may rank differently than with fp32 summaries.
- *   summaries: [B, Hkv, ceil(T/bs), D] of the given type, 16-byte aligned.
+ * The same three calls with the summaries stored as fp32, bf16 or fp8
+ * (summary_dtype: KSA_SUMMARIES_F32, _BF16 or _FP8).  Each block mean is
+ * computed in fp32 as above and stored in the chosen format: fewer bytes for
+ * the maintenance writes and, above all, for the scoring reads, which
+ * dominate at long context and small budget [KIN s.5 names the block mean;
+ * the storage precision is this library's option, not the source's].
+ *   BF16: each value rounded to the nearest bf16 (ties to even).
+ *   FP8:  each block's D values scaled by 2^-e, e the smallest exponent with
+ *         max |mean| <= 448 2^e, and rounded to the nearest fp8 e4m3 value
+ *         (ties to even); the block keeps the scale 2^e as an fp32.  Layout:
+ *         the values [B, Hkv, ceil(T/bs), D] bytes, then the scales
+ *         [B, Hkv, ceil(T/bs)] fp32 -- B Hkv ceil(T/bs) (D + 4) bytes in all.
+ *         head_dim 128 only (else KSA_ERR_UNSUPPORTED).
+ * Scores are accumulated in fp32 from the stored values, so blocks whose
+ * scores differ by less than the rounding of their means may rank
+ * differently than with fp32 summaries.
+ *   summaries: [B, Hkv, ceil(T/bs), D] of the given type (FP8: as above),
+ *              16-byte aligned.
  * Every other argument, limit and error as the fp32 calls, which are these
  * with KSA_SUMMARIES_F32.  An unknown summary_dtype is KSA_ERR_INVALID_ARG.
  */

@@ -37,7 +37,11 @@
  *  (R11) random-head aggregation: the random head of each row is an input
  *        drawn by the caller, and that head's own top-k set serves every head;
  *  (R12) attention recall of a selection is the share of the dense softmax
- *        weight (over every cached token) that falls on the selected tokens.
+ *        weight (over every cached token) that falls on the selected tokens;
+ *  (R13) fp8 block summaries are a storage format of the block mean: each
+ *        block's D means are scaled by 2^-e, e the smallest exponent with
+ *        max |mean| <= 448 2^e, rounded to the nearest e4m3 value (ties to
+ *        even) and scaled back; the scores read the stored values.
  *
  * Inputs: bf16 values arrive as their 16-bit patterns and are widened to fp64
  * exactly.  All arrays are dense row-major.  Threads: OpenMP over independent
@@ -144,6 +148,54 @@ uint16_t ksa_oracle_round_bf16(double x) {
   return (uint16_t)(sign | (uint16_t)(u >> 16));
 }
 
+/* ---- (R13) fp8 e4m3 block summaries ----------------------------------------
+ * e4m3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits.  Normal values
+ * (1 + m/8) 2^(E-7) for E = 1..15 except E = 15, m = 7 (not a number), so the
+ * largest is 1.75 * 2^8 = 448; subnormal values (m/8) 2^-6.  Every finite
+ * value is therefore a multiple of its binade's spacing 2^(E-10) (2^-9 below
+ * 2^-6).  Rounding: to the nearest value, ties to the even mantissa; a
+ * magnitude above 448 is held at 448.  Returns the rounded value. */
+double ksa_oracle_round_e4m3(double x) {
+  if (isnan(x)) return x;
+  const double a = fabs(x);
+  if (a == 0.0) return x;
+  int e;
+  frexp(a, &e); /* a = f 2^e, 0.5 <= f < 1: binade [2^(e-1), 2^e) */
+  int q = e - 4; /* spacing 2^(e-1-3) */
+  if (q < -9) q = -9; /* subnormals share the spacing of the lowest binade */
+  const double m = ldexp(a, -q); /* a in units of the spacing, exact */
+  double r = floor(m);
+  const double frac = m - r;
+  if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+  double v = ldexp(r, q);
+  if (v > 448.0) v = 448.0;
+  return signbit(x) ? -v : v;
+}
+
+/* The block's scale exponent: the smallest e with max_d |mean_d| <= 448 2^e
+ * (0 when the block mean is all zeros).  The stored block is the values
+ * round_e4m3(mean_d 2^-e) with the scale 2^e. */
+int ksa_oracle_e4m3_scale_exp(double amax) {
+  if (!(amax > 0.0)) return 0;
+  int e = (int)ceil(log2(amax / 448.0)) - 1;
+  while (amax > ldexp(448.0, e)) ++e; /* settle e exactly against 448 2^e */
+  while (e > -200 && amax <= ldexp(448.0, e - 1)) --e;
+  return e;
+}
+
+/* Stored form of D-dim block means, in place: each block of D values becomes
+ * round_e4m3(v 2^-e) 2^e with its own e. */
+void ksa_oracle_store_fp8_blocks(size_t n_blocks, int D, double *S) {
+  for (size_t j = 0; j < n_blocks; ++j) {
+    double *m = S + j * (size_t)D;
+    double amax = 0.0;
+    for (int d = 0; d < D; ++d)
+      if (fabs(m[d]) > amax) amax = fabs(m[d]);
+    const int e = ksa_oracle_e4m3_scale_exp(amax);
+    for (int d = 0; d < D; ++d) m[d] = ldexp(ksa_oracle_round_e4m3(ldexp(m[d], -e)), e);
+  }
+}
+
 void ksa_oracle_round_bf16_array(size_t n, const double *in, uint16_t *out) {
   for (size_t i = 0; i < n; ++i) out[i] = ksa_oracle_round_bf16(in[i]);
 }
@@ -243,13 +295,14 @@ int ksa_oracle_topk(int n, const double *s, int k, int32_t *out) {
 
 /*
  * (A1 -> A2 -> A3) composed: block ids per (b, g), ascending, -1 padded.
- * summary_bf16 != 0: the summaries are stored as bf16 (R10) before scoring.
+ * summary_fmt: 0 exact means; 1 stored as bf16 (R10); 2 stored as fp8 e4m3
+ * with a power-of-two scale per block (R13), before scoring.
  *   block_idx: [B, Hkv, k];  num_sel: [B, Hkv];
  *   scores_out (nullable): [B, Hkv, ceil(T/bs)].
  */
 void ksa_oracle_select_blocks_ex(int B, int Hq, int Hkv, int D, int T, int bs,
                                  const uint16_t *q, const uint16_t *K,
-                                 const int32_t *seq_lens, int k, int summary_bf16,
+                                 const int32_t *seq_lens, int k, int summary_fmt,
                                  int32_t *block_idx, int32_t *num_sel,
                                  double *scores_out) {
   const int nb_max = num_blocks(T, bs);
@@ -258,8 +311,10 @@ void ksa_oracle_select_blocks_ex(int B, int Hq, int Hkv, int D, int T, int bs,
   double *s = scores_out ? scores_out
                          : (double *)malloc(sizeof(double) * (size_t)B * Hkv * nb_max);
   ksa_oracle_block_summaries(B, Hkv, T, D, bs, K, seq_lens, S);
-  if (summary_bf16) {
+  if (summary_fmt == 1) {
     for (size_t i = 0; i < n_sum; ++i) S[i] = bf16_to_f64(ksa_oracle_round_bf16(S[i]));
+  } else if (summary_fmt == 2) {
+    ksa_oracle_store_fp8_blocks(n_sum / (size_t)D, D, S);
   }
   ksa_oracle_block_scores(B, Hq, Hkv, D, nb_max, bs, q, S, seq_lens, s);
 #pragma omp parallel for collapse(2) schedule(dynamic)

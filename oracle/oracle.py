@@ -60,6 +60,11 @@ class Oracle:
         L.ksa_oracle_round_bf16.argtypes = [c_double]
         L.ksa_oracle_round_bf16.restype = ctypes.c_uint16
         L.ksa_oracle_round_bf16_array.argtypes = [ctypes.c_size_t, _f64p, _u16p]
+        L.ksa_oracle_round_e4m3.argtypes = [c_double]
+        L.ksa_oracle_round_e4m3.restype = c_double
+        L.ksa_oracle_e4m3_scale_exp.argtypes = [c_double]
+        L.ksa_oracle_e4m3_scale_exp.restype = c_int
+        L.ksa_oracle_store_fp8_blocks.argtypes = [ctypes.c_size_t, c_int, _f64p]
         L.ksa_oracle_attention.argtypes = ([c_int] * 5 + [_u16p, _u16p, _u16p, _i32p,
                                            ctypes.c_void_p, ctypes.c_void_p, c_int, c_int,
                                            c_int, c_double, _f64p, nullable_f64,
@@ -110,6 +115,23 @@ class Oracle:
         self.lib.ksa_oracle_round_bf16_array(x.size, x.reshape(-1), out.reshape(-1))
         return out
 
+    def round_e4m3(self, x) -> np.ndarray:
+        """Nearest fp8 e4m3 value (ties to even, held at +-448) of fp64 values, same shape."""
+        x = np.asarray(x, dtype=np.float64)
+        return np.vectorize(self.lib.ksa_oracle_round_e4m3, otypes=[np.float64])(x)
+
+    def e4m3_scale_exp(self, amax: float) -> int:
+        """Smallest e with amax <= 448 * 2^e (0 for amax == 0)."""
+        return int(self.lib.ksa_oracle_e4m3_scale_exp(float(amax)))
+
+    def store_fp8(self, S: np.ndarray) -> np.ndarray:
+        """The stored values of block means [..., D] as fp8 e4m3 with a power-of-two scale
+        per block (a copy, fp64)."""
+        S = np.ascontiguousarray(S, dtype=np.float64).copy()
+        D = S.shape[-1]
+        self.lib.ksa_oracle_store_fp8_blocks(S.size // D, D, S.reshape(-1))
+        return S
+
     def block_summaries_bf16(self, K: np.ndarray, seq_lens: np.ndarray, bs: int) -> np.ndarray:
         """The block means stored as bf16 -> uint16 bits [B,Hkv,ceil(T/bs),D]."""
         return self.round_bf16(self.block_summaries(K, seq_lens, bs))
@@ -136,9 +158,10 @@ class Oracle:
         return out[:m].copy()
 
     def select_blocks(self, q, K, seq_lens, bs: int, k: int, want_scores: bool = False,
-                      summary_bf16: bool = False):
+                      summary_bf16: bool = False, summary_fp8: bool = False):
         """A1+A2+A3: (block_idx [B,Hkv,k] ascending -1 padded, num_sel [B,Hkv][, scores]).
-        summary_bf16: the block means are stored as bf16 before scoring."""
+        summary_bf16 / summary_fp8: the block means are stored as bf16 / as fp8 e4m3 with a
+        power-of-two scale per block before scoring."""
         q = np.ascontiguousarray(q, dtype=np.uint16)
         K = np.ascontiguousarray(K, dtype=np.uint16)
         B, Hq, D = q.shape
@@ -148,7 +171,8 @@ class Oracle:
         scores = np.empty((B, Hkv, -(-T // bs)), np.float64) if want_scores else None
         self.lib.ksa_oracle_select_blocks_ex(
             B, Hq, Hkv, D, T, bs, q, K, np.ascontiguousarray(seq_lens, np.int32), k,
-            int(summary_bf16), idx, cnt, scores.ctypes.data if want_scores else None)
+            2 if summary_fp8 else int(bool(summary_bf16)), idx, cnt,
+            scores.ctypes.data if want_scores else None)
         return (idx, cnt, scores) if want_scores else (idx, cnt)
 
     def select_tokens_per_head(self, q, K, seq_lens, k: int):

@@ -21,22 +21,25 @@ REL_TOL = 1e-2
 LSE_TOL = 1e-4
 
 
-def _row_scores(oracle, q_row, K, lens, bs, summary_bf16):
+def _row_scores(oracle, q_row, K, lens, bs, summary_bf16, summary_fp8=False):
     S = oracle.block_summaries(K[None], lens, bs)
     if summary_bf16:  # the scores the bf16-stored means give
         S = bf16_value(oracle.round_bf16(S))
+    if summary_fp8:  # ... or the fp8-stored ones
+        S = oracle.store_fp8(S)
     return oracle.block_scores(q_row[None], S, lens, bs)[0]  # [Hkv, nb]
 
 
 def gap_fix_row(oracle, q_row: np.ndarray, K_row: np.ndarray, L: int, bs: int, k: int,
-                delta: float = DELTA, max_iter: int = 20, summary_bf16: bool = False):
+                delta: float = DELTA, max_iter: int = 20, summary_bf16: bool = False,
+                summary_fp8: bool = False):
     """Plant a score gap >= delta at the top-k boundary of every kv-head of one row.
 
     q_row: uint16 [Hq, D] bits; K_row: uint16 [Hkv, T, D] bits (edited copy returned).
     Selected blocks that sit within delta of the best unselected score have all
     their valid keys moved along the group's query-sum direction until the
-    boundary gap is at least delta (scored from bf16-stored means when
-    summary_bf16).  Returns (K_row, number of blocks moved)."""
+    boundary gap is at least delta (scored from bf16- or fp8-stored means when
+    summary_bf16 / summary_fp8).  Returns (K_row, number of blocks moved)."""
     K = K_row.copy()
     Hq, D = q_row.shape
     Hkv, T, _ = K.shape
@@ -45,7 +48,7 @@ def gap_fix_row(oracle, q_row: np.ndarray, K_row: np.ndarray, L: int, bs: int, k
     lens = np.array([L], np.int32)
     moved = 0
     for _ in range(max_iter):
-        s = _row_scores(oracle, q_row, K, lens, bs, summary_bf16)
+        s = _row_scores(oracle, q_row, K, lens, bs, summary_bf16, summary_fp8)
         nb = -(-L // bs)
         if nb <= k:
             return K, moved
@@ -72,9 +75,10 @@ def gap_fix_row(oracle, q_row: np.ndarray, K_row: np.ndarray, L: int, bs: int, k
     raise AssertionError("could not plant the score gap")
 
 
-def min_boundary_gap(oracle, q_row, K_row, L, bs, k, summary_bf16: bool = False) -> float:
+def min_boundary_gap(oracle, q_row, K_row, L, bs, k, summary_bf16: bool = False,
+                     summary_fp8: bool = False) -> float:
     lens = np.array([L], np.int32)
-    s = _row_scores(oracle, q_row, K_row, lens, bs, summary_bf16)
+    s = _row_scores(oracle, q_row, K_row, lens, bs, summary_bf16, summary_fp8)
     nb = -(-L // bs)
     if nb <= k:
         return np.inf

@@ -25,6 +25,9 @@ def test_bytes_qwen3_0_6b_step():
     assert total == 403_439_616
     total16, attn16, summ16 = bench.algorithmic_bytes(sh, lens, "block", summary_bytes=2)
     assert summ16 == 67_108_864 and attn16 == attn and total16 == total - 67_108_864
+    # fp8: one byte per value plus a 4-byte scale per block
+    _, _, summ8 = bench.algorithmic_bytes(sh, lens, "block", summary_bytes=1, summary_extra=4)
+    assert summ8 == 64 * 8 * 512 * (128 + 4)
 
 
 def test_bytes_short_rows_and_dense():

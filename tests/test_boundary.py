@@ -126,8 +126,14 @@ def test_validation_of_the_newer_entry_points(ksa):
     # summary storage type out of range
     assert lib.ksa_build_block_summaries_ex(ctypes.byref(sh), FAKE, FAKE, 0, 7, FAKE, None,
                                             None) == 1
-    assert lib.ksa_select_blocks_ex(ctypes.byref(sh), FAKE, FAKE, 2, FAKE, 4, FAKE, FAKE, FAKE,
+    assert lib.ksa_select_blocks_ex(ctypes.byref(sh), FAKE, FAKE, 3, FAKE, 4, FAKE, FAKE, FAKE,
                                     BIG, None, None) == 1
+    # fp8 summaries (2) need head_dim 128
+    sh64 = _shape(ksa, D=64)
+    assert lib.ksa_build_block_summaries_ex(ctypes.byref(sh64), FAKE, FAKE, 0, 2, FAKE, None,
+                                            None) == 2
+    assert lib.ksa_select_blocks_ex(ctypes.byref(sh64), FAKE, FAKE, 2, FAKE, 4, FAKE, FAKE, FAKE,
+                                    BIG, None, None) == 2
     # window: k < 1, NULL output, unsupported block size
     assert lib.ksa_select_window(ctypes.byref(sh), FAKE, 0, FAKE, FAKE, None, None) == 1
     assert lib.ksa_select_window(ctypes.byref(sh), FAKE, 4, None, FAKE, None, None) == 1

@@ -737,6 +737,109 @@ def test_select_blocks_bf16_summaries(ksa, oracle, D, bs, k, nblk):
     assert st.item() == 0
 
 
+# one e4m3 step of one stored element (1/8 of its binade, at the block's scale) moves a score
+# by |group query sum| x step: here at most ~0.12; the planted gap is twice that
+DELTA_FP8 = 0.25
+
+
+def _fp8_values(S8):
+    """Decoded fp8 summaries [B, Hkv, nb, D] (fp64, host): the e4m3 values times the scales."""
+    vals = S8.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return vals * ksa_scales(S8)[..., None]
+
+
+def ksa_scales(S8):
+    import block_top_sparse_ksa_b200 as k
+    return k.fp8_summary_scales(S8).cpu().to(torch.float64).numpy()
+
+
+def test_summaries_fp8_storage(ksa, oracle):
+    """fp8 storage (D = 128): a block's scale is 2^e, e the smallest exponent with
+    max|mean| <= 448 2^e, and its values are the fp32 means times 2^-e rounded to the nearest
+    e4m3 value -- bit for bit what torch's float8_e4m3fn cast makes of the GPU's own fp32
+    means -- and against the oracle's rounding of the exact means the scales agree and a
+    value differs by at most one e4m3 step.  LAST_BLOCK writes one block and its scale."""
+    rng = np.random.default_rng(1150)
+    B, Hkv, D, bs = 3, 2, 128, 16
+    T = 9 * bs + 3
+    nbm = -(-T // bs)
+    # keys of very different sizes from block to block (scales 2^-8 .. 2^7)
+    mag = np.exp2(rng.integers(-8, 8, (B, Hkv, nbm, 1, 1))).repeat(bs, 3).reshape(B, Hkv, -1, 1)
+    K = bf16_bits(rng.standard_normal((B, Hkv, nbm * bs, D)) * mag)[:, :, :T]
+    K = np.ascontiguousarray(K)
+    lens = np.array([T, 1, 2 * bs + 5], np.int32)
+    Kd, Ld = to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    S32 = ksa.ksa_build_block_summaries(Kd, Ld, bs)
+    S8 = ksa.ksa_build_block_summaries(Kd, Ld, bs, summary_dtype="fp8")
+    assert S8.dtype == torch.uint8 and tuple(S8.shape) == (B, Hkv, nbm, D)
+    scales = ksa_scales(S8)
+    want_bytes = (S32.cpu().double() / torch.from_numpy(scales)[..., None]).float().to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got_bytes = S8.cpu().numpy()
+    ref = oracle.store_fp8(oracle.block_summaries(K, lens, bs))
+    got = _fp8_values(S8)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        m32 = np.abs(S32[b, :, :nb].cpu().double().numpy()).max(-1)
+        e = np.vectorize(oracle.e4m3_scale_exp)(m32)
+        np.testing.assert_array_equal(scales[b, :, :nb], np.exp2(e))
+        assert np.array_equal(got_bytes[b, :, :nb], want_bytes[b, :, :nb])
+        d = np.abs(got[b, :, :nb] - ref[b, :, :nb]) / scales[b, :, :nb, None]
+        big = np.maximum(np.abs(got[b, :, :nb]), np.abs(ref[b, :, :nb])) / scales[b, :, :nb, None]
+        step = np.exp2(np.floor(np.log2(np.maximum(big, 2.0 ** -6))) - 3)
+        assert np.all(d <= step), d.max()
+        assert np.mean(d > 0) < 1e-3
+    S2 = ksa.alloc_summaries(B, Hkv, nbm, D, "fp8")
+    S2.fill_(0x7F)  # e4m3 NaN everywhere
+    ksa.fp8_summary_scales(S2).fill_(float("nan"))
+    ksa.ksa_build_block_summaries(Kd, Ld, bs, ksa.SUMMARY_LAST_BLOCK, summaries=S2)
+    sc2 = ksa_scales(S2)
+    for b in range(B):
+        nb = -(-lens[b] // bs)
+        assert np.array_equal(S2[b, :, nb - 1].cpu().numpy(), got_bytes[b, :, nb - 1])
+        np.testing.assert_array_equal(sc2[b, :, nb - 1], scales[b, :, nb - 1])
+        assert np.all(S2[b, :, :nb - 1].cpu().numpy() == 0x7F)
+        assert np.all(np.isnan(sc2[b, :, :nb - 1]))
+
+
+@pytest.mark.parametrize("bs,k,nblk", [(16, 8, 40), (32, 6, 300), (16, 32, 1100)])
+def test_select_blocks_fp8_summaries(ksa, oracle, bs, k, nblk):
+    """Selection from fp8-stored summaries: the oracle's blocks for fp8-stored means, with a
+    planted gap; the fused decode-step form refreshes the last block (values and scale)."""
+    rng = np.random.default_rng(1250 + nblk)
+    B, Hq, Hkv, D = 3, 8, 2, 128
+    T = nblk * bs + 7
+    lens = np.array([T, 13 * bs + 1, 3 * bs], np.int32)
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    for b in range(B):
+        K[b], _ = gap_fix_row(oracle, q[b], K[b], int(lens[b]), bs, k, delta=DELTA_FP8,
+                              summary_fp8=True)
+        assert min_boundary_gap(oracle, q[b], K[b], int(lens[b]), bs, k,
+                                summary_fp8=True) >= DELTA_FP8
+    qd, Kd, Ld = to_dev_bf16(q), to_dev_bf16(K), torch.from_numpy(lens).to(DEV)
+    st = status_tensor()
+    S = ksa.ksa_build_block_summaries(Kd, Ld, bs, summary_dtype="fp8", dev_status=st)
+    idx, cnt = ksa.ksa_select_blocks(qd, S, Ld, bs, T, k, dev_status=st)
+    ref_idx, ref_cnt = oracle.select_blocks(q, K, lens, bs, k, summary_fp8=True)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    # fused form: stale last blocks (values and scales), refreshed in fp8 by the call
+    S_old = ksa.alloc_summaries(B, Hkv, S.shape[2], D, "fp8")
+    S_old.copy_(S)
+    sc_old = ksa.fp8_summary_scales(S_old)
+    sc_old.copy_(ksa.fp8_summary_scales(S))
+    for b in range(B):
+        jl = (lens[b] - 1) // bs
+        S_old[b, :, jl] = 0
+        sc_old[b, :, jl] = 0.0
+    idx2, cnt2 = ksa.ksa_decode_select_blocks(qd, Kd, S_old, Ld, bs, k, dev_status=st)
+    assert torch.equal(S_old, S)
+    assert torch.equal(sc_old.view(torch.int32), ksa.fp8_summary_scales(S).view(torch.int32))
+    assert torch.equal(idx2, idx) and torch.equal(cnt2, cnt)
+    assert st.item() == 0
+
+
 # ---------------------------------------------------------------------------
 # paged K/V cache (page = block)
 

@@ -62,8 +62,18 @@ MUTANTS = [
     ("bf16 subnormal spacing of the normal range", "if (q < -133) q = -133;",
      "if (q < -126) q = -126;", 0,
      [lambda o: pins.test_round_bf16_format_values(o, 2.0 ** -133, 0x0001)]),
-    ("bf16 summary storage never applied", "if (summary_bf16) {", "if (0) {", 0,
+    ("bf16 summary storage never applied", "if (summary_fmt == 1) {", "if (0) {", 0,
      [pins.test_select_blocks_bf16_storage_tie]),
+    ("e4m3 ties rounded away from zero",
+     "if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;\n  double v = ldexp(r, q);",
+     "if (frac >= 0.5) r += 1.0;\n  double v = ldexp(r, q);", 0,
+     [lambda o: pins.test_round_e4m3_format_values(o, 1.0625, 1.0)]),
+    ("e4m3 spacing one bit too fine", "int q = e - 4; /* spacing", "int q = e - 5; /* spacing", 0,
+     [pins.test_round_e4m3_matches_torch]),
+    ("e4m3 scale one binade too small", "while (amax > ldexp(448.0, e)) ++e;",
+     "while (amax > ldexp(448.0, e + 1)) ++e;", 0, [pins.test_e4m3_scale_exponent]),
+    ("fp8 summary storage never applied", "  } else if (summary_fmt == 2) {",
+     "  } else if (0) {", 0, [pins.test_select_blocks_fp8_storage]),
     ("page row ignores the kv-head",
      "pages + (((size_t)page * Hkv + g) * bs + t % bs) * D;",
      "pages + (((size_t)page * Hkv) * bs + t % bs) * D;", 0,

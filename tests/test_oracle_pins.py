@@ -818,3 +818,108 @@ def test_recall_with_huge_logits(oracle):
     assert r1[0, 0] == pytest.approx(math.exp(-64) / (1 + math.exp(-64) + math.exp(-128)),
                                      rel=1e-12)
 
+
+
+# --------------------------------------------------------------------------
+# fp8 (e4m3) block summaries: the stored form of a block mean (reading R13)
+
+
+def _e4m3_grid():
+    """Every finite non-negative e4m3 value, from the format's definition: normal
+    (1 + m/8) 2^(E-7) for E = 1..15 (not E = 15, m = 7), subnormal (m/8) 2^-6."""
+    vals = [(m / 8) * 2.0 ** -6 for m in range(8)]
+    vals += [(1 + m / 8) * 2.0 ** (E - 7) for E in range(1, 16) for m in range(8)
+             if not (E == 15 and m == 7)]
+    return np.array(vals)
+
+
+@pytest.mark.parametrize("x,want", [
+    (1.0, 1.0), (448.0, 448.0), (500.0, 448.0), (-1e9, -448.0),
+    (2.0 ** -9, 2.0 ** -9),              # the smallest subnormal
+    (2.0 ** -10, 0.0),                   # halfway to 0: even (0)
+    (3 * 2.0 ** -10, 2 * 2.0 ** -9),     # halfway between 1 and 2 units: even (2)
+    (1.0625, 1.0),                       # 1 + 1/16: halfway, even mantissa 0
+    (1.1875, 1.25),                      # 1 + 3/16: halfway, even mantissa 2
+    (-7.5, -7.5), (0.0703125, 0.0703125), (240.0, 240.0), (232.0, 224.0),
+])
+def test_round_e4m3_format_values(oracle, x, want):
+    assert oracle.round_e4m3(x) == want
+
+
+def test_round_e4m3_is_the_nearest_grid_value(oracle):
+    """Brute force over the grid: the nearest value, ties to the even mantissa (the even
+    index in the ordered grid)."""
+    grid = _e4m3_grid()
+    rng = np.random.default_rng(81)
+    xs = np.concatenate([rng.uniform(0, 448, 3000), np.exp2(rng.uniform(-11, 8.8, 3000)),
+                         (grid[:-1] + grid[1:]) / 2])  # every midpoint
+    for x in xs:
+        d = np.abs(grid - x)
+        best = np.flatnonzero(d == d.min())
+        want = grid[best[0]] if len(best) == 1 else grid[[i for i in best if i % 2 == 0][0]]
+        assert oracle.round_e4m3(x) == want, x
+        assert oracle.round_e4m3(-x) == -want
+
+
+def test_round_e4m3_matches_torch(oracle):
+    """torch's float8_e4m3fn cast rounds to nearest even as well (values within +-448)."""
+    rng = np.random.default_rng(82)
+    x = np.clip(rng.standard_normal(20000) * np.exp2(rng.integers(-12, 9, 20000)), -448, 448)
+    t = torch.tensor(x, dtype=torch.float64).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_e4m3(x), t)
+
+
+def test_e4m3_scale_exponent(oracle):
+    """e is the smallest exponent with amax <= 448 2^e."""
+    for e in range(-20, 10):
+        assert oracle.e4m3_scale_exp(448.0 * 2.0 ** e) == e
+        assert oracle.e4m3_scale_exp(np.nextafter(448.0 * 2.0 ** e, np.inf)) == e + 1
+    rng = np.random.default_rng(83)
+    for amax in np.exp2(rng.uniform(-30, 20, 500)):
+        e = oracle.e4m3_scale_exp(amax)
+        assert 448.0 * 2.0 ** (e - 1) < amax <= 448.0 * 2.0 ** e
+    assert oracle.e4m3_scale_exp(0.0) == 0
+
+
+def test_store_fp8_blocks(oracle):
+    """Each block is scaled by its own power of two: the largest |mean| lands in
+    (224, 448], every stored value is an e4m3 value times 2^e, and blocks whose means are
+    already such values are stored exactly."""
+    rng = np.random.default_rng(84)
+    S = rng.standard_normal((5, 3, 128)) * np.exp2(rng.integers(-6, 6, (5, 3, 1)))
+    T = oracle.store_fp8(S)
+    grid = np.concatenate([-_e4m3_grid()[::-1], _e4m3_grid()])
+    for blk, out in zip(S.reshape(-1, 128), T.reshape(-1, 128)):
+        e = oracle.e4m3_scale_exp(np.abs(blk).max())
+        assert 224.0 < np.abs(blk).max() / 2.0 ** e <= 448.0
+        assert np.all(np.isin(out / 2.0 ** e, grid))
+        assert np.max(np.abs(out - blk) / 2.0 ** e) <= 16.0  # half a spacing at 448 * 2^e
+    exact = np.array([[1.0, -0.5, 0.375, 448.0 / 64]])  # e4m3 values times 2^-6
+    np.testing.assert_array_equal(oracle.store_fp8(exact), exact)
+
+
+def test_select_blocks_fp8_storage(oracle):
+    """Stored as fp8, block means change the ranking where the rounding moves a score past
+    another, and not where every mean is stored exactly."""
+    D, bs = 4, 2
+    q = bf16_bits(np.array([[[1.0, 0, 0, 0]]]))
+    # every block's largest mean is 8: scale 2^-5 (8 <= 448 2^-5 = 14 < 2 * 8), so the first
+    # mean x is stored as round_e4m3(32 x) / 32, on a grid of 4 / 32 = 1/8 in [1, 2):
+    #   1.0625 -> 34, halfway between 32 and 36: the even mantissa, 32 -> 1.0
+    #   1.09375 -> 35 -> 36 -> 1.125;  1.125 -> 36 -> 1.125 (exact)
+    K = np.zeros((1, 1, 6, D))
+    K[0, 0, 0:2] = [1.0625, 8, 0, 0]
+    K[0, 0, 2:4] = [1.09375, 8, 0, 0]
+    K[0, 0, 4:6] = [1.125, 8, 0, 0]
+    K = bf16_bits(K)
+    L = np.array([6], np.int32)
+    idx, _, s_exact = oracle.select_blocks(q, K, L, bs, 1, want_scores=True)
+    idx8, _, s8 = oracle.select_blocks(q, K, L, bs, 1, want_scores=True, summary_fp8=True)
+    assert list(idx[0, 0]) == [2]                 # 1.125 is the best exact mean
+    assert s8[0, 0, 1] == s8[0, 0, 2] == 1.125    # 1.09375 is stored as 1.125: a tie ...
+    assert list(idx8[0, 0]) == [1]                # ... that the lower block wins
+    # means that are e4m3 values times 2^e are stored exactly: the exact path's result
+    K2 = bf16_bits(np.array([[[[0.5, 4, 0, 0], [0.5, 4, 0, 0], [0.25, 2, 0, 0], [0.25, 2, 0, 0]]]]))
+    i_a, _ = oracle.select_blocks(q, K2, np.array([4], np.int32), bs, 1)
+    i_b, _ = oracle.select_blocks(q, K2, np.array([4], np.int32), bs, 1, summary_fp8=True)
+    assert np.array_equal(i_a, i_b)
