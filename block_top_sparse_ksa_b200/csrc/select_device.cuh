@@ -186,18 +186,23 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
         const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
         if (lane + off < 32) incl += y;
       }
-      uint32_t run = incl - tot;
-      if (run < remaining && incl >= remaining) {  // the one lane holding the k-th key
-        for (int b = 31; b >= 0; --b) {
-          const uint32_t before = run, c = hist[32 * lane + b];
-          run += c;
-          if (run >= remaining) {
-            misc[0] = static_cast<uint32_t>(32 * lane + b);
-            misc[1] = before;
-            misc[2] = c;
-            break;
-          }
-        }
+      // the one lane whose buckets hold the k-th live key; then the whole warp walks that
+      // lane's 32 buckets from the top, one bucket per lane, with a prefix sum
+      const int owner = __ffs(__ballot_sync(0xffffffffu, incl - tot < remaining &&
+                                                             incl >= remaining)) - 1;
+      const uint32_t above_owner = __shfl_sync(0xffffffffu, incl - tot, owner);
+      const uint32_t c = hist[32 * owner + 31 - lane];
+      uint32_t pre = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, pre, off);
+        if (lane >= off) pre += y;
+      }
+      const int j = __ffs(__ballot_sync(0xffffffffu, above_owner + pre >= remaining)) - 1;
+      if (lane == j) {
+        misc[0] = static_cast<uint32_t>(32 * owner + 31 - j);
+        misc[1] = above_owner + pre - c;
+        misc[2] = c;
       }
     }
     __syncthreads();
@@ -246,8 +251,7 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
   __syncthreads();
   if (warp == 0) {
     // lane l owns words [WPL l, WPL l + WPL): the lowest-index `remaining` live keys join the
-    // selection (written back into selw), then every winner gets its place from a prefix
-    // count of the words
+    // selection (written back into selw); then each word's place in the output (livew)
     constexpr int WPL = (W + 31) / 32;
     const int w0 = lane * WPL, w1 = min(w0 + WPL, W);
     uint32_t nl = 0u;
@@ -286,12 +290,16 @@ __device__ __forceinline__ void fast_topk(const uint32_t *krow, int n, int k, in
     }
     ps -= ns;
     for (int w = w0; w < w1; ++w) {
-      uint32_t x = selw[w];
-      while (x != 0u) {
-        const int b = __ffs(x) - 1;
-        x &= x - 1u;
-        out[ps++] = 32 * w + b;
-      }
+      livew[w] = ps;
+      ps += __popc(selw[w]);
+    }
+  }
+  __syncthreads();
+  for (int w = tid; w < W; w += NT) {  // every thread writes the winners of its words
+    uint32_t x = selw[w], pos = livew[w];
+    while (x != 0u) {
+      out[pos++] = 32 * w + (__ffs(x) - 1);
+      x &= x - 1u;
     }
   }
 }
