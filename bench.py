@@ -296,17 +296,25 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
+def sources_digest(paths) -> str:
+    """First 16 hex digits of the SHA-256 of the files' bytes, concatenated in order."""
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def stored_traffic(kernel: str, workload: str, batch: int):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken at this batch and
-    the kernel source is unchanged since (else None)."""
+    """DRAM bytes per launch from a committed ncu capture, if it stands for this batch and the
+    kernel's sources are unchanged since (else None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
         ent = rec[kernel][workload]
         if int(ent["batch"]) != batch:
             return None
-        src = open(os.path.join(ROOT, ent["source"]), "rb").read()
-        if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha256_16"]:
+        if sources_digest(ent["sources"]) != ent["sources_sha256_16"]:
             return None
         return float(ent["dram_bytes_per_launch"])
     except Exception:

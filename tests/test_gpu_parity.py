@@ -222,6 +222,92 @@ def test_token_list_attention_shared(ksa, oracle, D, tpi):
     assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, tpi, shared=True) == 0
 
 
+def _list_with_runs(rng, n_units, cap, tpi, past_end=0):
+    """Ascending distinct units: a recency window ending at the last unit, runs of 15 to
+    100 tokens at unaligned starts, scattered singles up to cap, and `past_end` units
+    beyond the row's end."""
+    w = min(n_units, cap // 3)
+    picks = set(range(n_units - w, n_units + past_end))
+    for ln in (15, 16, 17, 33, 48, 100):
+        u = -(-ln // tpi)
+        s = int(rng.integers(0, max(1, n_units - w - u)))
+        picks.update(range(s, min(s + u, n_units)))
+    rest = np.setdiff1d(np.arange(n_units), np.fromiter(picks, np.int64))
+    extra = cap - len(picks)
+    if extra > 0:
+        picks.update(rng.choice(rest, size=min(extra, len(rest)), replace=False).tolist())
+    out = np.sort(np.fromiter(picks, np.int64)).astype(np.int32)
+    assert len(out) <= cap
+    return out
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("tpi", [1, 4])
+def test_token_list_runs_of_consecutive_rows(ksa, oracle, D, tpi):
+    """Token lists holding runs (a recency window, adjacent picks, runs that start and end
+    inside a stage) next to scattered picks; one row's list runs past its end."""
+    rng = np.random.default_rng(520 + D + tpi)
+    B, Hq, Hkv = 3, 16, 4
+    T = 3000
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = np.array([3000, 1999, 2500], np.int32)
+    cap = 900 // tpi
+    idx = np.full((B, cap), -1, np.int32)
+    cnt = np.zeros((B,), np.int32)
+    for b in range(B):
+        lst = _list_with_runs(rng, -(-int(lens[b]) // tpi), cap, tpi, past_end=2 if b == 1 else 0)
+        idx[b, :len(lst)] = lst
+        cnt[b] = len(lst)
+    st = _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, tpi, shared=True)
+    assert st == 2  # KSA_FLAG_INDEX_SKIPPED, from row 1's entries past its end
+
+
+@pytest.mark.parametrize("Hkv", [1, 2])
+def test_paged_token_list_runs(ksa, oracle, Hkv):
+    """Paged pools with runs of consecutive tokens that cross page boundaries, on pages in
+    sequence (with one kv-head, consecutive pool rows) and on shuffled pages: the result
+    equals the contiguous cache's bit for bit and the oracle's."""
+    rng = np.random.default_rng(1350 + Hkv)
+    B, Hq, D, bs, mb = 2, 8, 128, 16, 60
+    T = mb * bs
+    lens = np.array([T, 37 * bs + 5], np.int32)
+    n_pages = B * mb + 7
+    K_pages = rand_bits(rng, (n_pages, Hkv, bs, D))
+    V_pages = rand_bits(rng, (n_pages, Hkv, bs, D))
+    # row 0's pages in sequence, row 1's in sequence for its first half, then shuffled
+    tbl = np.zeros((B, mb), np.int32)
+    tbl[0] = np.arange(mb)
+    tail = mb + np.arange(mb)
+    tail[mb // 2:] = rng.permutation(tail[mb // 2:])
+    tbl[1] = tail
+    K = oracle.gather_pages(K_pages, tbl, lens)
+    V = oracle.gather_pages(V_pages, tbl, lens)
+    q = rand_bits(rng, (B, Hq, D))
+    cap = 400
+    lst = np.full((B, cap), -1, np.int32)
+    n_t = np.zeros((B,), np.int32)
+    for b in range(B):
+        pick = _list_with_runs(rng, int(lens[b]), cap, 1)
+        lst[b, :len(pick)] = pick
+        n_t[b] = len(pick)
+    qd, Ld = to_dev_bf16(q), torch.from_numpy(lens).to(DEV)
+    Kp, Vp = to_dev_bf16(K_pages), to_dev_bf16(V_pages)
+    Kc, Vc = to_dev_bf16(K), to_dev_bf16(V)
+    td = torch.from_numpy(tbl).to(DEV)
+    lst_d, n_d = torch.from_numpy(lst).to(DEV), torch.from_numpy(n_t).to(DEV)
+    st = status_tensor()
+    out_p, _ = ksa.ksa_sparse_decode_attn_paged(qd, Kp, Vp, td, Ld, lst_d, n_d, tokens_per_idx=1,
+                                                idx_shared=True, dev_status=st)
+    out_c, _ = ksa.ksa_sparse_decode_attn(qd, Kc, Vc, Ld, lst_d, n_d, tokens_per_idx=1,
+                                          idx_shared=True)
+    assert torch.equal(out_p, out_c)
+    ref, _, _ = oracle.attention(q, K, V, lens, lst, n_t, 1, True)
+    assert_out_close(out_p.cpu().numpy(), ref)
+    assert st.item() == 0
+
+
 def test_attention_edge_cases(ksa, oracle):
     rng = np.random.default_rng(600)
     B, Hq, Hkv, D, T, bs = 3, 4, 2, 128, 256, 16
