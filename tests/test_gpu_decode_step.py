@@ -76,6 +76,14 @@ CASES = [
     (2, 8, 2, 128, 3000 * 16, 16, 64, torch.float32, 0),      # 3000 blocks
     (4, 8, 2, 128, 512, 16, 64, torch.float32, 0),            # k covers every block
     (64, 16, 8, 128, 16384, 32, 32, torch.float32, 0),        # Qwen3-0.6B step shape
+    # between half and all of the resident attention CTAs' worth of rows (148 SMs x 3): the
+    # attention grid is one CTA per row
+    (32, 32, 8, 128, 8192, 16, 64, torch.float32, 0),         # 256 rows, 512 blocks
+    (32, 32, 8, 128, 32768, 16, 128, torch.float32, 0),       # the Qwen3-8B step shape
+    (28, 8, 8, 128, 4096, 16, 128, torch.float32, 1),         # rows kept whole and ranked
+    (150, 8, 2, 64, 4096, 16, 24, torch.bfloat16, 0),         # D 64, bf16 summaries
+    (55, 16, 8, 128, 10000, 32, 20, torch.bfloat16, 0),       # 440 rows
+    (28, 8, 8, 64, 5200 * 16, 16, 64, torch.float32, 0),      # 5200 blocks
 ]
 
 
@@ -99,11 +107,13 @@ def test_decode_step_equals_the_two_calls(ksa, B, Hq, Hkv, D, T, bs, k, sdt, odt
     assert torch.isfinite(got[2].float()).all()
 
 
-def test_decode_step_repeated_calls_on_one_workspace(ksa):
+@pytest.mark.parametrize("B", [16, 32])
+def test_decode_step_repeated_calls_on_one_workspace(ksa, B):
     """Calls back to back on one workspace, alternating two query sets and two caches: each
     result equals the first result for its inputs (every call leaves the workspace's
-    semaphores as it found them)."""
-    B, Hq, Hkv, D, T, bs, k = 16, 32, 8, 128, 16384, 16, 64
+    semaphores as it found them).  With 32 rows of 8 kv-heads the attention grid is one
+    CTA per row."""
+    Hq, Hkv, D, T, bs, k = 32, 8, 128, 16384, 16, 64
     qa, Ka, Va, la = _inputs(B, Hq, Hkv, D, T, bs, seed=1)
     qb, Kb, Vb, lb = _inputs(B, Hq, Hkv, D, T, bs, seed=2)
     Sa = _prefill(ksa, Ka, la, bs, torch.float32)
@@ -126,10 +136,11 @@ def test_decode_step_repeated_calls_on_one_workspace(ksa):
     assert not torch.equal(first["a"][2], first["b"][2])
 
 
-def test_decode_step_flags_bad_lengths_and_nan_scores(ksa):
+@pytest.mark.parametrize("B,Hkv", [(4, 2), (32, 8)])
+def test_decode_step_flags_bad_lengths_and_nan_scores(ksa, B, Hkv):
     """Device-side data errors flag the status word as in the two calls: a seq_len outside
     [1, T] is clamped, a NaN summary ranks lowest."""
-    B, Hq, Hkv, D, T, bs, k = 4, 8, 2, 128, 2048, 16, 8
+    Hq, D, T, bs, k = 8 * Hkv // 2, 128, 2048, 16, 8
     q, K, V, lens = _inputs(B, Hq, Hkv, D, T, bs, seed=3)
     S = _prefill(ksa, K, lens, bs, torch.float32)
     lens[3] = T + 5
