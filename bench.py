@@ -610,8 +610,8 @@ def run_block_e2e(args, dist, wl: BlockWorkload):
 def run_unified(args, dist, dev):
     import block_top_sparse_ksa_b200 as ksa
     from block_top_sparse_ksa_b200 import synth
-    sh = synth.LESSISMORE
-    inp = synth.lessismore_inputs(device=dev)
+    _, sh = resolve_workload(args.workload, args.batch)
+    inp = synth.lessismore_inputs(device=dev, shape=sh)
     B, Hq, Hkv, D, T = sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, sh.capacity
     ws = torch.empty((ksa.ksa_unified_select_workspace(B, Hq, Hkv, D, T, sh.per_head_topk,
                                                        sh.token_budget),),

@@ -210,11 +210,15 @@ __global__ void __launch_bounds__(kPickThreads) unified_pick_kernel(const Unifie
 // pass never piles equal digits of tied keys into one bin (scores on a coarse
 // grid tie a lot).  Once the candidates are all equal the threshold is found.
 // Keys above it vote; of the keys equal to it the lowest-index ones vote
-// (ballots and per-warp counts, in token order).
+// (ballots and per-warp counts, in token order).  Slots past the row's end
+// hold key 0, the lowest key there is, and take part like real keys: the
+// P-th largest is a real key (P < L), and where it is 0 the real zeros come
+// first in token order, so a padding slot never votes.
 template <int KPL>
 __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const UnifiedArgs a) {
   constexpr int NT = kPickRegThreads, NW = NT / 32;
   __shared__ __align__(16) uint32_t hist[NW][256];
+  __shared__ uint32_t spare[NT];  // the non-candidates' adds (never read)
   __shared__ uint32_t red[3][NW];
   __shared__ uint32_t xinfo[3];
   const int b = blockIdx.x / a.Hq, h = blockIdx.x % a.Hq;
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
     uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
 #pragma unroll
     for (int e = 0; e < KPL; ++e) {
-      if (tid + NT * e < L && (key[e] & pmask) == prefix) {
+      if ((key[e] & pmask) == prefix) {
         kmin = min(kmin, key[e]);
         kmax = max(kmax, key[e]);
         ++cnt;
@@ -284,8 +288,10 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
     __syncthreads();  // also: red was read by everyone
 #pragma unroll
     for (int e = 0; e < KPL; ++e) {
-      if (tid + NT * e < L && (key[e] & pmask) == prefix)
-        atomicAdd(&hist[warp][(key[e] >> sh) & 255u], 1u);
+      // every slot adds: non-candidates to a spare word of their own (a
+      // conditional add here costs the compiler a register per key)
+      const bool c = (key[e] & pmask) == prefix;
+      atomicAdd(c ? &hist[warp][(key[e] >> sh) & 255u] : &spare[tid], 1u);
     }
     __syncthreads();
     if (warp == 0) {  // lane l owns bins [8l, 8l + 8); counts from the top bin down
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
   if (!all_eq) {
 #pragma unroll
     for (int e = 0; e < KPL; ++e) {
-      const bool eq = tid + NT * e < L && key[e] == tau;
+      const bool eq = key[e] == tau;
       const uint32_t eb = __ballot_sync(0xffffffffu, eq);
       if (lane == 0) pre[e * NW + warp] = __popc(eb);
     }
@@ -369,9 +375,7 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
   uint32_t *bits = a.bits + (static_cast<size_t>(b) * a.Hq + h) * W32;
 #pragma unroll
   for (int e = 0; e < KPL; ++e) {
-    const int j = tid + NT * e;
-    const bool ok = j < L;
-    const bool gt = ok && key[e] > tau, eq = ok && key[e] == tau;
+    const bool gt = key[e] > tau, eq = key[e] == tau;
     bool sel = gt || eq;
     if (!all_eq) {
       const uint32_t eb = __ballot_sync(0xffffffffu, eq);
