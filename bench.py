@@ -670,7 +670,11 @@ def run_unified(args, dist, dev):
                      "kernel_sum_ms": t_sel + t_att3},
         # selection: scores, picks, (vote counting when the picks keep the row's keys in
         # registers: capacity <= 24576), shared set; then one attention launch per layer
-        "gpu_launches": ((4 if T <= 24576 else 3) + len(inp.layers)) * args.steps, "clocks": clk,
+        # selection: scores, per-head picks, then the shared set straight from the pick bit
+        # sets (register picks, < 64 heads), or votes + set; rows over 24576 tokens: scores,
+        # picks with votes, set
+        "gpu_launches": ((3 if T > 24576 or (Hq < 64 and -(-T // 32) <= 1024) else 4)
+                         + len(inp.layers)) * args.steps, "clocks": clk,
         "config": {"workload": sh.name, "batch_per_gpu": B, "num_q_heads": Hq,
                    "num_kv_heads": Hkv, "head_dim": D, "context": sh.seq_len,
                    "per_head_topk": sh.per_head_topk, "token_budget": sh.token_budget,

@@ -440,6 +440,157 @@ __global__ void __launch_bounds__(kPickThreads) unified_topk_list_kernel(const U
   if (threadIdx.x == 0) a.num_sel[static_cast<size_t>(b) * a.Hq + h] = k;
 }
 
+// Exclusive prefix sum of v over the block (thread order) and the total.
+// `scan` holds NT / 32 + 1 words of shared memory.  All threads must call.
+template <int NT>
+__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t *scan,
+                                                        uint32_t &total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) scan[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = lane < NW ? scan[lane] : 0u;
+    uint32_t wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += y;
+    }
+    if (lane < NW) scan[lane] = wi - w;
+    if (lane == 31) scan[NW] = wi;
+  }
+  __syncthreads();
+  const uint32_t r = scan[warp] + incl - v;
+  total = scan[NW];
+  __syncthreads();  // scan is reused by the next call
+  return r;
+}
+
+// Shared set straight from the per-head pick bit sets (the register-pick path,
+// fewer than 64 heads): CTA per row, thread t owns the 32 candidates of bit
+// word t.  It adds the row's Hq words into six bit planes (a ripple-carry
+// counter per token lane, so plane i holds bit i of every token's vote count),
+// counts the tokens of each vote value from the planes, finds the threshold
+// vote from the top value down, then -- with masks of the tokens above it and
+// equal to it, again from the planes -- two block scans give each thread its
+// share of the tied tokens (lowest first) and its output position, and it
+// writes its picks in token order.  The same set as the votes kernel followed
+// by unified_set_kernel, in one launch.
+__global__ void __launch_bounds__(kSetThreads) unified_set_bits_kernel(const UnifiedArgs a) {
+  constexpr int NT = kSetThreads, NW = NT / 32;
+  __shared__ uint32_t hist[NW][64];
+  __shared__ uint32_t scan[NW + 1];
+  __shared__ uint32_t info[2];
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int L = clamp_len(a.seq_lens[b], a.T, nullptr);
+  int32_t *out = a.token_idx + static_cast<size_t>(b) * a.budget;
+  if (L <= a.budget) {
+    for (int i = tid; i < a.budget; i += NT) out[i] = i < L ? i : -1;
+    if (tid == 0) a.num_sel[b] = L;
+    return;
+  }
+  const int n = L - a.R;  // candidates [0, L - R)
+  const int k = a.budget - a.R;
+  if (k > 0) {
+    // this thread's candidates: tokens 32 tid + j, j set in vm
+    const int base = tid * 32;
+    const uint32_t vm = base + 32 <= n ? 0xffffffffu : (base < n ? (1u << (n - base)) - 1u : 0u);
+    uint32_t c[6] = {0u, 0u, 0u, 0u, 0u, 0u};  // bit planes of the vote counts
+    if (vm != 0u) {  // (words past the candidates are not read: they may be stale)
+      const int W32 = (a.T + 31) / 32;
+      const uint32_t *bits = a.bits + static_cast<size_t>(b) * a.Hq * W32 + tid;
+#pragma unroll 8
+      for (int h = 0; h < a.Hq; ++h) {
+        uint32_t carry = __ldcg(bits + static_cast<size_t>(h) * W32);
+#pragma unroll
+        for (int i = 0; i < 6; ++i) {
+          const uint32_t t = c[i] & carry;
+          c[i] ^= carry;
+          carry = t;
+        }
+      }
+    }
+    // tokens of each vote value, per warp
+    for (int v = 0; v <= a.Hq; ++v) {
+      uint32_t m = vm;
+#pragma unroll
+      for (int i = 0; i < 6; ++i) m &= ((v >> i) & 1) ? c[i] : ~c[i];
+      const uint32_t cnt = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popc(m)));
+      if (lane == 0) hist[warp][v] = cnt;
+    }
+    __syncthreads();
+    if (tid < 64) {
+      uint32_t t = 0u;
+      for (int w = 0; w < NW; ++w) t += tid <= a.Hq ? hist[w][tid] : 0u;
+      hist[0][tid] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {  // lane l owns values 2l, 2l + 1; counts from the top value down
+      const uint32_t c1 = hist[0][2 * lane + 1], c0 = hist[0][2 * lane];
+      const uint32_t tot = c0 + c1;
+      uint32_t incl = tot;  // over lanes >= this one
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl += y;
+      }
+      const uint32_t above = incl - tot;
+      const uint32_t kk = static_cast<uint32_t>(k);
+      if (above < kk && above + c1 >= kk) {
+        info[0] = 2u * lane + 1u;
+        info[1] = above;
+      } else if (above + c1 < kk && above + tot >= kk) {
+        info[0] = 2u * lane;
+        info[1] = above + c1;
+      }
+    }
+    __syncthreads();
+    const uint32_t tau = info[0];
+    const uint32_t take_eq = static_cast<uint32_t>(k) - info[1];  // tied picks, lowest first
+    // masks of this thread's tokens with votes above tau and equal to it
+    uint32_t gt = 0u, eq = 0xffffffffu;
+#pragma unroll
+    for (int i = 5; i >= 0; --i) {
+      if ((tau >> i) & 1u) {
+        eq &= c[i];
+      } else {
+        gt |= eq & c[i];
+        eq &= ~c[i];
+      }
+    }
+    gt &= vm;
+    eq &= vm;
+    uint32_t tot;
+    const uint32_t my_eq = static_cast<uint32_t>(__popc(eq));
+    const uint32_t eq_before = block_exclusive_sum<NT>(my_eq, scan, tot);
+    const uint32_t eq_take = eq_before >= take_eq ? 0u : min(my_eq, take_eq - eq_before);
+    uint32_t keep = 0u, rest = eq;  // the lowest eq_take tied tokens
+    for (uint32_t q = 0u; q < eq_take; ++q) {
+      const uint32_t low = rest & (~rest + 1u);
+      keep |= low;
+      rest ^= low;
+    }
+    uint32_t sel = gt | keep;
+    uint32_t pos = block_exclusive_sum<NT>(static_cast<uint32_t>(__popc(sel)), scan, tot);
+    while (sel != 0u) {
+      out[pos++] = base + __ffs(sel) - 1;
+      sel &= sel - 1u;
+    }
+  }
+  for (int i = tid; i < a.R; i += NT) out[k + i] = n + i;
+  if (tid == 0) a.num_sel[b] = a.budget;
+}
+
 // Shared set: CTA per row.
 __global__ void __launch_bounds__(kSetThreads) unified_set_kernel(const UnifiedArgs a) {
   __shared__ uint32_t hist[256];
@@ -524,6 +675,9 @@ cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_
     else if (per <= 80) err = launch_pdl(unified_pick_reg_kernel<80>, pgrid, pblock, 0, stream, a);
     else err = launch_pdl(unified_pick_reg_kernel<96>, pgrid, pblock, 0, stream, a);
     if (err != cudaSuccess) return err;
+    if (a.Hq < 64 && (a.T + 31) / 32 <= kSetThreads)  // the set straight from the bit sets
+      return launch_pdl(unified_set_bits_kernel, dim3(static_cast<unsigned>(a.B)),
+                        dim3(kSetThreads), 0, stream, a);
     const long long nt = static_cast<long long>(a.B) * ((a.T + 31) / 32) * 32;
     err = launch_pdl(unified_votes_kernel, dim3(static_cast<unsigned>((nt + 255) / 256)),
                      dim3(256), 0, stream, a);
