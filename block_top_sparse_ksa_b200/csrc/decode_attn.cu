@@ -63,9 +63,18 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   // With index lists (rows of equal padded length) and between half and all of the
   // resident CTAs' worth of rows, one CTA per row: slices then end on row boundaries, and
   // no row is split, so no CTA ends with a partial merge (measured on the Qwen3-8B shape,
-  // 256 rows: attention 61.2 -> 55.0 us; two or more rows per CTA gained nothing).
+  // 256 rows: attention 61.2 -> 55.0 us; two or more rows per CTA gained nothing).  With
+  // block lists and fewer rows, each row is cut into s = n / rows equal parts, one per
+  // CTA, so every CTA holds one piece of one row (128 rows of 250 stages: 59.3 -> 53.0
+  // us).  Token lists keep every resident CTA: there the copy-issuing producer warps set
+  // the pace, and fewer CTAs measured slower (64.3 -> 66.0 us on the same rows).
   const long long rows = p.W / p.V;
-  if (MODE != kModeDense && 2 * rows >= n && rows <= n) n = rows;
+  if (MODE != kModeDense) {
+    if (2 * rows >= n && rows <= n)
+      n = rows;
+    else if (MODE == kModeTma && 2 * rows < n)
+      n = rows * (n / rows);
+  }
   p.N = static_cast<int>(n);
   // programmatic: the CTAs take their places and set up while the grid in
   // front (normally the small ranking launch) finishes
