@@ -13,11 +13,22 @@ constexpr int kStageTok = 16;  // tokens per pipeline stage (16 or 32: one or tw
 constexpr int kTiles = kStageTok / 16;
 constexpr uint32_t kFullMask = kStageTok >= 32 ? 0xffffffffu : ((1u << kStageTok) - 1u);
 constexpr int kConsumers = 4;
-constexpr int kAttnThreads = (kConsumers + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeParts = 4;  // split-row partials combined per round of loads
 
 enum { kModeDense = 0, kModeTma = 1, kModeCp = 2 };
+
+// Token lists take two producer warps (stages alternate between them): their
+// 16-byte copies are issued by the warps themselves, and one warp per CTA set
+// the pace.
+template <int MODE>
+__host__ __device__ constexpr int attn_producers() {
+  return MODE == kModeCp ? 2 : 1;
+}
+template <int MODE>
+__host__ __device__ constexpr int attn_threads() {
+  return (kConsumers + attn_producers<MODE>()) * 32;
+}
 
 template <int D>
 struct Cfg {
@@ -236,7 +247,7 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
 
   int issued = 0;  // stages the producer filled (TMA modes: uses of the lane's own buffer)
 
-  if (warp == kConsumers) {
+  if (warp >= kConsumers) {
     // ------------------------------------------------------------ producer
     uint32_t skipped = 0u;
     if (MODE != kModeCp) {
@@ -331,9 +342,14 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
         }
       }
     } else {
-      // token lists: the warp fills one stage at a time with 16-byte cp.async
-      // (row u of a stage <- list entry j*eps + u/tpi, token offset u%tpi); the
-      // list is read 32 entries at a time, one per lane, the next 32 in flight
+      // token lists: each producer warp fills its stages one at a time with
+      // 16-byte cp.async (row u of a stage <- list entry j*eps + u/tpi, token
+      // offset u%tpi); producer pw takes the CTA's stages i = pw (mod 2), so it
+      // only ever fills the buffers of that parity (kStages is even).  The list
+      // is read 32 entries at a time, one per lane, the next 32 in flight.
+      constexpr int NP = attn_producers<MODE>();
+      static_assert(NS % NP == 0, "a buffer belongs to one producer");
+      const int pw = warp - kConsumers;
       bool stop = false;
       int i = 0;
       for (int r = r_first; r <= r_last && !stop; ++r) {
@@ -355,6 +371,12 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
           nxt = (wbase + 32 + lane < ri.n_idx) ? c1 : -1;
         }
         for (int j = ja; j < jb; ++j, ++i) {
+          if (j * eps >= wbase + 32) {  // stages advance by at most one window
+            wbase += 32;
+            cur = nxt;
+            nxt = (wbase + 32 + lane < ri.n_idx) ? ri.list[wbase + 32 + lane] : -1;
+          }
+          if (i % NP != pw) continue;  // the other producer's stage
           const int buf = i % NS;
           if (i >= NS &&
               !__all_sync(0xffffffffu,
@@ -369,11 +391,6 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
           issued = i + 1;
           uint8_t *sK = stages + static_cast<size_t>(buf) * C::kStageBytes;
           uint8_t *sV = sK + C::kTileBytes;
-          if (j * eps >= wbase + 32) {  // stages advance by at most one window
-            wbase += 32;
-            cur = nxt;
-            nxt = (wbase + 32 + lane < ri.n_idx) ? ri.list[wbase + 32 + lane] : -1;
-          }
           const int e = j * eps + lane / tpi;
           const int id = __shfl_sync(0xffffffffu, cur, (e - wbase) & 31);
           bool valid = false;
@@ -625,13 +642,15 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
   }
 
   __syncthreads();
-  if (*abort_flag != 0u && warp == kConsumers) {
-    // a wait gave up: let every copy the producer issued land before the CTA
-    // exits (each wait bounded again)
+  if (*abort_flag != 0u && warp >= kConsumers) {
+    // a wait gave up: let every copy the producers issued land before the CTA
+    // exits (each wait bounded again); a token-list producer waits for its own
+    // buffers, those of its stages' parity
     if (MODE != kModeCp) {
       if (lane < NS && issued > 0) mbar_wait(&full[lane], static_cast<uint32_t>(issued - 1) & 1u);
     } else if (lane == 0) {
-      for (int buf = 0; buf < NS && buf < issued; ++buf) {
+      constexpr int NP = attn_producers<MODE>();
+      for (int buf = warp - kConsumers; buf < NS && buf < issued; buf += NP) {
         const int uses = (issued - 1 - buf) / NS + 1;
         mbar_wait(&full[buf], static_cast<uint32_t>(uses - 1) & 1u);
       }

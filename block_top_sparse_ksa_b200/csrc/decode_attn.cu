@@ -41,7 +41,7 @@ using namespace att;
 namespace {
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(kAttnThreads, 3)
+__global__ void __launch_bounds__(attn_threads<MODE>(), 3)
     sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap,
                               const __grid_constant__ CUtensorMap vmap, const AttnDev p) {
   extern __shared__ uint8_t smem_raw[];
@@ -54,7 +54,8 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   const size_t smem = attn_smem_bytes(D, p.gw);
   int occ = 0;
   const cudaError_t err = kernel_occupancy(
-      reinterpret_cast<const void *>(sparse_decode_attn_kernel<D, MODE>), kAttnThreads, smem, &occ);
+      reinterpret_cast<const void *>(sparse_decode_attn_kernel<D, MODE>), attn_threads<MODE>(),
+      smem, &occ);
   if (err != cudaSuccess) return err;
   occ = occ < 1 ? 1 : (occ > kAttnMaxCtasPerSm ? kAttnMaxCtasPerSm : occ);
   long long n = static_cast<long long>(num_sms) * occ;
@@ -78,7 +79,8 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   p.N = static_cast<int>(n);
   // programmatic: the CTAs take their places and set up while the grid in
   // front (normally the small ranking launch) finishes
-  return launch_programmatic(sparse_decode_attn_kernel<D, MODE>, dim3(p.N), dim3(kAttnThreads),
+  return launch_programmatic(sparse_decode_attn_kernel<D, MODE>, dim3(p.N),
+                             dim3(attn_threads<MODE>()),
                              smem, stream, km, vm, p);
 }
 

@@ -315,17 +315,29 @@ def test_device_status_read_back_validation(ksa):
     assert flags.value == 7  # untouched on a refused call
 
 
+# The one kernel allowed a spill: the token-list attention at head_dim 128 runs two producer
+# warps, so three CTAs of six warps hold at most 96 registers a thread (five warps of one
+# sub-partition share its 16K registers), and it spills a few words; measured against the
+# one-producer form without spills it is faster (65.5 -> 59.9 us per LessIsMore layer).
+SPILL_ALLOWED = {"sparse_decode_attn_kernelILi128ELi2E": 64}  # kernel -> max bytes
+
+
 def test_no_kernel_spills_registers(ksa):
     """The last build's ptxas report: every kernel fits its registers (the selection and pick
-    kernels keep whole rows of keys in registers; a spill would send them to local memory)."""
+    kernels keep whole rows of keys in registers; a spill would send them to local memory),
+    but for the listed one, within its bound."""
     from block_top_sparse_ksa_b200 import build
     if not os.path.exists(build.REPORT):
         build.build(force=True)
     text = open(build.REPORT).read()
-    entries = re.findall(r"Compiling entry function '([^']+)'", text)
-    spills = re.findall(r"(\d+) bytes spill stores, (\d+) bytes spill loads", text)
-    assert len(entries) >= 30 and len(spills) >= len(entries)
-    assert all(a == "0" and b == "0" for a, b in spills), spills
+    blocks = re.split(r"Compiling entry function '", text)[1:]
+    assert len(blocks) >= 30
+    for blk in blocks:
+        name = blk.split("'", 1)[0]
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", blk)
+        assert m, name
+        allowed = max([v for k, v in SPILL_ALLOWED.items() if k in name], default=0)
+        assert int(m.group(1)) <= allowed and int(m.group(2)) <= allowed, (name, m.groups())
 
 
 def test_validation_of_the_decode_step_and_append(ksa):
