@@ -30,7 +30,7 @@ __host__ __device__ constexpr int attn_threads() {
   return (kConsumers + attn_producers<MODE>()) * 32;
 }
 
-template <int D>
+template <int D, bool DEEP = false>
 struct Cfg {
   static constexpr int kHalves = D / 64;              // 64-column (128-byte) halves of a row
   static constexpr int kHalfBytes = kStageTok * 128;  // one 64-column half of a stage tile
@@ -41,8 +41,10 @@ struct Cfg {
   // the same warp and that warp awaits the buffer's phases strictly in order.
   // (With buffers shared between warps a fast warp could wait on a phase two
   // ahead of the barrier, which a parity wait cannot tell from a finished one.)
-  // Two buffers per warp: a warp computes on one while its next stage lands.
-  static constexpr int kStages = (kStageTok == 16 ? 8 : 4) * (D == 128 ? 1 : 2);
+  // Two buffers per warp: a warp computes on one while its next stage lands;
+  // three in the deep form (two CTAs per SM, one per row: more bytes in flight
+  // per CTA).
+  static constexpr int kStages = (kStageTok == 16 ? (DEEP ? 12 : 8) : 4) * (D == 128 ? 1 : 2);
   static_assert(kStages % kConsumers == 0, "stage buffers must map to one consumer warp each");
   static constexpr int kKT = D / 16;
   // stage buffers, 2 mbarriers + 1 mask per stage, flags; plus 1 KB alignment slack
@@ -204,10 +206,10 @@ __device__ __forceinline__ void merge_partials(const AttnDev &p, int r, int tid)
 }
 
 // One CTA's share of the attention (the body of the attention kernel).
-template <int D, int MODE>
+template <int D, int MODE, bool DEEP = false>
 __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensorMap &vmap,
                                          const AttnDev &p, uint8_t *smem_raw) {
-  using C = Cfg<D>;
+  using C = Cfg<D, DEEP>;
   constexpr int NS = C::kStages;
   constexpr int KT = C::kKT;
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -664,8 +666,9 @@ __device__ __forceinline__ void attn_cta(const CUtensorMap &kmap, const CUtensor
 // encoded.
 bool attn_prepare(const AttnArgs &a, void *ws, CUtensorMap *km, CUtensorMap *vm, AttnDev *p,
                   int *mode);
-// Dynamic shared memory of the attention CTA for G query heads per row.
-size_t attn_smem_bytes(int D, int G);
+// Dynamic shared memory of the attention CTA for G query heads per row (deep:
+// the form with three stage buffers per consumer warp).
+size_t attn_smem_bytes(int D, int G, bool deep = false);
 
 }  // namespace att
 }  // namespace ksa

@@ -40,25 +40,32 @@ using namespace att;
 
 namespace {
 
-template <int D, int MODE>
-__global__ void __launch_bounds__(attn_threads<MODE>(), 3)
+template <int D, int MODE, bool DEEP = false>
+__global__ void __launch_bounds__(attn_threads<MODE>(), DEEP ? 2 : 3)
     sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap,
                               const __grid_constant__ CUtensorMap vmap, const AttnDev p) {
   extern __shared__ uint8_t smem_raw[];
-  attn_cta<D, MODE>(kmap, vmap, p, smem_raw);
+  attn_cta<D, MODE, DEEP>(kmap, vmap, p, smem_raw);
+}
+
+template <int D, int MODE, bool DEEP>
+cudaError_t resident_ctas(const AttnDev &p, int num_sms, long long *n) {
+  int occ = 0;
+  const cudaError_t err = kernel_occupancy(
+      reinterpret_cast<const void *>(sparse_decode_attn_kernel<D, MODE, DEEP>),
+      attn_threads<MODE>(), attn_smem_bytes(D, p.gw, DEEP), &occ);
+  if (err != cudaSuccess) return err;
+  occ = occ < 1 ? 1 : (occ > kAttnMaxCtasPerSm ? kAttnMaxCtasPerSm : occ);
+  *n = static_cast<long long>(num_sms) * occ;
+  return cudaSuccess;
 }
 
 template <int D, int MODE>
 cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, int num_sms,
                        cudaStream_t stream) {
-  const size_t smem = attn_smem_bytes(D, p.gw);
-  int occ = 0;
-  const cudaError_t err = kernel_occupancy(
-      reinterpret_cast<const void *>(sparse_decode_attn_kernel<D, MODE>), attn_threads<MODE>(),
-      smem, &occ);
+  long long n = 0;
+  cudaError_t err = resident_ctas<D, MODE, false>(p, num_sms, &n);
   if (err != cudaSuccess) return err;
-  occ = occ < 1 ? 1 : (occ > kAttnMaxCtasPerSm ? kAttnMaxCtasPerSm : occ);
-  long long n = static_cast<long long>(num_sms) * occ;
   if (n > p.W) n = p.W;
   if (n < 1) n = 1;
   // With index lists (rows of equal padded length) and between half and all of the
@@ -70,18 +77,35 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   // us).  Token lists keep every resident CTA: there the copy-issuing producer warps set
   // the pace, and fewer CTAs measured slower (64.3 -> 66.0 us on the same rows).
   const long long rows = p.W / p.V;
+  bool deep = false;
   if (MODE != kModeDense) {
-    if (2 * rows >= n && rows <= n)
+    if (2 * rows >= n && rows <= n) {
       n = rows;
-    else if (MODE == kModeTma && 2 * rows < n)
+      // block lists, one CTA per row: where the rows also fit two deep CTAs per SM
+      // (three buffers per consumer warp), those run instead -- the SMs that hold two
+      // rows set the time, and they then keep half as many bytes again in flight
+      if constexpr (MODE == kModeTma) {
+        long long n_deep = 0;
+        err = resident_ctas<D, MODE, true>(p, num_sms, &n_deep);
+        if (err != cudaSuccess) return err;
+        deep = rows <= n_deep;
+      }
+    } else if (MODE == kModeTma && 2 * rows < n) {
       n = rows * (n / rows);
+    }
   }
   p.N = static_cast<int>(n);
   // programmatic: the CTAs take their places and set up while the grid in
   // front (normally the small ranking launch) finishes
-  return launch_programmatic(sparse_decode_attn_kernel<D, MODE>, dim3(p.N),
-                             dim3(attn_threads<MODE>()),
-                             smem, stream, km, vm, p);
+  if constexpr (MODE == kModeTma) {
+    if (deep)
+      return launch_programmatic(sparse_decode_attn_kernel<D, MODE, true>, dim3(p.N),
+                                 dim3(attn_threads<MODE>()), attn_smem_bytes(D, p.gw, true),
+                                 stream, km, vm, p);
+  }
+  return launch_programmatic(sparse_decode_attn_kernel<D, MODE, false>, dim3(p.N),
+                             dim3(attn_threads<MODE>()), attn_smem_bytes(D, p.gw, false), stream,
+                             km, vm, p);
 }
 
 }  // namespace
@@ -96,8 +120,9 @@ size_t attn_workspace_bytes(int B, int Hq, int Hkv, int D, int num_sms) {
 
 namespace att {
 
-size_t attn_smem_bytes(int D, int G) {
-  const size_t fixed = D == 128 ? Cfg<128>::kFixedSmem : Cfg<64>::kFixedSmem;
+size_t attn_smem_bytes(int D, int G, bool deep) {
+  const size_t fixed = deep ? (D == 128 ? Cfg<128, true>::kFixedSmem : Cfg<64, true>::kFixedSmem)
+                            : (D == 128 ? Cfg<128>::kFixedSmem : Cfg<64>::kFixedSmem);
   return fixed + static_cast<size_t>(kConsumers) * (2 * G + G * D) * 4;
 }
 
