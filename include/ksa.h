@@ -379,8 +379,7 @@ ksa_status ksa_sparse_decode_attn_paged(const ksa_shape *shape, const uint16_t *
  * with cudaMemsetAsync on `stream` and launches the attention kernel.
  * The first call on a device looks up the scratch's device address
  * (cudaGetSymbolAddress), and so does the first call after the device's
- * context has changed (cudaDeviceReset); make that first call before any
- * stream capture.
+ * context has changed (cudaDeviceReset).
  * Every call shares the one scratch area, so calls that may overlap on the
  * GPU (different streams, or different host threads) race: issue them one
  * after another on one stream.
