@@ -71,19 +71,23 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   // With index lists (rows of equal padded length) and between half and all of the
   // resident CTAs' worth of rows, one CTA per row: slices then end on row boundaries, and
   // no row is split, so no CTA ends with a partial merge (measured on the Qwen3-8B shape,
-  // 256 rows: attention 61.2 -> 55.0 us; two or more rows per CTA gained nothing).  With
-  // block lists and fewer rows, each row is cut into s = n / rows equal parts, one per
-  // CTA, so every CTA holds one piece of one row (128 rows of 250 stages: 59.3 -> 53.0
-  // us).  Token lists keep every resident CTA: there the copy-issuing producer warps set
-  // the pace, and fewer CTAs measured slower (64.3 -> 66.0 us on the same rows).
+  // 256 rows: attention 61.2 -> 55.0 us).  With block lists:
+  //  * one CTA per row, where the rows also fit two deep CTAs per SM (three buffers per
+  //    consumer warp), those run: the SMs that hold two rows set the time, and they then
+  //    keep half as many bytes again in flight (Qwen3-8B step 100.2 -> 97.7 us);
+  //  * more rows than resident CTAs: r whole rows per deep CTA, r the fewest that fit the
+  //    deep grid, where r divides the rows (Qwen3-0.6B shape, 512 rows: attention 57.1 ->
+  //    53.7 us; the 8-stage form with several rows per CTA gained nothing);
+  //  * fewer than half the resident CTAs' worth of rows: each row is cut into s = n / rows
+  //    equal parts, one per CTA, so every CTA holds one piece of one row (128 rows of 250
+  //    stages: 59.3 -> 53.0 us).
+  // Token lists keep every resident CTA: there the copy-issuing producer warps set the
+  // pace, and fewer CTAs measured slower (64.3 -> 66.0 us on the same rows).
   const long long rows = p.W / p.V;
   bool deep = false;
   if (MODE != kModeDense) {
     if (2 * rows >= n && rows <= n) {
       n = rows;
-      // block lists, one CTA per row: where the rows also fit two deep CTAs per SM
-      // (three buffers per consumer warp), those run instead -- the SMs that hold two
-      // rows set the time, and they then keep half as many bytes again in flight
       if constexpr (MODE == kModeTma) {
         long long n_deep = 0;
         err = resident_ctas<D, MODE, true>(p, num_sms, &n_deep);
@@ -92,6 +96,15 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
       }
     } else if (MODE == kModeTma && 2 * rows < n) {
       n = rows * (n / rows);
+    } else if constexpr (MODE == kModeTma) {  // rows > n
+      long long n_deep = 0;
+      err = resident_ctas<D, MODE, true>(p, num_sms, &n_deep);
+      if (err != cudaSuccess) return err;
+      const long long r = (rows + n_deep - 1) / n_deep;  // rows per deep CTA
+      if (rows % r == 0 && 2 * (rows / r) >= n_deep) {
+        n = rows / r;
+        deep = true;
+      }
     }
   }
   p.N = static_cast<int>(n);
