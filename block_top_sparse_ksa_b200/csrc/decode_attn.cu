@@ -75,9 +75,13 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   //  * one CTA per row, where the rows also fit two deep CTAs per SM (three buffers per
   //    consumer warp), those run: the SMs that hold two rows set the time, and they then
   //    keep half as many bytes again in flight (Qwen3-8B step 100.2 -> 97.7 us);
-  //  * more rows than resident CTAs: r whole rows per deep CTA, r the fewest that fit the
-  //    deep grid, where r divides the rows (Qwen3-0.6B shape, 512 rows: attention 57.1 ->
-  //    53.7 us; the 8-stage form with several rows per CTA gained nothing);
+  //  * more rows than resident CTAs but at most twice the deep grid, an even number,
+  //    filling at least 85% of the deep grid with pairs: two whole rows per deep CTA (an
+  //    SM holding two CTAs carries twice an SM holding one, so the fill bounds the
+  //    imbalance).  Qwen3-0.6B shape, 512 rows in 256 CTAs: attention 57.1 -> 53.7 us.
+  //    More rows per CTA measured slower than stream-K on the sweep shapes (80 rows per
+  //    CTA at 4K/256: 441 -> 491 us; 4 rows in 160 CTAs at 128K/8192: 424 -> 532 us), and
+  //    the 8-stage form with several rows per CTA gained nothing;
   //  * fewer than half the resident CTAs' worth of rows: each row is cut into s = n / rows
   //    equal parts, one per CTA, so every CTA holds one piece of one row (128 rows of 250
   //    stages: 59.3 -> 53.0 us).
@@ -100,9 +104,8 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
       long long n_deep = 0;
       err = resident_ctas<D, MODE, true>(p, num_sms, &n_deep);
       if (err != cudaSuccess) return err;
-      const long long r = (rows + n_deep - 1) / n_deep;  // rows per deep CTA
-      if (rows % r == 0 && 2 * (rows / r) >= n_deep) {
-        n = rows / r;
+      if (rows <= 2 * n_deep && rows % 2 == 0 && 20 * (rows / 2) >= 17 * n_deep) {
+        n = rows / 2;
         deep = true;
       }
     }

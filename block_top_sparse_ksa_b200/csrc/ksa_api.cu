@@ -732,7 +732,8 @@ size_t ksa_select_tokens_one_head_workspace(const ksa_shape *shape, int32_t k_to
   const size_t heads = static_cast<size_t>(shape->batch) * shape->num_q_heads;
   return ksa::unified_workspace_bytes(shape->batch, shape->num_q_heads, shape->capacity) +
          ((heads * k_tokens * sizeof(int32_t) + 255) & ~static_cast<size_t>(255)) +
-         ((heads * sizeof(int32_t) + 255) & ~static_cast<size_t>(255));
+         ((heads * sizeof(int32_t) + 255) & ~static_cast<size_t>(255)) +
+         ((static_cast<size_t>(shape->batch) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255));
 }
 
 ksa_status ksa_select_tokens_one_head(const ksa_shape *shape, const uint16_t *q,
@@ -761,22 +762,22 @@ ksa_status ksa_select_tokens_one_head(const ksa_shape *shape, const uint16_t *q,
   if (!aligned(ws, 256)) return fail(KSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   int32_t *lists = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + base);
   int32_t *counts = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + base + lists_bytes);
+  const size_t counts_bytes = (heads * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+  int32_t *dev_heads = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + base +
+                                                   lists_bytes + counts_bytes);
   // every head's own set into the workspace (the per-head kernels) ...
   st = ksa_select_tokens_per_head(shape, q, K, seq_lens, k_tokens, lists, counts, ws, base,
                                   dev_status, stream);
   if (st != KSA_OK) return st;
-  // ... then each row's chosen head's list and count, in stream order
+  // ... then the heads drawn for the rows (one copy; the host array is read before the
+  // copy call returns) and each row's chosen list and count (one gather launch)
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t k = static_cast<size_t>(k_tokens);
-  for (int b = 0; b < B; ++b) {
-    const size_t src = static_cast<size_t>(b) * Hq + head_of_row[b];
-    cudaError_t err = cudaMemcpyAsync(token_idx + b * k, lists + src * k, k * sizeof(int32_t),
-                                      cudaMemcpyDeviceToDevice, s);
-    if (err == cudaSuccess)
-      err = cudaMemcpyAsync(num_sel + b, counts + src, sizeof(int32_t), cudaMemcpyDeviceToDevice,
-                            s);
-    if (err != cudaSuccess) return cuda_status(err, "ksa_select_tokens_one_head copy");
-  }
+  cudaError_t err = cudaMemcpyAsync(dev_heads, head_of_row, static_cast<size_t>(B) * sizeof(int32_t),
+                                    cudaMemcpyHostToDevice, s);
+  if (err != cudaSuccess) return cuda_status(err, "ksa_select_tokens_one_head heads copy");
+  err = ksa::launch_gather_head_lists(lists, counts, dev_heads, B, Hq, k_tokens, token_idx,
+                                      num_sel, s);
+  if (err != cudaSuccess) return cuda_status(err, "ksa_select_tokens_one_head gather");
   return KSA_OK;
 }
 

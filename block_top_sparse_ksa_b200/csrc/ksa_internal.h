@@ -121,6 +121,11 @@ size_t unified_workspace_bytes(int B, int Hq, int T);
 cudaError_t launch_unified_select(const UnifiedArgs &a, int num_sms, cudaStream_t stream);
 // Per-head token top-k lists (P = k = budget; token_idx [B, Hq, k], num_sel [B, Hq]).
 cudaError_t launch_tokens_per_head(const UnifiedArgs &a, cudaStream_t stream);
+// Row b's list and count <- those of query head head[b] (device array [B]), from
+// lists [B, Hq, k] and counts [B, Hq].
+cudaError_t launch_gather_head_lists(const int32_t *lists, const int32_t *counts,
+                                     const int32_t *head, int B, int Hq, int k,
+                                     int32_t *token_idx, int32_t *num_sel, cudaStream_t stream);
 
 // Resident CTAs per SM of `func` launched with `threads` threads and `smem`
 // bytes of dynamic shared memory, on the current device.  The first query per

@@ -636,6 +636,27 @@ cudaError_t launch_scores(const UnifiedArgs &a, cudaStream_t stream) {
                     a, n_chunks);
 }
 
+// Random-head aggregation's last step: row b's set is query head head[b]'s
+// list and count.  One thread per list entry (and per count).
+__global__ void __launch_bounds__(256) gather_head_lists_kernel(const int32_t *lists,
+                                                                const int32_t *counts,
+                                                                const int32_t *head, int B,
+                                                                int Hq, int k, int32_t *token_idx,
+                                                                int32_t *num_sel) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long n = static_cast<long long>(B) * k;
+  if (e < n) {
+    const int b = static_cast<int>(e / k), i = static_cast<int>(e - static_cast<long long>(b) * k);
+    const size_t src = static_cast<size_t>(b) * Hq + head[b];
+    token_idx[e] = lists[src * k + i];
+  } else if (e < n + B) {
+    const int b = static_cast<int>(e - n);
+    num_sel[b] = counts[static_cast<size_t>(b) * Hq + head[b]];
+  }
+}
+
 }  // namespace
 
 size_t unified_workspace_bytes(int B, int Hq, int T) {
@@ -644,6 +665,14 @@ size_t unified_workspace_bytes(int B, int Hq, int T) {
   const size_t bits =
       (static_cast<size_t>(B) * Hq * ((T + 31) / 32) * sizeof(uint32_t) + 255) & ~static_cast<size_t>(255);
   return keys + votes + bits;
+}
+
+cudaError_t launch_gather_head_lists(const int32_t *lists, const int32_t *counts,
+                                     const int32_t *head, int B, int Hq, int k,
+                                     int32_t *token_idx, int32_t *num_sel, cudaStream_t stream) {
+  const long long n = static_cast<long long>(B) * k + B;
+  return launch_pdl(gather_head_lists_kernel, dim3(static_cast<unsigned>((n + 255) / 256)),
+                    dim3(256), 0, stream, lists, counts, head, B, Hq, k, token_idx, num_sel);
 }
 
 cudaError_t launch_tokens_per_head(const UnifiedArgs &a, cudaStream_t stream) {

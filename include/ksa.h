@@ -170,9 +170,10 @@ ksa_status ksa_select_tokens_per_head(const ksa_shape *shape, const uint16_t *q,
  *   token_idx: [B, k_tokens] int32;  num_sel: [B] int32 (written)
  *   ws: device scratch of ksa_select_tokens_one_head_workspace() bytes,
  *       256-byte aligned, no initialisation needed.
- * It runs the per-head kernels into the workspace, then copies each row's
- * chosen list with one cudaMemcpyAsync per row (and one per count) on
- * `stream`.  A head outside [0, Hq) is KSA_ERR_INVALID_ARG before any launch.
+ * It runs the per-head kernels into the workspace, copies head_of_row into
+ * the workspace (one host-to-device cudaMemcpyAsync on `stream`), and gathers
+ * each row's chosen list and count with one launch.  A head outside [0, Hq)
+ * is KSA_ERR_INVALID_ARG before any launch.
  * Limits: as ksa_select_tokens_per_head.
  */
 size_t ksa_select_tokens_one_head_workspace(const ksa_shape *shape, int32_t k_tokens);

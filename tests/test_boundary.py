@@ -279,7 +279,7 @@ def test_validation_of_random_head_selection(ksa):
     assert call(good, 4, None, 0) == 3
     per_head = lib.ksa_select_tokens_per_head_workspace(ctypes.byref(sh), 4)
     one_head = lib.ksa_select_tokens_one_head_workspace(ctypes.byref(sh), 4)
-    assert one_head >= per_head + 3 * 8 * 4 * 4 + 3 * 8 * 4
+    assert one_head >= per_head + 3 * 8 * 4 * 4 + 3 * 8 * 4 + 3 * 4  # lists, counts, heads
     assert call(good, 4, FAKE, one_head - 1) == 3
 
 
