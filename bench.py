@@ -334,18 +334,24 @@ def warm_up(step, warmup: int, min_s: float) -> int:
     return n
 
 
-def timed_steps(step, steps: int, dist, stream):
+def timed_steps(step, steps: int, dist, stream, side=(), join=None):
     """K steps back to back between two events on `stream`, bracketed by barrier +
-    synchronize.  Returns (device ms over all K steps, host enqueue us per step)."""
+    synchronize.  Streams in `side` start after the start event; `join()` (if given) makes
+    `stream` wait for their last work before the end event.  Returns (device ms over all K
+    steps, host enqueue us per step)."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
     start.record(stream)
+    for s in side:
+        s.wait_event(start)
     h0 = time.perf_counter()
     for i in range(steps):
         step(i)
     h1 = time.perf_counter()
+    if join is not None:
+        join()
     end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
@@ -569,8 +575,11 @@ def run_block_e2e(args, dist, wl: BlockWorkload):
     """The same step through the public API with host buffers.  Per step: the new query and
     the new token's K/V rows go host->device from pinned memory, ksa_append_kv writes the
     rows into their cache slot (token L_b - 1: the lengths stay fixed, so every step is the
-    same workload), then the selection and attention calls, and the output comes back
-    device->host.  The copies are inside the timed region."""
+    same workload), then ksa_decode_step, and the output comes back device->host.  Every
+    step's copies are inside the timed region.  Two forms: serial (every copy on the compute
+    stream, in step order), and pipelined (as a serving loop runs it: the uploads on one copy
+    stream and the downloads on another, with double buffers and events, so a step's copies
+    overlap the neighbouring steps' kernels; the value reported)."""
     import block_top_sparse_ksa_b200 as ksa
     sh = wl.shape
     B, Hq, Hkv, D = sh.batch, sh.num_q_heads, sh.num_kv_heads, sh.head_dim
@@ -578,33 +587,80 @@ def run_block_e2e(args, dist, wl: BlockWorkload):
     nq = wl.nq
     h_q = wl.qs.cpu().pin_memory()
     h_kv = torch.randn((nq, 2, B, Hkv, D), dtype=torch.float32).to(torch.bfloat16).pin_memory()
-    h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
-    d_q = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
-    d_kv = torch.empty((2, B, Hkv, D), dtype=torch.bfloat16, device=dev)
+    h_out = [torch.empty((B, Hq, D), dtype=torch.float32).pin_memory() for _ in range(2)]
+    d_q = [torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    d_kv = [torch.empty((2, B, Hkv, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    d_out = [torch.empty((B, Hq, D), dtype=torch.float32, device=dev) for _ in range(2)]
     stream = wl.stream
     lens = wl.inp.seq_lens
 
-    def step(i):
-        d_q.copy_(h_q[i % nq], non_blocking=True)
-        d_kv.copy_(h_kv[i % nq], non_blocking=True)
-        ksa.ksa_append_kv(d_kv[0], d_kv[1], wl.inp.K, wl.inp.V, lens, stream=stream)
+    def compute(i, q, kv, out):
+        ksa.ksa_append_kv(kv[0], kv[1], wl.inp.K, wl.inp.V, lens, stream=stream)
         if wl.kind == "dense":
-            wl.attend(i, d_q)
+            ksa.ksa_sparse_decode_attn(q, wl.inp.K, wl.inp.V, lens, out=out,
+                                       workspace=wl.ws_att, stream=stream)
         else:
-            wl.decode_step(i, d_q)
-        h_out.copy_(wl.out, non_blocking=True)
+            ksa.ksa_decode_step(q, wl.inp.K, wl.inp.V, wl.S, lens, sh.block_size, sh.k_blocks,
+                                block_idx=wl.idx, num_sel=wl.cnt, out=out,
+                                workspace=wl.ws_step, stream=stream)
 
-    warm_up(step, args.warmup, 0.0)
-    ms, host_us = timed_steps(step, args.steps, dist, stream)
+    def serial_step(i):
+        d_q[0].copy_(h_q[i % nq], non_blocking=True)
+        d_kv[0].copy_(h_kv[i % nq], non_blocking=True)
+        compute(i, d_q[0], d_kv[0], d_out[0])
+        h_out[0].copy_(d_out[0], non_blocking=True)
+
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]  # whether buffer set s has been through a step yet
+    last = [None]
+
+    def piped_step(i):
+        s = i & 1
+        with torch.cuda.stream(up):
+            if used[s]:
+                up.wait_event(ev_comp[s])  # step i - 2 has read d_q[s], d_kv[s]
+            d_q[s].copy_(h_q[i % nq], non_blocking=True)
+            d_kv[s].copy_(h_kv[i % nq], non_blocking=True)
+            ev_up[s].record(up)
+        stream.wait_event(ev_up[s])
+        if used[s]:
+            stream.wait_event(ev_down[s])  # step i - 2's output has left d_out[s]
+        compute(i, d_q[s], d_kv[s], d_out[s])
+        ev_comp[s].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_comp[s])
+            h_out[s].copy_(d_out[s], non_blocking=True)
+            ev_down[s].record(down)
+        used[s] = True
+        last[0] = s
+
+    def join():
+        stream.wait_event(ev_down[last[0]])
+
+    warm_up(serial_step, args.warmup, 0.0)
+    ms_ser, host_ser = timed_steps(serial_step, args.steps, dist, stream)
+    value_ser, ms_step_ser = weak_scaling(dist, B, ms_ser, args.steps)
+    warm_up(piped_step, args.warmup, 0.0)
+    ms, host_us = timed_steps(piped_step, args.steps, dist, stream, side=(up, down), join=join)
     value, ms_step = weak_scaling(dist, B, ms, args.steps)
+    torch.cuda.synchronize()
+    ref = d_out[last[0]].cpu()
+    assert torch.equal(h_out[last[0]], ref), "the last step's download differs from its output"
     h2d = (B * Hq * D + 2 * B * Hkv * D) * 2
     d2h = B * Hq * D * 4
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
             "host_enqueue_us_per_step": host_us,
             "gpu_launches": (wl.launches_per_step + 1) * args.steps,  # + the append
+            "serial": {"value": value_ser, "ms_per_step": ms_step_ser,
+                       "host_enqueue_us_per_step": host_ser},
             "note": "per step: q and the new token's K/V rows host->device (pinned), "
-                    "ksa_append_kv, ksa_decode_step, out device->host"}
+                    "ksa_append_kv, ksa_decode_step, out device->host; value: uploads and "
+                    "downloads on two copy streams with double buffers, overlapping the "
+                    "neighbouring steps' kernels; serial: every copy on the compute stream"}
 
 
 def run_unified(args, dist, dev):
