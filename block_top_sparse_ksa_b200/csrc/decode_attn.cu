@@ -82,11 +82,10 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
   //    More rows per CTA measured slower than stream-K on the sweep shapes (80 rows per
   //    CTA at 4K/256: 441 -> 491 us; 4 rows in 160 CTAs at 128K/8192: 424 -> 532 us), and
   //    the 8-stage form with several rows per CTA gained nothing;
-  //  * fewer than half the resident CTAs' worth of rows: each row is cut into s = n / rows
-  //    equal parts, one per CTA, so every CTA holds one piece of one row (128 rows of 250
-  //    stages: 59.3 -> 53.0 us).
-  // Token lists keep every resident CTA: there the copy-issuing producer warps set the
-  // pace, and fewer CTAs measured slower (64.3 -> 66.0 us on the same rows).
+  //  * fewer than half the resident CTAs' worth of rows (token lists too): each row is cut
+  //    into s = n / rows equal parts, one per CTA, so every CTA holds one piece of one row
+  //    (128 rows of 250 stages: block lists 59.3 -> 53.0 us, token lists 59.3 -> 55.9 us;
+  //    with one producer warp per CTA the token lists had measured slower this way).
   const long long rows = p.W / p.V;
   bool deep = false;
   if (MODE != kModeDense) {
@@ -98,7 +97,7 @@ cudaError_t launch_one(const CUtensorMap &km, const CUtensorMap &vm, AttnDev p, 
         if (err != cudaSuccess) return err;
         deep = rows <= n_deep;
       }
-    } else if (MODE == kModeTma && 2 * rows < n) {
+    } else if (2 * rows < n) {
       n = rows * (n / rows);
     } else if constexpr (MODE == kModeTma) {  // rows > n
       long long n_deep = 0;
