@@ -245,17 +245,8 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
   uint32_t prefix = 0u, pmask = 0u;
   uint32_t remaining = static_cast<uint32_t>(a.P);  // still to take among the candidates
   uint32_t tau = 0u, n_eq = 0u;
-  for (int pass = 0; pass < 5; ++pass) {  // at most 4 passes of 8 bits, then all equal
-    // min / max / count of the candidates (keys matching the digits fixed so far)
-    uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
-#pragma unroll
-    for (int e = 0; e < KPL; ++e) {
-      if ((key[e] & pmask) == prefix) {
-        kmin = min(kmin, key[e]);
-        kmax = max(kmax, key[e]);
-        ++cnt;
-      }
-    }
+  // min / max / count of the candidates, block-wide (every thread gets them)
+  auto block_range = [&](uint32_t &kmin, uint32_t &kmax, uint32_t &cnt) {
     kmin = __reduce_min_sync(0xffffffffu, kmin);
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     cnt = __reduce_add_sync(0xffffffffu, cnt);
@@ -274,6 +265,16 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
       kmax = max(kmax, red[1][w]);
       cnt += red[2][w];
     }
+  };
+  // the first pass's candidates are all the slots
+  uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = KPL;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    kmin = min(kmin, key[e]);
+    kmax = max(kmax, key[e]);
+  }
+  block_range(kmin, kmax, cnt);
+  for (int pass = 0; pass < 5; ++pass) {  // at most 4 passes of 8 bits, then all equal
     if (kmin == kmax) {  // every candidate equal: the threshold
       tau = kmin;
       n_eq = cnt;
@@ -331,6 +332,19 @@ __global__ void __launch_bounds__(kPickRegThreads) unified_pick_reg_kernel(const
     tau = prefix;
     __syncthreads();  // xinfo, hist and red are rewritten by the next pass
     if (sh == 0) break;  // every bit fixed
+    // the next pass's candidates: keys matching the digits fixed so far
+    kmin = 0xffffffffu;
+    kmax = 0u;
+    cnt = 0u;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      if ((key[e] & pmask) == prefix) {
+        kmin = min(kmin, key[e]);
+        kmax = max(kmax, key[e]);
+        ++cnt;
+      }
+    }
+    block_range(kmin, kmax, cnt);
   }
   __syncthreads();  // red is read above before it is rewritten below
   const uint32_t take_eq = remaining;  // keys equal to tau to take, lowest token first
@@ -473,17 +487,26 @@ __device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t *sc
   return r;
 }
 
+// Full adder on 32 bit lanes at once: a + b + c = 2 hi + lo in every lane.
+__device__ __forceinline__ void csa(uint32_t &hi, uint32_t &lo, uint32_t a, uint32_t b,
+                                    uint32_t c) {
+  const uint32_t u = a ^ b;
+  hi = (a & b) | (u & c);
+  lo = u ^ c;
+}
+
 // Shared set straight from the per-head pick bit sets (the register-pick path,
 // fewer than 64 heads): CTA per row, thread t owns the 32 candidates of bit
-// word t.  It adds the row's Hq words into six bit planes (a ripple-carry
-// counter per token lane, so plane i holds bit i of every token's vote count),
+// word t.  It adds the row's Hq words into six bit planes (a counter per token
+// lane, so plane i holds bit i of every token's vote count: carry-save adders
+// take sixteen heads at a time, ripple-carry adds the rest),
 // counts the tokens of each vote value from the planes, finds the threshold
 // vote from the top value down, then -- with masks of the tokens above it and
 // equal to it, again from the planes -- two block scans give each thread its
 // share of the tied tokens (lowest first) and its output position, and it
 // writes its picks in token order.  The same set as the votes kernel followed
 // by unified_set_kernel, in one launch.
-__global__ void __launch_bounds__(kSetThreads) unified_set_bits_kernel(const UnifiedArgs a) {
+__global__ void __launch_bounds__(kSetThreads, 1) unified_set_bits_kernel(const UnifiedArgs a) {
   constexpr int NT = kSetThreads, NW = NT / 32;
   __shared__ uint32_t hist[NW][64];
   __shared__ uint32_t scan[NW + 1];
@@ -509,8 +532,35 @@ __global__ void __launch_bounds__(kSetThreads) unified_set_bits_kernel(const Uni
     if (vm != 0u) {  // (words past the candidates are not read: they may be stale)
       const int W32 = (a.T + 31) / 32;
       const uint32_t *bits = a.bits + static_cast<size_t>(b) * a.Hq * W32 + tid;
-#pragma unroll 8
-      for (int h = 0; h < a.Hq; ++h) {
+      int h = 0;
+      // sixteen heads at a time through a tree of carry-save adders: c[0..3]
+      // take the weights 1..8 and the tree's weight-16 output adds into c[4],
+      // c[5] (a count stays below 64, so nothing carries past c[5])
+      for (; h + 16 <= a.Hq; h += 16) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = __ldcg(bits + static_cast<size_t>(h + i) * W32);
+        uint32_t t2a, t2b, f4a, f4b, e8a, e8b, s16;
+        csa(t2a, c[0], c[0], w[0], w[1]);
+        csa(t2b, c[0], c[0], w[2], w[3]);
+        csa(f4a, c[1], c[1], t2a, t2b);
+        csa(t2a, c[0], c[0], w[4], w[5]);
+        csa(t2b, c[0], c[0], w[6], w[7]);
+        csa(f4b, c[1], c[1], t2a, t2b);
+        csa(e8a, c[2], c[2], f4a, f4b);
+        csa(t2a, c[0], c[0], w[8], w[9]);
+        csa(t2b, c[0], c[0], w[10], w[11]);
+        csa(f4a, c[1], c[1], t2a, t2b);
+        csa(t2a, c[0], c[0], w[12], w[13]);
+        csa(t2b, c[0], c[0], w[14], w[15]);
+        csa(f4b, c[1], c[1], t2a, t2b);
+        csa(e8b, c[2], c[2], f4a, f4b);
+        csa(s16, c[3], c[3], e8a, e8b);
+        const uint32_t t = c[4] & s16;
+        c[4] ^= s16;
+        c[5] ^= t;
+      }
+      for (; h < a.Hq; ++h) {  // the rest one at a time: a ripple-carry add
         uint32_t carry = __ldcg(bits + static_cast<size_t>(h) * W32);
 #pragma unroll
         for (int i = 0; i < 6; ++i) {
@@ -520,13 +570,17 @@ __global__ void __launch_bounds__(kSetThreads) unified_set_bits_kernel(const Uni
         }
       }
     }
-    // tokens of each vote value, per warp
-    for (int v = 0; v <= a.Hq; ++v) {
-      uint32_t m = vm;
+    // tokens of each vote value, per warp (warps past the candidates count none)
+    if (__any_sync(0xffffffffu, vm != 0u)) {
+      for (int v = 0; v <= a.Hq; ++v) {
+        uint32_t m = vm;
 #pragma unroll
-      for (int i = 0; i < 6; ++i) m &= ((v >> i) & 1) ? c[i] : ~c[i];
-      const uint32_t cnt = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popc(m)));
-      if (lane == 0) hist[warp][v] = cnt;
+        for (int i = 0; i < 6; ++i) m &= ((v >> i) & 1) ? c[i] : ~c[i];
+        const uint32_t cnt = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popc(m)));
+        if (lane == 0) hist[warp][v] = cnt;
+      }
+    } else {
+      for (int v = lane; v <= a.Hq; v += 32) hist[warp][v] = 0u;
     }
     __syncthreads();
     if (tid < 64) {

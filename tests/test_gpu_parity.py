@@ -400,6 +400,23 @@ def test_unified_select_exact(ksa, oracle, L, P, budget, R):
     assert np.array_equal(idx.cpu().numpy(), ref_idx)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(20, 4), (48, 8), (63, 9), (64, 8)])
+def test_unified_select_head_counts(ksa, oracle, Hq, Hkv):
+    # the shared set adds the heads' pick bits sixteen at a time, the rest one at a
+    # time; vote counts up to 63 stay exact; 64 heads and more count votes per token
+    rng = np.random.default_rng(720 + Hq)
+    B, D, L = 2, 64, 3000
+    T = L + 5
+    q = dyadic_bits(rng, (B, Hq, D))
+    K = dyadic_bits(rng, (B, Hkv, T, D))
+    lens = np.array([L, L - 777], np.int32)
+    idx, cnt = ksa.ksa_unified_select(to_dev_bf16(q), to_dev_bf16(K),
+                                      torch.from_numpy(lens).to(DEV), 600, 800, 200)
+    ref_idx, ref_cnt = oracle.unified_select(q, K, lens, 600, 800, 200)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+
+
 def test_unified_default_window_is_quarter(ksa, oracle):
     rng = np.random.default_rng(710)
     B, Hq, Hkv, D, T = 1, 8, 2, 64, 1200
