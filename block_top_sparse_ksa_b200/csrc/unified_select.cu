@@ -502,7 +502,7 @@ __device__ __forceinline__ void csa(uint32_t &hi, uint32_t &lo, uint32_t a, uint
 // take sixteen heads at a time, ripple-carry adds the rest),
 // counts the tokens of each vote value from the planes, finds the threshold
 // vote from the top value down, then -- with masks of the tokens above it and
-// equal to it, again from the planes -- two block scans give each thread its
+// equal to it, again from the planes -- one block scan gives each thread its
 // share of the tied tokens (lowest first) and its output position, and it
 // writes its picks in token order.  The same set as the votes kernel followed
 // by unified_set_kernel, in one launch.
@@ -624,9 +624,14 @@ __global__ void __launch_bounds__(kSetThreads, 1) unified_set_bits_kernel(const 
     }
     gt &= vm;
     eq &= vm;
+    // one scan of the packed counts (each total is at most 32 NT < 2^16): the tied
+    // tokens before this thread, and those above tau; the kept tied tokens before it
+    // are the first take_eq of the row's, so its first output slot follows from both
     uint32_t tot;
     const uint32_t my_eq = static_cast<uint32_t>(__popc(eq));
-    const uint32_t eq_before = block_exclusive_sum<NT>(my_eq, scan, tot);
+    const uint32_t before = block_exclusive_sum<NT>(
+        (static_cast<uint32_t>(__popc(gt)) << 16) | my_eq, scan, tot);
+    const uint32_t eq_before = before & 0xffffu, gt_before = before >> 16;
     const uint32_t eq_take = eq_before >= take_eq ? 0u : min(my_eq, take_eq - eq_before);
     uint32_t keep = 0u, rest = eq;  // the lowest eq_take tied tokens
     for (uint32_t q = 0u; q < eq_take; ++q) {
@@ -635,7 +640,7 @@ __global__ void __launch_bounds__(kSetThreads, 1) unified_set_bits_kernel(const 
       rest ^= low;
     }
     uint32_t sel = gt | keep;
-    uint32_t pos = block_exclusive_sum<NT>(static_cast<uint32_t>(__popc(sel)), scan, tot);
+    uint32_t pos = gt_before + min(eq_before, take_eq);
     while (sel != 0u) {
       out[pos++] = base + __ffs(sel) - 1;
       sel &= sel - 1u;
