@@ -222,6 +222,36 @@ def test_token_list_attention_shared(ksa, oracle, D, tpi):
     assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, tpi, shared=True) == 0
 
 
+# Row counts, in SMs, that reach each way the attention launch splits its work (for one
+# query-head group of 4 at head_dim 128, three CTAs per SM, two in the deep form): rows cut
+# into equal parts, one deep CTA per row, one CTA per row, two whole rows per deep CTA, and
+# the stream-K split (an odd count, and more rows than two deep grids hold).
+PARTITION_ROWS = [(0.5, 0), (2.0, -8), (3.0, -4), (4.0, -16), (4.0, -15), (5.0, 0)]
+
+
+@pytest.mark.parametrize("tpi", [16, 1])
+@pytest.mark.parametrize("per_sm,extra", PARTITION_ROWS)
+def test_attention_partition_forms(ksa, oracle, tpi, per_sm, extra):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B = max(1, int(per_sm * sms) + extra)
+    rng = np.random.default_rng(900 + B + tpi)
+    Hq, Hkv, D, T = 4, 1, 128, 320
+    q = rand_bits(rng, (B, Hq, D))
+    K = rand_bits(rng, (B, Hkv, T, D))
+    V = rand_bits(rng, (B, Hkv, T, D))
+    lens = rng.integers(T // 2, T + 1, size=B).astype(np.int32)
+    lens[0], lens[-1] = T, 7
+    cap = 6 if tpi == 16 else 48
+    idx = np.full((B, Hkv, cap), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    for b in range(B):
+        units = -(-int(lens[b]) // tpi)
+        n = int(rng.integers(1, min(cap, units) + 1))
+        idx[b, 0, :n] = np.sort(rng.choice(units, size=n, replace=False))
+        cnt[b, 0] = n
+    assert _attn_check(ksa, oracle, q, K, V, lens, idx, cnt, tpi) == 0
+
+
 def _list_with_runs(rng, n_units, cap, tpi, past_end=0):
     """Ascending distinct units: a recency window ending at the last unit, runs of 15 to
     100 tokens at unaligned starts, scattered singles up to cap, and `past_end` units
