@@ -229,13 +229,14 @@ def test_token_list_attention_shared(ksa, oracle, D, tpi):
 PARTITION_ROWS = [(0.5, 0), (2.0, -8), (3.0, -4), (4.0, -16), (4.0, -15), (5.0, 0)]
 
 
+@pytest.mark.parametrize("D,Hq", [(128, 4), (64, 8)])
 @pytest.mark.parametrize("tpi", [16, 1])
 @pytest.mark.parametrize("per_sm,extra", PARTITION_ROWS)
-def test_attention_partition_forms(ksa, oracle, tpi, per_sm, extra):
+def test_attention_partition_forms(ksa, oracle, D, Hq, tpi, per_sm, extra):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     B = max(1, int(per_sm * sms) + extra)
-    rng = np.random.default_rng(900 + B + tpi)
-    Hq, Hkv, D, T = 4, 1, 128, 320
+    rng = np.random.default_rng(900 + B + tpi + D)
+    Hkv, T = 1, 320
     q = rand_bits(rng, (B, Hq, D))
     K = rand_bits(rng, (B, Hkv, T, D))
     V = rand_bits(rng, (B, Hkv, T, D))
